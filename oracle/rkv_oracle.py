@@ -1,0 +1,160 @@
+"""fp64 CPU oracle for decode-time KV-cache scoring, selection and compaction.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import or run anything in this directory.  The
+product path (the CUDA library and its Python binding) never calls it and shares
+no code with it.
+
+Source: the R-KV article (QbitAI repost, "R-KV三步走：冗余识别+重要性评估+动态淘汰"),
+which names the method's steps in this order:
+
+* 边生成边压缩 (decoding-time compression): the step runs on the cache of one
+  (sequence, layer, KV head) while decoding;
+* 重要性打分 (importance): multi-head attention estimates each token's
+  contribution to what follows;
+* 冗余打分 (redundancy): cosine similarity between key vectors finds repeated
+  content;
+* 联合淘汰 (joint eviction): keep high-importance, low-redundancy tokens within
+  the KV budget, best at lambda ~ 0.1.
+
+The page gives only these ingredients.  The exact formulas written out below
+are the reading this engine adopts for them (plain attention softmax averaged
+over window queries and the GQA group; row-mean cosine similarity with the
+diagonal excluded, then a softmax over tokens; s = lam*a - (1-lam)*r; keep the
+last w tokens and the top-B of the rest, ties to the lower index).
+
+Notation: one unit has N cached keys K [N, d] (and values V), window w, group G,
+queries Q [G, w, d]; query (g, t) sits at position N - w + t and attends to keys
+j <= N - w + t.  Candidates C = {0 .. N-w-1}.  Everything is float64; inputs
+are the exact widening of the bf16 values.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def key_norms(K: np.ndarray) -> np.ndarray:
+    """||k_i|| for every key (冗余打分 needs cosine similarity, i.e. unit keys)."""
+    return np.sqrt(np.einsum("nd,nd->n", K, K))
+
+
+def unit_keys(K: np.ndarray) -> np.ndarray:
+    """k_hat_i = k_i / ||k_i||, with k_hat_i = 0 for a zero key."""
+    nrm = key_norms(K)
+    inv = np.zeros_like(nrm)
+    nz = nrm > 0
+    inv[nz] = 1.0 / nrm[nz]
+    return K * inv[:, None]
+
+
+def attention_probs(Q: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """p[g, t, j]: causal softmax of q_{g,t} . k_j / sqrt(d) over j <= N-w+t
+    (重要性打分: the attention that the most recent decode queries pay to each
+    cached token).  Masked entries are exactly 0."""
+    G, w, d = Q.shape
+    N = K.shape[0]
+    z = np.einsum("gtd,nd->gtn", Q, K) / np.sqrt(d)
+    pos = N - w + np.arange(w)                       # position of query t
+    visible = np.arange(N)[None, :] <= pos[:, None]  # [w, N]
+    z = np.where(visible[None], z, -np.inf)
+    zmax = z.max(axis=2, keepdims=True)
+    e = np.exp(z - zmax)
+    return e / e.sum(axis=2, keepdims=True)
+
+
+def importance(Q: np.ndarray, K: np.ndarray):
+    """Importance (重要性打分).
+
+    a_bar_j = mean over (g, t) of p[g, t, j]; a_i = a_bar_i / sum_{j in C} a_bar_j
+    for i in C.  Returns (a_bar [N], a [N - w])."""
+    G, w, d = Q.shape
+    N = K.shape[0]
+    abar = attention_probs(Q, K).mean(axis=(0, 1))
+    c = N - w
+    if c <= 0:
+        return abar, np.zeros(0)
+    return abar, abar[:c] / abar[:c].sum()
+
+
+def redundancy_mean(K: np.ndarray, w: int, block: int = 2048):
+    """Redundancy (冗余打分), straight from the definition, in row blocks.
+
+    S_ij = k_hat_i . k_hat_j; m_i = sum_{j != i, j < N} S_ij / (N - 1) for i in C;
+    r = softmax over C of m.  The N x N matrix is never held whole.
+    Returns (m [N - w], r [N - w])."""
+    N = K.shape[0]
+    c = N - w
+    if c <= 0:
+        return np.zeros(0), np.zeros(0)
+    kh = unit_keys(K)
+    m = np.empty(c)
+    for i0 in range(0, c, block):
+        i1 = min(c, i0 + block)
+        S = kh[i0:i1] @ kh.T                              # [rows, N]
+        S[np.arange(i1 - i0), np.arange(i0, i1)] = 0.0    # exclude j == i
+        m[i0:i1] = S.sum(axis=1) / (N - 1)
+    return m, softmax(m)
+
+
+def redundancy_mean_closed_form(K: np.ndarray, w: int):
+    """The same m as :func:`redundancy_mean`, by linearity of the row sum:
+    sum_{j != i} k_hat_i . k_hat_j = k_hat_i . U - k_hat_i . k_hat_i with
+    U = sum_j k_hat_j.  O(N d) instead of O(N^2 d); exact up to rounding."""
+    N = K.shape[0]
+    c = N - w
+    if c <= 0:
+        return np.zeros(0), np.zeros(0)
+    kh = unit_keys(K)
+    U = kh.sum(axis=0)
+    m = (kh[:c] @ U - np.einsum("nd,nd->n", kh[:c], kh[:c])) / (N - 1)
+    return m, softmax(m)
+
+
+def softmax(x: np.ndarray) -> np.ndarray:
+    if x.size == 0:
+        return x.copy()
+    e = np.exp(x - x.max())
+    return e / e.sum()
+
+
+def joint_score(a: np.ndarray, r: np.ndarray, lam: float) -> np.ndarray:
+    """Joint eviction score (联合淘汰): s_i = lam * a_i - (1 - lam) * r_i."""
+    return lam * a - (1.0 - lam) * r
+
+
+def select(s: np.ndarray, N: int, w: int, budget: int):
+    """Kept indices (联合淘汰 under the KV budget).
+
+    Rank candidates by (s descending, index ascending); keep the first
+    min(budget, N - w); return them in ascending order followed by the window
+    N - w .. N - 1.  If N - w <= budget every token is kept."""
+    c = N - w
+    if c <= budget:
+        return np.arange(N, dtype=np.int64)
+    order = np.lexsort((np.arange(c), -s))     # primary key: -s; then index
+    kept = np.sort(order[:budget])
+    return np.concatenate([kept, np.arange(c, N)]).astype(np.int64)
+
+
+def compact(K: np.ndarray, V: np.ndarray, idx: np.ndarray):
+    """Gather-based compaction of the surviving rows (the R-KV-style baseline
+    named in the ThinKV summary): K'[j] = K[idx[j]], V'[j] = V[idx[j]]."""
+    return K[idx], V[idx]
+
+
+def run_unit(Q, K, V, w: int, budget: int, lam: float, redundancy="rowblocks"):
+    """Whole path for one unit.  ``redundancy`` picks the definition
+    (``rowblocks``) or the closed form (``closed``)."""
+    N = K.shape[0]
+    abar, a = importance(Q, K)
+    if redundancy == "rowblocks":
+        m, r = redundancy_mean(K, w)
+    elif redundancy == "closed":
+        m, r = redundancy_mean_closed_form(K, w)
+    else:
+        raise ValueError(redundancy)
+    s = joint_score(a, r, lam)
+    idx = select(s, N, w, budget)
+    Kc, Vc = compact(K, V, idx)
+    return dict(abar=abar, a=a, m=m, r=r, s=s, idx=idx, K=Kc, V=Vc,
+                norms=key_norms(K))

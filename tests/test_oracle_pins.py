@@ -1,0 +1,316 @@
+"""Pins for the fp64 oracle: things other than the oracle itself that fix what
+it must compute (R-KV article, "R-KV三步走": 重要性打分, 冗余打分, 联合淘汰).
+
+* a hand-derived 6-token worked example (tests/golden/worked_6token.json);
+* a second, loop-only transcription on tiny inputs;
+* textbook special cases (w = 1, G = 1 reduces importance to a plain softmax,
+  checked against scipy);
+* brute force over every budget-subset for N <= 12;
+* invariants: B >= N - w keeps everything, lambda = 1 is pure attention top-B,
+  lambda = 0 keeps the least redundant, permutation equivariance, cosine scale
+  invariance, exact duplicates tie, heavily repeated keys are the most
+  redundant, GQA averaging is linear in the heads;
+* mutation checks: a planted mistake in a copy of the oracle fails the pins.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+
+from oracle import loops
+from oracle import rkv_oracle as ora
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden", "worked_6token.json")
+
+
+def _worked():
+    with open(GOLD) as f:
+        g = json.load(f)
+    K = np.array(g["K"], dtype=np.float64)
+    Q = np.array(g["Q"], dtype=np.float64).reshape(g["group"], g["window"], g["d"])
+    return g, Q, K
+
+
+def check_worked_example(o):
+    """Return a list of mismatches of oracle module ``o`` against the fixture."""
+    g, Q, K = _worked()
+    w, B, tol = g["window"], g["budget"], g["tolerance"]
+    bad = []
+    p = o.attention_probs(Q, K)[0]
+    if not np.allclose(p, g["p"], atol=tol, rtol=0):
+        bad.append("p")
+    abar, a = o.importance(Q, K)
+    if not np.allclose(abar, g["abar"], atol=tol, rtol=0):
+        bad.append("abar")
+    if not np.allclose(a, g["a"], atol=tol, rtol=0):
+        bad.append("a")
+    for fn in (o.redundancy_mean, o.redundancy_mean_closed_form):
+        m, r = fn(K, w)
+        if not np.allclose(m, g["m"], atol=tol, rtol=0):
+            bad.append(fn.__name__ + ".m")
+        if not np.allclose(r, g["r"], atol=tol, rtol=0):
+            bad.append(fn.__name__ + ".r")
+    m, r = o.redundancy_mean(K, w)
+    s = o.joint_score(a, r, 0.1)
+    if not np.allclose(s, g["s"]["0.1"], atol=tol, rtol=0):
+        bad.append("s")
+    for lam, want in g["idx"].items():
+        s = o.joint_score(a, r, float(lam))
+        idx = o.select(s, K.shape[0], w, B)
+        if list(idx) != want:
+            bad.append("idx@" + lam)
+    return bad
+
+
+def test_worked_example():
+    assert check_worked_example(ora) == []
+
+
+def test_worked_example_through_run_unit():
+    g, Q, K = _worked()
+    V = np.arange(12, dtype=np.float64).reshape(6, 2)
+    out = ora.run_unit(Q, K, V, g["window"], g["budget"], 0.1)
+    assert list(out["idx"]) == g["idx"]["0.1"]
+    np.testing.assert_array_equal(out["V"], V[[2, 3, 4, 5]])
+    np.testing.assert_array_equal(out["K"], K[[2, 3, 4, 5]])
+
+
+def _rand_unit(rng, N, d, G, w, dup=0.0):
+    K = rng.standard_normal((N, d))
+    if dup:
+        for i in range(1, N):
+            if rng.random() < dup:
+                K[i] = K[rng.integers(0, i)]
+    Q = rng.standard_normal((G, w, d))
+    return Q, K
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_matches_loop_transcription(seed):
+    rng = np.random.default_rng(seed)
+    N = int(rng.integers(4, 40))
+    w = int(rng.integers(1, min(N - 1, 6) + 1))
+    d = int(rng.choice([2, 3, 8, 16]))
+    G = int(rng.integers(1, 4))
+    B = int(rng.integers(0, N))
+    lam = float(rng.choice([0.0, 0.1, 0.5, 1.0]))
+    Q, K = _rand_unit(rng, N, d, G, w, dup=0.2)
+    V = rng.standard_normal((N, d))
+    ref = loops.run_unit(Q.tolist(), K.tolist(), w, B, lam)
+    out = ora.run_unit(Q, K, V, w, B, lam)
+    np.testing.assert_allclose(out["abar"], ref["abar"], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(out["a"], ref["a"], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(out["m"], ref["m"], rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(out["r"], ref["r"], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(out["s"], ref["s"], rtol=1e-10, atol=1e-14)
+    assert list(out["idx"]) == ref["idx"]
+
+
+@pytest.mark.parametrize("N", [300, 2049, 4100])
+def test_closed_form_equals_definition(N):
+    rng = np.random.default_rng(N)
+    K = rng.standard_normal((N, 128)) * rng.uniform(0.5, 4, size=128)
+    K[5] = K[3]          # an exact duplicate
+    K[7] = 0.0           # a zero key
+    m1, r1 = ora.redundancy_mean(K, 8, block=512)
+    m2, r2 = ora.redundancy_mean_closed_form(K, 8)
+    np.testing.assert_allclose(m2, m1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r2, r1, rtol=1e-10, atol=0)
+    assert m1[7] == 0.0
+
+
+@pytest.mark.parametrize("N", [1, 17, 512])
+def test_single_query_is_textbook_softmax(N):
+    rng = np.random.default_rng(N)
+    d = 128
+    K = rng.standard_normal((N, d))
+    Q = rng.standard_normal((1, 1, d))
+    abar, a = ora.importance(Q, K)
+    want = scipy.special.softmax(K @ Q[0, 0] / math.sqrt(d))
+    np.testing.assert_allclose(abar, want, rtol=1e-12)
+    if N > 1:
+        np.testing.assert_allclose(a, want[:-1] / want[:-1].sum(), rtol=1e-12)
+
+
+def test_causal_mask_hides_later_keys():
+    rng = np.random.default_rng(3)
+    Q, K = _rand_unit(rng, 20, 8, 2, 4)
+    p = ora.attention_probs(Q, K)
+    for t in range(4):
+        last = 20 - 4 + t
+        assert np.all(p[:, t, last + 1:] == 0)
+        assert np.all(p[:, t, :last + 1] > 0)
+        np.testing.assert_allclose(p[:, t].sum(axis=1), 1.0, rtol=1e-13)
+
+
+def test_gqa_average_is_linear_in_heads():
+    rng = np.random.default_rng(4)
+    Q, K = _rand_unit(rng, 50, 16, 3, 4)
+    abar, _ = ora.importance(Q, K)
+    per_head = [ora.importance(Q[g:g + 1], K)[0] for g in range(3)]
+    np.testing.assert_allclose(abar, np.mean(per_head, axis=0), rtol=1e-13)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_selection_matches_subset_brute_force(seed):
+    rng = np.random.default_rng(100 + seed)
+    N = int(rng.integers(5, 13))
+    w = int(rng.integers(1, 4))
+    B = int(rng.integers(1, N - w + 1))
+    Q, K = _rand_unit(rng, N, 4, 2, w, dup=0.3)
+    for lam in (0.0, 0.1, 1.0):
+        _, a = ora.importance(Q, K)
+        _, r = ora.redundancy_mean(K, w)
+        s = ora.joint_score(a, r, lam)
+        assert list(ora.select(s, N, w, B)) == loops.select_by_subsets(
+            s.tolist(), N, w, B)
+
+
+def test_ties_break_to_lower_index():
+    s = np.array([0.5, 0.2, 0.5, 0.5, 0.1])
+    assert list(ora.select(s, 7, 2, 2)) == [0, 2, 5, 6]
+    assert list(ora.select(s, 7, 2, 3)) == [0, 2, 3, 5, 6]
+
+
+@pytest.mark.parametrize("B", [6, 7, 100])
+def test_budget_at_least_candidates_keeps_all(B):
+    rng = np.random.default_rng(B)
+    Q, K = _rand_unit(rng, 12, 8, 1, 6)
+    out = ora.run_unit(Q, K, K, 6, B, 0.1)
+    assert list(out["idx"]) == list(range(12))
+
+
+def test_lambda_one_is_pure_attention_topB():
+    rng = np.random.default_rng(7)
+    Q, K = _rand_unit(rng, 400, 32, 4, 8)
+    out = ora.run_unit(Q, K, K, 8, 50, 1.0)
+    _, a = ora.importance(Q, K)
+    thr = np.sort(a)[::-1][49]
+    kept = out["idx"][:-8]
+    assert len(kept) == 50 and np.all(a[kept] >= thr)
+    assert np.all(np.delete(a, kept) <= thr)
+
+
+def test_lambda_zero_keeps_least_redundant():
+    rng = np.random.default_rng(8)
+    Q, K = _rand_unit(rng, 400, 32, 4, 8, dup=0.2)
+    out = ora.run_unit(Q, K, K, 8, 60, 0.0)
+    m, _ = ora.redundancy_mean_closed_form(K, 8)
+    kept = out["idx"][:-8]
+    assert m[kept].max() <= np.delete(m, kept).min() + 1e-15
+
+
+def test_candidate_permutation_equivariance():
+    rng = np.random.default_rng(9)
+    N, w, B = 300, 8, 40
+    Q, K = _rand_unit(rng, N, 16, 2, w)
+    V = rng.standard_normal((N, 16))
+    perm = np.concatenate([rng.permutation(N - w), np.arange(N - w, N)])
+    o1 = ora.run_unit(Q, K, V, w, B, 0.1)
+    o2 = ora.run_unit(Q, K[perm], V[perm], w, B, 0.1)
+    np.testing.assert_allclose(o2["a"], o1["a"][perm[:N - w]], rtol=1e-12)
+    np.testing.assert_allclose(o2["r"], o1["r"][perm[:N - w]], rtol=1e-12)
+    # kept sets map onto each other (no exact ties in continuous random data)
+    kept1 = set(o1["idx"][:-w].tolist())
+    kept2 = set(perm[o2["idx"][:-w]].tolist())
+    assert kept1 == kept2
+
+
+def test_cosine_scale_invariance():
+    rng = np.random.default_rng(10)
+    K = rng.standard_normal((200, 32))
+    m1, r1 = ora.redundancy_mean(K, 4)
+    m2, r2 = ora.redundancy_mean(K * rng.uniform(0.1, 10, size=(200, 1)), 4)
+    np.testing.assert_allclose(m2, m1, rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(r2, r1, rtol=1e-11)
+
+
+def test_exact_duplicates_tie_and_repeats_are_most_redundant():
+    rng = np.random.default_rng(11)
+    # margin of a 16-fold key: 15/(N-1) ~ 0.05; spread of m among i.i.d.
+    # keys: 1/sqrt(d N) ~ 0.005, so the repeats must top the ranking
+    N, d = 300, 128
+    K = rng.standard_normal((N, d))
+    rep = list(range(10, 290, 18))                       # 16 copies of key 10
+    K[rep] = K[10]
+    K[20] = 3.0 * K[30]                                  # same direction
+    m, r = ora.redundancy_mean(K, 8)
+    # identical up to the summation order of the BLAS row blocks
+    np.testing.assert_allclose(m[rep], m[rep[0]], rtol=1e-13, atol=0)
+    np.testing.assert_allclose(r[rep], r[rep[0]], rtol=1e-13, atol=0)
+    assert m[20] == pytest.approx(m[30], abs=1e-15)
+    assert set(np.argsort(m)[::-1][:len(rep)].tolist()) == set(rep)
+
+
+def test_degenerate_no_candidates():
+    rng = np.random.default_rng(12)
+    Q, K = _rand_unit(rng, 6, 4, 1, 6)
+    out = ora.run_unit(Q, K, K, 6, 3, 0.1)
+    assert out["a"].size == 0 and out["r"].size == 0
+    assert list(out["idx"]) == list(range(6))
+
+
+# ---- mutation checks: each planted mistake must fail a pin ----------------
+
+class _Mutant:
+    def __init__(self, **over):
+        for k in dir(ora):
+            if not k.startswith("__"):
+                setattr(self, k, getattr(ora, k))
+        for k, v in over.items():
+            setattr(self, k, v)
+
+
+def _no_causal_mask(Q, K):
+    G, w, d = Q.shape
+    z = np.einsum("gtd,nd->gtn", Q, K) / np.sqrt(d)
+    e = np.exp(z - z.max(axis=2, keepdims=True))
+    return e / e.sum(axis=2, keepdims=True)
+
+
+def _no_scale(Q, K):
+    return ora.attention_probs(Q * np.sqrt(Q.shape[2]), K)
+
+
+def _diag_kept(K, w, block=2048):
+    N = K.shape[0]
+    kh = ora.unit_keys(K)
+    m = (kh[:N - w] @ kh.T).sum(axis=1) / (N - 1)
+    return m, ora.softmax(m)
+
+
+def _not_normalised(K, w, block=2048):
+    N = K.shape[0]
+    S = K[:N - w] @ K.T
+    S[np.arange(N - w), np.arange(N - w)] = 0
+    m = S.sum(axis=1) / (N - 1)
+    return m, ora.softmax(m)
+
+
+def _wrong_sign(a, r, lam):
+    return lam * a + (1 - lam) * r
+
+
+def _ties_high(s, N, w, budget):
+    c = N - w
+    if c <= budget:
+        return np.arange(N)
+    order = np.lexsort((-np.arange(c), -s))
+    return np.concatenate([np.sort(order[:budget]), np.arange(c, N)])
+
+
+@pytest.mark.parametrize("over", [
+    dict(attention_probs=_no_causal_mask),
+    dict(attention_probs=_no_scale),
+    dict(redundancy_mean=_diag_kept, redundancy_mean_closed_form=_diag_kept),
+    dict(redundancy_mean=_not_normalised,
+         redundancy_mean_closed_form=_not_normalised),
+    dict(joint_score=_wrong_sign),
+    dict(select=_ties_high),
+], ids=["no-causal-mask", "no-1/sqrt(d)", "diagonal-kept", "raw-dot-not-cosine",
+        "wrong-sign", "ties-to-high-index"])
+def test_planted_mistake_fails_worked_example(over):
+    assert check_worked_example(_Mutant(**over)) != []
