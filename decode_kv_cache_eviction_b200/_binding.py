@@ -1,0 +1,223 @@
+"""Thin ctypes binding of ``librkv.so`` (argument marshalling only).
+
+Every computation runs in the library's CUDA kernels; this module only turns
+torch tensors into pointers and stream handles, checks dtypes and shapes, and
+turns status codes into exceptions.  There is no fallback: if the library is
+missing, loading fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librkv.so")
+
+RKV_OK = 0
+RKV_ERR_INVALID_ARG = -1
+RKV_ERR_UNSUPPORTED = -2
+RKV_ERR_CUDA = -3
+RKV_ERR_TIMEOUT = -4
+RKV_ERR_OOM = -5
+RKV_ERR_CAPACITY = -6
+RKV_ERR_DEVICE = -7
+
+RKV_REDUNDANCY_GEMM = 0
+RKV_REDUNDANCY_CLOSED_FORM = 1
+RKV_FLAG_GEMM_SINGLE_CTA = 1
+
+# Every function declared in include/rkv.h.
+EXPORTS = ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact",
+           "rkv_compress", "rkv_check_status", "rkv_launch_count", "rkv_set_timing",
+           "rkv_read_timing", "rkv_status_string", "rkv_version")
+KERNELS = ("score", "plan", "gemm", "select", "compact")
+
+
+class RkvConfig(ctypes.Structure):
+    _fields_ = [("head_dim", ctypes.c_int), ("group", ctypes.c_int),
+                ("window", ctypes.c_int), ("max_units", ctypes.c_int),
+                ("max_tokens", ctypes.c_int64), ("redundancy", ctypes.c_int),
+                ("flags", ctypes.c_int)]
+
+
+class RkvBatch(ctypes.Structure):
+    _fields_ = [("num_units", ctypes.c_int), ("tok_off", ctypes.c_void_p),
+                ("tok_off_host", ctypes.c_void_p), ("K", ctypes.c_void_p),
+                ("V", ctypes.c_void_p), ("Q", ctypes.c_void_p)]
+
+
+class RkvError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+
+
+_lib = None
+
+
+def lib():
+    """Load ``librkv.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m decode_kv_cache_eviction_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    L.rkv_create.argtypes = [ctypes.POINTER(RkvConfig), ctypes.POINTER(vp)]
+    L.rkv_destroy.argtypes = [vp]
+    L.rkv_score.argtypes = [vp, ctypes.POINTER(RkvBatch), vp, vp, vp, vp]
+    L.rkv_select.argtypes = [vp, ctypes.POINTER(RkvBatch), vp, vp, f32, i32, vp, vp, vp]
+    L.rkv_compact.argtypes = [vp, ctypes.POINTER(RkvBatch), vp, vp, i32, vp, vp, vp]
+    L.rkv_compress.argtypes = [vp, ctypes.POINTER(RkvBatch), f32, i32, vp, vp, vp, vp, vp,
+                               vp, vp]
+    L.rkv_check_status.argtypes = [vp, vp]
+    L.rkv_launch_count.argtypes = [vp]
+    L.rkv_launch_count.restype = i64
+    L.rkv_set_timing.argtypes = [vp, i32]
+    L.rkv_read_timing.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_double),
+                                  ctypes.POINTER(i64)]
+    L.rkv_status_string.argtypes = [i32]
+    L.rkv_status_string.restype = ctypes.c_char_p
+    L.rkv_version.argtypes = []
+    for name in ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact",
+                 "rkv_compress", "rkv_check_status", "rkv_set_timing", "rkv_read_timing",
+                 "rkv_version"):
+        getattr(L, name).restype = i32
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return lib().rkv_status_string(code).decode()
+
+
+def _check(code: int, what: str):
+    if code != RKV_OK:
+        raise RkvError(code, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class Batch:
+    """Views of one batch of unit caches (tensors stay owned by the caller).
+
+    K, V: [T, d] bf16 CUDA tensors; Q: [U, G, w, d] bf16; tok_off: host int64
+    offsets [U+1] (a device copy is made once, here)."""
+
+    def __init__(self, K, V, Q, tok_off):
+        for name, t in (("K", K), ("V", V), ("Q", Q)):
+            if t is not None:
+                if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+                    raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+        self.K, self.V, self.Q = K, V, Q
+        off = np.ascontiguousarray(np.asarray(tok_off, dtype=np.int64))
+        self.tok_off_host = off
+        dev = (K if K is not None else Q).device
+        self.tok_off = torch.from_numpy(off).to(dev)
+        self.c = RkvBatch(len(off) - 1, self.tok_off.data_ptr(),
+                          off.ctypes.data, _ptr(K), _ptr(V), _ptr(Q))
+
+    @property
+    def num_units(self):
+        return len(self.tok_off_host) - 1
+
+    @property
+    def num_tokens(self):
+        return int(self.tok_off_host[-1])
+
+
+class Engine:
+    """One engine = one configuration and its device workspace."""
+
+    def __init__(self, group: int, window: int, max_units: int, max_tokens: int,
+                 head_dim: int = 128, redundancy: str = "gemm", single_cta_gemm=False):
+        mode = {"gemm": RKV_REDUNDANCY_GEMM, "closed": RKV_REDUNDANCY_CLOSED_FORM}[redundancy]
+        self.cfg = RkvConfig(head_dim, group, window, max_units, max_tokens, mode,
+                             RKV_FLAG_GEMM_SINGLE_CTA if single_cta_gemm else 0)
+        self.group, self.window = group, window
+        h = ctypes.c_void_p()
+        _check(lib().rkv_create(ctypes.byref(self.cfg), ctypes.byref(h)), "rkv_create")
+        self.h = h
+
+    def close(self):
+        if getattr(self, "h", None):
+            lib().rkv_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- calls ----------------------------------------------------------------
+    def score(self, batch: Batch, a, r, m=None, stream=None):
+        _check(lib().rkv_score(self.h, ctypes.byref(batch.c), _ptr(a), _ptr(r), _ptr(m),
+                               _stream(stream)), "rkv_score")
+
+    def select(self, batch: Batch, a, r, lam: float, budget: int, idx, n_kept, stream=None):
+        _check(lib().rkv_select(self.h, ctypes.byref(batch.c), _ptr(a), _ptr(r),
+                                float(lam), int(budget), _ptr(idx), _ptr(n_kept),
+                                _stream(stream)), "rkv_select")
+
+    def compact(self, batch: Batch, idx, n_kept, budget: int, K_out, V_out, stream=None):
+        _check(lib().rkv_compact(self.h, ctypes.byref(batch.c), _ptr(idx), _ptr(n_kept),
+                                 int(budget), _ptr(K_out), _ptr(V_out), _stream(stream)),
+               "rkv_compact")
+
+    def compress(self, batch: Batch, lam: float, budget: int, a, r, idx, n_kept, K_out,
+                 V_out, stream=None):
+        _check(lib().rkv_compress(self.h, ctypes.byref(batch.c), float(lam), int(budget),
+                                  _ptr(a), _ptr(r), _ptr(idx), _ptr(n_kept), _ptr(K_out),
+                                  _ptr(V_out), _stream(stream)), "rkv_compress")
+
+    def check_status(self, stream=None):
+        _check(lib().rkv_check_status(self.h, _stream(stream)), "device status")
+
+    def set_timing(self, enable: bool):
+        _check(lib().rkv_set_timing(self.h, 1 if enable else 0), "rkv_set_timing")
+
+    def read_timing(self):
+        """{kernel: (total_ms, launches)} since the previous read."""
+        out = {}
+        for k, name in enumerate(KERNELS):
+            ms, n = ctypes.c_double(), ctypes.c_int64()
+            _check(lib().rkv_read_timing(self.h, k, ctypes.byref(ms), ctypes.byref(n)),
+                   "rkv_read_timing")
+            out[name] = (ms.value, n.value)
+        lib().rkv_set_timing(self.h, 1)   # forget what was read
+        return out
+
+    @property
+    def launches(self) -> int:
+        return int(lib().rkv_launch_count(self.h))
+
+    # -- allocation helpers (caller-owned outputs) ------------------------------
+    def alloc_scores(self, batch: Batch):
+        T = batch.num_tokens
+        dev = batch.K.device
+        return (torch.empty(T, dtype=torch.float32, device=dev),
+                torch.empty(T, dtype=torch.float32, device=dev))
+
+    def alloc_outputs(self, batch: Batch, budget: int):
+        U, W = batch.num_units, budget + self.window
+        dev = batch.K.device
+        return (torch.empty((U, W), dtype=torch.int32, device=dev),
+                torch.empty(U, dtype=torch.int32, device=dev),
+                torch.empty((U, W, 128), dtype=torch.bfloat16, device=dev),
+                torch.empty((U, W, 128), dtype=torch.bfloat16, device=dev))

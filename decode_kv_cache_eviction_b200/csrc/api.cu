@@ -1,0 +1,458 @@
+// C ABI of the engine: argument validation, workspace, tensor maps, launches.
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "../../include/rkv.h"
+#include "ptx.cuh"
+#include "rkv_internal.cuh"
+
+using namespace rkv;
+
+struct rkv_engine {
+  rkv_config cfg;
+  int device = 0;
+  int nsm = 0;
+  int rp = 32;                 // padded G*w (MMA N of the logits tile)
+  int lmax = 0;                // tokens per score CTA the layout is sized for
+  int nstages = 0;             // score K-tile ring depth
+  int score_smem = 0;
+  int score_clusters[5] = {};  // active clusters for cluster sizes 1, 2, 4, 8, 16
+  int max_cs = 16;
+  int max_n = 0;               // largest supported N_u
+  bool pair = true;
+  int gemm_ctas = 0;
+  float* rho = nullptr;        // [max_tokens]
+  int* item_off = nullptr;     // [max_units + 1]
+  int* unit_cnt = nullptr;     // [max_units]
+  int* status = nullptr;       // [1]
+  int64_t launches = 0;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  // per-kernel timing (rkv_set_timing)
+  static constexpr int kMaxEv = 4096;
+  bool timing = false;
+  cudaEvent_t ev[kMaxEv][2] = {};
+  int ev_kernel[kMaxEv] = {};
+  int nev = 0;
+  bool ev_made = false;
+};
+
+namespace {
+
+constexpr int kSmemCap = 227 * 1024;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_fail(cudaError_t e) {
+  (void)e;
+  cudaGetLastError();
+  return RKV_ERR_CUDA;
+}
+
+int make_map(rkv_engine* e, CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = e->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RKV_OK : RKV_ERR_CUDA;
+}
+
+// Host-side checks of a batch against the engine; fills T and the largest N.
+int check_batch(const rkv_engine* e, const rkv_batch* b, int64_t* T, int* nmax, int* cmax) {
+  if (!b) return RKV_ERR_INVALID_ARG;
+  if (b->num_units < 0) return RKV_ERR_INVALID_ARG;
+  if (b->num_units > e->cfg.max_units) return RKV_ERR_CAPACITY;
+  if (!b->tok_off_host || !b->tok_off) return RKV_ERR_INVALID_ARG;
+  const int64_t* off = b->tok_off_host;
+  if (off[0] != 0) return RKV_ERR_INVALID_ARG;
+  int nm = 0;
+  for (int u = 0; u < b->num_units; ++u) {
+    const int64_t n = off[u + 1] - off[u];
+    if (n < e->cfg.window) return RKV_ERR_INVALID_ARG;
+    if (n > e->max_n) return RKV_ERR_UNSUPPORTED;
+    if (n > nm) nm = static_cast<int>(n);
+  }
+  const int64_t t = off[b->num_units];
+  if (t > e->cfg.max_tokens) return RKV_ERR_CAPACITY;
+  if (!aligned(b->tok_off, 8)) return RKV_ERR_INVALID_ARG;
+  *T = t;
+  *nmax = nm;
+  *cmax = nm - e->cfg.window;
+  return RKV_OK;
+}
+
+// Record the start event of a launch of `kernel` (when timing is on).
+void t_begin(rkv_engine* e, int kernel, cudaStream_t st) {
+  if (!e->timing || e->nev >= rkv_engine::kMaxEv) return;
+  e->ev_kernel[e->nev] = kernel;
+  cudaEventRecord(e->ev[e->nev][0], st);
+}
+void t_end(rkv_engine* e, cudaStream_t st) {
+  if (!e->timing || e->nev >= rkv_engine::kMaxEv) return;
+  cudaEventRecord(e->ev[e->nev][1], st);
+  ++e->nev;
+}
+
+int cs_index(int cs) {
+  int i = 0;
+  while ((1 << i) < cs) ++i;
+  return i;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rkv_version(void) { return 10000; }
+
+const char* rkv_status_string(int s) {
+  switch (s) {
+    case RKV_OK: return "ok";
+    case RKV_ERR_INVALID_ARG: return "invalid argument";
+    case RKV_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case RKV_ERR_CUDA: return "CUDA runtime error";
+    case RKV_ERR_TIMEOUT: return "device wait timed out";
+    case RKV_ERR_OOM: return "device allocation failed";
+    case RKV_ERR_CAPACITY: return "batch exceeds engine capacity";
+    case RKV_ERR_DEVICE: return "kept index outside its unit";
+    default: return "unknown status";
+  }
+}
+
+int rkv_create(const rkv_config* cfg, rkv_engine** out) {
+  if (!cfg || !out) return RKV_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (cfg->group < 1 || cfg->window < 1 || cfg->max_units < 1 || cfg->max_tokens < 1)
+    return RKV_ERR_INVALID_ARG;
+  if (cfg->redundancy != RKV_REDUNDANCY_GEMM && cfg->redundancy != RKV_REDUNDANCY_CLOSED_FORM)
+    return RKV_ERR_INVALID_ARG;
+  if ((cfg->flags & ~RKV_FLAG_GEMM_SINGLE_CTA) != 0) return RKV_ERR_INVALID_ARG;
+  if (cfg->head_dim != kHeadDim) return RKV_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(cfg->group) * cfg->window > kMaxRows) return RKV_ERR_UNSUPPORTED;
+  if (cfg->max_tokens >= (static_cast<int64_t>(1) << 31)) return RKV_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(cfg->max_units) * cfg->group * cfg->window >=
+      (static_cast<int64_t>(1) << 31))
+    return RKV_ERR_UNSUPPORTED;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail(cudaErrorNoDevice);
+  int major = 0, minor = 0, nsm = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cuda_fail(cudaErrorUnknown);
+  if (major != 10 || minor != 0) return RKV_ERR_UNSUPPORTED;
+
+  rkv_engine* e = new (std::nothrow) rkv_engine();
+  if (!e) return RKV_ERR_OOM;
+  e->cfg = *cfg;
+  e->device = dev;
+  e->nsm = nsm;
+  e->rp = cfg->group * cfg->window <= 16 ? 16 : 32;
+  e->pair = (cfg->flags & RKV_FLAG_GEMM_SINGLE_CTA) == 0;
+
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn) {
+    delete e;
+    return cuda_fail(cudaErrorUnknown);
+  }
+  e->encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+
+  // Score kernel layout: 3072 tokens per CTA, deepest K ring that fits.
+  const bool closed = cfg->redundancy == RKV_REDUNDANCY_CLOSED_FORM;
+  e->lmax = 3072;
+  e->nstages = 0;
+  for (int ns = 8; ns >= 3; --ns) {
+    if (static_cast<int>(score_layout(e->rp, closed, e->lmax, ns).total) + 1024 <= kSmemCap) {
+      e->nstages = ns;
+      break;
+    }
+  }
+  e->score_smem = score_layout(e->rp, closed, e->lmax, e->nstages).total + 1024;
+  if (score_configure(e->rp, closed, e->score_smem, 16) != cudaSuccess) {
+    delete e;
+    return cuda_fail(cudaErrorUnknown);
+  }
+  e->max_cs = 0;
+  for (int i = 0; i < 5; ++i) {
+    e->score_clusters[i] = score_max_clusters(e->rp, closed, e->score_smem, 1 << i);
+    if (e->score_clusters[i] > 0) e->max_cs = 1 << i;
+    else break;
+  }
+  if (e->max_cs == 0) {
+    delete e;
+    return RKV_ERR_UNSUPPORTED;
+  }
+  e->max_n = e->max_cs * e->lmax;
+  if (e->max_n > kMaxTokensPerUnit) e->max_n = kMaxTokensPerUnit;
+
+  if (select_configure() != cudaSuccess) {
+    delete e;
+    return cuda_fail(cudaErrorUnknown);
+  }
+  if (!closed) {
+    if (gemm_configure(e->pair) != cudaSuccess) {
+      delete e;
+      return cuda_fail(cudaErrorUnknown);
+    }
+    e->gemm_ctas = gemm_max_ctas(e->pair);
+    if (e->gemm_ctas <= 0) {
+      delete e;
+      return RKV_ERR_UNSUPPORTED;
+    }
+  }
+
+  bool ok = cudaMalloc(&e->status, 16) == cudaSuccess;
+  ok = ok && cudaMalloc(&e->item_off, sizeof(int) * (cfg->max_units + 1)) == cudaSuccess;
+  ok = ok && cudaMalloc(&e->unit_cnt, sizeof(int) * cfg->max_units) == cudaSuccess;
+  if (!closed) ok = ok && cudaMalloc(&e->rho, sizeof(float) * cfg->max_tokens) == cudaSuccess;
+  ok = ok && cudaMemset(e->status, 0, 16) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    cudaFree(e->status);
+    cudaFree(e->item_off);
+    cudaFree(e->unit_cnt);
+    cudaFree(e->rho);
+    delete e;
+    return RKV_ERR_OOM;
+  }
+  *out = e;
+  return RKV_OK;
+}
+
+int rkv_set_timing(rkv_engine* e, int enable) {
+  if (!e) return RKV_ERR_INVALID_ARG;
+  if (enable && !e->ev_made) {
+    for (int i = 0; i < rkv_engine::kMaxEv; ++i)
+      for (int k = 0; k < 2; ++k)
+        if (cudaEventCreate(&e->ev[i][k]) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+    e->ev_made = true;
+  }
+  e->timing = enable != 0;
+  e->nev = 0;
+  return RKV_OK;
+}
+
+int rkv_read_timing(rkv_engine* e, int kernel, double* total_ms, int64_t* launches) {
+  if (!e || !total_ms || !launches || kernel < 0 || kernel >= RKV_NUM_KERNELS)
+    return RKV_ERR_INVALID_ARG;
+  double tot = 0.0;
+  int64_t n = 0;
+  for (int i = 0; i < e->nev; ++i) {
+    if (e->ev_kernel[i] != kernel) continue;
+    if (cudaEventSynchronize(e->ev[i][1]) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, e->ev[i][0], e->ev[i][1]) != cudaSuccess)
+      return cuda_fail(cudaErrorUnknown);
+    tot += ms;
+    ++n;
+  }
+  *total_ms = tot;
+  *launches = n;
+  return RKV_OK;
+}
+
+int rkv_destroy(rkv_engine* e) {
+  if (!e) return RKV_OK;
+  cudaDeviceSynchronize();
+  if (e->ev_made)
+    for (int i = 0; i < rkv_engine::kMaxEv; ++i)
+      for (int k = 0; k < 2; ++k) cudaEventDestroy(e->ev[i][k]);
+  cudaFree(e->status);
+  cudaFree(e->item_off);
+  cudaFree(e->unit_cnt);
+  cudaFree(e->rho);
+  delete e;
+  return RKV_OK;
+}
+
+int64_t rkv_launch_count(const rkv_engine* e) { return e ? e->launches : 0; }
+
+int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
+              rkv_stream_t stream) {
+  if (!e) return RKV_ERR_INVALID_ARG;
+  int64_t T = 0;
+  int nmax = 0, cmax = 0;
+  int rc = check_batch(e, b, &T, &nmax, &cmax);
+  if (rc != RKV_OK) return rc;
+  if (!a || !r || !b->K || !b->Q) return RKV_ERR_INVALID_ARG;
+  if (!aligned(b->K, 16) || !aligned(b->Q, 16) || !aligned(a, 4) || !aligned(r, 4) ||
+      (m && !aligned(m, 4)))
+    return RKV_ERR_INVALID_ARG;
+  const int U = b->num_units;
+  if (U == 0) return RKV_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool closed = e->cfg.redundancy == RKV_REDUNDANCY_CLOSED_FORM;
+  const int R = e->cfg.group * e->cfg.window;
+
+  // cluster size: about 1024 tokens per CTA, at most what the layout holds
+  int cs = 1;
+  while (cs < e->max_cs && (nmax + cs - 1) / cs > 1024) cs <<= 1;
+  while ((((nmax + cs - 1) / cs + kTile - 1) / kTile) * kTile > e->lmax) {
+    if (cs >= e->max_cs) return RKV_ERR_UNSUPPORTED;
+    cs <<= 1;
+  }
+  int ncl = e->score_clusters[cs_index(cs)];
+  if (ncl > U) ncl = U;
+
+  CUtensorMap kmap, qmap;
+  if (make_map(e, &kmap, b->K, static_cast<uint64_t>(T), kTile) != RKV_OK) return RKV_ERR_CUDA;
+  if (make_map(e, &qmap, b->Q, static_cast<uint64_t>(U) * R, e->rp) != RKV_OK)
+    return RKV_ERR_CUDA;
+
+  ScoreParams p;
+  p.tok_off = b->tok_off;
+  p.num_units = U;
+  p.R = R;
+  p.w = e->cfg.window;
+  p.cs = cs;
+  p.lmax = e->lmax;
+  p.nstages = e->nstages;
+  p.scale_log2 = kLog2e / sqrtf(static_cast<float>(kHeadDim));
+  p.a_out = a;
+  p.r_out = r;
+  p.m_out = m;
+  p.rho_out = closed ? nullptr : e->rho;
+  p.status = e->status;
+  t_begin(e, RKV_KERNEL_SCORE, st);
+  cudaError_t err = launch_score(kmap, qmap, p, e->rp, closed, ncl, st);
+  t_end(e, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  ++e->launches;
+  if (closed) return RKV_OK;
+
+  // redundancy GEMM
+  const int rows_per_item = e->pair ? 256 : 128;
+  t_begin(e, RKV_KERNEL_PLAN, st);
+  err = launch_plan(b->tok_off, U, e->cfg.window, rows_per_item, e->item_off, e->unit_cnt, st);
+  t_end(e, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  ++e->launches;
+  CUtensorMap amap, bmap;
+  if (make_map(e, &amap, b->K, static_cast<uint64_t>(T), 128) != RKV_OK) return RKV_ERR_CUDA;
+  if (make_map(e, &bmap, b->K, static_cast<uint64_t>(T), e->pair ? 128 : 256) != RKV_OK)
+    return RKV_ERR_CUDA;
+  GemmParams g;
+  g.tok_off = b->tok_off;
+  g.item_off = e->item_off;
+  g.num_units = U;
+  g.w = e->cfg.window;
+  g.rho = e->rho;
+  g.m_dst = m ? m : r;
+  g.r_dst = r;
+  g.unit_cnt = e->unit_cnt;
+  g.status = e->status;
+  int64_t items = 0;
+  for (int u = 0; u < U; ++u) {
+    const int64_t c = b->tok_off_host[u + 1] - b->tok_off_host[u] - e->cfg.window;
+    if (c > 0) items += (c + rows_per_item - 1) / rows_per_item;
+  }
+  if (items == 0) return RKV_OK;
+  int64_t nctas = e->gemm_ctas;
+  const int64_t need = items * (e->pair ? 2 : 1);
+  if (nctas > need) nctas = need;
+  t_begin(e, RKV_KERNEL_GEMM, st);
+  err = launch_gemm(amap, bmap, g, e->pair, static_cast<int>(nctas), st);
+  t_end(e, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  ++e->launches;
+  return RKV_OK;
+}
+
+int rkv_select(rkv_engine* e, const rkv_batch* b, const float* a, const float* r, float lambda,
+               int budget, int32_t* idx, int32_t* n_kept, rkv_stream_t stream) {
+  if (!e) return RKV_ERR_INVALID_ARG;
+  int64_t T = 0;
+  int nmax = 0, cmax = 0;
+  int rc = check_batch(e, b, &T, &nmax, &cmax);
+  if (rc != RKV_OK) return rc;
+  if (!(lambda >= 0.f && lambda <= 1.f) || budget < 0) return RKV_ERR_INVALID_ARG;
+  if (!a || !r || !idx || !n_kept) return RKV_ERR_INVALID_ARG;
+  if (!aligned(a, 4) || !aligned(r, 4) || !aligned(idx, 4) || !aligned(n_kept, 4))
+    return RKV_ERR_INVALID_ARG;
+  const int U = b->num_units;
+  if (U == 0) return RKV_OK;
+  if (static_cast<int64_t>(budget) + e->cfg.window >= (static_cast<int64_t>(1) << 30) ||
+      static_cast<int64_t>(U) * (budget + e->cfg.window) >= (static_cast<int64_t>(1) << 31))
+    return RKV_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_begin(e, RKV_KERNEL_SELECT, st);
+  cudaError_t err = launch_select(b->tok_off, U, e->cfg.window, cmax, a, r, lambda, budget, idx,
+                                  n_kept, st);
+  t_end(e, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  ++e->launches;
+  return RKV_OK;
+}
+
+int rkv_compact(rkv_engine* e, const rkv_batch* b, const int32_t* idx, const int32_t* n_kept,
+                int budget, void* K_out, void* V_out, rkv_stream_t stream) {
+  if (!e) return RKV_ERR_INVALID_ARG;
+  int64_t T = 0;
+  int nmax = 0, cmax = 0;
+  int rc = check_batch(e, b, &T, &nmax, &cmax);
+  if (rc != RKV_OK) return rc;
+  if (budget < 0 || !idx || !n_kept || !K_out || !V_out || !b->K || !b->V)
+    return RKV_ERR_INVALID_ARG;
+  if (!aligned(b->K, 16) || !aligned(b->V, 16) || !aligned(K_out, 16) || !aligned(V_out, 16) ||
+      !aligned(idx, 4) || !aligned(n_kept, 4))
+    return RKV_ERR_INVALID_ARG;
+  const int U = b->num_units;
+  if (U == 0) return RKV_OK;
+  const int64_t W = static_cast<int64_t>(budget) + e->cfg.window;
+  if (U * W >= (static_cast<int64_t>(1) << 31)) return RKV_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_begin(e, RKV_KERNEL_COMPACT, st);
+  cudaError_t err = launch_compact(b->tok_off, U, static_cast<int>(W), idx, n_kept, b->K, b->V,
+                                   K_out, V_out, e->status, e->nsm, st);
+  t_end(e, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  ++e->launches;
+  return RKV_OK;
+}
+
+int rkv_compress(rkv_engine* e, const rkv_batch* b, float lambda, int budget, float* a, float* r,
+                 int32_t* idx, int32_t* n_kept, void* K_out, void* V_out, rkv_stream_t stream) {
+  if (!e) return RKV_ERR_INVALID_ARG;
+  // validate everything before enqueuing anything
+  int64_t T = 0;
+  int nmax = 0, cmax = 0;
+  int rc = check_batch(e, b, &T, &nmax, &cmax);
+  if (rc != RKV_OK) return rc;
+  if (!(lambda >= 0.f && lambda <= 1.f) || budget < 0 || !a || !r || !idx || !n_kept ||
+      !K_out || !V_out || !b->K || !b->V || !b->Q)
+    return RKV_ERR_INVALID_ARG;
+  if (!aligned(b->V, 16) || !aligned(K_out, 16) || !aligned(V_out, 16))
+    return RKV_ERR_INVALID_ARG;
+  rc = rkv_score(e, b, a, r, nullptr, stream);
+  if (rc != RKV_OK) return rc;
+  rc = rkv_select(e, b, a, r, lambda, budget, idx, n_kept, stream);
+  if (rc != RKV_OK) return rc;
+  return rkv_compact(e, b, idx, n_kept, budget, K_out, V_out, stream);
+}
+
+int rkv_check_status(rkv_engine* e, rkv_stream_t stream) {
+  if (!e) return RKV_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+  int h = 0;
+  if (cudaMemcpy(&h, e->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return cuda_fail(cudaErrorUnknown);
+  if (h != 0 && cudaMemset(e->status, 0, sizeof(int)) != cudaSuccess)
+    return cuda_fail(cudaErrorUnknown);
+  if (h & kStatusTimeout) return RKV_ERR_TIMEOUT;
+  if (h & kStatusBadIndex) return RKV_ERR_DEVICE;
+  if (h != 0) return RKV_ERR_CUDA;
+  return RKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,136 @@
+// Internal declarations shared by the kernels and the C ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rkv {
+
+constexpr int kHeadDim = 128;        // d (the only supported head size)
+constexpr int kTile = 128;           // tokens per K tile (TMA box rows, MMA M)
+constexpr int kTileBytes = kTile * kHeadDim * 2;
+constexpr int kMaxTokensPerUnit = 49152;
+constexpr int kMaxRows = 32;         // G * w limit (MMA N of the logits tile)
+constexpr int kScoreThreads = 384;   // 12 warps
+constexpr int kGemmThreads = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------- score
+struct ScoreParams {
+  const int64_t* tok_off;  // [U+1]
+  int num_units;
+  int R;                   // G * w real query rows
+  int w;
+  int cs;                  // CTAs per cluster (one unit per cluster)
+  int lmax;                // tokens per CTA, multiple of 128
+  int nstages;             // K tile ring depth
+  float scale_log2;        // log2(e) / sqrt(d)
+  float* a_out;            // [T]
+  float* r_out;            // [T]
+  float* m_out;            // [T] or null
+  float* rho_out;          // [T] (1/||k||) or null
+  int* status;
+};
+
+struct ScoreLayout {
+  uint32_t stages, q, abar, marr, rhoc, rhot, ufin, mrow, invl, red1, red2, rsum, xbuf, bars,
+      slot, flags, total;
+};
+
+__host__ __device__ inline int score_xb(int rp) { return 2 * rp + 128 + 4; }
+
+__host__ __device__ inline ScoreLayout score_layout(int rp, bool closed, int lmax, int ns) {
+  ScoreLayout L;
+  uint32_t o = 0;
+  L.stages = o; o += ns * kTileBytes;
+  L.q = o; o += 2 * rp * 256;
+  L.abar = o; o += lmax * 4;
+  L.marr = o; if (closed) o += lmax * 4;
+  L.rhoc = o; if (closed) o += lmax * 4;
+  L.rhot = o; o += 2 * 128 * 4;
+  L.ufin = o; o += 128 * 4;
+  L.mrow = o; o += rp * 4;
+  L.invl = o; o += rp * 4;
+  L.red1 = o; o += 4 * rp * 2 * 4;
+  L.red2 = o; o += 4 * 128 * 4;
+  L.rsum = o; o += 16 * 4;
+  L.xbuf = o; o += 2 * score_xb(rp) * 4;
+  o = (o + 15u) & ~15u;
+  L.bars = o; o += (2 * ns + 14) * 8;
+  L.slot = o; o += 16;
+  L.flags = o; o += 16;
+  L.total = o;
+  return L;
+}
+
+// ---------------------------------------------------------------- redundancy GEMM
+struct GemmParams {
+  const int64_t* tok_off;  // [U+1]
+  const int* item_off;     // [U+1] prefix of row blocks per unit
+  int num_units;
+  int w;
+  const float* rho;        // [T] 1/||k||
+  float* m_dst;            // [T] receives m (may equal r_dst)
+  float* r_dst;            // [T] receives r
+  int* unit_cnt;           // [U] zeroed by the plan kernel
+  int* status;
+};
+
+template <bool kPair>
+struct GemmCfg {
+  static constexpr int kCtaGroup = kPair ? 2 : 1;
+  static constexpr int kRowsPerCta = 128;                    // A rows held by a CTA
+  static constexpr int kRowsPerItem = kPair ? 256 : 128;
+  static constexpr int kN = 256;                             // key columns per tile
+  static constexpr int kBRows = kPair ? 128 : 256;           // key rows a CTA loads
+  static constexpr int kStages = kPair ? 5 : 2;
+  static constexpr int kABytes = kRowsPerCta * 256;          // 32 KiB
+  static constexpr int kBBytes = kBRows * 256;
+  static constexpr int kMmaM = kPair ? 256 : 128;
+};
+
+struct GemmLayout {
+  uint32_t a, b, rho, rowx, fin, bars, slot, flags, total;
+};
+template <bool kPair>
+__host__ __device__ inline GemmLayout gemm_layout() {
+  using C = GemmCfg<kPair>;
+  GemmLayout L;
+  uint32_t o = 0;
+  L.a = o; o += C::kABytes;
+  L.b = o; o += C::kStages * C::kBBytes;
+  L.rho = o; o += 2 * 256 * 4;
+  L.rowx = o; o += 128 * 4;
+  L.fin = o; o += 32 * 4;
+  L.bars = o; o += (2 + 2 * C::kStages + 4) * 8;
+  L.slot = o; o += 16;
+  L.flags = o; o += 16;
+  L.total = o;
+  return L;
+}
+
+// ---------------------------------------------------------------- launches
+// Each returns a cudaError_t of the launch (cudaSuccess when enqueued).
+cudaError_t launch_score(const CUtensorMap& kmap, const CUtensorMap& qmap, const ScoreParams& p,
+                         int rp, bool closed, int nclusters, cudaStream_t st);
+cudaError_t score_configure(int rp, bool closed, int smem_bytes, int cs);
+int score_max_clusters(int rp, bool closed, int smem_bytes, int cs);
+
+cudaError_t launch_plan(const int64_t* tok_off, int U, int w, int rows_per_item, int* item_off,
+                        int* unit_cnt, cudaStream_t st);
+cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const GemmParams& p,
+                        bool pair, int nctas, cudaStream_t st);
+cudaError_t gemm_configure(bool pair);
+int gemm_max_ctas(bool pair);
+
+cudaError_t launch_select(const int64_t* tok_off, int U, int w, int cmax, const float* a,
+                          const float* r, float lam, int budget, int32_t* idx, int32_t* n_kept,
+                          cudaStream_t st);
+cudaError_t select_configure();
+
+cudaError_t launch_compact(const int64_t* tok_off, int U, int W, const int32_t* idx,
+                           const int32_t* n_kept, const void* K, const void* V, void* Ko,
+                           void* Vo, int* status, int nsm, cudaStream_t st);
+
+}  // namespace rkv

@@ -1,0 +1,174 @@
+/*
+ * rkv.h -- C ABI of the decode-time KV-cache compression engine (R-KV hot path)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Method: the R-KV article (QbitAI repost, section "R-KV三步走：冗余识别+重要性评估+
+ * 动态淘汰").  While decoding, each (sequence, layer, KV head) cache is scored by
+ *   - importance (重要性打分): attention that the last w decode queries pay to each
+ *     cached token, softmax per query, averaged over the window and the GQA group;
+ *   - redundancy (冗余打分): cosine similarity between each key and all other cached
+ *     keys, averaged over the row (diagonal excluded), then a softmax over tokens;
+ * and the joint eviction step (联合淘汰: high importance, low redundancy, lambda ~ 0.1)
+ * keeps the last w tokens plus the top-B of the rest and compacts K/V into a B+w
+ * slot buffer (gather compaction, named as the R-KV-style baseline in the ThinKV
+ * summary, "Continuous Thinking" section).
+ *
+ * Terms used below.  A *unit* is one (sequence, layer, KV head).  Unit u has
+ * N_u cached tokens, stored as rows tok_off[u] .. tok_off[u+1]-1 of K and V.
+ * d = head_dim (= 128), G = query heads per KV head, w = window.  Query (g, t)
+ * of unit u is Q[u][g][t][:] and sits at position N_u - w + t; it attends to
+ * keys 0 .. N_u - w + t.  The candidates are C_u = {0 .. N_u - w - 1}.
+ *
+ * Conventions (every call):
+ *   - All data pointers are DEVICE pointers, owned by the caller, unless the
+ *     parameter says "host".  Inputs are read only.  K, V, Q, K_out, V_out
+ *     must be 16-byte aligned; float/int32 arrays 4-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t) and never synchronise
+ *     the host, except rkv_check_status.  They never throw.
+ *   - Return value: RKV_OK (0) or a negative RKV_ERR_* code.  Arguments are
+ *     validated on the host before anything is enqueued; on an error nothing is
+ *     enqueued.  Faults found on the device (a wait that timed out, a kept index
+ *     outside its unit) are recorded in the engine's device status word and
+ *     reported by rkv_check_status.
+ *   - One engine may be used from one host thread at a time.  Calls that share
+ *     an engine must be ordered on one stream (the engine's workspace is reused).
+ */
+#ifndef RKV_H_
+#define RKV_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* rkv_stream_t; /* identical to cudaStream_t */
+typedef struct rkv_engine rkv_engine;     /* opaque; owns device workspace only */
+
+enum {
+  RKV_OK = 0,
+  RKV_ERR_INVALID_ARG = -1, /* null/unaligned pointer, bad size, N_u < w, ... */
+  RKV_ERR_UNSUPPORTED = -2, /* head_dim != 128, G*w > 32, N_u > 49152, not sm_100 */
+  RKV_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
+  RKV_ERR_TIMEOUT = -4,     /* a device-side wait ran out of time (see rkv_check_status) */
+  RKV_ERR_OOM = -5,         /* workspace allocation failed */
+  RKV_ERR_CAPACITY = -6,    /* batch larger than the engine's max_units / max_tokens */
+  RKV_ERR_DEVICE = -7       /* a kept index outside its unit (see rkv_check_status) */
+};
+
+/* How rkv_score computes the redundancy row mean m_i. */
+enum {
+  /* Tensor-core K K^T tile products with the norm scaling, diagonal mask,
+   * row mean and token softmax fused into the epilogue (N x N never stored). */
+  RKV_REDUNDANCY_GEMM = 0,
+  /* The same m_i by linearity of the row sum:
+   * sum_{j != i} khat_i . khat_j = khat_i . (sum_j khat_j) - khat_i . khat_i. */
+  RKV_REDUNDANCY_CLOSED_FORM = 1
+};
+
+typedef struct {
+  int head_dim;       /* d; must be 128 */
+  int group;          /* G >= 1: query heads per KV head */
+  int window;         /* w >= 1: window queries and always-kept tail tokens */
+  int max_units;      /* capacity: units per batch (>= 1) */
+  int64_t max_tokens; /* capacity: total cached rows per batch (>= 1) */
+  int redundancy;     /* RKV_REDUNDANCY_GEMM or RKV_REDUNDANCY_CLOSED_FORM */
+  int flags;          /* 0, or RKV_FLAG_* bits */
+} rkv_config;
+
+/* rkv_config.flags */
+enum {
+  /* Redundancy GEMM on single CTAs (M = 128 tcgen05 MMAs) instead of CTA
+   * pairs (M = 256, cta_group::2).  Same results; slower. */
+  RKV_FLAG_GEMM_SINGLE_CTA = 1
+};
+
+typedef struct {
+  int num_units;               /* U, 0 <= U <= max_units */
+  const int64_t* tok_off;      /* device [U+1]: row offsets, tok_off[0] = 0, nondecreasing */
+  const int64_t* tok_off_host; /* HOST copy of the same [U+1] values (validation, sizing) */
+  const void* K;               /* device bf16 [T, d] row-major keys, T = tok_off[U] */
+  const void* V;               /* device bf16 [T, d] row-major values */
+  const void* Q;               /* device bf16 [U, G, w, d]: window queries (post-RoPE) */
+} rkv_batch;
+
+/* Create an engine and allocate its device workspace on the current device.
+ * Fails with RKV_ERR_UNSUPPORTED on a device that is not sm_100. */
+int rkv_create(const rkv_config* cfg, rkv_engine** out);
+
+/* Free the workspace (waits for the device to finish using it). NULL is a no-op. */
+int rkv_destroy(rkv_engine* eng);
+
+/* Importance and redundancy scores (R-KV 重要性打分 and 冗余打分).
+ *   a [T] fp32: a_i = abar_i / sum_{j in C} abar_j for i in C, where
+ *               abar_i = mean over (g, t) of softmax_j(q_{g,t} . k_j / sqrt(d))[i];
+ *   r [T] fp32: r_i = exp(m_i) / sum_{j in C} exp(m_j) for i in C, where
+ *               m_i = sum_{j != i, j < N} khat_i . khat_j / (N - 1),
+ *               khat = k / ||k|| (0 for a zero key);
+ *   m [T] fp32, optional (NULL to skip): the row means m_i.
+ * Row tok_off[u] + i holds token i of unit u; window rows (i >= N_u - w) are 0. */
+int rkv_score(rkv_engine* eng, const rkv_batch* batch, float* a, float* r, float* m,
+              rkv_stream_t stream);
+
+/* Joint eviction (R-KV 联合淘汰): s_i = lambda * a_i - (1 - lambda) * r_i for i in C
+ * (fp32); keep the min(budget, N_u - w) candidates ranked first by (s descending,
+ * index ascending), in ascending index order, followed by the window
+ * N_u - w .. N_u - 1.  When N_u - w <= budget every token 0 .. N_u - 1 is kept.
+ *   idx [U, budget + w] int32: kept token indices (unit-local); unused slots -1;
+ *   n_kept [U] int32: number of valid slots of each unit.
+ * lambda must lie in [0, 1]; budget >= 0. */
+int rkv_select(rkv_engine* eng, const rkv_batch* batch, const float* a, const float* r,
+               float lambda, int budget, int32_t* idx, int32_t* n_kept, rkv_stream_t stream);
+
+/* Gather compaction: K_out[u][j] = K[tok_off[u] + idx[u][j]] (and V likewise) for
+ * j < n_kept[u]; rows n_kept[u] .. budget + w - 1 are zero.  Bit-exact copies.
+ *   K_out, V_out: device bf16 [U, budget + w, d] (must not overlap K, V).
+ * An index outside 0 .. N_u - 1 zero-fills its row and sets RKV_ERR_DEVICE. */
+int rkv_compact(rkv_engine* eng, const rkv_batch* batch, const int32_t* idx,
+                const int32_t* n_kept, int budget, void* K_out, void* V_out,
+                rkv_stream_t stream);
+
+/* rkv_score, rkv_select and rkv_compact in one call.  a and r are caller-owned
+ * scratch [T] fp32 (they hold the scores afterwards). */
+int rkv_compress(rkv_engine* eng, const rkv_batch* batch, float lambda, int budget,
+                 float* a, float* r, int32_t* idx, int32_t* n_kept, void* K_out,
+                 void* V_out, rkv_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the engine's device status word:
+ * RKV_OK, RKV_ERR_TIMEOUT (a device wait gave up; outputs are invalid) or
+ * RKV_ERR_DEVICE (an out-of-range kept index reached rkv_compact). */
+int rkv_check_status(rkv_engine* eng, rkv_stream_t stream);
+
+/* Number of kernel launches enqueued by this engine since creation. */
+int64_t rkv_launch_count(const rkv_engine* eng);
+
+/* Kernels, for per-kernel timing. */
+enum {
+  RKV_KERNEL_SCORE = 0,   /* importance (+ closed-form redundancy) */
+  RKV_KERNEL_PLAN = 1,    /* per-unit row-block offsets for the GEMM */
+  RKV_KERNEL_GEMM = 2,    /* redundancy GEMM + fused epilogue + token softmax */
+  RKV_KERNEL_SELECT = 3,  /* joint score + top-B */
+  RKV_KERNEL_COMPACT = 4, /* K/V gather */
+  RKV_NUM_KERNELS = 5
+};
+
+/* Per-kernel timing.  While enabled, the engine records a pair of CUDA events
+ * on the launch stream around each of its kernel launches (up to 4096 pairs
+ * between reads).  rkv_read_timing synchronises on those events and returns,
+ * for `kernel`, the summed device time in milliseconds and the number of
+ * launches since the previous read (of any kernel), then forgets them.
+ * rkv_set_timing(eng, 0) disables recording and drops unread events. */
+int rkv_set_timing(rkv_engine* eng, int enable);
+int rkv_read_timing(rkv_engine* eng, int kernel, double* total_ms, int64_t* launches);
+
+/* Static description of a status code. */
+const char* rkv_status_string(int status);
+
+/* ABI version (major * 10000 + minor * 100 + patch). */
+int rkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RKV_H_ */

@@ -1,0 +1,239 @@
+"""GPU engine vs the fp64 oracle, through the C ABI (see tests/parity.py for the
+tolerances).  Ordered from the integer kernels (select, compaction) to the
+score kernels, then edge cases, then the full-size workloads on sampled units."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from decode_kv_cache_eviction_b200 import Batch, Engine, RkvError
+from decode_kv_cache_eviction_b200 import workloads as W
+from oracle import rkv_oracle as ora
+
+from parity import check_unit, make_batch, run_engine
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def rand_batch(lengths, G, w, seed=0, dup=0.2, zero_rows=()):
+    rng = np.random.default_rng(seed)
+    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    T = int(off[-1])
+    K = rng.standard_normal((T, 128)).astype(np.float32)
+    for u in range(len(lengths)):
+        for i in range(1, lengths[u]):
+            if rng.random() < dup:
+                K[off[u] + i] = K[off[u] + rng.integers(0, i)]
+    for z in zero_rows:
+        K[z] = 0
+    V = rng.standard_normal((T, 128)).astype(np.float32)
+    Q = rng.standard_normal((len(lengths), G, w, 128)).astype(np.float32)
+    t = lambda x: torch.from_numpy(x).to(DEV).to(torch.bfloat16)
+    return Batch(t(K), t(V), t(Q), off)
+
+
+# ----------------------------------------------------------------- select alone
+@pytest.mark.parametrize("lam", [0.0, 0.1, 1.0])
+@pytest.mark.parametrize("lengths,budget", [([1000], 100), ([4096, 300, 9], 256),
+                                            ([20000, 33000], 4096), ([5000], 0)])
+def test_select_bit_exact_given_scores(lam, lengths, budget):
+    w = 8
+    b = rand_batch(lengths, 1, w, seed=len(lengths) + budget)
+    rng = np.random.default_rng(budget)
+    T = b.num_tokens
+    a = rng.random(T).astype(np.float32) * 1e-3
+    r = rng.random(T).astype(np.float32) * 1e-3
+    a[::7] = a[3]  # plenty of exact ties
+    r[::7] = r[3]
+    eng = Engine(1, w, max_units=len(lengths), max_tokens=T, redundancy="closed")
+    ta, tr = torch.from_numpy(a).to(DEV), torch.from_numpy(r).to(DEV)
+    idx, nk, _, _ = eng.alloc_outputs(b, budget)
+    eng.select(b, ta, tr, lam, budget, idx, nk)
+    eng.check_status()
+    idx, nk = idx.cpu().numpy(), nk.cpu().numpy()
+    lam32 = np.float32(lam)
+    for u, N in enumerate(lengths):
+        r0 = int(b.tok_off_host[u])
+        c = N - w
+        s32 = ora.joint_score(a[r0:r0 + c], r[r0:r0 + c], lam32)   # fp32 on both sides
+        assert s32.dtype == np.float32
+        want = ora.select(s32, N, w, budget)
+        assert nk[u] == len(want)
+        np.testing.assert_array_equal(idx[u, :nk[u]], want)
+        assert np.all(idx[u, nk[u]:] == -1)
+
+
+# ----------------------------------------------------------------- compaction alone
+def test_compact_bit_exact_and_bad_index_flag():
+    lengths, w, budget = [700, 64, 1500], 4, 100
+    b = rand_batch(lengths, 1, w, seed=3)
+    eng = Engine(1, w, max_units=3, max_tokens=b.num_tokens, redundancy="closed")
+    U, Wd = 3, budget + w
+    rng = np.random.default_rng(0)
+    idx = np.full((U, Wd), -1, np.int32)
+    nk = np.array([Wd, 64, 77], np.int32)
+    for u, N in enumerate(lengths):
+        idx[u, :nk[u]] = np.sort(rng.choice(N, size=nk[u], replace=False))
+    tidx, tnk = torch.from_numpy(idx).to(DEV), torch.from_numpy(nk).to(DEV)
+    _, _, Ko, Vo = eng.alloc_outputs(b, budget)
+    eng.compact(b, tidx, tnk, budget, Ko, Vo)
+    eng.check_status()
+    for u in range(U):
+        src = torch.from_numpy(idx[u, :nk[u]].astype(np.int64) + b.tok_off_host[u]).to(DEV)
+        assert torch.equal(Ko[u, :nk[u]].view(torch.int16), b.K[src].view(torch.int16))
+        assert torch.equal(Vo[u, :nk[u]].view(torch.int16), b.V[src].view(torch.int16))
+        assert torch.count_nonzero(Ko[u, nk[u]:].view(torch.int16)) == 0
+    # an index outside its unit zero-fills the row and is reported
+    idx[1, 5] = 64
+    tidx = torch.from_numpy(idx).to(DEV)
+    eng.compact(b, tidx, tnk, budget, Ko, Vo)
+    with pytest.raises(RkvError) as ei:
+        eng.check_status()
+    assert ei.value.code == -7
+    assert torch.count_nonzero(Ko[1, 5].view(torch.int16)) == 0
+    eng.check_status()   # the status word was cleared
+
+
+# ----------------------------------------------------------------- worked example
+def test_worked_example_on_gpu():
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_6token.json")))
+    K = np.zeros((6, 128), np.float32)
+    K[:, :2] = np.array(g["K"])
+    Q = np.zeros((1, 1, 2, 128), np.float32)
+    Q[0, 0, :, :2] = np.array(g["Q"][0])
+    # zero padding keeps every dot product and norm, but the kernel scales
+    # logits by 1/sqrt(128) instead of 1/sqrt(2): pre-scale the queries by
+    # sqrt(128/2) = 8 (exact in bf16) so the logits match the d = 2 example
+    Q *= 8.0
+    t = lambda x: torch.from_numpy(x).to(DEV).to(torch.bfloat16)
+    b = Batch(t(K), t(K), t(Q), np.array([0, 6]))
+    for mode in ("closed", "gemm"):
+        for lam, want in g["idx"].items():
+            out = run_engine(b, 1, 2, float(lam), 2, mode=mode)
+            np.testing.assert_allclose(out["a"][:4], g["a"], atol=5e-6)
+            np.testing.assert_allclose(out["r"][:4], g["r"], atol=5e-6)
+            np.testing.assert_allclose(out["m"][:4], g["m"], atol=5e-6)
+            assert out["idx"][0].tolist() == want, (mode, lam)
+
+
+# ----------------------------------------------------------------- score kernels, small
+@pytest.mark.parametrize("mode", ["closed", "gemm"])
+@pytest.mark.parametrize("G,w", [(1, 8), (4, 8), (2, 3), (5, 5), (1, 1), (32, 1)])
+def test_score_small_ragged(mode, G, w):
+    lengths = [w, w + 1, 127, 128, 129, 1000, 2500, 5000]
+    zero_rows = [3 + lengths[0] + lengths[1]]   # a zero key inside unit 2
+    b = rand_batch(lengths, G, w, seed=G * 10 + w, zero_rows=zero_rows)
+    budget = 64
+    for lam in (0.1,):
+        out = run_engine(b, G, w, lam, budget, mode=mode)
+        for u in range(len(lengths)):
+            check_unit(out, b, u, w, lam, budget)
+
+
+@pytest.mark.parametrize("mode", ["closed", "gemm"])
+def test_budget_edges(mode):
+    lengths = [300, 300, 300]
+    w = 8
+    b = rand_batch(lengths, 4, w, seed=7)
+    for budget in (0, 1, 291, 292, 300):
+        out = run_engine(b, 4, w, 0.1, budget, mode=mode)
+        for u in range(3):
+            check_unit(out, b, u, w, 0.1, budget)
+
+
+def test_gemm_single_cta_and_pair_agree():
+    b = rand_batch([3000, 4100, 700], 4, 8, seed=11)
+    o1 = run_engine(b, 4, 8, 0.1, 256, mode="gemm", single_cta=True)
+    o2 = run_engine(b, 4, 8, 0.1, 256, mode="gemm", single_cta=False)
+    o3 = run_engine(b, 4, 8, 0.1, 256, mode="closed")
+    for u in range(3):
+        check_unit(o1, b, u, 8, 0.1, 256)
+    np.testing.assert_allclose(o1["m"], o2["m"], rtol=1e-5, atol=1e-7)
+    np.testing.assert_allclose(o2["r"], o3["r"], rtol=1e-4, atol=1e-9)
+
+
+def test_largest_supported_unit():
+    N = 49152
+    b = rand_batch([N], 4, 8, seed=1, dup=0.0)
+    for mode in ("closed", "gemm"):
+        out = run_engine(b, 4, 8, 0.1, 4096, mode=mode)
+        check_unit(out, b, 0, 8, 0.1, 4096)
+
+
+def test_rejects_too_long_unit_and_capacity():
+    b = rand_batch([49153], 1, 8, seed=0, dup=0.0)
+    eng = Engine(1, 8, max_units=1, max_tokens=b.num_tokens, redundancy="closed")
+    a, r = eng.alloc_scores(b)
+    with pytest.raises(RkvError) as ei:
+        eng.score(b, a, r)
+    assert ei.value.code == -2
+    small = Engine(1, 8, max_units=1, max_tokens=100, redundancy="closed")
+    with pytest.raises(RkvError) as ei:
+        small.score(b, a, r)
+    assert ei.value.code == -6
+    bad = Batch(b.K, b.V, b.Q, np.array([0, 5]))   # N < w
+    with pytest.raises(RkvError) as ei:
+        eng.score(bad, a, r)
+    assert ei.value.code == -1
+
+
+def test_repeated_calls_are_deterministic():
+    b = rand_batch([4000, 6000], 4, 8, seed=5)
+    for mode in ("closed", "gemm"):
+        eng = Engine(4, 8, max_units=2, max_tokens=b.num_tokens, redundancy=mode)
+        o1 = run_engine(b, 4, 8, 0.1, 512, engine=eng)
+        o2 = run_engine(b, 4, 8, 0.1, 512, engine=eng)
+        assert np.array_equal(o1["a"], o2["a"]) and np.array_equal(o1["r"], o2["r"])
+        assert np.array_equal(o1["idx"], o2["idx"])
+
+
+# ----------------------------------------------------------------- full workloads
+def _sampled(name, n_sample, modes=("gemm", "closed")):
+    wl = W.WORKLOADS[name]
+    gb = W.generate(wl, seed=0, device=DEV)
+    b = make_batch(gb)
+    U = b.num_units
+    rng = np.random.default_rng(123)
+    units = sorted(set([0, U - 1] + rng.choice(U, size=min(U, n_sample), replace=False).tolist()))
+    for mode in modes:
+        for lam in wl.lambdas:
+            out = run_engine(b, wl.group, wl.window, lam, wl.budget, mode=mode)
+            for u in units:
+                check_unit(out, b, u, wl.window, lam, wl.budget)
+            del out
+            torch.cuda.empty_cache()
+    return b, units
+
+
+def test_workload_tiny_full():
+    _sampled("tiny", 1)
+
+
+def test_workload_llama3_layer_full():
+    _sampled("llama3_8b_layer", 8)
+
+
+def test_workload_tiny_definition_redundancy():
+    """Redundancy checked against the row-block definition (not the closed form)."""
+    wl = W.WORKLOADS["tiny"]
+    b = make_batch(W.generate(wl, seed=1, device=DEV))
+    out = run_engine(b, wl.group, wl.window, 0.1, wl.budget, mode="gemm")
+    check_unit(out, b, 0, wl.window, 0.1, wl.budget, redundancy="rowblocks")
+
+
+@pytest.mark.slow
+def test_workload_r1_llama8b_cache_sampled():
+    _sampled("r1_llama8b_cache", 6)
+
+
+@pytest.mark.slow
+def test_workload_long_trace_32k_sampled():
+    _sampled("long_trace_32k", 6)
+
+
+@pytest.mark.slow
+def test_workload_ragged_serving_sampled():
+    _sampled("ragged_serving", 8)
