@@ -170,9 +170,14 @@ def test_rejects_too_long_unit_and_capacity():
     with pytest.raises(RkvError) as ei:
         eng.score(b, a, r)
     assert ei.value.code == -2
+    b2 = rand_batch([200], 1, 8, seed=0, dup=0.0)
     small = Engine(1, 8, max_units=1, max_tokens=100, redundancy="closed")
     with pytest.raises(RkvError) as ei:
-        small.score(b, a, r)
+        small.score(b2, a, r)
+    assert ei.value.code == -6
+    two = rand_batch([100, 100], 1, 8, seed=0, dup=0.0)
+    with pytest.raises(RkvError) as ei:
+        small.score(two, a, r)
     assert ei.value.code == -6
     bad = Batch(b.K, b.V, b.Q, np.array([0, 5]))   # N < w
     with pytest.raises(RkvError) as ei:
