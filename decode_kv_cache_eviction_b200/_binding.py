@@ -33,7 +33,7 @@ RKV_FLAG_GEMM_SINGLE_CTA = 1
 # Every function declared in include/rkv.h.
 EXPORTS = ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact",
            "rkv_compress", "rkv_check_status", "rkv_launch_count", "rkv_set_timing",
-           "rkv_read_timing", "rkv_status_string", "rkv_version")
+           "rkv_read_timing", "rkv_score_noalloc", "rkv_status_string", "rkv_version")
 KERNELS = ("score", "plan", "gemm", "select", "compact")
 
 
@@ -83,12 +83,13 @@ def lib():
     L.rkv_set_timing.argtypes = [vp, i32]
     L.rkv_read_timing.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_double),
                                   ctypes.POINTER(i64)]
+    L.rkv_score_noalloc.argtypes = [i32, i32, ctypes.POINTER(RkvBatch), vp, vp, vp, vp]
     L.rkv_status_string.argtypes = [i32]
     L.rkv_status_string.restype = ctypes.c_char_p
     L.rkv_version.argtypes = []
     for name in ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact",
                  "rkv_compress", "rkv_check_status", "rkv_set_timing", "rkv_read_timing",
-                 "rkv_version"):
+                 "rkv_score_noalloc", "rkv_version"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -111,6 +112,13 @@ def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def score_noalloc(group: int, window: int, batch: "Batch", a, r, m=None, stream=None):
+    """rkv_score_noalloc: GEMM-mode scores using only the library's static device
+    scratch (no engine, no allocation by the library)."""
+    _check(lib().rkv_score_noalloc(int(group), int(window), ctypes.byref(batch.c), _ptr(a),
+                                   _ptr(r), _ptr(m), _stream(stream)), "rkv_score_noalloc")
 
 
 class Batch:

@@ -161,6 +161,35 @@ enum {
 int rkv_set_timing(rkv_engine* eng, int enable);
 int rkv_read_timing(rkv_engine* eng, int kernel, double* total_ms, int64_t* launches);
 
+/* Scoring without any device allocation (no engine object).
+ *
+ * The paper has no counterpart to this call; it exists for callers that cannot
+ * allocate device memory themselves or through the library: serving stacks that
+ * reserve nearly all HBM up front for their own KV block pool and hand out no
+ * further memory, or host frameworks that load this library as a plug-in and
+ * forbid it from calling cudaMalloc behind their allocator's back.
+ *
+ * Computes exactly what rkv_score computes for an engine created with
+ * RKV_REDUNDANCY_GEMM (CTA-pair GEMM), with head_dim = 128 and the given group and
+ * window.  Its scratch (1/||k|| per row, per-unit row-block offsets and
+ * counters, a status word) lives in one file-scope __device__ array of about
+ * 4.1 MB that every GPU which loads the library holds until the process exits;
+ * nothing is allocated or freed per call.  Limits: at most RKV_NOALLOC_MAX_UNITS
+ * units and RKV_NOALLOC_MAX_TOKENS rows per call (larger batches return
+ * RKV_ERR_CAPACITY before anything is enqueued), and the rkv_score limits
+ * (G*w <= 32, N_u <= 49152).
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and sets kernel attributes with that device current;
+ * make that first call before any stream capture.  All calls share the one
+ * array and each call rewrites what it reads, so successive calls on one
+ * stream are safe, but calls that overlap on the GPU (other streams, other host
+ * threads without ordering) race on it.  A device-side wait that times out is
+ * recorded only in the array's status word: this call has no status query. */
+enum { RKV_NOALLOC_MAX_UNITS = 4096, RKV_NOALLOC_MAX_TOKENS = 1048576 };
+int rkv_score_noalloc(int group, int window, const rkv_batch* batch, float* a, float* r,
+                      float* m, rkv_stream_t stream);
+
 /* Static description of a status code. */
 const char* rkv_status_string(int status);
 
