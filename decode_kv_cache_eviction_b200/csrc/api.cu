@@ -16,7 +16,6 @@ struct rkv_engine {
   int device = 0;
   int nsm = 0;
   int rp = 32;                 // padded G*w (MMA N of the logits tile)
-  int lmax = 0;                // tokens per score CTA the layout is sized for
   int nstages = 0;             // score K-tile ring depth
   int score_smem = 0;
   int score_clusters[5] = {};  // active clusters for cluster sizes 1, 2, 4, 8, 16
@@ -167,18 +166,12 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   }
   e->encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
 
-  // Score kernel layout: 3072 tokens per CTA, deepest K ring that fits.
+  // Score kernel: deepest K-tile ring that fits; logits of up to 512/rp tiles
+  // per CTA stay in TMEM, so a unit may hold up to max_cs * 512/rp * 128 tokens.
   const bool closed = cfg->redundancy == RKV_REDUNDANCY_CLOSED_FORM;
-  e->lmax = 3072;
-  e->nstages = 0;
-  for (int ns = 8; ns >= 3; --ns) {
-    if (static_cast<int>(score_layout(e->rp, closed, e->lmax, ns).total) + 1024 <= kSmemCap) {
-      e->nstages = ns;
-      break;
-    }
-  }
-  e->score_smem = score_layout(e->rp, closed, e->lmax, e->nstages).total + 1024;
-  if (score_configure(e->rp, closed, e->score_smem, 16) != cudaSuccess) {
+  e->nstages = score_stages(e->rp, closed, kSmemCap);
+  e->score_smem = score_layout(e->rp, closed, e->nstages).total + 1024;
+  if (e->nstages == 0 || score_configure(e->rp, closed, e->score_smem, 16) != cudaSuccess) {
     delete e;
     return cuda_fail(cudaErrorUnknown);
   }
@@ -192,7 +185,7 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
     delete e;
     return RKV_ERR_UNSUPPORTED;
   }
-  e->max_n = e->max_cs * e->lmax;
+  e->max_n = e->max_cs * score_lmax(e->rp);
   if (e->max_n > kMaxTokensPerUnit) e->max_n = kMaxTokensPerUnit;
 
   if (select_configure() != cudaSuccess) {
@@ -294,13 +287,8 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   const bool closed = e->cfg.redundancy == RKV_REDUNDANCY_CLOSED_FORM;
   const int R = e->cfg.group * e->cfg.window;
 
-  // cluster size: about 1024 tokens per CTA, at most what the layout holds
-  int cs = 1;
-  while (cs < e->max_cs && (nmax + cs - 1) / cs > 1024) cs <<= 1;
-  while ((((nmax + cs - 1) / cs + kTile - 1) / kTile) * kTile > e->lmax) {
-    if (cs >= e->max_cs) return RKV_ERR_UNSUPPORTED;
-    cs <<= 1;
-  }
+  const int cs = score_cluster_size(nmax, e->rp, e->max_cs);
+  if (cs == 0) return RKV_ERR_UNSUPPORTED;
   int ncl = e->score_clusters[cs_index(cs)];
   if (ncl > U) ncl = U;
 
@@ -315,7 +303,6 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   p.R = R;
   p.w = e->cfg.window;
   p.cs = cs;
-  p.lmax = e->lmax;
   p.nstages = e->nstages;
   p.scale_log2 = kLog2e / sqrtf(static_cast<float>(kHeadDim));
   p.a_out = a;

@@ -28,7 +28,6 @@ constexpr int kMaxUnits = RKV_NOALLOC_MAX_UNITS;
 constexpr int64_t kMaxTokens = RKV_NOALLOC_MAX_TOKENS;
 constexpr int kMaxDevices = 64;
 constexpr int kSmemCap = 227 * 1024;
-constexpr int kLmax = 3072;  // tokens per score CTA the layout is sized for
 
 struct Scratch {
   float rho[kMaxTokens];
@@ -87,14 +86,9 @@ int setup(int dev, DeviceState** out) {
   d.scratch = static_cast<Scratch*>(ptr);
   for (int k = 0; k < 2; ++k) {
     const int rp = k ? 32 : 16;
-    for (int ns = 8; ns >= 3; --ns) {
-      if (static_cast<int>(score_layout(rp, false, kLmax, ns).total) + 1024 <= kSmemCap) {
-        d.nstages[k] = ns;
-        break;
-      }
-    }
-    d.smem[k] = score_layout(rp, false, kLmax, d.nstages[k]).total + 1024;
-    if (score_configure(rp, false, d.smem[k], 16) != cudaSuccess) {
+    d.nstages[k] = score_stages(rp, false, kSmemCap);
+    d.smem[k] = score_layout(rp, false, d.nstages[k]).total + 1024;
+    if (d.nstages[k] == 0 || score_configure(rp, false, d.smem[k], 16) != cudaSuccess) {
       cudaGetLastError();
       return RKV_ERR_CUDA;
     }
@@ -168,12 +162,8 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   const int R = group * window;
   const int rp = R <= 16 ? 16 : 32;
   const int k = rp == 32 ? 1 : 0;
-  int cs = 1;
-  while (cs < d->max_cs[k] && (nmax + cs - 1) / cs > 1024) cs <<= 1;
-  while ((((nmax + cs - 1) / cs + kTile - 1) / kTile) * kTile > kLmax) {
-    if (cs >= d->max_cs[k]) return RKV_ERR_UNSUPPORTED;
-    cs <<= 1;
-  }
+  const int cs = score_cluster_size(nmax, rp, d->max_cs[k]);
+  if (cs == 0) return RKV_ERR_UNSUPPORTED;
   int ci = 0;
   while ((1 << ci) < cs) ++ci;
   int ncl = d->clusters[k][ci];
@@ -195,7 +185,6 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   p.R = R;
   p.w = window;
   p.cs = cs;
-  p.lmax = kLmax;
   p.nstages = d->nstages[k];
   p.scale_log2 = kLog2e / sqrtf(static_cast<float>(kHeadDim));
   p.a_out = a;

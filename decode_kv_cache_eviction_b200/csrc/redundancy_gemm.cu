@@ -184,11 +184,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int etid = threadIdx.x - 128;   // 0..255
-    const int half = (warp - 4) >> 2;     // column half of the tile
+    const int ew = warp - 4;              // epilogue warp 0..7
+    const int half = ew >> 2;             // column half of the tile
     const int q = warp & 3;               // TMEM lane quarter
     const int rloc = q * 32 + lane;       // row of this CTA's A block
-    const int hidx = q * 32 + lane;       // 0..127 within the half
-    float* rho_s = reinterpret_cast<float*>(sm + L.rho);
+    // private rho slices of this warp: [2][128] floats (the 128 columns of its half)
+    float* rho_w = reinterpret_cast<float*>(sm + L.rho) + ew * 256;
     float* rowx = reinterpret_cast<float*>(sm + L.rowx);
     float* fin = reinterpret_cast<float*>(sm + L.fin);
     const uint32_t acc_empty_lead = kPair ? mapa(smem_u32(acc_empty), 0) : smem_u32(acc_empty);
@@ -204,54 +205,68 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int i = rbase + rloc;
       float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
       const int ntiles = (N + C::kN - 1) / C::kN;
+      // rho of the 4 columns this lane stages, one tile ahead
+      auto load_rho = [&](int j0, float (&dst)[4]) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int col = j0 + half * 128 + lane * 4 + e;
+          dst[e] = col < N ? __ldg(&p.rho[base + col]) : 0.f;
+        }
+      };
+      float rpre[4];
+      load_rho(0, rpre);
       for (int t = 0; t < ntiles; ++t) {
         const int j0 = t * C::kN;
-        {
-          const int col = j0 + half * 128 + hidx;
-          rho_s[ab * 256 + half * 128 + hidx] = col < N ? __ldg(&p.rho[base + col]) : 0.f;
-        }
-        named_bar_sync(1 + half, 128);
+        float* rs = rho_w + (t & 1) * 128;
+        *reinterpret_cast<float4*>(rs + lane * 4) = make_float4(rpre[0], rpre[1], rpre[2], rpre[3]);
+        __syncwarp();
+        if (t + 1 < ntiles) load_rho(j0 + C::kN, rpre);
         mbar_wait(&acc_full[ab], aph, abort, p.status);
         __syncwarp();
         tc_fence_after();
+        const uint32_t tbase =
+            tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + half * 128;
+        uint32_t va[32], vb[32], vc[32], vd[32];
+        tmem_ld32(tbase, va);
+        tmem_ld32(tbase + 32, vb);
+        tmem_ld32(tbase + 64, vc);
+        tmem_ld32(tbase + 96, vd);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {   // the accumulator is in registers: hand it back to the MMA
+          if constexpr (kPair) mbar_arrive_cluster_relaxed(acc_empty_lead + ab * 8);
+          else mbar_arrive(&acc_empty[ab]);
+        }
+        if (++ab == 2) { ab = 0; aph ^= 1; }
         const int cw0 = j0 + half * 128;             // first column of this warp's half
         const int rw0 = rbase + q * 32;              // first row of this warp
-        const bool diag = (rw0 < cw0 + 128) && (cw0 < rw0 + 32);
-        const float* rs = rho_s + ab * 256 + half * 128;
-        const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + half * 128;
-#pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t v[32];
-          tmem_ld32(tbase + ch * 32, v);
-          tmem_wait_ld();
-          if (!diag) {
+        if (!((rw0 < cw0 + 128) && (cw0 < rw0 + 32))) {
+          auto fold = [&](const uint32_t (&v)[32], int off) {
 #pragma unroll
             for (int cc = 0; cc < 32; cc += 4) {
-              const float4 r4 = *reinterpret_cast<const float4*>(rs + ch * 32 + cc);
+              const float4 r4 = *reinterpret_cast<const float4*>(rs + off + cc);
               s0 = fmaf(__uint_as_float(v[cc + 0]), r4.x, s0);
               s1 = fmaf(__uint_as_float(v[cc + 1]), r4.y, s1);
               s2 = fmaf(__uint_as_float(v[cc + 2]), r4.z, s2);
               s3 = fmaf(__uint_as_float(v[cc + 3]), r4.w, s3);
             }
-          } else {
-            const int jd = i - (cw0 + ch * 32);      // column of the diagonal in this chunk
+          };
+          fold(va, 0); fold(vb, 32); fold(vc, 64); fold(vd, 96);
+        } else {
+          const int jd = i - cw0;                    // this row's diagonal column in the half
+          auto fold = [&](const uint32_t (&v)[32], int off) {
 #pragma unroll
             for (int cc = 0; cc < 32; cc += 4) {
-              const float4 r4 = *reinterpret_cast<const float4*>(rs + ch * 32 + cc);
-              s0 = fmaf(cc + 0 == jd ? 0.f : __uint_as_float(v[cc + 0]), r4.x, s0);
-              s1 = fmaf(cc + 1 == jd ? 0.f : __uint_as_float(v[cc + 1]), r4.y, s1);
-              s2 = fmaf(cc + 2 == jd ? 0.f : __uint_as_float(v[cc + 2]), r4.z, s2);
-              s3 = fmaf(cc + 3 == jd ? 0.f : __uint_as_float(v[cc + 3]), r4.w, s3);
+              const float4 r4 = *reinterpret_cast<const float4*>(rs + off + cc);
+              s0 = fmaf(off + cc + 0 == jd ? 0.f : __uint_as_float(v[cc + 0]), r4.x, s0);
+              s1 = fmaf(off + cc + 1 == jd ? 0.f : __uint_as_float(v[cc + 1]), r4.y, s1);
+              s2 = fmaf(off + cc + 2 == jd ? 0.f : __uint_as_float(v[cc + 2]), r4.z, s2);
+              s3 = fmaf(off + cc + 3 == jd ? 0.f : __uint_as_float(v[cc + 3]), r4.w, s3);
             }
-          }
+          };
+          fold(va, 0); fold(vb, 32); fold(vc, 64); fold(vd, 96);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if constexpr (kPair) mbar_arrive_cluster(acc_empty_lead + ab * 8);
-          else mbar_arrive(&acc_empty[ab]);
-        }
-        if (++ab == 2) { ab = 0; aph ^= 1; }
       }
       // ---- item end: combine halves, write m, count the unit's finished blocks
       float tot = (s0 + s1) + (s2 + s3);

@@ -10,7 +10,7 @@ namespace rkv {
 constexpr int kHeadDim = 128;        // d (the only supported head size)
 constexpr int kTile = 128;           // tokens per K tile (TMA box rows, MMA M)
 constexpr int kTileBytes = kTile * kHeadDim * 2;
-constexpr int kMaxTokensPerUnit = 49152;
+constexpr int kMaxTokensPerUnit = 49152;  // select keeps a unit's keys in shared memory
 constexpr int kMaxRows = 32;         // G * w limit (MMA N of the logits tile)
 constexpr int kScoreThreads = 384;   // 12 warps
 constexpr int kGemmThreads = 384;
@@ -23,7 +23,6 @@ struct ScoreParams {
   int R;                   // G * w real query rows
   int w;
   int cs;                  // CTAs per cluster (one unit per cluster)
-  int lmax;                // tokens per CTA, multiple of 128
   int nstages;             // K tile ring depth
   float scale_log2;        // log2(e) / sqrt(d)
   float* a_out;            // [T]
@@ -34,34 +33,66 @@ struct ScoreParams {
 };
 
 struct ScoreLayout {
-  uint32_t stages, q, abar, marr, rhoc, rhot, ufin, mrow, invl, red1, red2, rsum, xbuf, bars,
-      slot, flags, total;
+  uint32_t stages, q, abar, marr, rhoc, rhot, ufin, gath, mrow, invl, red1, red2, rsum, rowt,
+      xbuf, bars, slot, flags, total;
 };
 
-__host__ __device__ inline int score_xb(int rp) { return 2 * rp + 128 + 4; }
+constexpr int kMaxClusterSize = 16;
+constexpr int kTmemColsTotal = 512;
 
-__host__ __device__ inline ScoreLayout score_layout(int rp, bool closed, int lmax, int ns) {
+// Logit tiles of one CTA live in TMEM for the whole unit: 512 columns hold
+// 512 / rp tiles of 128 tokens.
+__host__ __device__ inline int score_res_tiles(int rp) { return kTmemColsTotal / rp; }
+__host__ __device__ inline int score_lmax(int rp) { return score_res_tiles(rp) * kTile; }
+// Floats of one CTA's round-1 partials: (max, sum) per query row [, U].
+__host__ __device__ inline int score_xb(int rp, bool closed) { return 2 * rp + (closed ? 128 : 0); }
+constexpr int kScoreBarsFixed = 32 + 1 + 2 + 2 + 2;  // tile-ready, TMEM-free, Q, Q, exchange
+
+__host__ __device__ inline ScoreLayout score_layout(int rp, bool closed, int ns) {
   ScoreLayout L;
   uint32_t o = 0;
+  const int lmax = score_lmax(rp);
   L.stages = o; o += ns * kTileBytes;
   L.q = o; o += 2 * rp * 256;
   L.abar = o; o += lmax * 4;
   L.marr = o; if (closed) o += lmax * 4;
   L.rhoc = o; if (closed) o += lmax * 4;
-  L.rhot = o; o += 2 * 128 * 4;
-  L.ufin = o; o += 128 * 4;
+  L.rhot = o; if (closed) o += 2 * 128 * 4;
+  L.ufin = o; if (closed) o += 128 * 4;
+  L.gath = o; o += kMaxClusterSize * score_xb(rp, closed) * 4;
   L.mrow = o; o += rp * 4;
   L.invl = o; o += rp * 4;
   L.red1 = o; o += 4 * rp * 2 * 4;
-  L.red2 = o; o += 4 * 128 * 4;
+  L.red2 = o; if (closed) o += 4 * 128 * 4;
   L.rsum = o; o += 16 * 4;
-  L.xbuf = o; o += 2 * score_xb(rp) * 4;
+  L.rowt = o; o += 32 * 4;
+  L.xbuf = o; o += (score_xb(rp, closed) + 2 * kMaxClusterSize + 4) * 4;
   o = (o + 15u) & ~15u;
-  L.bars = o; o += (2 * ns + 14) * 8;
+  L.bars = o; o += (2 * ns + kScoreBarsFixed) * 8;
   L.slot = o; o += 16;
   L.flags = o; o += 16;
   L.total = o;
   return L;
+}
+
+// Deepest K-tile ring that fits next to the rest of the layout.
+__host__ __device__ inline int score_stages(int rp, bool closed, int smem_cap) {
+  for (int ns = 8; ns >= 2; --ns)
+    if (static_cast<int>(score_layout(rp, closed, ns).total) + 1024 <= smem_cap) return ns;
+  return 0;
+}
+
+// Cluster size for a batch whose longest unit has nmax tokens: about 1024
+// tokens per CTA, enough CTAs for the TMEM-resident logits, at most max_cs.
+// Returns 0 if the unit does not fit.
+inline int score_cluster_size(int nmax, int rp, int max_cs) {
+  int cs = 1;
+  while (cs < max_cs && (nmax + cs - 1) / cs > 1024) cs <<= 1;
+  while ((((nmax + cs - 1) / cs + kTile - 1) / kTile) * kTile > score_lmax(rp)) {
+    if (cs >= max_cs) return 0;
+    cs <<= 1;
+  }
+  return cs;
 }
 
 // ---------------------------------------------------------------- redundancy GEMM
@@ -100,7 +131,7 @@ __host__ __device__ inline GemmLayout gemm_layout() {
   uint32_t o = 0;
   L.a = o; o += C::kABytes;
   L.b = o; o += C::kStages * C::kBBytes;
-  L.rho = o; o += 2 * 256 * 4;
+  L.rho = o; o += 8 * 2 * 128 * 4;   // per epilogue warp: two 128-column slices
   L.rowx = o; o += 128 * 4;
   L.fin = o; o += 32 * 4;
   L.bars = o; o += (2 + 2 * C::kStages + 4) * 8;

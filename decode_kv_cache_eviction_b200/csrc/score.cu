@@ -1,35 +1,53 @@
 // Score kernel: importance (R-KV 重要性打分) and, in closed-form mode, the
-// redundancy row mean (R-KV 冗余打分) for every unit, in one pass over K.
+// redundancy row mean (R-KV 冗余打分) for every unit, with K read from HBM once.
 //
 // One thread-block cluster of `cs` CTAs owns one unit at a time; CTA `rank`
-// owns the contiguous token chunk [rank*L, rank*L + L) (L a multiple of 128).
-// Each chunk is streamed twice as 128-token K tiles through a TMA ring:
+// owns the contiguous token chunk [rank*L, rank*L + L) (L a multiple of 128,
+// at most 512 / RP tiles).  Per unit:
 //
-//   pass 1 (forward order, loads kept in L2 with evict_last):
-//     - logits z = K_tile . Q^T on tcgen05 (M = 128 tokens, N = padded G*w,
-//       fp32 accumulator in TMEM); per-thread online softmax statistics
-//       (running max and sum of 2^(y - max), y = z * log2(e) / sqrt(d));
-//     - key norms ||k|| on CUDA cores -> rho = 1/||k||;
-//     - (closed form) U = sum_j rho_j k_j.
-//   cluster exchange #1: merge (max, sum) per query row and U over the cluster
-//     through distributed shared memory.
-//   pass 2 (reverse order, so the most recently loaded tiles -- most likely
-//     still in L2 -- come first):
-//     - logits again; abar_j = (1/(G w)) sum_rows 2^(y - M_row) / L_row;
-//     - (closed form) m_j = (rho_j k_j . U - khat_j . khat_j) / (N - 1).
-//   cluster exchange #2: sum of abar over candidates and of exp(m).
+//   pass 1 (K tiles streamed by TMA, kept in L2 with evict_last in closed form):
+//     - logits z = K_tile . Q^T on tcgen05 (M = 128 tokens, N = RP padded
+//       query rows, fp32 accumulator).  Tile k's logits stay in TMEM columns
+//       [k*RP, (k+1)*RP) for the whole unit, so pass 2 needs no second MMA;
+//     - per-thread online softmax statistics (running max, sum of
+//       2^(y - max), y = z * log2(e) / sqrt(d)) with a lazy max;
+//     - key norms on CUDA cores -> rho = 1/||k||; (closed form) U = sum rho_j k_j.
+//   cluster exchange #1: every CTA gathers all CTAs' (max, sum) per query row
+//     [and partial U] through distributed shared memory and merges them in
+//     rank order, so every CTA holds identical values.
+//   pass 2:
+//     - abar_j = (1/(G w)) sum_rows 2^(y - M_row) / L_row from the TMEM logits;
+//     - (closed form) K tiles again, most recent first (likely still in L2):
+//       m_j = (rho_j k_j . U - khat_j . khat_j) / (N - 1) on CUDA cores.
+//   cluster exchange #2: sums of abar and of exp(m) over the candidates.
 //   write a = abar / sum, r = exp(m) / sum (window rows get 0).
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM
-// owner, warps 4-7 logits/softmax (thread = token row of the tile, lane
-// quarter = warp % 4), warps 8-11 norms / U / k.U (thread = token row).
+// owner, warps 4-7 softmax (thread = token row of a tile; TMEM lane quarter =
+// warp % 4), warps 8-11 norms and U (thread = token row).
 #include "ptx.cuh"
 #include "rkv_internal.cuh"
 
 namespace rkv {
 namespace {
 
-constexpr int kNAcc = 4;  // TMEM accumulator buffers
+constexpr float kNegBig = -1e30f;  // initial running max (finite: no inf - inf)
+constexpr float kLazy = 8.f;       // log2 headroom before the running max moves
+
+#ifdef RKV_TRACE
+// Optional phase trace (build with -DRKV_TRACE): globaltimer stamps per CTA for
+// the first kTraceUnits units it processes, kTraceSlots stamps each.
+constexpr int kTraceCtas = 256, kTraceUnits = 8, kTraceSlots = 8;
+__device__ unsigned long long g_score_trace[kTraceCtas * kTraceUnits * kTraceSlots];
+#define RKV_STAMP(it, slot)                                                              \
+  do {                                                                                   \
+    if ((it) < kTraceUnits && blockIdx.x < kTraceCtas)                                   \
+      g_score_trace[(blockIdx.x * kTraceUnits + (it)) * kTraceSlots + (slot)] =          \
+          globaltimer_ns();                                                              \
+  } while (0)
+#else
+#define RKV_STAMP(it, slot) do { } while (0)
+#endif
 
 struct UnitSched {
   int64_t base;  // first row of the unit in K
@@ -62,67 +80,98 @@ __device__ __forceinline__ void tmem_ld_rows(uint32_t taddr, uint32_t (&v)[RP]) 
 // Merge two (max, sum) softmax statistics in the log2 domain.
 __device__ __forceinline__ void merge_stat(float& m, float& s, float om, float os) {
   const float M = fmaxf(m, om);
-  if (M == -INFINITY) {
-    m = M;
-    s = 0.f;
-    return;
-  }
   s = s * ex2(m - M) + os * ex2(om - M);
   m = M;
 }
 
-// Exchange `nvals` floats at `xb` (this CTA's partials) with every CTA of the
-// cluster: release-arrive on each CTA's barrier, then wait for all of them.
+// Thread rr (< cs) releases to CTA rr: a cluster-scope fence (cumulative over
+// the CTA barrier before it) followed by a relaxed arrive.  Then every
+// consumer thread waits until all CTAs of the cluster have released.
 __device__ __forceinline__ void cluster_exchange(uint64_t* bar, uint32_t parity, int cs,
                                                  int ctid, volatile int* abort, int* status) {
-  fence_acq_rel_cluster();
   named_bar_sync(1, 256);
-  if (ctid == 0) {
-    const uint32_t local = smem_u32(bar);
-    for (int rr = 0; rr < cs; ++rr) mbar_arrive_cluster(mapa(local, rr));
+  if (ctid < cs) {
+    fence_acq_rel_cluster();
+    mbar_arrive_cluster_relaxed(mapa(smem_u32(bar), ctid));
   }
   mbar_wait<true>(bar, parity, abort, status);
   __syncwarp();
+}
+
+// Copy `n` floats at `src` (same offset in every CTA) from all `cs` CTAs into
+// the local array dst[rank * n + k]; all loads are issued before any store.
+__device__ __forceinline__ void cluster_gather(float* dst, const float* src, int n, int cs,
+                                               int ctid) {
+  constexpr int kMaxPer = (kMaxClusterSize * (2 * 32 + 128) + 255) / 256;
+  const uint32_t local = smem_u32(src);
+  const int total = n * cs;
+  float v[kMaxPer];
+#pragma unroll
+  for (int k = 0; k < kMaxPer; ++k) {
+    const int e = ctid + k * 256;
+    if (e < total) {
+      const int rr = e / n;
+      v[k] = ld_cluster_f32(mapa(local + 4u * static_cast<uint32_t>(e - rr * n), rr));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kMaxPer; ++k) {
+    const int e = ctid + k * 256;
+    if (e < total) dst[e] = v[k];
+  }
+}
+
+// Load the 16 swizzled 16-byte chunks of K-tile row `row` (128 bf16).
+__device__ __forceinline__ void load_row(uint32_t sb, int row, uint4 (&xs)[16]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+      const uint32_t ad = sb + h * (kTileBytes / 2) + row * 128 + ((cc ^ (row & 7)) << 4);
+      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(xs[h * 8 + cc].x), "=r"(xs[h * 8 + cc].y), "=r"(xs[h * 8 + cc].z),
+                     "=r"(xs[h * 8 + cc].w)
+                   : "r"(ad));
+    }
+  }
 }
 
 template <int RP, bool CLOSED>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                  const ScoreParams p) {
+  constexpr int XB = 2 * RP + (CLOSED ? 128 : 0);   // round-1 partial floats per CTA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   const int NS = p.nstages;
-  const ScoreLayout L = score_layout(RP, CLOSED, p.lmax, NS);
+  const ScoreLayout L = score_layout(RP, CLOSED, NS);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = static_cast<int>(cluster_ctarank());
   const int cid = static_cast<int>(cluster_id_x());
   const int ncl = static_cast<int>(cluster_count_x());
   const int cs = p.cs;
-  const int XB = score_xb(RP);
 
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* empty = full + NS;
-  uint64_t* acc_full = empty + NS;
-  uint64_t* acc_empty = acc_full + kNAcc;
-  uint64_t* qfull = acc_empty + kNAcc;
+  uint64_t* tready = empty + NS;   // [32] logits of tile k are in TMEM
+  uint64_t* tfree = tready + 32;   // softmax warps are done with the unit's TMEM
+  uint64_t* qfull = tfree + 1;
   uint64_t* qempty = qfull + 2;
   uint64_t* redbar = qempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.slot);
   volatile int* abort = reinterpret_cast<volatile int*>(sm + L.flags);
   float* rsum = reinterpret_cast<float*>(sm + L.rsum);
   float* xbuf = reinterpret_cast<float*>(sm + L.xbuf);
-  constexpr uint32_t kTmemCols = (kNAcc * RP < 32) ? 32 : kNAcc * RP;
+  float* gath = reinterpret_cast<float*>(sm + L.gath);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);  // MMA commit + 4 norm warps
+      mbar_init(&empty[s], 1 + 4);  // MMA thread + 4 norm warps
     }
-    for (int b = 0; b < kNAcc; ++b) {
-      mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
-    }
+    for (int k = 0; k < 32; ++k) mbar_init(&tready[k], 1);
+    mbar_init(tfree, 4);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&qfull[b], 1);
       mbar_init(&qempty[b], 1);
@@ -132,7 +181,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc<1>(tmem_slot, kTmemCols);
+    tmem_alloc<1>(tmem_slot, kTmemColsTotal);
     tmem_relinquish<1>();
   }
   tc_fence_before();
@@ -158,18 +207,21 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           tma_load_2d(qd, &qmap, &qfull[qb], 0, u * p.R, keep);
           tma_load_2d(qd + RP * 128, &qmap, &qfull[qb], 64, u * p.R, keep);
         }
-        for (int pass = 0; pass < 2; ++pass) {
+        for (int pass = 0; pass < (CLOSED ? 2 : 1); ++pass) {
           for (int kk = 0; kk < s.nt; ++kk) {
             const int k = pass ? s.nt - 1 - kk : kk;
             if (mbar_wait(&empty[stage], ph ^ 1, abort, p.status)) {
               uint8_t* dst = sm + L.stages + stage * kTileBytes;
               const int y = static_cast<int>(s.base + s.start + kTile * k);
+              // read once (GEMM form), or kept for the pass-2 re-read (closed form)
+              const uint64_t pol = (CLOSED && pass == 0) ? keep : drop;
               mbar_arrive_expect_tx(&full[stage], kTileBytes);
-              tma_load_2d(dst, &kmap, &full[stage], 0, y, pass ? drop : keep);
-              tma_load_2d(dst + kTileBytes / 2, &kmap, &full[stage], 64, y, pass ? drop : keep);
+              tma_load_2d(dst, &kmap, &full[stage], 0, y, pol);
+              tma_load_2d(dst + kTileBytes / 2, &kmap, &full[stage], 64, y, pol);
             }
             if (++stage == NS) { stage = 0; ph ^= 1; }
           }
+          if (pass == 0) RKV_STAMP(it, 7);
         }
       }
     }
@@ -178,44 +230,53 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, RP);
-      int stage = 0, ab = 0;
-      uint32_t ph = 0, aph = 0;
+      int stage = 0;
+      uint32_t ph = 0;
       int it = 0;
       for (int u = cid; u < p.num_units; u += ncl, ++it) {
         const UnitSched s = unit_sched(p, u, rank);
         const int qb = it & 1;
         bool ok = mbar_wait(&qfull[qb], (it >> 1) & 1, abort, p.status);
+        // the previous unit's logits must have been read out of TMEM
+        ok = mbar_wait(tfree, (it & 1) ^ 1, abort, p.status) && ok;
         const uint32_t qaddr = smem_u32(sm + L.q + qb * RP * 256);
-        for (int pass = 0; pass < 2; ++pass) {
-          for (int kk = 0; kk < s.nt; ++kk) {
-            bool go = mbar_wait(&full[stage], ph, abort, p.status);
-            go = mbar_wait(&acc_empty[ab], aph ^ 1, abort, p.status) && go && ok;
-            tc_fence_after();
-            if (go) {
-              const uint32_t kaddr = smem_u32(sm + L.stages + stage * kTileBytes);
-              const uint32_t d = tmem + ab * RP;
+        for (int k = 0; k < s.nt; ++k) {
+          const bool go = mbar_wait(&full[stage], ph, abort, p.status) && ok;
+          tc_fence_after();
+          if (go) {
+            const uint32_t kaddr = smem_u32(sm + L.stages + stage * kTileBytes);
+            const uint32_t d = tmem + k * RP;
 #pragma unroll
-              for (int kq = 0; kq < 8; ++kq) {
-                const uint32_t ko = (kq >> 2) * (kTileBytes / 2) + (kq & 3) * 32;
-                const uint32_t qo = (kq >> 2) * (RP * 128) + (kq & 3) * 32;
-                mma_bf16<1>(d, desc_kmajor_sw128(kaddr + ko), desc_kmajor_sw128(qaddr + qo),
-                            idesc, kq > 0);
-              }
-              mma_commit(&empty[stage]);
-              mma_commit(&acc_full[ab]);
+            for (int kq = 0; kq < 8; ++kq) {
+              const uint32_t ko = (kq >> 2) * (kTileBytes / 2) + (kq & 3) * 32;
+              const uint32_t qo = (kq >> 2) * (RP * 128) + (kq & 3) * 32;
+              mma_bf16<1>(d, desc_kmajor_sw128(kaddr + ko), desc_kmajor_sw128(qaddr + qo),
+                          idesc, kq > 0);
             }
-            if (++stage == NS) { stage = 0; ph ^= 1; }
-            if (++ab == kNAcc) { ab = 0; aph ^= 1; }
+            mma_commit(&empty[stage]);
+            mma_commit(&tready[k]);
+          } else {
+            mbar_arrive(&empty[stage]);
           }
+          if (++stage == NS) { stage = 0; ph ^= 1; }
         }
         if (ok) mma_commit(&qempty[qb]);
+        else mbar_arrive(&qempty[qb]);
+        if constexpr (CLOSED) {
+          // pass-2 tiles feed only the norm warps: keep the ring's arrival count
+          for (int k = 0; k < s.nt; ++k) {
+            mbar_wait(&full[stage], ph, abort, p.status);
+            mbar_arrive(&empty[stage]);
+            if (++stage == NS) { stage = 0; ph ^= 1; }
+          }
+        }
       }
     }
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ consumers
     const int ctid = threadIdx.x - 128;      // 0..255
-    const bool is_soft = warp < 8;           // warps 4-7: logits / softmax
+    const bool is_soft = warp < 8;           // warps 4-7: softmax
     const int q4 = warp & 3;                 // TMEM lane quarter
     const int row = q4 * 32 + lane;          // token row of the tile
     float* abar_s = reinterpret_cast<float*>(sm + L.abar);
@@ -228,75 +289,95 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     float* red1 = reinterpret_cast<float*>(sm + L.red1);
     float* red2 = reinterpret_cast<float*>(sm + L.red2);
     const float invR = 1.f / static_cast<float>(p.R);
+    // bit r set for real query rows; row_t[r] = window step t of query row
+    // r = g*w + t (read only for tiles that reach the window)
+    const uint32_t rmask = p.R >= 32 ? 0xffffffffu : ((1u << p.R) - 1u);
+    const int* row_t = reinterpret_cast<const int*>(sm + L.rowt);
+    if (ctid < 32) reinterpret_cast<int*>(sm + L.rowt)[ctid] = ctid % p.w;
+    named_bar_sync(1, 256);
 
-    int stage = 0, ab = 0, ntile1 = 0;
-    uint32_t ph = 0, aph = 0;
+    int stage = 0, ntile1 = 0;
+    uint32_t ph = 0;
+    uint32_t tph = 0;  // phase bit of tready[k]
     int it = 0;
     for (int u = cid; u < p.num_units; u += ncl, ++it) {
       const UnitSched s = unit_sched(p, u, rank);
-      const int N = s.n, c = s.c, w = p.w;
+      const int N = s.n, c = s.c;
       float st_m[RP], st_s[RP];  // pass 1: running stats; pass 2: row max and 1/sum
 #pragma unroll
-      for (int r = 0; r < RP; ++r) { st_m[r] = -INFINITY; st_s[r] = 0.f; }
+      for (int r = 0; r < RP; ++r) { st_m[r] = kNegBig; st_s[r] = 0.f; }
       float U4[4] = {0.f, 0.f, 0.f, 0.f};
-      float part = 0.f;  // pass 2: sum of abar (softmax warps) or of exp(m) (norm warps)
+      float part = 0.f;  // pass 2: sum of abar (softmax) or of exp(m) (norm warps)
+      if (ctid == 0) RKV_STAMP(it, 0);
 
       // ================================================= pass 1
       for (int k = 0; k < s.nt; ++k) {
         const int t0 = s.start + kTile * k;
+        const int j = t0 + row;
         if (is_soft) {
-          mbar_wait(&acc_full[ab], aph, abort, p.status);
+          mbar_wait(&tready[k], (tph >> k) & 1u, abort, p.status);
+          tph ^= 1u << k;
           __syncwarp();
           tc_fence_after();
           uint32_t v[RP];
-          tmem_ld_rows<RP>(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + ab * RP, v);
+          tmem_ld_rows<RP>(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + k * RP, v);
           tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[ab]);
-          if (++ab == kNAcc) { ab = 0; aph ^= 1; }
-          const int j = t0 + row;
+          // y = log2-scaled logit, -inf where masked (padding row, beyond N,
+          // causal); only a tile that reaches the window needs the causal limit
+          float y[RP];
           if (t0 + kTile <= c) {
 #pragma unroll
+            for (int r = 0; r < RP; ++r)
+              y[r] = ((rmask >> r) & 1u) ? __uint_as_float(v[r]) * p.scale_log2 : -INFINITY;
+          } else {
+#pragma unroll
             for (int r = 0; r < RP; ++r) {
-              if (r < p.R) {
-                const float y = __uint_as_float(v[r]) * p.scale_log2;
-                if (y > st_m[r]) { st_s[r] = st_s[r] * ex2(st_m[r] - y) + 1.f; st_m[r] = y; }
-                else st_s[r] += ex2(y - st_m[r]);
+              const bool vis = ((rmask >> r) & 1u) && j < N && j <= c + row_t[r];
+              y[r] = vis ? __uint_as_float(v[r]) * p.scale_log2 : -INFINITY;
+            }
+          }
+          // Lazy running max: the reference max only moves when a logit exceeds
+          // it by more than 2^kLazy, so terms 2^(y - max) stay below 256 and the
+          // common case is branch-free.
+          bool need = false;
+#pragma unroll
+          for (int r = 0; r < RP; ++r) need |= y[r] > st_m[r] + kLazy;
+          if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+              if (y[r] > st_m[r]) {
+                st_s[r] = st_s[r] * ex2(st_m[r] - y[r]) + 1.f;
+                st_m[r] = y[r];
+              } else {
+                st_s[r] += ex2(y[r] - st_m[r]);
               }
             }
           } else {
 #pragma unroll
-            for (int r = 0; r < RP; ++r) {
-              if (r < p.R && j < N && j <= c + (r % w)) {
-                const float y = __uint_as_float(v[r]) * p.scale_log2;
-                if (y > st_m[r]) { st_s[r] = st_s[r] * ex2(st_m[r] - y) + 1.f; st_m[r] = y; }
-                else st_s[r] += ex2(y - st_m[r]);
-              }
-            }
+            for (int r = 0; r < RP; ++r) st_s[r] += ex2(y[r] - st_m[r]);
           }
         } else {
-          // norm warps: ||k|| of row `row`, rho, (closed) U accumulation
+          // norm warps: ||k|| of row `row`, rho, (closed form) U accumulation
           mbar_wait(&full[stage], ph, abort, p.status);
+          __syncwarp();
           const uint32_t sb = smem_u32(sm + L.stages + stage * kTileBytes);
-          const int j = t0 + row;
-          float n2a = 0.f, n2b = 0.f;
+          uint4 xs[16];
+          load_row(sb, row, xs);
+          float nq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-              uint4 x;
-              const uint32_t ad = sb + h * (kTileBytes / 2) + row * 128 + ((cc ^ (row & 7)) << 4);
-              asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                           : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w) : "r"(ad));
-              float f;
-              f = bf_lo(x.x); n2a = fmaf(f, f, n2a); f = bf_hi(x.x); n2b = fmaf(f, f, n2b);
-              f = bf_lo(x.y); n2a = fmaf(f, f, n2a); f = bf_hi(x.y); n2b = fmaf(f, f, n2b);
-              f = bf_lo(x.z); n2a = fmaf(f, f, n2a); f = bf_hi(x.z); n2b = fmaf(f, f, n2b);
-              f = bf_lo(x.w); n2a = fmaf(f, f, n2a); f = bf_hi(x.w); n2b = fmaf(f, f, n2b);
-            }
+          for (int k8 = 0; k8 < 16; ++k8) {
+            float f;
+            f = bf_lo(xs[k8].x); nq[0] = fmaf(f, f, nq[0]);
+            f = bf_hi(xs[k8].x); nq[1] = fmaf(f, f, nq[1]);
+            f = bf_lo(xs[k8].y); nq[2] = fmaf(f, f, nq[2]);
+            f = bf_hi(xs[k8].y); nq[3] = fmaf(f, f, nq[3]);
+            f = bf_lo(xs[k8].z); nq[4] = fmaf(f, f, nq[4]);
+            f = bf_hi(xs[k8].z); nq[5] = fmaf(f, f, nq[5]);
+            f = bf_lo(xs[k8].w); nq[6] = fmaf(f, f, nq[6]);
+            f = bf_hi(xs[k8].w); nq[7] = fmaf(f, f, nq[7]);
           }
-          const float n2 = n2a + n2b;
+          const float n2 =
+              ((nq[0] + nq[1]) + (nq[2] + nq[3])) + ((nq[4] + nq[5]) + (nq[6] + nq[7]));
           const float rho = (j < N && n2 > 0.f) ? 1.f / sqrtf(n2) : 0.f;
           if constexpr (CLOSED) {
             rhoc[j - s.start] = rho;
@@ -307,6 +388,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             const int hh = lane >> 4;
             const uint32_t cidx = (lane & 15) >> 1;
             const uint32_t sub = (lane & 1) * 8;
+            float U8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
             for (int rr = 0; rr < 32; ++rr) {
               const int rw = q4 * 32 + rr;
@@ -315,11 +397,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                   sb + hh * (kTileBytes / 2) + rw * 128 + ((cidx ^ (rw & 7)) << 4) + sub;
               uint32_t x0, x1;
               asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(x0), "=r"(x1) : "r"(ad));
-              U4[0] = fmaf(rr_rho, bf_lo(x0), U4[0]);
-              U4[1] = fmaf(rr_rho, bf_hi(x0), U4[1]);
-              U4[2] = fmaf(rr_rho, bf_lo(x1), U4[2]);
-              U4[3] = fmaf(rr_rho, bf_hi(x1), U4[3]);
+              float* Ua = U8 + (rr & 1) * 4;
+              Ua[0] = fmaf(rr_rho, bf_lo(x0), Ua[0]);
+              Ua[1] = fmaf(rr_rho, bf_hi(x0), Ua[1]);
+              Ua[2] = fmaf(rr_rho, bf_lo(x1), Ua[2]);
+              Ua[3] = fmaf(rr_rho, bf_hi(x1), Ua[3]);
             }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) U4[i] += U8[i] + U8[4 + i];
           } else {
             if (j < N && p.rho_out) p.rho_out[s.base + j] = rho;
           }
@@ -331,6 +416,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       }
 
       // ================================================= exchange 1
+      if (ctid == 0) RKV_STAMP(it, 1);
+      if (ctid == 128) RKV_STAMP(it, 2);
       if (is_soft) {
 #pragma unroll
         for (int r = 0; r < RP; ++r) {
@@ -353,10 +440,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         for (int i = 0; i < 4; ++i) red2[q4 * 128 + lane * 4 + i] = U4[i];
       }
       named_bar_sync(1, 256);
-      float* xa = xbuf;  // exchange buffer of round 1
+      float* xa = xbuf;  // this CTA's round-1 partials
       if (ctid < RP) {
-        float m = -INFINITY, sacc = 0.f;
-        for (int q = 0; q < 4; ++q) merge_stat(m, sacc, red1[(q * RP + ctid) * 2], red1[(q * RP + ctid) * 2 + 1]);
+        float m = kNegBig, sacc = 0.f;
+        for (int q = 0; q < 4; ++q)
+          merge_stat(m, sacc, red1[(q * RP + ctid) * 2], red1[(q * RP + ctid) * 2 + 1]);
         xa[2 * ctid] = m;
         xa[2 * ctid + 1] = sacc;
       }
@@ -365,98 +453,100 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         xa[2 * RP + e] = red2[e] + red2[128 + e] + red2[256 + e] + red2[384 + e];
       }
       cluster_exchange(&redbar[0], it & 1, cs, ctid, abort, p.status);
+      cluster_gather(gath, xa, XB, cs, ctid);
+      named_bar_sync(1, 256);
       if (ctid < RP) {
-        float m = -INFINITY, sacc = 0.f;
-        const uint32_t la = smem_u32(&xa[2 * ctid]);
-        for (int rr = 0; rr < cs; ++rr) {
-          const uint32_t ra = mapa(la, rr);
-          merge_stat(m, sacc, ld_cluster_f32(ra), ld_cluster_f32(ra + 4));
-        }
+        float m = kNegBig, sacc = 0.f;
+        for (int rr = 0; rr < cs; ++rr)
+          merge_stat(m, sacc, gath[rr * XB + 2 * ctid], gath[rr * XB + 2 * ctid + 1]);
         mrow[ctid] = m;
         invl[ctid] = sacc > 0.f ? 1.f / sacc : 0.f;
       }
       if (CLOSED && ctid >= 128) {
         const int e = ctid - 128;
-        const uint32_t la = smem_u32(&xa[2 * RP + e]);
         float acc = 0.f;
-        for (int rr = 0; rr < cs; ++rr) acc += ld_cluster_f32(mapa(la, rr));
+        for (int rr = 0; rr < cs; ++rr) acc += gath[rr * XB + 2 * RP + e];
         ufin[e] = acc;
       }
       named_bar_sync(1, 256);
       if (is_soft) {
 #pragma unroll
         for (int r = 0; r < RP; ++r) {
-          st_m[r] = (r < p.R) ? mrow[r] : 0.f;
-          st_s[r] = (r < p.R) ? invl[r] : 0.f;
+          // padding rows: a huge max and zero weight, so they add exactly 0
+          st_m[r] = ((rmask >> r) & 1u) ? mrow[r] : 1e30f;
+          st_s[r] = ((rmask >> r) & 1u) ? invl[r] : 0.f;
         }
       }
+      if (ctid == 0) RKV_STAMP(it, 3);
 
-      // ================================================= pass 2 (reverse)
+      // ================================================= pass 2
       const float inv_nm1 = N > 1 ? 1.f / static_cast<float>(N - 1) : 0.f;
-      for (int kk = 0; kk < s.nt; ++kk) {
-        const int k = s.nt - 1 - kk;
-        const int t0 = s.start + kTile * k;
-        const int j = t0 + row;
-        if (is_soft) {
-          mbar_wait(&acc_full[ab], aph, abort, p.status);
-          __syncwarp();
-          tc_fence_after();
+      if (is_soft) {
+        for (int k = 0; k < s.nt; ++k) {
+          const int t0 = s.start + kTile * k;
+          const int j = t0 + row;
           uint32_t v[RP];
-          tmem_ld_rows<RP>(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + ab * RP, v);
+          tmem_ld_rows<RP>(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + k * RP, v);
           tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[ab]);
-          if (++ab == kNAcc) { ab = 0; aph ^= 1; }
-          float pj = 0.f;
+          float pq[4] = {0.f, 0.f, 0.f, 0.f};
           if (t0 + kTile <= c) {
 #pragma unroll
             for (int r = 0; r < RP; ++r)
-              if (r < p.R) pj = fmaf(ex2(fmaf(__uint_as_float(v[r]), p.scale_log2, -st_m[r])), st_s[r], pj);
+              pq[r & 3] = fmaf(ex2(fmaf(__uint_as_float(v[r]), p.scale_log2, -st_m[r])),
+                               st_s[r], pq[r & 3]);
           } else {
 #pragma unroll
             for (int r = 0; r < RP; ++r)
-              if (r < p.R && j < N && j <= c + (r % w))
-                pj = fmaf(ex2(fmaf(__uint_as_float(v[r]), p.scale_log2, -st_m[r])), st_s[r], pj);
+              if (((rmask >> r) & 1u) && j < N && j <= c + row_t[r])
+                pq[r & 3] = fmaf(ex2(fmaf(__uint_as_float(v[r]), p.scale_log2, -st_m[r])),
+                                 st_s[r], pq[r & 3]);
           }
           if (j < c) {
-            const float ab_ = pj * invR;
+            const float ab_ = ((pq[0] + pq[1]) + (pq[2] + pq[3])) * invR;
             abar_s[j - s.start] = ab_;
             part += ab_;
           }
-        } else {
+        }
+        // the unit's logits have been read: TMEM may take the next unit
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tfree);
+      } else if (CLOSED) {
+        for (int kk = 0; kk < s.nt; ++kk) {
+          const int k = s.nt - 1 - kk;
+          const int j = s.start + kTile * k + row;
           mbar_wait(&full[stage], ph, abort, p.status);
-          if constexpr (CLOSED) {
-            const uint32_t sb = smem_u32(sm + L.stages + stage * kTileBytes);
-            float da = 0.f, db = 0.f;
+          __syncwarp();
+          const uint32_t sb = smem_u32(sm + L.stages + stage * kTileBytes);
+          uint4 xs[16];
+          load_row(sb, row, xs);
+          float dq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-#pragma unroll
-              for (int cc = 0; cc < 8; ++cc) {
-                uint4 x;
-                const uint32_t ad = sb + h * (kTileBytes / 2) + row * 128 + ((cc ^ (row & 7)) << 4);
-                asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                             : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w) : "r"(ad));
-                const float4 ua = *reinterpret_cast<const float4*>(&ufin[h * 64 + cc * 8]);
-                const float4 ub = *reinterpret_cast<const float4*>(&ufin[h * 64 + cc * 8 + 4]);
-                da = fmaf(bf_lo(x.x), ua.x, da); db = fmaf(bf_hi(x.x), ua.y, db);
-                da = fmaf(bf_lo(x.y), ua.z, da); db = fmaf(bf_hi(x.y), ua.w, db);
-                da = fmaf(bf_lo(x.z), ub.x, da); db = fmaf(bf_hi(x.z), ub.y, db);
-                da = fmaf(bf_lo(x.w), ub.z, da); db = fmaf(bf_hi(x.w), ub.w, db);
-              }
-            }
-            if (j < c) {
-              const float rho = rhoc[j - s.start];
-              const float m = (rho * (da + db) - (rho > 0.f ? 1.f : 0.f)) * inv_nm1;
-              marr[j - s.start] = m;
-              part += ex2(m * kLog2e);
-            }
+          for (int k8 = 0; k8 < 16; ++k8) {
+            const float4 ua = *reinterpret_cast<const float4*>(&ufin[k8 * 8]);
+            const float4 ub = *reinterpret_cast<const float4*>(&ufin[k8 * 8 + 4]);
+            dq[0] = fmaf(bf_lo(xs[k8].x), ua.x, dq[0]);
+            dq[1] = fmaf(bf_hi(xs[k8].x), ua.y, dq[1]);
+            dq[2] = fmaf(bf_lo(xs[k8].y), ua.z, dq[2]);
+            dq[3] = fmaf(bf_hi(xs[k8].y), ua.w, dq[3]);
+            dq[0] = fmaf(bf_lo(xs[k8].z), ub.x, dq[0]);
+            dq[1] = fmaf(bf_hi(xs[k8].z), ub.y, dq[1]);
+            dq[2] = fmaf(bf_lo(xs[k8].w), ub.z, dq[2]);
+            dq[3] = fmaf(bf_hi(xs[k8].w), ub.w, dq[3]);
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[stage]);
           if (++stage == NS) { stage = 0; ph ^= 1; }
+          if (j < c) {
+            const float rho = rhoc[j - s.start];
+            const float dot = (dq[0] + dq[1]) + (dq[2] + dq[3]);
+            const float m = (rho * dot - (rho > 0.f ? 1.f : 0.f)) * inv_nm1;
+            marr[j - s.start] = m;
+            part += ex2(m * kLog2e);
+          }
         }
       }
+      if (ctid == 0) RKV_STAMP(it, 4);
 
       // ================================================= exchange 2 and output
       part = warp_reduce_sum(part);
@@ -468,19 +558,21 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         xb2[1] = rsum[4] + rsum[5] + rsum[6] + rsum[7];
       }
       cluster_exchange(&redbar[1], it & 1, cs, ctid, abort, p.status);
+      float* g2 = xbuf + XB + 4;   // [cs][2] gathered sums
+      if (ctid < 2 * cs) g2[ctid] = ld_cluster_f32(mapa(smem_u32(&xb2[ctid & 1]), ctid >> 1));
+      named_bar_sync(1, 256);
       if (ctid == 0) {
         float sa = 0.f, se = 0.f;
-        const uint32_t la = smem_u32(&xb2[0]);
         for (int rr = 0; rr < cs; ++rr) {
-          const uint32_t ra = mapa(la, rr);
-          sa += ld_cluster_f32(ra);
-          se += ld_cluster_f32(ra + 4);
+          sa += g2[2 * rr];
+          se += g2[2 * rr + 1];
         }
         rsum[8] = sa > 0.f ? 1.f / sa : 0.f;
         rsum[9] = se > 0.f ? 1.f / se : 0.f;
       }
       named_bar_sync(1, 256);
       const float inv_sa = rsum[8], inv_se = rsum[9];
+      if (ctid == 0) RKV_STAMP(it, 5);
       for (int i = ctid; i < s.len; i += 256) {
         const int j = s.start + i;
         const int64_t g = s.base + j;
@@ -497,6 +589,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           if (p.m_out) p.m_out[g] = 0.f;
         }
       }
+      if (ctid == 0) RKV_STAMP(it, 6);
     }
   }
 
@@ -505,7 +598,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc<1>(tmem, kTmemCols);
+    tmem_dealloc<1>(tmem, kTmemColsTotal);
   }
 }
 
@@ -520,6 +613,12 @@ void* pick(int rp, bool closed) {
 }
 
 }  // namespace
+
+#ifdef RKV_TRACE
+cudaError_t score_trace_read(void* dst, size_t bytes) {
+  return cudaMemcpyFromSymbol(dst, g_score_trace, bytes);
+}
+#endif
 
 cudaError_t score_configure(int rp, bool closed, int smem_bytes, int cs) {
   void* f = pick(rp, closed);
@@ -552,7 +651,7 @@ int score_max_clusters(int rp, bool closed, int smem_bytes, int cs) {
 
 cudaError_t launch_score(const CUtensorMap& kmap, const CUtensorMap& qmap, const ScoreParams& p,
                          int rp, bool closed, int nclusters, cudaStream_t st) {
-  const ScoreLayout L = score_layout(rp, closed, p.lmax, p.nstages);
+  const ScoreLayout L = score_layout(rp, closed, p.nstages);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nclusters * p.cs, 1, 1);
   cfg.blockDim = dim3(kScoreThreads, 1, 1);

@@ -13,6 +13,9 @@
  * slot buffer (gather compaction, named as the R-KV-style baseline in the ThinKV
  * summary, "Continuous Thinking" section).
  *
+ * Limits: head_dim = 128, G*w <= 32; N_u <= 32768 when G*w > 16, else N_u <= 49152
+ * (each cluster of up to 16 CTAs keeps a unit's logits in tensor memory).
+ *
  * Terms used below.  A *unit* is one (sequence, layer, KV head).  Unit u has
  * N_u cached tokens, stored as rows tok_off[u] .. tok_off[u+1]-1 of K and V.
  * d = head_dim (= 128), G = query heads per KV head, w = window.  Query (g, t)
@@ -48,7 +51,7 @@ typedef struct rkv_engine rkv_engine;     /* opaque; owns device workspace only 
 enum {
   RKV_OK = 0,
   RKV_ERR_INVALID_ARG = -1, /* null/unaligned pointer, bad size, N_u < w, ... */
-  RKV_ERR_UNSUPPORTED = -2, /* head_dim != 128, G*w > 32, N_u > 49152, not sm_100 */
+  RKV_ERR_UNSUPPORTED = -2, /* head_dim != 128, G*w > 32, N_u too long, not sm_100 */
   RKV_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
   RKV_ERR_TIMEOUT = -4,     /* a device-side wait ran out of time (see rkv_check_status) */
   RKV_ERR_OOM = -5,         /* workspace allocation failed */
@@ -177,7 +180,7 @@ int rkv_read_timing(rkv_engine* eng, int kernel, double* total_ms, int64_t* laun
  * nothing is allocated or freed per call.  Limits: at most RKV_NOALLOC_MAX_UNITS
  * units and RKV_NOALLOC_MAX_TOKENS rows per call (larger batches return
  * RKV_ERR_CAPACITY before anything is enqueued), and the rkv_score limits
- * (G*w <= 32, N_u <= 49152).
+ * (G*w <= 32; N_u <= 32768 when G*w > 16, else N_u <= 49152).
  *
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) and sets kernel attributes with that device current;

@@ -155,11 +155,13 @@ def test_gemm_single_cta_and_pair_agree():
     np.testing.assert_allclose(o2["r"], o3["r"], rtol=1e-4, atol=1e-9)
 
 
-def test_largest_supported_unit():
-    N = 49152
-    b = rand_batch([N], 4, 8, seed=1, dup=0.0)
+@pytest.mark.parametrize("G,N", [(4, 32768), (2, 49152)])
+def test_largest_supported_unit(G, N):
+    # logits of a unit stay in tensor memory: 32768 tokens at G*w = 32,
+    # 49152 (the select limit) at G*w <= 16
+    b = rand_batch([N], G, 8, seed=1, dup=0.0)
     for mode in ("closed", "gemm"):
-        out = run_engine(b, 4, 8, 0.1, 4096, mode=mode)
+        out = run_engine(b, G, 8, 0.1, 4096, mode=mode)
         check_unit(out, b, 0, 8, 0.1, 4096)
 
 
@@ -169,6 +171,11 @@ def test_rejects_too_long_unit_and_capacity():
     a, r = eng.alloc_scores(b)
     with pytest.raises(RkvError) as ei:
         eng.score(b, a, r)
+    assert ei.value.code == -2
+    b4 = rand_batch([32769], 4, 8, seed=0, dup=0.0)
+    eng4 = Engine(4, 8, max_units=1, max_tokens=b4.num_tokens, redundancy="gemm")
+    with pytest.raises(RkvError) as ei:
+        eng4.score(b4, *eng4.alloc_scores(b4))
     assert ei.value.code == -2
     b2 = rand_batch([200], 1, 8, seed=0, dup=0.0)
     small = Engine(1, 8, max_units=1, max_tokens=100, redundancy="closed")
