@@ -12,7 +12,7 @@ constexpr int kTile = 128;           // tokens per K tile (TMA box rows, MMA M)
 constexpr int kTileBytes = kTile * kHeadDim * 2;
 constexpr int kMaxTokensPerUnit = 49152;  // select keeps a unit's keys in shared memory
 constexpr int kMaxRows = 32;         // G * w limit (MMA N of the logits tile)
-constexpr int kScoreThreads = 384;   // 12 warps
+constexpr int kScoreThreads = 512;   // 16 warps
 constexpr int kGemmThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -33,8 +33,8 @@ struct ScoreParams {
 };
 
 struct ScoreLayout {
-  uint32_t stages, q, abar, marr, rhoc, rhot, ufin, gath, mrow, invl, red1, red2, rsum, rowt,
-      xbuf, bars, slot, flags, total;
+  uint32_t stages, q, abar, marr, rhoc, rhot, ufin, gath, gath2, mrow, invl, red1, red2, rsum,
+      rowt, xbuf, bars, slot, flags, total;
 };
 
 constexpr int kMaxClusterSize = 16;
@@ -59,14 +59,15 @@ __host__ __device__ inline ScoreLayout score_layout(int rp, bool closed, int ns)
   L.rhoc = o; if (closed) o += lmax * 4;
   L.rhot = o; if (closed) o += 2 * 128 * 4;
   L.ufin = o; if (closed) o += 128 * 4;
-  L.gath = o; o += kMaxClusterSize * score_xb(rp, closed) * 4;
+  L.gath = o; o += kMaxClusterSize * score_xb(rp, closed) * 4;   // round-1 inbox
+  L.gath2 = o; o += kMaxClusterSize * 4 * 4;                       // round-2 inbox
   L.mrow = o; o += rp * 4;
   L.invl = o; o += rp * 4;
   L.red1 = o; o += 4 * rp * 2 * 4;
   L.red2 = o; if (closed) o += 4 * 128 * 4;
-  L.rsum = o; o += 16 * 4;
+  L.rsum = o; o += 32 * 4;
   L.rowt = o; o += 32 * 4;
-  L.xbuf = o; o += (score_xb(rp, closed) + 2 * kMaxClusterSize + 4) * 4;
+  L.xbuf = o; o += (score_xb(rp, closed) + 4) * 4;
   o = (o + 15u) & ~15u;
   L.bars = o; o += (2 * ns + kScoreBarsFixed) * 8;
   L.slot = o; o += 16;

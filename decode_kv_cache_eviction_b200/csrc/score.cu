@@ -12,9 +12,10 @@
 //     - per-thread online softmax statistics (running max, sum of
 //       2^(y - max), y = z * log2(e) / sqrt(d)) with a lazy max;
 //     - key norms on CUDA cores -> rho = 1/||k||; (closed form) U = sum rho_j k_j.
-//   cluster exchange #1: every CTA gathers all CTAs' (max, sum) per query row
-//     [and partial U] through distributed shared memory and merges them in
-//     rank order, so every CTA holds identical values.
+//   cluster exchange #1: every CTA pushes its (max, sum) per query row [and
+//     partial U] into every CTA's inbox with st.async (completing bytes on the
+//     receiver's mbarrier); each CTA merges the inbox in rank order, so every
+//     CTA holds identical values.
 //   pass 2:
 //     - abar_j = (1/(G w)) sum_rows 2^(y - M_row) / L_row from the TMEM logits;
 //     - (closed form) K tiles again, most recent first (likely still in L2):
@@ -22,9 +23,10 @@
 //   cluster exchange #2: sums of abar and of exp(m) over the candidates.
 //   write a = abar / sum, r = exp(m) / sum (window rows get 0).
 //
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM
-// owner, warps 4-7 softmax (thread = token row of a tile; TMEM lane quarter =
-// warp % 4), warps 8-11 norms and U (thread = token row).
+// Warp roles (512 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM
+// owner, warps 4-11 softmax (thread = token row of a tile; TMEM lane quarter =
+// warp % 4; warps 4-7 take the first half of the query rows, 8-11 the second),
+// warps 12-15 norms and U (thread = token row).
 #include "ptx.cuh"
 #include "rkv_internal.cuh"
 
@@ -71,10 +73,12 @@ __device__ __forceinline__ UnitSched unit_sched(const ScoreParams& p, int u, int
   return s;
 }
 
-template <int RP>
-__device__ __forceinline__ void tmem_ld_rows(uint32_t taddr, uint32_t (&v)[RP]) {
-  if constexpr (RP == 16) tmem_ld16(taddr, v);
-  else tmem_ld32(taddr, v);
+constexpr int kConsumers = 384;   // softmax + norm threads
+
+template <int RH>
+__device__ __forceinline__ void tmem_ld_rows(uint32_t taddr, uint32_t (&v)[RH]) {
+  if constexpr (RH == 8) tmem_ld8(taddr, v);
+  else tmem_ld16(taddr, v);
 }
 
 // Merge two (max, sum) softmax statistics in the log2 domain.
@@ -84,40 +88,19 @@ __device__ __forceinline__ void merge_stat(float& m, float& s, float om, float o
   m = M;
 }
 
-// Thread rr (< cs) releases to CTA rr: a cluster-scope fence (cumulative over
-// the CTA barrier before it) followed by a relaxed arrive.  Then every
-// consumer thread waits until all CTAs of the cluster have released.
-__device__ __forceinline__ void cluster_exchange(uint64_t* bar, uint32_t parity, int cs,
-                                                 int ctid, volatile int* abort, int* status) {
-  named_bar_sync(1, 256);
-  if (ctid < cs) {
-    fence_acq_rel_cluster();
-    mbar_arrive_cluster_relaxed(mapa(smem_u32(bar), ctid));
-  }
-  mbar_wait<true>(bar, parity, abort, status);
-  __syncwarp();
-}
-
-// Copy `n` floats at `src` (same offset in every CTA) from all `cs` CTAs into
-// the local array dst[rank * n + k]; all loads are issued before any store.
-__device__ __forceinline__ void cluster_gather(float* dst, const float* src, int n, int cs,
-                                               int ctid) {
-  constexpr int kMaxPer = (kMaxClusterSize * (2 * 32 + 128) + 255) / 256;
-  const uint32_t local = smem_u32(src);
-  const int total = n * cs;
-  float v[kMaxPer];
-#pragma unroll
-  for (int k = 0; k < kMaxPer; ++k) {
-    const int e = ctid + k * 256;
-    if (e < total) {
-      const int rr = e / n;
-      v[k] = ld_cluster_f32(mapa(local + 4u * static_cast<uint32_t>(e - rr * n), rr));
-    }
-  }
-#pragma unroll
-  for (int k = 0; k < kMaxPer; ++k) {
-    const int e = ctid + k * 256;
-    if (e < total) dst[e] = v[k];
+// Push this CTA's n4 16-byte chunks at `src` into slot `rank` of the inbox
+// (same offset) of every CTA of the cluster with st.async; each store
+// completes its bytes on the receiving CTA's barrier `bar`, which expects
+// cs * n4 * 16 bytes per round.  No fence is needed: the receiver sees the
+// data once its barrier phase completes.
+__device__ __forceinline__ void cluster_push(const float* src, float* inbox, int n4, int cs,
+                                             int rank, uint64_t* bar, int ctid) {
+  const uint32_t inbox_base = smem_u32(inbox) + static_cast<uint32_t>(rank * n4 * 16);
+  const uint32_t bar_local = smem_u32(bar);
+  for (int e = ctid; e < n4 * cs; e += kConsumers) {
+    const int dst = e / n4, ch = e - dst * n4;
+    const float4 v = reinterpret_cast<const float4*>(src)[ch];
+    st_async_v4(mapa(inbox_base + ch * 16, dst), mapa(bar_local, dst), v);
   }
 }
 
@@ -141,6 +124,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                  const ScoreParams p) {
   constexpr int XB = 2 * RP + (CLOSED ? 128 : 0);   // round-1 partial floats per CTA
+  constexpr int RH = RP / 2;                         // query rows per softmax warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -171,11 +155,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       mbar_init(&empty[s], 1 + 4);  // MMA thread + 4 norm warps
     }
     for (int k = 0; k < 32; ++k) mbar_init(&tready[k], 1);
-    mbar_init(tfree, 4);
+    mbar_init(tfree, 8);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&qfull[b], 1);
       mbar_init(&qempty[b], 1);
-      mbar_init(&redbar[b], cs);
+      mbar_init(&redbar[b], 1);   // local arrive.expect_tx; bytes from every CTA
     }
     *abort = 0;
     fence_mbar_init();
@@ -275,10 +259,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ consumers
-    const int ctid = threadIdx.x - 128;      // 0..255
-    const bool is_soft = warp < 8;           // warps 4-7: softmax
+    const int ctid = threadIdx.x - 128;      // 0..383
+    const bool is_soft = warp < 12;          // warps 4-11: softmax
     const int q4 = warp & 3;                 // TMEM lane quarter
     const int row = q4 * 32 + lane;          // token row of the tile
+    const int r0 = ((warp - 4) >> 2) * RH;   // first query row of a softmax warp
     float* abar_s = reinterpret_cast<float*>(sm + L.abar);
     float* marr = reinterpret_cast<float*>(sm + L.marr);
     float* rhoc = reinterpret_cast<float*>(sm + L.rhoc);
@@ -294,7 +279,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const uint32_t rmask = p.R >= 32 ? 0xffffffffu : ((1u << p.R) - 1u);
     const int* row_t = reinterpret_cast<const int*>(sm + L.rowt);
     if (ctid < 32) reinterpret_cast<int*>(sm + L.rowt)[ctid] = ctid % p.w;
-    named_bar_sync(1, 256);
+    named_bar_sync(1, kConsumers);
 
     int stage = 0, ntile1 = 0;
     uint32_t ph = 0;
@@ -303,9 +288,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     for (int u = cid; u < p.num_units; u += ncl, ++it) {
       const UnitSched s = unit_sched(p, u, rank);
       const int N = s.n, c = s.c;
-      float st_m[RP], st_s[RP];  // pass 1: running stats; pass 2: row max and 1/sum
+      float st_m[RH], st_s[RH];  // pass 1: running stats; pass 2: row max and 1/sum
 #pragma unroll
-      for (int r = 0; r < RP; ++r) { st_m[r] = kNegBig; st_s[r] = 0.f; }
+      for (int r = 0; r < RH; ++r) { st_m[r] = kNegBig; st_s[r] = 0.f; }
+      for (int i = ctid; i < s.len; i += kConsumers) abar_s[i] = 0.f;
       float U4[4] = {0.f, 0.f, 0.f, 0.f};
       float part = 0.f;  // pass 2: sum of abar (softmax) or of exp(m) (norm warps)
       if (ctid == 0) RKV_STAMP(it, 0);
@@ -319,20 +305,20 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           tph ^= 1u << k;
           __syncwarp();
           tc_fence_after();
-          uint32_t v[RP];
-          tmem_ld_rows<RP>(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + k * RP, v);
+          uint32_t v[RH];
+          tmem_ld_rows<RH>(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + k * RP + r0, v);
           tmem_wait_ld();
           // y = log2-scaled logit, -inf where masked (padding row, beyond N,
           // causal); only a tile that reaches the window needs the causal limit
-          float y[RP];
+          float y[RH];
           if (t0 + kTile <= c) {
 #pragma unroll
-            for (int r = 0; r < RP; ++r)
-              y[r] = ((rmask >> r) & 1u) ? __uint_as_float(v[r]) * p.scale_log2 : -INFINITY;
+            for (int r = 0; r < RH; ++r)
+              y[r] = ((rmask >> (r0 + r)) & 1u) ? __uint_as_float(v[r]) * p.scale_log2 : -INFINITY;
           } else {
 #pragma unroll
-            for (int r = 0; r < RP; ++r) {
-              const bool vis = ((rmask >> r) & 1u) && j < N && j <= c + row_t[r];
+            for (int r = 0; r < RH; ++r) {
+              const bool vis = ((rmask >> (r0 + r)) & 1u) && j < N && j <= c + row_t[r0 + r];
               y[r] = vis ? __uint_as_float(v[r]) * p.scale_log2 : -INFINITY;
             }
           }
@@ -341,10 +327,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           // common case is branch-free.
           bool need = false;
 #pragma unroll
-          for (int r = 0; r < RP; ++r) need |= y[r] > st_m[r] + kLazy;
+          for (int r = 0; r < RH; ++r) need |= y[r] > st_m[r] + kLazy;
           if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-            for (int r = 0; r < RP; ++r) {
+            for (int r = 0; r < RH; ++r) {
               if (y[r] > st_m[r]) {
                 st_s[r] = st_s[r] * ex2(st_m[r] - y[r]) + 1.f;
                 st_m[r] = y[r];
@@ -354,7 +340,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             }
           } else {
 #pragma unroll
-            for (int r = 0; r < RP; ++r) st_s[r] += ex2(y[r] - st_m[r]);
+            for (int r = 0; r < RH; ++r) st_s[r] += ex2(y[r] - st_m[r]);
           }
         } else {
           // norm warps: ||k|| of row `row`, rho, (closed form) U accumulation
@@ -417,10 +403,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
       // ================================================= exchange 1
       if (ctid == 0) RKV_STAMP(it, 1);
-      if (ctid == 128) RKV_STAMP(it, 2);
+      if (ctid == 256) RKV_STAMP(it, 2);
       if (is_soft) {
 #pragma unroll
-        for (int r = 0; r < RP; ++r) {
+        for (int r = 0; r < RH; ++r) {
 #pragma unroll
           for (int o = 16; o; o >>= 1) {
             const float om = __shfl_xor_sync(0xffffffffu, st_m[r], o);
@@ -430,16 +416,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
         if (lane == 0) {
 #pragma unroll
-          for (int r = 0; r < RP; ++r) {
-            red1[(q4 * RP + r) * 2 + 0] = st_m[r];
-            red1[(q4 * RP + r) * 2 + 1] = st_s[r];
+          for (int r = 0; r < RH; ++r) {
+            red1[(q4 * RP + r0 + r) * 2 + 0] = st_m[r];
+            red1[(q4 * RP + r0 + r) * 2 + 1] = st_s[r];
           }
         }
       } else if (CLOSED) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) red2[q4 * 128 + lane * 4 + i] = U4[i];
       }
-      named_bar_sync(1, 256);
+      named_bar_sync(1, kConsumers);
       float* xa = xbuf;  // this CTA's round-1 partials
       if (ctid < RP) {
         float m = kNegBig, sacc = 0.f;
@@ -448,33 +434,37 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         xa[2 * ctid] = m;
         xa[2 * ctid + 1] = sacc;
       }
-      if (CLOSED && ctid >= 128) {
-        const int e = ctid - 128;
+      if (CLOSED && ctid >= 256) {
+        const int e = ctid - 256;
         xa[2 * RP + e] = red2[e] + red2[128 + e] + red2[256 + e] + red2[384 + e];
       }
-      cluster_exchange(&redbar[0], it & 1, cs, ctid, abort, p.status);
-      cluster_gather(gath, xa, XB, cs, ctid);
-      named_bar_sync(1, 256);
+      if (ctid == 0) mbar_arrive_expect_tx(&redbar[0], cs * XB * 4);
+      named_bar_sync(1, kConsumers);
+      cluster_push(xa, gath, XB / 4, cs, rank, &redbar[0], ctid);
+      mbar_wait<true>(&redbar[0], it & 1, abort, p.status);
+      __syncwarp();
       if (ctid < RP) {
-        float m = kNegBig, sacc = 0.f;
+        float m = kNegBig;
+        for (int rr = 0; rr < cs; ++rr) m = fmaxf(m, gath[rr * XB + 2 * ctid]);
+        float sacc = 0.f;
         for (int rr = 0; rr < cs; ++rr)
-          merge_stat(m, sacc, gath[rr * XB + 2 * ctid], gath[rr * XB + 2 * ctid + 1]);
+          sacc = fmaf(gath[rr * XB + 2 * ctid + 1], ex2(gath[rr * XB + 2 * ctid] - m), sacc);
         mrow[ctid] = m;
         invl[ctid] = sacc > 0.f ? 1.f / sacc : 0.f;
       }
-      if (CLOSED && ctid >= 128) {
-        const int e = ctid - 128;
+      if (CLOSED && ctid >= 256) {
+        const int e = ctid - 256;
         float acc = 0.f;
         for (int rr = 0; rr < cs; ++rr) acc += gath[rr * XB + 2 * RP + e];
         ufin[e] = acc;
       }
-      named_bar_sync(1, 256);
+      named_bar_sync(1, kConsumers);
       if (is_soft) {
 #pragma unroll
-        for (int r = 0; r < RP; ++r) {
+        for (int r = 0; r < RH; ++r) {
           // padding rows: a huge max and zero weight, so they add exactly 0
-          st_m[r] = ((rmask >> r) & 1u) ? mrow[r] : 1e30f;
-          st_s[r] = ((rmask >> r) & 1u) ? invl[r] : 0.f;
+          st_m[r] = ((rmask >> (r0 + r)) & 1u) ? mrow[r0 + r] : 1e30f;
+          st_s[r] = ((rmask >> (r0 + r)) & 1u) ? invl[r0 + r] : 0.f;
         }
       }
       if (ctid == 0) RKV_STAMP(it, 3);
@@ -485,25 +475,26 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         for (int k = 0; k < s.nt; ++k) {
           const int t0 = s.start + kTile * k;
           const int j = t0 + row;
-          uint32_t v[RP];
-          tmem_ld_rows<RP>(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + k * RP, v);
+          uint32_t v[RH];
+          tmem_ld_rows<RH>(tmem + (static_cast<uint32_t>(q4 * 32) << 16) + k * RP + r0, v);
           tmem_wait_ld();
           float pq[4] = {0.f, 0.f, 0.f, 0.f};
           if (t0 + kTile <= c) {
 #pragma unroll
-            for (int r = 0; r < RP; ++r)
+            for (int r = 0; r < RH; ++r)
               pq[r & 3] = fmaf(ex2(fmaf(__uint_as_float(v[r]), p.scale_log2, -st_m[r])),
                                st_s[r], pq[r & 3]);
           } else {
 #pragma unroll
-            for (int r = 0; r < RP; ++r)
-              if (((rmask >> r) & 1u) && j < N && j <= c + row_t[r])
+            for (int r = 0; r < RH; ++r)
+              if (((rmask >> (r0 + r)) & 1u) && j < N && j <= c + row_t[r0 + r])
                 pq[r & 3] = fmaf(ex2(fmaf(__uint_as_float(v[r]), p.scale_log2, -st_m[r])),
                                  st_s[r], pq[r & 3]);
           }
           if (j < c) {
+            // two warps (row halves) add into the zeroed slot: a + b either way
             const float ab_ = ((pq[0] + pq[1]) + (pq[2] + pq[3])) * invR;
-            abar_s[j - s.start] = ab_;
+            atomicAdd(&abar_s[j - s.start], ab_);
             part += ab_;
           }
         }
@@ -551,29 +542,34 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       // ================================================= exchange 2 and output
       part = warp_reduce_sum(part);
       if (lane == 0) rsum[warp - 4] = part;
-      named_bar_sync(1, 256);
+      named_bar_sync(1, kConsumers);
       float* xb2 = xbuf + XB;
+      float* g2 = reinterpret_cast<float*>(sm + L.gath2);   // [cs][4] received sums
       if (ctid == 0) {
-        xb2[0] = rsum[0] + rsum[1] + rsum[2] + rsum[3];
-        xb2[1] = rsum[4] + rsum[5] + rsum[6] + rsum[7];
+        xb2[0] = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) +
+                 ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
+        xb2[1] = (rsum[8] + rsum[9]) + (rsum[10] + rsum[11]);
+        xb2[2] = 0.f;
+        xb2[3] = 0.f;
+        mbar_arrive_expect_tx(&redbar[1], cs * 16);
       }
-      cluster_exchange(&redbar[1], it & 1, cs, ctid, abort, p.status);
-      float* g2 = xbuf + XB + 4;   // [cs][2] gathered sums
-      if (ctid < 2 * cs) g2[ctid] = ld_cluster_f32(mapa(smem_u32(&xb2[ctid & 1]), ctid >> 1));
-      named_bar_sync(1, 256);
+      named_bar_sync(1, kConsumers);
+      cluster_push(xb2, g2, 1, cs, rank, &redbar[1], ctid);
+      mbar_wait<true>(&redbar[1], it & 1, abort, p.status);
+      __syncwarp();
       if (ctid == 0) {
         float sa = 0.f, se = 0.f;
         for (int rr = 0; rr < cs; ++rr) {
-          sa += g2[2 * rr];
-          se += g2[2 * rr + 1];
+          sa += g2[4 * rr];
+          se += g2[4 * rr + 1];
         }
-        rsum[8] = sa > 0.f ? 1.f / sa : 0.f;
-        rsum[9] = se > 0.f ? 1.f / se : 0.f;
+        rsum[16] = sa > 0.f ? 1.f / sa : 0.f;
+        rsum[17] = se > 0.f ? 1.f / se : 0.f;
       }
-      named_bar_sync(1, 256);
-      const float inv_sa = rsum[8], inv_se = rsum[9];
+      named_bar_sync(1, kConsumers);
+      const float inv_sa = rsum[16], inv_se = rsum[17];
       if (ctid == 0) RKV_STAMP(it, 5);
-      for (int i = ctid; i < s.len; i += 256) {
+      for (int i = ctid; i < s.len; i += kConsumers) {
         const int j = s.start + i;
         const int64_t g = s.base + j;
         if (j < c) {
