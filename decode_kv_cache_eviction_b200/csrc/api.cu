@@ -23,7 +23,8 @@ struct rkv_engine {
   int max_n = 0;               // largest supported N_u
   bool pair = true;
   int gemm_ctas = 0;
-  float* rho = nullptr;        // [max_tokens]
+  float* rho = nullptr;        // [max_tokens + kRhoAlign * max_units] padded 1/||k||
+  int64_t* rho_off = nullptr;  // [max_units + 1]
   int* item_off = nullptr;     // [max_units + 1]
   int* unit_cnt = nullptr;     // [max_units]
   int* status = nullptr;       // [1]
@@ -207,7 +208,11 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   bool ok = cudaMalloc(&e->status, 16) == cudaSuccess;
   ok = ok && cudaMalloc(&e->item_off, sizeof(int) * (cfg->max_units + 1)) == cudaSuccess;
   ok = ok && cudaMalloc(&e->unit_cnt, sizeof(int) * cfg->max_units) == cudaSuccess;
-  if (!closed) ok = ok && cudaMalloc(&e->rho, sizeof(float) * cfg->max_tokens) == cudaSuccess;
+  if (!closed) {
+    const int64_t nrho = cfg->max_tokens + static_cast<int64_t>(kRhoAlign) * cfg->max_units;
+    ok = ok && cudaMalloc(&e->rho, sizeof(float) * nrho) == cudaSuccess;
+    ok = ok && cudaMalloc(&e->rho_off, sizeof(int64_t) * (cfg->max_units + 1)) == cudaSuccess;
+  }
   ok = ok && cudaMemset(e->status, 0, 16) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
@@ -215,6 +220,7 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
     cudaFree(e->item_off);
     cudaFree(e->unit_cnt);
     cudaFree(e->rho);
+    cudaFree(e->rho_off);
     delete e;
     return RKV_ERR_OOM;
   }
@@ -264,6 +270,7 @@ int rkv_destroy(rkv_engine* e) {
   cudaFree(e->item_off);
   cudaFree(e->unit_cnt);
   cudaFree(e->rho);
+  cudaFree(e->rho_off);
   delete e;
   return RKV_OK;
 }
@@ -309,21 +316,26 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   p.r_out = r;
   p.m_out = m;
   p.rho_out = closed ? nullptr : e->rho;
+  p.rho_off = closed ? nullptr : e->rho_off;
   p.status = e->status;
+  const int rows_per_item = e->pair ? 256 : 128;
+  cudaError_t err;
+  if (!closed) {   // row blocks for the GEMM and the padded rho layout the score kernel writes
+    t_begin(e, RKV_KERNEL_PLAN, st);
+    err = launch_plan(b->tok_off, U, e->cfg.window, rows_per_item, e->item_off, e->unit_cnt,
+                      e->rho_off, st);
+    t_end(e, st);
+    if (err != cudaSuccess) return cuda_fail(err);
+    ++e->launches;
+  }
   t_begin(e, RKV_KERNEL_SCORE, st);
-  cudaError_t err = launch_score(kmap, qmap, p, e->rp, closed, ncl, st);
+  err = launch_score(kmap, qmap, p, e->rp, closed, ncl, st);
   t_end(e, st);
   if (err != cudaSuccess) return cuda_fail(err);
   ++e->launches;
   if (closed) return RKV_OK;
 
   // redundancy GEMM
-  const int rows_per_item = e->pair ? 256 : 128;
-  t_begin(e, RKV_KERNEL_PLAN, st);
-  err = launch_plan(b->tok_off, U, e->cfg.window, rows_per_item, e->item_off, e->unit_cnt, st);
-  t_end(e, st);
-  if (err != cudaSuccess) return cuda_fail(err);
-  ++e->launches;
   CUtensorMap amap, bmap;
   if (make_map(e, &amap, b->K, static_cast<uint64_t>(T), 128) != RKV_OK) return RKV_ERR_CUDA;
   if (make_map(e, &bmap, b->K, static_cast<uint64_t>(T), e->pair ? 128 : 256) != RKV_OK)
@@ -334,6 +346,7 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   g.num_units = U;
   g.w = e->cfg.window;
   g.rho = e->rho;
+  g.rho_off = e->rho_off;
   g.m_dst = m ? m : r;
   g.r_dst = r;
   g.unit_cnt = e->unit_cnt;

@@ -30,7 +30,8 @@ constexpr int kMaxDevices = 64;
 constexpr int kSmemCap = 227 * 1024;
 
 struct Scratch {
-  float rho[kMaxTokens];
+  float rho[kMaxTokens + static_cast<int64_t>(kRhoAlign) * kMaxUnits];
+  int64_t rho_off[kMaxUnits + 1];
   int item_off[kMaxUnits + 1];
   int unit_cnt[kMaxUnits];
   int status[4];
@@ -191,12 +192,14 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   p.r_out = r;
   p.m_out = m;
   p.rho_out = s->rho;
+  p.rho_off = s->rho_off;
   p.status = s->status;
-  if (launch_score(kmap, qmap, p, rp, false, ncl, st) != cudaSuccess) {
+  if (launch_plan(b->tok_off, U, window, 256, s->item_off, s->unit_cnt, s->rho_off, st) !=
+      cudaSuccess) {
     cudaGetLastError();
     return RKV_ERR_CUDA;
   }
-  if (launch_plan(b->tok_off, U, window, 256, s->item_off, s->unit_cnt, st) != cudaSuccess) {
+  if (launch_score(kmap, qmap, p, rp, false, ncl, st) != cudaSuccess) {
     cudaGetLastError();
     return RKV_ERR_CUDA;
   }
@@ -212,6 +215,7 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   g.num_units = U;
   g.w = window;
   g.rho = s->rho;
+  g.rho_off = s->rho_off;
   g.m_dst = m ? m : r;
   g.r_dst = r;
   g.unit_cnt = s->unit_cnt;

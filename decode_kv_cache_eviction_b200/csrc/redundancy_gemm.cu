@@ -57,6 +57,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* b_empty = b_full + NSB;
   uint64_t* acc_full = b_empty + NSB;
   uint64_t* acc_empty = acc_full + 2;
+  uint64_t* rho_full = acc_empty + 2;      // [kRhoSlots] rho tile landed
+  uint64_t* rho_empty = rho_full + kRhoSlots;  // [kRhoSlots] epilogue done with it
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.slot);
   volatile int* abort = reinterpret_cast<volatile int*>(sm + L.flags);
   volatile int* last_flag = reinterpret_cast<volatile int*>(sm + L.flags + 4);
@@ -71,6 +73,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kPair ? 16 : 8);
+    }
+    for (int b = 0; b < kRhoSlots; ++b) {
+      mbar_init(&rho_full[b], 1);
+      mbar_init(&rho_empty[b], 8);   // this CTA's 8 epilogue warps
     }
     *abort = 0;
     fence_mbar_init();
@@ -96,9 +102,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t ph = 0;
       int ai = 0;
+      uint32_t rt = 0;   // rho tiles loaded so far
+      float* rho_ring = reinterpret_cast<float*>(sm + L.rho);
       for (int item = group_id; item < n_items; item += ngroups, ++ai) {
         const int u = find_unit(p.item_off, p.num_units, item);
         const int blk = item - __ldg(&p.item_off[u]);
+        const float* rho_u = p.rho + __ldg(&p.rho_off[u]);
         const int64_t base = __ldg(&p.tok_off[u]);
         const int N = static_cast<int>(__ldg(&p.tok_off[u + 1]) - base);
         const int ya = static_cast<int>(base + blk * C::kRowsPerItem + rank * 128);
@@ -131,6 +140,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
           if (++stage == NSB) { stage = 0; ph ^= 1; }
+          // the 256 column weights of this tile (every CTA of a pair loads its own)
+          const uint32_t rs = rt % kRhoSlots;
+          if (mbar_wait(&rho_empty[rs], ((rt / kRhoSlots) & 1) ^ 1, abort, p.status)) {
+            mbar_arrive_expect_tx(&rho_full[rs], 256 * 4);
+            bulk_load(rho_ring + rs * 256, rho_u + t * C::kN, 256 * 4, &rho_full[rs]);
+          }
+          ++rt;
         }
       }
     }
@@ -188,13 +204,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int half = ew >> 2;             // column half of the tile
     const int q = warp & 3;               // TMEM lane quarter
     const int rloc = q * 32 + lane;       // row of this CTA's A block
-    // private rho slices of this warp: [2][128] floats (the 128 columns of its half)
-    float* rho_w = reinterpret_cast<float*>(sm + L.rho) + ew * 256;
+    const float* rho_ring = reinterpret_cast<const float*>(sm + L.rho);
     float* rowx = reinterpret_cast<float*>(sm + L.rowx);
     float* fin = reinterpret_cast<float*>(sm + L.fin);
     const uint32_t acc_empty_lead = kPair ? mapa(smem_u32(acc_empty), 0) : smem_u32(acc_empty);
     int ab = 0;
     uint32_t aph = 0;
+    uint32_t rt = 0;   // rho tiles consumed so far
     for (int item = group_id; item < n_items; item += ngroups) {
       const int u = find_unit(p.item_off, p.num_units, item);
       const int blk = item - __ldg(&p.item_off[u]);
@@ -205,23 +221,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int i = rbase + rloc;
       float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
       const int ntiles = (N + C::kN - 1) / C::kN;
-      // rho of the 4 columns this lane stages, one tile ahead
-      auto load_rho = [&](int j0, float (&dst)[4]) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int col = j0 + half * 128 + lane * 4 + e;
-          dst[e] = col < N ? __ldg(&p.rho[base + col]) : 0.f;
-        }
-      };
-      float rpre[4];
-      load_rho(0, rpre);
-      for (int t = 0; t < ntiles; ++t) {
+      for (int t = 0; t < ntiles; ++t, ++rt) {
         const int j0 = t * C::kN;
-        float* rs = rho_w + (t & 1) * 128;
-        *reinterpret_cast<float4*>(rs + lane * 4) = make_float4(rpre[0], rpre[1], rpre[2], rpre[3]);
-        __syncwarp();
-        if (t + 1 < ntiles) load_rho(j0 + C::kN, rpre);
+        const uint32_t rs_slot = rt % kRhoSlots;
+        const float* rs = rho_ring + rs_slot * 256 + half * 128;
         mbar_wait(&acc_full[ab], aph, abort, p.status);
+        mbar_wait(&rho_full[rs_slot], (rt / kRhoSlots) & 1, abort, p.status);
         __syncwarp();
         tc_fence_after();
         const uint32_t tbase =
@@ -267,6 +272,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           };
           fold(va, 0); fold(vb, 32); fold(vc, 64); fold(vd, 96);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rho_empty[rs_slot]);
       }
       // ---- item end: combine halves, write m, count the unit's finished blocks
       float tot = (s0 + s1) + (s2 + s3);
@@ -274,7 +281,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       named_bar_sync(3, 256);
       if (half == 0 && i < c) {
         tot += rowx[rloc];
-        const float rho_i = __ldg(&p.rho[base + i]);
+        const float rho_i = __ldg(&p.rho[__ldg(&p.rho_off[u]) + i]);
         p.m_dst[base + i] = rho_i * tot / static_cast<float>(N - 1);
       }
       __threadfence();
@@ -314,47 +321,64 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// One block: items per unit and their prefix, and zeroed unit counters.
+// One block: items per unit and their prefix, 256-aligned rho segment
+// offsets, and zeroed unit counters.
 __global__ void plan_kernel(const int64_t* tok_off, int U, int w, int rows_per_item,
-                            int* item_off, int* unit_cnt) {
-  __shared__ int wsum[32];
+                            int* item_off, int* unit_cnt, int64_t* rho_off) {
+  __shared__ long long wsum[2][32];
   const int tid = threadIdx.x, nt = blockDim.x;
   const int per = (U + nt - 1) / nt;
   const int u0 = min(U, tid * per), u1 = min(U, u0 + per);
-  int local = 0;
+  long long li = 0, lr = 0;   // this thread's items and padded rho length
   for (int u = u0; u < u1; ++u) {
-    const int c = static_cast<int>(tok_off[u + 1] - tok_off[u]) - w;
-    local += c > 0 ? (c + rows_per_item - 1) / rows_per_item : 0;
+    const int64_t n = tok_off[u + 1] - tok_off[u];
+    const int64_t c = n - w;
+    li += c > 0 ? (c + rows_per_item - 1) / rows_per_item : 0;
+    lr += (n + kRhoAlign - 1) / kRhoAlign * kRhoAlign;
     unit_cnt[u] = 0;
   }
-  // block exclusive scan of `local`
-  int incl = local;
+  // block exclusive scans of li and lr
+  long long ii = li, ir = lr;
   const int lane = tid & 31, wp = tid >> 5;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+    const long long yi = __shfl_up_sync(0xffffffffu, ii, o);
+    const long long yr = __shfl_up_sync(0xffffffffu, ir, o);
+    if (lane >= o) { ii += yi; ir += yr; }
   }
-  if (lane == 31) wsum[wp] = incl;
+  if (lane == 31) { wsum[0][wp] = ii; wsum[1][wp] = ir; }
   __syncthreads();
   if (wp == 0) {
-    int x = lane < (nt >> 5) ? wsum[lane] : 0;
+    long long xi = lane < (nt >> 5) ? wsum[0][lane] : 0;
+    long long xr = lane < (nt >> 5) ? wsum[1][lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
+      const long long yi = __shfl_up_sync(0xffffffffu, xi, o);
+      const long long yr = __shfl_up_sync(0xffffffffu, xr, o);
+      if (lane >= o) { xi += yi; xr += yr; }
     }
-    wsum[lane] = x;
+    wsum[0][lane] = xi;
+    wsum[1][lane] = xr;
   }
   __syncthreads();
-  int run = incl - local + (wp > 0 ? wsum[wp - 1] : 0);
+  long long ri = ii - li + (wp > 0 ? wsum[0][wp - 1] : 0);
+  long long rr = ir - lr + (wp > 0 ? wsum[1][wp - 1] : 0);
   for (int u = u0; u < u1; ++u) {
-    item_off[u] = run;
-    const int c = static_cast<int>(tok_off[u + 1] - tok_off[u]) - w;
-    run += c > 0 ? (c + rows_per_item - 1) / rows_per_item : 0;
+    item_off[u] = static_cast<int>(ri);
+    rho_off[u] = rr;
+    const int64_t n = tok_off[u + 1] - tok_off[u];
+    const int64_t c = n - w;
+    ri += c > 0 ? (c + rows_per_item - 1) / rows_per_item : 0;
+    rr += (n + kRhoAlign - 1) / kRhoAlign * kRhoAlign;
   }
-  if (u1 == U && u0 < u1) item_off[U] = run;
-  if (U == 0 && tid == 0) item_off[0] = 0;
+  if (u1 == U && u0 < u1) {
+    item_off[U] = static_cast<int>(ri);
+    rho_off[U] = rr;
+  }
+  if (U == 0 && tid == 0) {
+    item_off[0] = 0;
+    rho_off[0] = 0;
+  }
 }
 
 }  // namespace
@@ -401,8 +425,8 @@ int gemm_max_ctas(bool pair) {
 }
 
 cudaError_t launch_plan(const int64_t* tok_off, int U, int w, int rows_per_item, int* item_off,
-                        int* unit_cnt, cudaStream_t st) {
-  plan_kernel<<<1, 1024, 0, st>>>(tok_off, U, w, rows_per_item, item_off, unit_cnt);
+                        int* unit_cnt, int64_t* rho_off, cudaStream_t st) {
+  plan_kernel<<<1, 1024, 0, st>>>(tok_off, U, w, rows_per_item, item_off, unit_cnt, rho_off);
   return cudaGetLastError();
 }
 

@@ -28,7 +28,8 @@ struct ScoreParams {
   float* a_out;            // [T]
   float* r_out;            // [T]
   float* m_out;            // [T] or null
-  float* rho_out;          // [T] (1/||k||) or null
+  float* rho_out;          // 1/||k|| at rho_off[u] + j (pads zeroed), or null
+  const int64_t* rho_off;  // [U+1] 256-aligned per-unit offsets into rho_out
   int* status;
 };
 
@@ -102,7 +103,8 @@ struct GemmParams {
   const int* item_off;     // [U+1] prefix of row blocks per unit
   int num_units;
   int w;
-  const float* rho;        // [T] 1/||k||
+  const float* rho;        // 1/||k|| at rho_off[u] + j, zero up to rho_off[u+1]
+  const int64_t* rho_off;  // [U+1] multiples of kRhoAlign
   float* m_dst;            // [T] receives m (may equal r_dst)
   float* r_dst;            // [T] receives r
   int* unit_cnt;           // [U] zeroed by the plan kernel
@@ -122,6 +124,9 @@ struct GemmCfg {
   static constexpr int kMmaM = kPair ? 256 : 128;
 };
 
+constexpr int kRhoAlign = 256;   // per-unit rho segments start at multiples of this
+constexpr int kRhoSlots = 8;     // ring of 256-column rho tiles in the GEMM kernel
+
 struct GemmLayout {
   uint32_t a, b, rho, rowx, fin, bars, slot, flags, total;
 };
@@ -132,10 +137,10 @@ __host__ __device__ inline GemmLayout gemm_layout() {
   uint32_t o = 0;
   L.a = o; o += C::kABytes;
   L.b = o; o += C::kStages * C::kBBytes;
-  L.rho = o; o += 8 * 2 * 128 * 4;   // per epilogue warp: two 128-column slices
+  L.rho = o; o += kRhoSlots * 256 * 4;
   L.rowx = o; o += 128 * 4;
   L.fin = o; o += 32 * 4;
-  L.bars = o; o += (2 + 2 * C::kStages + 4) * 8;
+  L.bars = o; o += (2 + 2 * C::kStages + 4 + 2 * kRhoSlots) * 8;
   L.slot = o; o += 16;
   L.flags = o; o += 16;
   L.total = o;
@@ -150,7 +155,7 @@ cudaError_t score_configure(int rp, bool closed, int smem_bytes, int cs);
 int score_max_clusters(int rp, bool closed, int smem_bytes, int cs);
 
 cudaError_t launch_plan(const int64_t* tok_off, int U, int w, int rows_per_item, int* item_off,
-                        int* unit_cnt, cudaStream_t st);
+                        int* unit_cnt, int64_t* rho_off, cudaStream_t st);
 cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const GemmParams& p,
                         bool pair, int nctas, cudaStream_t st);
 cudaError_t gemm_configure(bool pair);

@@ -5,7 +5,7 @@
 // owns the contiguous token chunk [rank*L, rank*L + L) (L a multiple of 128,
 // at most 512 / RP tiles).  Per unit:
 //
-//   pass 1 (K tiles streamed by TMA, kept in L2 with evict_last in closed form):
+//   pass 1 (K tiles streamed by TMA; in closed form left in L2 for pass 2):
 //     - logits z = K_tile . Q^T on tcgen05 (M = 128 tokens, N = RP padded
 //       query rows, fp32 accumulator).  Tile k's logits stay in TMEM columns
 //       [k*RP, (k+1)*RP) for the whole unit, so pass 2 needs no second MMA;
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&kmap);
       prefetch_tmap(&qmap);
-      const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
+      const uint64_t keep = policy_evict_normal(), drop = policy_evict_first();
       int stage = 0;
       uint32_t ph = 0;
       int it = 0;
@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) U4[i] += U8[i] + U8[4 + i];
           } else {
-            if (j < N && p.rho_out) p.rho_out[s.base + j] = rho;
+            if (j < N && p.rho_out) p.rho_out[p.rho_off[u] + j] = rho;
           }
           ++ntile1;
           __syncwarp();
@@ -584,6 +584,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           p.r_out[g] = 0.f;
           if (p.m_out) p.m_out[g] = 0.f;
         }
+      }
+      if (!CLOSED && p.rho_out && rank == 0) {
+        const int64_t pe = p.rho_off[u + 1];
+        for (int64_t g = p.rho_off[u] + N + ctid; g < pe; g += kConsumers) p.rho_out[g] = 0.f;
       }
       if (ctid == 0) RKV_STAMP(it, 6);
     }

@@ -174,9 +174,9 @@ int rkv_read_timing(rkv_engine* eng, int kernel, double* total_ms, int64_t* laun
  *
  * Computes exactly what rkv_score computes for an engine created with
  * RKV_REDUNDANCY_GEMM (CTA-pair GEMM), with head_dim = 128 and the given group and
- * window.  Its scratch (1/||k|| per row, per-unit row-block offsets and
+ * window.  Its scratch (1/||k|| per row, per-unit row-block and row offsets and
  * counters, a status word) lives in one file-scope __device__ array of about
- * 4.1 MB that every GPU which loads the library holds until the process exits;
+ * 8.5 MB that every GPU which loads the library holds until the process exits;
  * nothing is allocated or freed per call.  Limits: at most RKV_NOALLOC_MAX_UNITS
  * units and RKV_NOALLOC_MAX_TOKENS rows per call (larger batches return
  * RKV_ERR_CAPACITY before anything is enqueued), and the rkv_score limits
