@@ -37,6 +37,13 @@ METRIC = "KV tokens scored+evicted/sec on 1 B200; % of HBM / tensor-core rooflin
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (read + write) per launch of a kernel on long_trace_32k, from one
+# ncu capture of the 16-unit profiling case scaled by 1024/16 units (traffic
+# grows in proportion to the units processed).  Set to None whenever the
+# kernel changes after its capture; the figures are in profiles/.
+NCU_TRAFFIC_LONG_TRACE = {"gemm": (136.739072e6 + 4.948224e6) * 64,
+                          "score": (134.491648e6 + 3.696384e6) * 64}
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -321,9 +328,12 @@ def run_engine(args, dist: Dist):
     value = tokens * dist.world / (ms * 1e-3)
     dom = "gemm" if args.redundancy == "gemm" else "score"
     roof = dict(rep[dom])
+    traffic = None
+    if wl.name == "long_trace_32k" and args.redundancy == "gemm":
+        traffic = NCU_TRAFFIC_LONG_TRACE.get(dom)
     roofline = {"kernel": dom, "bound": roof["bound"], "achieved": roof["achieved"],
                 "peak": roof["peak"], "unit": roof["unit"], "frac": roof["frac"],
-                "traffic": None,
+                "traffic": traffic, "traffic_unit": "bytes per launch (ncu, scaled)",
                 "peak_source": ("%s (%s)" % (src, "bf16_tflops_sustained" if dom == "gemm"
                                               else "hbm_gbs"))}
 

@@ -1,0 +1,32 @@
+"""Small profiling case for ncu (python -m decode_kv_cache_eviction_b200.profile_case): a long_trace_32k-shaped batch (N = 32768,
+G = 4, w = 8, B = 4096, 30% span duplicates) with --units units, compressed
+--iters times.  Used only as the target of the ncu commands recorded in this
+directory; it is not part of the library."""
+import argparse
+import os
+import sys
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))  # repo root
+
+import torch  # noqa: E402
+
+from decode_kv_cache_eviction_b200 import Batch, Engine, workloads as W  # noqa: E402
+
+ap = argparse.ArgumentParser()
+ap.add_argument("--units", type=int, default=32)
+ap.add_argument("--n", type=int, default=32768)
+ap.add_argument("--mode", default="gemm", choices=["gemm", "closed"])
+ap.add_argument("--iters", type=int, default=3)
+a = ap.parse_args()
+wl = W.custom(name="long_trace_32k", n_kv_head=a.units, group=4, window=8, budget=4096,
+              n_min=a.n, dup_frac=0.3, dup_noise=0.05, span_len=(32, 256))
+gb = W.generate(wl, seed=0, device="cuda")
+b = Batch(gb.K, gb.V, gb.Q, gb.tok_off)
+eng = Engine(4, 8, b.num_units, b.num_tokens, redundancy=a.mode)
+ra, rr = eng.alloc_scores(b)
+idx, nk, Ko, Vo = eng.alloc_outputs(b, 4096)
+for _ in range(a.iters):
+    eng.compress(b, 0.1, 4096, ra, rr, idx, nk, Ko, Vo)
+eng.check_status()
+torch.cuda.synchronize()
+print("ok", b.num_units, b.num_tokens)
