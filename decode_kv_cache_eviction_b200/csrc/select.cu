@@ -1,19 +1,33 @@
 // Joint eviction (R-KV 联合淘汰): s_i = lambda * a_i - (1 - lambda) * r_i and a
-// deterministic top-B of the candidates, one CTA per unit.
+// deterministic top-B of the candidates.
 //
-// The fp32 scores are mapped to order-preserving uint32 keys and kept in shared
-// memory (one HBM read of a and r).  A 4-pass radix select (8-bit digits, most
-// significant first) finds the exact key T of the B-th largest score and how
-// many keys equal to T must be taken; equal keys are taken lowest index first.
-// The kept set is then written in ascending index order: each warp owns a
-// contiguous segment of the candidates, counts its "greater" and "equal" keys,
-// and after one block-level prefix over the warps it writes its positions with
-// ballots, with no further block synchronisation.
+// Persistent CTAs (1024 threads) walk the units; while one unit is selected,
+// the next unit's a and r are prefetched into L2.  Per unit:
+//   1. s is computed in fp32 and mapped to order-preserving uint32 keys held
+//      in shared memory (one read of a and r); the block also finds the
+//      smallest and largest key.
+//   2. Radix select of the exact key T of the B-th largest score, most
+//      significant digit first.  Bits above the highest bit in which the min
+//      and max keys differ are common to all keys, so the first 8-bit digit is
+//      taken just below them: it spreads the keys over the bins even when all
+//      scores share sign and exponent.  Histograms are kept per group of four
+//      warps (plain shared-memory atomics).  After the first digit the
+//      surviving keys (usually ~1/256 of them) are compacted into a short list
+//      and the remaining digits only look at that list.
+//   3. Keys equal to T are taken lowest index first.  The kept set is written
+//      in ascending index order: each warp owns a contiguous segment of the
+//      candidates, counts its "greater" and "equal" keys, and after one
+//      block-level prefix over the warps writes its positions with ballots.
 #include "ptx.cuh"
 #include "rkv_internal.cuh"
 
 namespace rkv {
 namespace {
+
+constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kHistGroups = 8;    // histograms shared by four warps each
+constexpr int kListCap = 4096;    // keys kept for the digits after the first
 
 __device__ __forceinline__ uint32_t order_key(float s) {
   uint32_t b = __float_as_uint(s);
@@ -21,158 +35,249 @@ __device__ __forceinline__ uint32_t order_key(float s) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-template <int NT>
-__global__ void __launch_bounds__(NT) select_kernel(const int64_t* __restrict__ tok_off, int w,
-                                                    const float* __restrict__ a,
-                                                    const float* __restrict__ r, float lam,
-                                                    int budget, int32_t* __restrict__ idx,
-                                                    int32_t* __restrict__ n_kept) {
-  constexpr int NW = NT / 32;
+__device__ __forceinline__ void prefetch_l2(const void* p, size_t bytes) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(p) & ~static_cast<uintptr_t>(15);
+  const uintptr_t a1 = (reinterpret_cast<uintptr_t>(p) + bytes + 15) & ~static_cast<uintptr_t>(15);
+  for (uintptr_t q = a0; q < a1; q += 32768) {
+    const uintptr_t e = q + 32768 < a1 ? q + 32768 : a1;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(q),
+                 "r"(static_cast<uint32_t>(e - q))
+                 : "memory");
+  }
+}
+
+__global__ void __launch_bounds__(kSelThreads, 1)
+    select_kernel(const int64_t* __restrict__ tok_off, int U, int w, const float* __restrict__ a,
+                  const float* __restrict__ r, float lam, int budget, int32_t* __restrict__ idx,
+                  int32_t* __restrict__ n_kept) {
   extern __shared__ uint32_t keys[];
-  __shared__ int hist[257];
-  __shared__ int sh[2];
-  __shared__ int wgt[NW], weq[NW], eqb[NW], outb[NW];
-  const int u = blockIdx.x;
+  __shared__ uint32_t hist8[kHistGroups][256];
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t list[kListCap];
+  __shared__ int sh[8];
+  __shared__ uint32_t wmin[kSelWarps], wmax[kSelWarps];
+  __shared__ int wgt[kSelWarps], weq[kSelWarps], eqb[kSelWarps], outb[kSelWarps];
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
-  const int64_t base = tok_off[u];
-  const int N = static_cast<int>(tok_off[u + 1] - base);
-  const int c = N - w;
-  const int W = budget + w;
-  int32_t* out = idx + static_cast<int64_t>(u) * W;
-
-  if (c <= budget) {  // every token is kept
-    for (int i = tid; i < W; i += NT) out[i] = i < N ? i : -1;
-    if (tid == 0) n_kept[u] = N;
-    return;
-  }
   const float lw = lam, rw = 1.f - lam;
-  for (int i = tid; i < c; i += NT) {
-    const float s = __fsub_rn(__fmul_rn(lw, a[base + i]), __fmul_rn(rw, r[base + i]));
-    keys[i] = order_key(s);
-  }
-  __syncthreads();
+  const int W = budget + w;
 
-  // ---- radix select of the budget-th largest key
-  int want = budget;
-  uint32_t prefix = 0, pmask = 0;
-  const int cround = (c + 31) & ~31;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int b = tid; b < 257; b += NT) hist[b] = 0;
-    __syncthreads();
-    for (int i = tid; i < cround; i += NT) {
-      uint32_t bin = 256;
-      if (i < c) {
-        const uint32_t k = keys[i];
-        if ((k & pmask) == prefix) bin = (k >> shift) & 255u;
+  for (int u = blockIdx.x; u < U; u += gridDim.x) {
+    const int64_t base = tok_off[u];
+    const int N = static_cast<int>(tok_off[u + 1] - base);
+    const int c = N - w;
+    int32_t* out = idx + static_cast<int64_t>(u) * W;
+    if (tid == 0 && u + static_cast<int>(gridDim.x) < U) {
+      const int u2 = u + gridDim.x;
+      const int64_t b2 = tok_off[u2];
+      const int64_t c2 = tok_off[u2 + 1] - b2 - w;
+      if (c2 > budget) {
+        prefetch_l2(a + b2, static_cast<size_t>(c2) * 4);
+        prefetch_l2(r + b2, static_cast<size_t>(c2) * 4);
       }
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (bin < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+    }
+    if (c <= budget) {  // every token is kept
+      for (int i = tid; i < W; i += kSelThreads) out[i] = i < N ? i : -1;
+      if (tid == 0) n_kept[u] = N;
+      continue;
+    }
+
+    // ---- 1. keys, min and max
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int i = tid; i < c; i += kSelThreads) {
+      const float s = __fsub_rn(__fmul_rn(lw, a[base + i]), __fmul_rn(rw, r[base + i]));
+      const uint32_t k = order_key(s);
+      keys[i] = k;
+      kmin = min(kmin, k);
+      kmax = max(kmax, k);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    if (lane == 0) {
+      wmin[wp] = kmin;
+      wmax[wp] = kmax;
     }
     __syncthreads();
     if (wp == 0) {
-      int cnt[8], tot = 0;
+      kmin = wmin[lane];
+      kmax = wmax[lane];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        cnt[k] = hist[255 - 8 * lane - k];
-        tot += cnt[k];
+      for (int o = 16; o; o >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
       }
-      int incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+      if (lane == 0) {
+        sh[4] = static_cast<int>(kmin);
+        sh[5] = static_cast<int>(kmax);
       }
-      const int excl = incl - tot;
-      const unsigned hit = __ballot_sync(0xffffffffu, excl < want && want <= incl);
-      if (lane == __ffs(hit) - 1) {
-        int run = excl;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (run + cnt[k] >= want) {
-            sh[0] = 255 - 8 * lane - k;
-            sh[1] = run;
-            break;
-          }
-          run += cnt[k];
+    }
+    __syncthreads();
+    kmin = static_cast<uint32_t>(sh[4]);
+    kmax = static_cast<uint32_t>(sh[5]);
+
+    // ---- 2. radix select below the common prefix
+    const uint32_t diff = kmin ^ kmax;
+    int lo = diff ? 32 - __clz(diff) : 0;     // bits [0, lo) still undetermined
+    uint32_t pmask = lo >= 32 ? 0u : ~((1u << lo) - 1u);
+    uint32_t prefix = kmin & pmask;
+    int want = budget;                        // keys still to take among the prefix matches
+    bool in_list = false;
+    int nlist = 0;
+    while (lo > 0) {
+      const int d = min(8, lo);
+      const int shift = lo - d;
+      const uint32_t dmask = (1u << d) - 1u;
+      for (int b = tid; b < kHistGroups * 256; b += kSelThreads) (&hist8[0][0])[b] = 0u;
+      __syncthreads();
+      uint32_t* hg = hist8[wp >> 2];
+      if (!in_list) {
+        for (int i = tid; i < c; i += kSelThreads) {
+          const uint32_t k = keys[i];
+          if ((k & pmask) == prefix) atomicAdd(&hg[(k >> shift) & dmask], 1u);
+        }
+      } else {
+        for (int i = tid; i < nlist; i += kSelThreads) {
+          const uint32_t k = list[i];
+          if ((k & pmask) == prefix) atomicAdd(&hg[(k >> shift) & dmask], 1u);
         }
       }
+      __syncthreads();
+      if (tid < 256) {
+        uint32_t t = 0;
+#pragma unroll
+        for (int g = 0; g < kHistGroups; ++g) t += hist8[g][tid];
+        hist[tid] = t;
+      }
+      __syncthreads();
+      if (wp == 0) {
+        // lane l owns bins 255-8l .. 248-8l (descending)
+        int cnt[8], tot = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          cnt[k] = static_cast<int>(hist[255 - 8 * lane - k]);
+          tot += cnt[k];
+        }
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const int excl = incl - tot;
+        const unsigned hit = __ballot_sync(0xffffffffu, excl < want && want <= incl);
+        if (lane == __ffs(hit) - 1) {
+          int run = excl;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            if (run + cnt[k] >= want) {
+              sh[0] = 255 - 8 * lane - k;
+              sh[1] = run;
+              sh[2] = cnt[k];
+              break;
+            }
+            run += cnt[k];
+          }
+        }
+        if (lane == 0) sh[3] = 0;
+      }
+      __syncthreads();
+      want -= sh[1];
+      prefix |= static_cast<uint32_t>(sh[0]) << shift;
+      pmask |= dmask << shift;
+      lo = shift;
+      const int cnt_bin = sh[2];
+      if (!in_list && lo > 0 && cnt_bin <= kListCap) {
+        // survivors of this digit -> short list (order irrelevant for T)
+        for (int i0 = wp * 32; i0 < ((c + 31) & ~31); i0 += kSelThreads) {
+          const int i = i0 + lane;
+          const uint32_t k = i < c ? keys[i] : 0u;
+          const bool m = i < c && (k & pmask) == prefix;
+          const unsigned bal = __ballot_sync(0xffffffffu, m);
+          int slot = 0;
+          if (lane == 0 && bal) slot = atomicAdd(&sh[3], __popc(bal));
+          slot = __shfl_sync(0xffffffffu, slot, 0);
+          if (m) list[slot + __popc(bal & ((1u << lane) - 1u))] = k;
+        }
+        __syncthreads();
+        nlist = sh[3];
+        in_list = true;
+      }
+      __syncthreads();
     }
-    __syncthreads();
-    want -= sh[1];
-    prefix |= static_cast<uint32_t>(sh[0]) << shift;
-    pmask |= 255u << shift;
-    __syncthreads();
-  }
-  const uint32_t T = prefix;  // key of the budget-th largest score
-  const int take_eq = want;   // keys equal to T that are kept (lowest indices)
+    const uint32_t T = prefix;  // key of the budget-th largest score
+    const int take_eq = want;   // keys equal to T that are kept (lowest indices)
 
-  // ---- per-warp segments, counts, then ordered output
-  const int seg = (((c + NW - 1) / NW) + 31) & ~31;
-  const int s0 = wp * seg, s1 = min(c, s0 + seg);
-  int gt = 0, eq = 0;
-  for (int i0 = s0; i0 < s1; i0 += 32) {
-    const int i = i0 + lane;
-    const bool v = i < s1;
-    const uint32_t k = v ? keys[i] : 0u;
-    gt += __popc(__ballot_sync(0xffffffffu, v && k > T));
-    eq += __popc(__ballot_sync(0xffffffffu, v && k == T));
-  }
-  if (lane == 0) {
-    wgt[wp] = gt;
-    weq[wp] = eq;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int eb = 0, ob = 0;
-    for (int x = 0; x < NW; ++x) {
-      eqb[x] = eb;
-      outb[x] = ob;
-      ob += wgt[x] + min(max(take_eq - eb, 0), weq[x]);
-      eb += weq[x];
+    // ---- 3. per-warp segments, counts, then ordered output
+    const int seg = (((c + kSelWarps - 1) / kSelWarps) + 31) & ~31;
+    const int s0 = wp * seg, s1 = min(c, s0 + seg);
+    int gt = 0, eq = 0;
+    for (int i0 = s0; i0 < s1; i0 += 32) {
+      const int i = i0 + lane;
+      const bool v = i < s1;
+      const uint32_t k = v ? keys[i] : 0u;
+      gt += __popc(__ballot_sync(0xffffffffu, v && k > T));
+      eq += __popc(__ballot_sync(0xffffffffu, v && k == T));
     }
+    if (lane == 0) {
+      wgt[wp] = gt;
+      weq[wp] = eq;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int eb = 0, ob = 0;
+      for (int x = 0; x < kSelWarps; ++x) {
+        eqb[x] = eb;
+        outb[x] = ob;
+        ob += wgt[x] + min(max(take_eq - eb, 0), weq[x]);
+        eb += weq[x];
+      }
+    }
+    __syncthreads();
+    int eseen = eqb[wp], oseen = outb[wp];
+    const unsigned lt = (1u << lane) - 1u;
+    for (int i0 = s0; i0 < s1; i0 += 32) {
+      const int i = i0 + lane;
+      const bool v = i < s1;
+      const uint32_t k = v ? keys[i] : 0u;
+      const bool g = v && k > T, e = v && k == T;
+      const unsigned be = __ballot_sync(0xffffffffu, e);
+      const bool f = g || (e && eseen + __popc(be & lt) < take_eq);
+      const unsigned bf = __ballot_sync(0xffffffffu, f);
+      if (f) out[oseen + __popc(bf & lt)] = i;
+      eseen += __popc(be);
+      oseen += __popc(bf);
+    }
+    for (int t = tid; t < w; t += kSelThreads) out[budget + t] = c + t;
+    if (tid == 0) n_kept[u] = budget + w;
+    __syncthreads();  // shared state is reused by the next unit
   }
-  __syncthreads();
-  int eseen = eqb[wp], oseen = outb[wp];
-  const unsigned lt = (1u << lane) - 1u;
-  for (int i0 = s0; i0 < s1; i0 += 32) {
-    const int i = i0 + lane;
-    const bool v = i < s1;
-    const uint32_t k = v ? keys[i] : 0u;
-    const bool g = v && k > T, e = v && k == T;
-    const unsigned be = __ballot_sync(0xffffffffu, e);
-    const bool f = g || (e && eseen + __popc(be & lt) < take_eq);
-    const unsigned bf = __ballot_sync(0xffffffffu, f);
-    if (f) out[oseen + __popc(bf & lt)] = i;
-    eseen += __popc(be);
-    oseen += __popc(bf);
-  }
-  for (int t = tid; t < w; t += NT) out[budget + t] = c + t;
-  if (tid == 0) n_kept[u] = budget + w;
 }
 
 }  // namespace
 
 cudaError_t select_configure() {
-  const int smem = kMaxTokensPerUnit * 4;
-  cudaError_t e;
-  e = cudaFuncSetAttribute(select_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(select_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kMaxTokensPerUnit * 4);
 }
 
 cudaError_t launch_select(const int64_t* tok_off, int U, int w, int cmax, const float* a,
                           const float* r, float lam, int budget, int32_t* idx, int32_t* n_kept,
                           cudaStream_t st) {
   const size_t smem = cmax > budget ? static_cast<size_t>(cmax) * 4 : 0;
-  if (cmax > 16384)
-    select_kernel<1024><<<U, 1024, smem, st>>>(tok_off, w, a, r, lam, budget, idx, n_kept);
-  else if (cmax > 4096)
-    select_kernel<512><<<U, 512, smem, st>>>(tok_off, w, a, r, lam, budget, idx, n_kept);
-  else
-    select_kernel<256><<<U, 256, smem, st>>>(tok_off, w, a, r, lam, budget, idx, n_kept);
+  int dev = 0, nsm = 0, per = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, select_kernel, kSelThreads, smem) !=
+          cudaSuccess ||
+      per < 1) {
+    cudaGetLastError();
+    per = 1;
+  }
+  int grid = nsm * per;
+  if (grid > U) grid = U;
+  select_kernel<<<grid, kSelThreads, smem, st>>>(tok_off, U, w, a, r, lam, budget, idx, n_kept);
   return cudaGetLastError();
 }
 
