@@ -54,6 +54,22 @@ def redundancy(K, w):
     return m, [v / tot for v in e]
 
 
+def redundancy_max(K, w):
+    """Row max of the cosine-similarity matrix, diagonal excluded, then a
+    softmax over the candidates."""
+    N = len(K)
+    c = N - w
+    unit = []
+    for k in K:
+        n = math.sqrt(_dot(k, k))
+        unit.append([x / n for x in k] if n > 0 else [0.0] * len(k))
+    m = [max(_dot(unit[i], unit[j]) for j in range(N) if j != i) for i in range(c)]
+    mx = max(m)
+    e = [math.exp(v - mx) for v in m]
+    tot = math.fsum(e)
+    return m, [v / tot for v in e]
+
+
 def select(s, N, w, budget):
     """Sort candidates by (score descending, index ascending)."""
     c = N - w

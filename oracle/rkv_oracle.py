@@ -110,6 +110,26 @@ def redundancy_mean_closed_form(K: np.ndarray, w: int):
     return m, softmax(m)
 
 
+def redundancy_max(K: np.ndarray, w: int, block: int = 2048):
+    """Redundancy as the nearest duplicate (冗余打分, row-max reading): the
+    largest cosine similarity to any other cached key,
+    m_i = max_{j != i, j < N} k_hat_i . k_hat_j for i in C; r = softmax over C.
+    A key with an exact copy elsewhere gets m = 1, the largest possible value.
+    Returns (m [N - w], r [N - w])."""
+    N = K.shape[0]
+    c = N - w
+    if c <= 0:
+        return np.zeros(0), np.zeros(0)
+    kh = unit_keys(K)
+    m = np.empty(c)
+    for i0 in range(0, c, block):
+        i1 = min(c, i0 + block)
+        S = kh[i0:i1] @ kh.T
+        S[np.arange(i1 - i0), np.arange(i0, i1)] = -np.inf   # exclude j == i
+        m[i0:i1] = S.max(axis=1)
+    return m, softmax(m)
+
+
 def softmax(x: np.ndarray) -> np.ndarray:
     if x.size == 0:
         return x.copy()
@@ -143,14 +163,17 @@ def compact(K: np.ndarray, V: np.ndarray, idx: np.ndarray):
 
 
 def run_unit(Q, K, V, w: int, budget: int, lam: float, redundancy="rowblocks"):
-    """Whole path for one unit.  ``redundancy`` picks the definition
-    (``rowblocks``) or the closed form (``closed``)."""
+    """Whole path for one unit.  ``redundancy`` picks the row-mean definition
+    (``rowblocks``), its closed form (``closed``) or the row-max reading
+    (``max``)."""
     N = K.shape[0]
     abar, a = importance(Q, K)
     if redundancy == "rowblocks":
         m, r = redundancy_mean(K, w)
     elif redundancy == "closed":
         m, r = redundancy_mean_closed_form(K, w)
+    elif redundancy == "max":
+        m, r = redundancy_max(K, w)
     else:
         raise ValueError(redundancy)
     s = joint_score(a, r, lam)

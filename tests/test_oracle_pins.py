@@ -314,3 +314,44 @@ def _ties_high(s, N, w, budget):
         "wrong-sign", "ties-to-high-index"])
 def test_planted_mistake_fails_worked_example(over):
     assert check_worked_example(_Mutant(**over)) != []
+
+
+# ---- row-max redundancy (nearest duplicate) --------------------------------
+
+@pytest.mark.parametrize("seed", range(6))
+def test_row_max_matches_loop_transcription(seed):
+    rng = np.random.default_rng(200 + seed)
+    N = int(rng.integers(3, 40))
+    w = int(rng.integers(1, min(N - 1, 5) + 1))
+    Q, K = _rand_unit(rng, N, 8, 1, w, dup=0.2)
+    m_ref, r_ref = loops.redundancy_max(K.tolist(), w)
+    m, r = ora.redundancy_max(K, w, block=7)
+    np.testing.assert_allclose(m, m_ref, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(r, r_ref, rtol=1e-12)
+
+
+def test_row_max_exact_duplicates_are_maximal():
+    rng = np.random.default_rng(21)
+    K = rng.standard_normal((500, 128))
+    K[100] = K[7]
+    K[300] = 2.5 * K[40]          # same direction counts as a duplicate
+    m, r = ora.redundancy_max(K, 8)
+    assert m[7] == pytest.approx(1.0, abs=1e-12) and m[100] == pytest.approx(1.0, abs=1e-12)
+    assert m[40] == pytest.approx(1.0, abs=1e-12) and m[300] == pytest.approx(1.0, abs=1e-12)
+    others = np.delete(m, [7, 100, 40, 300])
+    assert others.max() < 0.6      # i.i.d. 128-d keys are far from each other
+    assert r[7] == pytest.approx(r.max(), rel=1e-12)
+
+
+def test_row_max_worked_example():
+    g, Q, K = _worked()
+    # unit keys (1,0),(1,0),(0,1),(-1,0),(1,1)/sqrt2,(0,-1): nearest other key of
+    # each candidate, by hand: k0 ~ k1 (1), k1 ~ k0 (1), k2 ~ k4 (1/sqrt2), k3 ~ k2 (0)
+    m, _ = ora.redundancy_max(K, g["window"])
+    np.testing.assert_allclose(m, [1.0, 1.0, 1 / np.sqrt(2), 0.0], atol=1e-12)
+
+
+def test_row_max_zero_key_and_window_keys_count():
+    K = np.array([[1.0, 0.0], [0.0, 0.0], [0.0, 1.0], [1.0, 0.0]])
+    m, _ = ora.redundancy_max(K, 1)   # candidates 0..2; key 3 (window) duplicates key 0
+    np.testing.assert_allclose(m, [1.0, 0.0, 0.0], atol=1e-15)
