@@ -52,10 +52,12 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="engine", choices=["engine", "reference"])
     ap.add_argument("--workload", default="long_trace_32k", choices=W.WORKLOAD_ORDER)
-    ap.add_argument("--redundancy", default="gemm", choices=["gemm", "closed"])
+    ap.add_argument("--redundancy", default="gemm", choices=["gemm", "closed", "max"])
     ap.add_argument("--lam", type=float, default=0.1)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-chunk", type=int, default=0,
+                    help="rows per chunk of the host-buffer pipeline (0: library default)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
@@ -151,6 +153,10 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+# oracle redundancy function that each engine mode computes
+ORACLE_MODE = {"gemm": "rowblocks", "closed": "closed", "max": "max"}
+
+
 def algorithmic(batch: Batch, wl: W.Workload):
     """Per-launch algorithmic work of each kernel (bytes or flops)."""
     n = np.diff(batch.tok_off_host).astype(np.float64)
@@ -223,7 +229,7 @@ def cpu_baseline(batch: Batch, wl: W.Workload, lam: float, seconds: float, redun
     rng = np.random.default_rng(7)
     order = rng.permutation(batch.num_units)
     toks, t_used, done = 0, 0.0, 0
-    mode = "rowblocks" if redundancy == "gemm" else "closed"
+    mode = ORACLE_MODE[redundancy]
     for u in order:
         r0, r1 = int(batch.tok_off_host[u]), int(batch.tok_off_host[u + 1])
         k = batch.K[r0:r1].float().cpu().numpy().astype(np.float64)
@@ -268,7 +274,7 @@ def run_reference(args, dist: Dist):
                              dup_noise=wl.dup_noise, span_len=wl.span_len,
                              key_scale=wl.key_scale, n_kv_head=len(units)),
                     seed=args.seed, device="cpu")
-    mode = "rowblocks" if args.redundancy == "gemm" else "closed"
+    mode = ORACLE_MODE[args.redundancy]
     times, toks = [], []
     for i in range(len(units)):
         r0, r1 = int(gb.tok_off[i]), int(gb.tok_off[i + 1])
@@ -326,7 +332,7 @@ def run_engine(args, dist: Dist):
     eng, ms, rep, launches = measure(args.redundancy)
     clocks = clk.stop() if clk else None
     value = tokens * dist.world / (ms * 1e-3)
-    dom = "gemm" if args.redundancy == "gemm" else "score"
+    dom = "score" if args.redundancy == "closed" else "gemm"
     roof = dict(rep[dom])
     traffic = None
     if wl.name == "long_trace_32k" and args.redundancy == "gemm":
@@ -367,45 +373,37 @@ def run_engine(args, dist: Dist):
 
 
 def measure_e2e(eng, batch: Batch, wl: W.Workload, args, dist: Dist):
-    """Same metric through the public call with host inputs and outputs: pinned
-    host K, V, Q, offsets -> device, rkv_compress, kept indices and compacted
-    K/V -> pinned host, all inside the timed region."""
+    """Same metric through the public host-buffer call (rkv_compress_host):
+    page-locked host K, V, Q and offsets in, kept indices and compacted K/V out
+    to page-locked host memory, the library's chunked copy-in / compute /
+    copy-out pipeline inside the timed region."""
     hK = torch.empty(batch.K.shape, dtype=batch.K.dtype, pin_memory=True)
     hV = torch.empty(batch.V.shape, dtype=batch.V.dtype, pin_memory=True)
     hQ = torch.empty(batch.Q.shape, dtype=batch.Q.dtype, pin_memory=True)
-    hoff = torch.from_numpy(batch.tok_off_host.copy()).pin_memory()
     hK.copy_(batch.K)
     hV.copy_(batch.V)
     hQ.copy_(batch.Q)
-    dK, dV, dQ = (torch.empty_like(t) for t in (batch.K, batch.V, batch.Q))
-    b2 = Batch(dK, dV, dQ, batch.tok_off_host)
-    a, r = eng.alloc_scores(b2)
-    idx, nk, Ko, Vo = eng.alloc_outputs(b2, wl.budget)
-    h_idx = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
-    h_nk = torch.empty(nk.shape, dtype=nk.dtype, pin_memory=True)
-    h_Ko = torch.empty(Ko.shape, dtype=Ko.dtype, pin_memory=True)
-    h_Vo = torch.empty(Vo.shape, dtype=Vo.dtype, pin_memory=True)
+    off = batch.tok_off_host
+    outs = eng.alloc_host_outputs(batch.num_units, wl.budget)
 
     def step():
-        dK.copy_(hK, non_blocking=True)
-        dV.copy_(hV, non_blocking=True)
-        dQ.copy_(hQ, non_blocking=True)
-        b2.tok_off.copy_(hoff, non_blocking=True)
-        eng.compress(b2, args.lam, wl.budget, a, r, idx, nk, Ko, Vo)
-        h_idx.copy_(idx, non_blocking=True)
-        h_nk.copy_(nk, non_blocking=True)
-        h_Ko.copy_(Ko, non_blocking=True)
-        h_Vo.copy_(Vo, non_blocking=True)
+        eng.compress_host(hK, hV, hQ, off, args.lam, wl.budget, *outs,
+                          chunk_tokens=args.e2e_chunk)
 
     ms, _, _ = timed(step, args.e2e_steps, 1, dist)
     eng.check_status()
-    ok = torch.equal(h_nk, nk.cpu())
-    h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hQ, hoff))
-    d2h = sum(t.numel() * t.element_size() for t in (h_idx, h_nk, h_Ko, h_Vo))
+    # the host path must reproduce the device path's kept indices exactly
+    a, r = eng.alloc_scores(batch)
+    idx, nk = eng.alloc_outputs(batch, wl.budget)[:2]
+    eng.score(batch, a, r)
+    eng.select(batch, a, r, args.lam, wl.budget, idx, nk)
+    ok = torch.equal(outs[1], nk.cpu()) and torch.equal(outs[0], idx.cpu())
+    h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hQ)) + 8 * len(off)
+    d2h = sum(t.numel() * t.element_size() for t in outs)
     return {"value": batch.num_tokens * dist.world / (ms * 1e-3), "unit": UNIT,
             "ms_per_step": ms, "steps": args.e2e_steps, "warmup": 1,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "outputs_consistent": bool(ok)}
+            "api": "rkv_compress_host", "outputs_consistent": bool(ok)}
 
 
 def main():

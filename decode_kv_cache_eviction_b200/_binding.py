@@ -28,11 +28,12 @@ RKV_ERR_DEVICE = -7
 
 RKV_REDUNDANCY_GEMM = 0
 RKV_REDUNDANCY_CLOSED_FORM = 1
+RKV_REDUNDANCY_MAX = 2
 RKV_FLAG_GEMM_SINGLE_CTA = 1
 
 # Every function declared in include/rkv.h.
 EXPORTS = ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact",
-           "rkv_compress", "rkv_check_status", "rkv_launch_count", "rkv_set_timing",
+           "rkv_compress", "rkv_compress_host", "rkv_check_status", "rkv_launch_count", "rkv_set_timing",
            "rkv_read_timing", "rkv_score_noalloc", "rkv_status_string", "rkv_version")
 KERNELS = ("score", "plan", "gemm", "select", "compact")
 
@@ -42,6 +43,11 @@ class RkvConfig(ctypes.Structure):
                 ("window", ctypes.c_int), ("max_units", ctypes.c_int),
                 ("max_tokens", ctypes.c_int64), ("redundancy", ctypes.c_int),
                 ("flags", ctypes.c_int)]
+
+
+class RkvHostBatch(ctypes.Structure):
+    _fields_ = [("num_units", ctypes.c_int), ("tok_off", ctypes.c_void_p),
+                ("K", ctypes.c_void_p), ("V", ctypes.c_void_p), ("Q", ctypes.c_void_p)]
 
 
 class RkvBatch(ctypes.Structure):
@@ -77,6 +83,8 @@ def lib():
     L.rkv_compact.argtypes = [vp, ctypes.POINTER(RkvBatch), vp, vp, i32, vp, vp, vp]
     L.rkv_compress.argtypes = [vp, ctypes.POINTER(RkvBatch), f32, i32, vp, vp, vp, vp, vp,
                                vp, vp]
+    L.rkv_compress_host.argtypes = [vp, ctypes.POINTER(RkvHostBatch), f32, i32, vp, vp, vp, vp,
+                                    i64, vp]
     L.rkv_check_status.argtypes = [vp, vp]
     L.rkv_launch_count.argtypes = [vp]
     L.rkv_launch_count.restype = i64
@@ -88,7 +96,8 @@ def lib():
     L.rkv_status_string.restype = ctypes.c_char_p
     L.rkv_version.argtypes = []
     for name in ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact",
-                 "rkv_compress", "rkv_check_status", "rkv_set_timing", "rkv_read_timing",
+                 "rkv_compress", "rkv_compress_host", "rkv_check_status", "rkv_set_timing",
+                 "rkv_read_timing",
                  "rkv_score_noalloc", "rkv_version"):
         getattr(L, name).restype = i32
     _lib = L
@@ -154,7 +163,8 @@ class Engine:
 
     def __init__(self, group: int, window: int, max_units: int, max_tokens: int,
                  head_dim: int = 128, redundancy: str = "gemm", single_cta_gemm=False):
-        mode = {"gemm": RKV_REDUNDANCY_GEMM, "closed": RKV_REDUNDANCY_CLOSED_FORM}[redundancy]
+        mode = {"gemm": RKV_REDUNDANCY_GEMM, "closed": RKV_REDUNDANCY_CLOSED_FORM,
+                "max": RKV_REDUNDANCY_MAX}[redundancy]
         self.cfg = RkvConfig(head_dim, group, window, max_units, max_tokens, mode,
                              RKV_FLAG_GEMM_SINGLE_CTA if single_cta_gemm else 0)
         self.group, self.window = group, window
@@ -194,6 +204,23 @@ class Engine:
                                   _ptr(a), _ptr(r), _ptr(idx), _ptr(n_kept), _ptr(K_out),
                                   _ptr(V_out), _stream(stream)), "rkv_compress")
 
+    def compress_host(self, K, V, Q, tok_off, lam: float, budget: int, idx, n_kept, K_out,
+                      V_out, chunk_tokens: int = 0, stream=None):
+        """The whole path from host tensors to host tensors (``rkv_compress_host``).
+        K, V [T, d], Q [U, G, w, d] bf16 and the outputs are CPU tensors (pinned for
+        overlapped copies); ``tok_off`` is an int64 sequence of U + 1 row offsets.
+        Outputs are complete once ``stream`` (default: torch's current) is synced."""
+        for t in (K, V, Q, idx, n_kept, K_out, V_out):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError("compress_host takes contiguous host tensors")
+        off = np.ascontiguousarray(np.asarray(tok_off, dtype=np.int64))
+        hb = RkvHostBatch(len(off) - 1, off.ctypes.data, K.data_ptr(), V.data_ptr(),
+                          Q.data_ptr())
+        _check(lib().rkv_compress_host(self.h, ctypes.byref(hb), float(lam), int(budget),
+                                       _ptr(idx), _ptr(n_kept), _ptr(K_out), _ptr(V_out),
+                                       int(chunk_tokens), _stream(stream)),
+               "rkv_compress_host")
+
     def check_status(self, stream=None):
         _check(lib().rkv_check_status(self.h, _stream(stream)), "device status")
 
@@ -221,6 +248,14 @@ class Engine:
         dev = batch.K.device
         return (torch.empty(T, dtype=torch.float32, device=dev),
                 torch.empty(T, dtype=torch.float32, device=dev))
+
+    def alloc_host_outputs(self, num_units: int, budget: int, pin: bool = True):
+        """Host (page-locked unless ``pin`` is False) outputs for compress_host."""
+        U, W = num_units, budget + self.window
+        return (torch.empty((U, W), dtype=torch.int32, pin_memory=pin),
+                torch.empty(U, dtype=torch.int32, pin_memory=pin),
+                torch.empty((U, W, 128), dtype=torch.bfloat16, pin_memory=pin),
+                torch.empty((U, W, 128), dtype=torch.bfloat16, pin_memory=pin))
 
     def alloc_outputs(self, batch: Batch, budget: int):
         U, W = batch.num_units, budget + self.window

@@ -6,38 +6,11 @@
 #include <new>
 
 #include "../../include/rkv.h"
+#include "engine.cuh"
 #include "ptx.cuh"
 #include "rkv_internal.cuh"
 
 using namespace rkv;
-
-struct rkv_engine {
-  rkv_config cfg;
-  int device = 0;
-  int nsm = 0;
-  int rp = 32;                 // padded G*w (MMA N of the logits tile)
-  int nstages = 0;             // score K-tile ring depth
-  int score_smem = 0;
-  int score_clusters[5] = {};  // active clusters for cluster sizes 1, 2, 4, 8, 16
-  int max_cs = 16;
-  int max_n = 0;               // largest supported N_u
-  bool pair = true;
-  int gemm_ctas = 0;
-  float* rho = nullptr;        // [max_tokens + kRhoAlign * max_units] padded 1/||k||
-  int64_t* rho_off = nullptr;  // [max_units + 1]
-  int* item_off = nullptr;     // [max_units + 1]
-  int* unit_cnt = nullptr;     // [max_units]
-  int* status = nullptr;       // [1]
-  int64_t launches = 0;
-  PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-  // per-kernel timing (rkv_set_timing)
-  static constexpr int kMaxEv = 4096;
-  bool timing = false;
-  cudaEvent_t ev[kMaxEv][2] = {};
-  int ev_kernel[kMaxEv] = {};
-  int nev = 0;
-  bool ev_made = false;
-};
 
 namespace {
 
@@ -130,7 +103,8 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   *out = nullptr;
   if (cfg->group < 1 || cfg->window < 1 || cfg->max_units < 1 || cfg->max_tokens < 1)
     return RKV_ERR_INVALID_ARG;
-  if (cfg->redundancy != RKV_REDUNDANCY_GEMM && cfg->redundancy != RKV_REDUNDANCY_CLOSED_FORM)
+  if (cfg->redundancy != RKV_REDUNDANCY_GEMM && cfg->redundancy != RKV_REDUNDANCY_CLOSED_FORM &&
+      cfg->redundancy != RKV_REDUNDANCY_MAX)
     return RKV_ERR_INVALID_ARG;
   if ((cfg->flags & ~RKV_FLAG_GEMM_SINGLE_CTA) != 0) return RKV_ERR_INVALID_ARG;
   if (cfg->head_dim != kHeadDim) return RKV_ERR_UNSUPPORTED;
@@ -156,6 +130,7 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   e->nsm = nsm;
   e->rp = cfg->group * cfg->window <= 16 ? 16 : 32;
   e->pair = (cfg->flags & RKV_FLAG_GEMM_SINGLE_CTA) == 0;
+  e->rowmax = cfg->redundancy == RKV_REDUNDANCY_MAX;
 
   cudaDriverEntryPointQueryResult q;
   void* fn = nullptr;
@@ -194,11 +169,11 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
     return cuda_fail(cudaErrorUnknown);
   }
   if (!closed) {
-    if (gemm_configure(e->pair) != cudaSuccess) {
+    if (gemm_configure(e->pair, e->rowmax) != cudaSuccess) {
       delete e;
       return cuda_fail(cudaErrorUnknown);
     }
-    e->gemm_ctas = gemm_max_ctas(e->pair);
+    e->gemm_ctas = gemm_max_ctas(e->pair, e->rowmax);
     if (e->gemm_ctas <= 0) {
       delete e;
       return RKV_ERR_UNSUPPORTED;
@@ -266,6 +241,7 @@ int rkv_destroy(rkv_engine* e) {
   if (e->ev_made)
     for (int i = 0; i < rkv_engine::kMaxEv; ++i)
       for (int k = 0; k < 2; ++k) cudaEventDestroy(e->ev[i][k]);
+  rkv_host_pipeline_free(e);
   cudaFree(e->status);
   cudaFree(e->item_off);
   cudaFree(e->unit_cnt);
@@ -361,7 +337,7 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   const int64_t need = items * (e->pair ? 2 : 1);
   if (nctas > need) nctas = need;
   t_begin(e, RKV_KERNEL_GEMM, st);
-  err = launch_gemm(amap, bmap, g, e->pair, static_cast<int>(nctas), st);
+  err = launch_gemm(amap, bmap, g, e->pair, e->rowmax, static_cast<int>(nctas), st);
   t_end(e, st);
   if (err != cudaSuccess) return cuda_fail(err);
   ++e->launches;

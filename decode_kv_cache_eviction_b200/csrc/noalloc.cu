@@ -101,11 +101,11 @@ int setup(int dev, DeviceState** out) {
     }
     if (d.max_cs[k] == 0) return RKV_ERR_UNSUPPORTED;
   }
-  if (gemm_configure(true) != cudaSuccess) {
+  if (gemm_configure(true, false) != cudaSuccess) {
     cudaGetLastError();
     return RKV_ERR_CUDA;
   }
-  d.gemm_ctas = gemm_max_ctas(true);
+  d.gemm_ctas = gemm_max_ctas(true, false);
   if (d.gemm_ctas <= 0) return RKV_ERR_UNSUPPORTED;
   d.ready = true;
   *out = &d;
@@ -222,7 +222,7 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   g.status = s->status;
   int64_t nctas = d->gemm_ctas;
   if (nctas > 2 * items) nctas = 2 * items;
-  if (launch_gemm(amap, bmap, g, true, static_cast<int>(nctas), st) != cudaSuccess) {
+  if (launch_gemm(amap, bmap, g, true, false, static_cast<int>(nctas), st) != cudaSuccess) {
     cudaGetLastError();
     return RKV_ERR_CUDA;
   }

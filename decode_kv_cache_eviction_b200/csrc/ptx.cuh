@@ -378,4 +378,22 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Packed fp32 pair arithmetic (sm_100): one instruction for two lanes of work.
+// (d0, d1) += (a0, a1) * (b0, b1), each element rounded once like fmaf.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 d, a, b;\n\t"
+      "mov.b64 d, {%0, %1};\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "fma.rn.f32x2 d, a, b, d;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// (p0, p1) = (a0, a1) * (b0, b1)
+__device__ __forceinline__ void mul2(float& p0, float& p1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 p, a, b;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 p, a, b;\n\tmov.b64 {%0, %1}, p;\n\t}"
+      : "=f"(p0), "=f"(p1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 }  // namespace rkv

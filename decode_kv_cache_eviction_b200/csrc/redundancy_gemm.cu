@@ -12,18 +12,41 @@
 // into per-row partial sums, so the N x N similarity matrix never reaches HBM.
 // The last CTA to finish a unit (atomic counter) applies the token softmax.
 //
+// Row-max variant (kMax): the same tiles, folded with a max instead of a
+// weighted sum, give the nearest-duplicate redundancy
+//   m_i = rho_i * max_{j != i, j < N} rho_j * (k_i . k_j)
+// (rho_i >= 0, so the row scaling commutes with the max).  Columns past the end
+// of the unit are masked explicitly there, since a zero weight is not neutral
+// for a max.
+//
 // Work item = (unit, block of rows).  In pair mode a cluster of two CTAs runs
 // one M = 256 MMA (cta_group::2): each CTA holds 128 A rows and half of each
 // 256-key B tile, which halves the shared-memory traffic per SM.
 //
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer (leader CTA
-// only in pair mode) and TMEM owner, warps 4-11 epilogue (warp % 4 selects the
-// TMEM lane quarter, (warp - 4) / 4 the 128-column half of the tile).
+// Warp roles (640 threads = 5 warps per SM sub-partition): warp 0 TMA producer,
+// warp 1 MMA issuer (leader CTA only in pair mode) and TMEM owner, warps 4-19
+// epilogue (warp % 4 selects the TMEM lane quarter, (warp - 4) / 4 the
+// 64-column quarter of the tile).
 #include "ptx.cuh"
 #include "rkv_internal.cuh"
 
 namespace rkv {
 namespace {
+
+#ifdef RKV_TRACE
+// Optional per-tile trace (build with -DRKV_TRACE): for the first kGT tiles of
+// each CTA, globaltimer stamps of the MMA thread and of epilogue warp 4.
+constexpr int kGTCtas = 160, kGT = 64;
+__device__ unsigned long long g_gemm_trace[kGTCtas * 2 * kGT * 4];
+#define RKV_GSTAMP(role, tile, slot)                                                      \
+  do {                                                                                   \
+    if ((tile) < kGT && blockIdx.x < kGTCtas)                                            \
+      g_gemm_trace[((blockIdx.x * 2 + (role)) * kGT + (tile)) * 4 + (slot)] =            \
+          globaltimer_ns();                                                              \
+  } while (0)
+#else
+#define RKV_GSTAMP(role, tile, slot) do { } while (0)
+#endif
 
 __device__ __forceinline__ int find_unit(const int* item_off, int U, int item) {
   int lo = 0, hi = U - 1;  // largest u with item_off[u] <= item
@@ -35,7 +58,7 @@ __device__ __forceinline__ int find_unit(const int* item_off, int U, int item) {
   return lo;
 }
 
-template <bool kPair>
+template <bool kPair, bool kMax>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     redundancy_gemm_kernel(const __grid_constant__ CUtensorMap amap,
                            const __grid_constant__ CUtensorMap bmap, const GemmParams p) {
@@ -72,11 +95,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kPair ? 16 : 8);
+      mbar_init(&acc_empty[b], kPair ? 32 : 16);
     }
     for (int b = 0; b < kRhoSlots; ++b) {
       mbar_init(&rho_full[b], 1);
-      mbar_init(&rho_empty[b], 8);   // this CTA's 8 epilogue warps
+      mbar_init(&rho_empty[b], 16);   // this CTA's 16 epilogue warps
     }
     *abort = 0;
     fence_mbar_init();
@@ -157,7 +180,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t idesc = idesc_bf16_f32(C::kMmaM, C::kN);
       int stage = 0, ab = 0;
       uint32_t ph = 0, aph = 0;
-      int ai = 0;
+      int ai = 0, tcount = 0;
       for (int item = group_id; item < n_items; item += ngroups, ++ai) {
         const int u = find_unit(p.item_off, p.num_units, item);
         const int64_t base = __ldg(&p.tok_off[u]);
@@ -165,9 +188,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool aok = mbar_wait(a_full, ai & 1, abort, p.status);
         const uint32_t aaddr = smem_u32(sm + L.a);
         const int ntiles = (N + C::kN - 1) / C::kN;
-        for (int t = 0; t < ntiles; ++t) {
+        for (int t = 0; t < ntiles; ++t, ++tcount) {
+          RKV_GSTAMP(0, tcount, 0);
           bool go = mbar_wait(&b_full[stage], ph, abort, p.status);
+          RKV_GSTAMP(0, tcount, 1);
           go = mbar_wait(&acc_empty[ab], aph ^ 1, abort, p.status) && go && aok;
+          RKV_GSTAMP(0, tcount, 2);
           tc_fence_after();
           if (go) {
             const uint32_t baddr = smem_u32(sm + L.b + stage * C::kBBytes);
@@ -187,6 +213,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               mma_commit(&acc_full[ab]);
             }
           }
+          RKV_GSTAMP(0, tcount, 3);
           if (++stage == NSB) { stage = 0; ph ^= 1; }
           if (++ab == 2) { ab = 0; aph ^= 1; }
         }
@@ -199,9 +226,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
-    const int etid = threadIdx.x - 128;   // 0..255
-    const int ew = warp - 4;              // epilogue warp 0..7
-    const int half = ew >> 2;             // column half of the tile
+    const int etid = threadIdx.x - 128;   // 0..511
+    const int ew = warp - 4;              // epilogue warp 0..15
+    const int cg = ew >> 2;               // 64-column group of the tile
     const int q = warp & 3;               // TMEM lane quarter
     const int rloc = q * 32 + lane;       // row of this CTA's A block
     const float* rho_ring = reinterpret_cast<const float*>(sm + L.rho);
@@ -219,23 +246,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int c = N - p.w;
       const int rbase = blk * C::kRowsPerItem + rank * 128;   // unit-local first row
       const int i = rbase + rloc;
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+      constexpr float kInit = kMax ? -INFINITY : 0.f;
+      float s0 = kInit, s1 = kInit, s2 = kInit, s3 = kInit;
       const int ntiles = (N + C::kN - 1) / C::kN;
       for (int t = 0; t < ntiles; ++t, ++rt) {
         const int j0 = t * C::kN;
         const uint32_t rs_slot = rt % kRhoSlots;
-        const float* rs = rho_ring + rs_slot * 256 + half * 128;
+        const float* rs = rho_ring + rs_slot * 256 + cg * 64;
+        if (etid == 0) RKV_GSTAMP(1, rt, 0);
         mbar_wait(&acc_full[ab], aph, abort, p.status);
         mbar_wait(&rho_full[rs_slot], (rt / kRhoSlots) & 1, abort, p.status);
+        if (etid == 0) RKV_GSTAMP(1, rt, 1);
         __syncwarp();
         tc_fence_after();
         const uint32_t tbase =
-            tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + half * 128;
-        uint32_t va[32], vb[32], vc[32], vd[32];
-        tmem_ld32(tbase, va);
-        tmem_ld32(tbase + 32, vb);
-        tmem_ld32(tbase + 64, vc);
-        tmem_ld32(tbase + 96, vd);
+            tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + cg * 64;
+        const int cw0 = j0 + cg * 64;                // first column of this warp's group
+        const int rw0 = rbase + q * 32;              // first row of this warp
+        const bool masked = ((rw0 < cw0 + 64) && (cw0 < rw0 + 32)) || (kMax && cw0 + 64 > N);
+        const int jd = i - cw0;
+        const int jn = kMax ? N - cw0 : 64;
+        constexpr uint32_t neutral = kMax ? 0xff800000u : 0u;   // -inf, or 0
+        // 32 columns at a time, so that the values, four partial sums and the
+        // weights fit the 96 registers a thread has at 640 threads per CTA.
+        // Masked groups (rare): the diagonal column i - cw0 and, for the row
+        // max, the columns past the unit are neutralised (-inf * rho is -inf or
+        // NaN, both ignored by fmaxf).  Sums use packed fp32x2 FMAs.
+        uint32_t v[32];
+        auto half = [&](int off) {
+          if (masked) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (k + off == jd || k + off >= jn) v[k] = neutral;
+          }
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 4) {
+            const float4 r4 = *reinterpret_cast<const float4*>(rs + off + cc);
+            if constexpr (kMax) {
+              float p0, p1, p2, p3;
+              mul2(p0, p1, __uint_as_float(v[cc + 0]), __uint_as_float(v[cc + 1]), r4.x, r4.y);
+              mul2(p2, p3, __uint_as_float(v[cc + 2]), __uint_as_float(v[cc + 3]), r4.z, r4.w);
+              s0 = fmaxf(s0, p0); s1 = fmaxf(s1, p1); s2 = fmaxf(s2, p2); s3 = fmaxf(s3, p3);
+            } else {
+              fma2(s0, s1, __uint_as_float(v[cc + 0]), __uint_as_float(v[cc + 1]), r4.x, r4.y);
+              fma2(s2, s3, __uint_as_float(v[cc + 2]), __uint_as_float(v[cc + 3]), r4.z, r4.w);
+            }
+          }
+        };
+        tmem_ld32(tbase, v);
+        tmem_wait_ld();
+        if (etid == 0) RKV_GSTAMP(1, rt, 2);
+        half(0);
+        tmem_ld32(tbase + 32, v);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -244,69 +306,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           else mbar_arrive(&acc_empty[ab]);
         }
         if (++ab == 2) { ab = 0; aph ^= 1; }
-        const int cw0 = j0 + half * 128;             // first column of this warp's half
-        const int rw0 = rbase + q * 32;              // first row of this warp
-        if (!((rw0 < cw0 + 128) && (cw0 < rw0 + 32))) {
-          auto fold = [&](const uint32_t (&v)[32], int off) {
-#pragma unroll
-            for (int cc = 0; cc < 32; cc += 4) {
-              const float4 r4 = *reinterpret_cast<const float4*>(rs + off + cc);
-              s0 = fmaf(__uint_as_float(v[cc + 0]), r4.x, s0);
-              s1 = fmaf(__uint_as_float(v[cc + 1]), r4.y, s1);
-              s2 = fmaf(__uint_as_float(v[cc + 2]), r4.z, s2);
-              s3 = fmaf(__uint_as_float(v[cc + 3]), r4.w, s3);
-            }
-          };
-          fold(va, 0); fold(vb, 32); fold(vc, 64); fold(vd, 96);
-        } else {
-          const int jd = i - cw0;                    // this row's diagonal column in the half
-          auto fold = [&](const uint32_t (&v)[32], int off) {
-#pragma unroll
-            for (int cc = 0; cc < 32; cc += 4) {
-              const float4 r4 = *reinterpret_cast<const float4*>(rs + off + cc);
-              s0 = fmaf(off + cc + 0 == jd ? 0.f : __uint_as_float(v[cc + 0]), r4.x, s0);
-              s1 = fmaf(off + cc + 1 == jd ? 0.f : __uint_as_float(v[cc + 1]), r4.y, s1);
-              s2 = fmaf(off + cc + 2 == jd ? 0.f : __uint_as_float(v[cc + 2]), r4.z, s2);
-              s3 = fmaf(off + cc + 3 == jd ? 0.f : __uint_as_float(v[cc + 3]), r4.w, s3);
-            }
-          };
-          fold(va, 0); fold(vb, 32); fold(vc, 64); fold(vd, 96);
-        }
+        half(32);
+        if (etid == 0) RKV_GSTAMP(1, rt, 3);
         __syncwarp();
         if (lane == 0) mbar_arrive(&rho_empty[rs_slot]);
       }
-      // ---- item end: combine halves, write m, count the unit's finished blocks
-      float tot = (s0 + s1) + (s2 + s3);
-      if (half == 1) rowx[rloc] = tot;
-      named_bar_sync(3, 256);
-      if (half == 0 && i < c) {
-        tot += rowx[rloc];
+      // ---- item end: combine the four column groups, write m, count finished blocks
+      float tot = kMax ? fmaxf(fmaxf(s0, s1), fmaxf(s2, s3)) : (s0 + s1) + (s2 + s3);
+      if (cg > 0) rowx[(cg - 1) * 128 + rloc] = tot;
+      named_bar_sync(3, 512);
+      if (cg == 0 && i < c) {
         const float rho_i = __ldg(&p.rho[__ldg(&p.rho_off[u]) + i]);
-        p.m_dst[base + i] = rho_i * tot / static_cast<float>(N - 1);
+        if constexpr (kMax) {
+          tot = fmaxf(fmaxf(tot, rowx[rloc]), fmaxf(rowx[128 + rloc], rowx[256 + rloc]));
+          p.m_dst[base + i] = rho_i * tot;
+        } else {
+          tot += (rowx[rloc] + rowx[128 + rloc]) + rowx[256 + rloc];
+          p.m_dst[base + i] = rho_i * tot / static_cast<float>(N - 1);
+        }
       }
       __threadfence();
-      named_bar_sync(3, 256);
+      named_bar_sync(3, 512);
       if (etid == 0) {
         const int nblk = __ldg(&p.item_off[u + 1]) - __ldg(&p.item_off[u]);
         const int done = atomicAdd(&p.unit_cnt[u], 1) + 1;
         *last_flag = done == nblk * (kPair ? 2 : 1);
       }
-      named_bar_sync(3, 256);
+      named_bar_sync(3, 512);
       if (*last_flag) {
         // ---- token softmax over the unit's candidates (|m| <= 1: no max shift)
         __threadfence();
         float sum = 0.f;
-        for (int ii = etid; ii < c; ii += 256) sum += ex2(__ldcg(&p.m_dst[base + ii]) * kLog2e);
+        for (int ii = etid; ii < c; ii += 512) sum += ex2(__ldcg(&p.m_dst[base + ii]) * kLog2e);
         sum = warp_reduce_sum(sum);
-        if (lane == 0) fin[warp - 4] = sum;
-        named_bar_sync(3, 256);
+        if (lane == 0) fin[ew] = sum;
+        named_bar_sync(3, 512);
         float totl = 0.f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) totl += fin[k];
+        for (int k = 0; k < 16; ++k) totl += fin[k];
         const float inv = 1.f / totl;
-        for (int ii = etid; ii < c; ii += 256)
+        for (int ii = etid; ii < c; ii += 512)
           p.r_dst[base + ii] = ex2(__ldcg(&p.m_dst[base + ii]) * kLog2e) * inv;
-        named_bar_sync(3, 256);
+        named_bar_sync(3, 512);
       }
     }
   }
@@ -383,17 +424,30 @@ __global__ void plan_kernel(const int64_t* tok_off, int U, int w, int rows_per_i
 
 }  // namespace
 
-cudaError_t gemm_configure(bool pair) {
+#ifdef RKV_TRACE
+cudaError_t gemm_trace_read(void* dst, size_t bytes) {
+  return cudaMemcpyFromSymbol(dst, g_gemm_trace, bytes);
+}
+#endif
+
+namespace {
+void* gemm_fn(bool pair, bool rowmax) {
+  if (pair) return rowmax ? reinterpret_cast<void*>(&redundancy_gemm_kernel<true, true>)
+                          : reinterpret_cast<void*>(&redundancy_gemm_kernel<true, false>);
+  return rowmax ? reinterpret_cast<void*>(&redundancy_gemm_kernel<false, true>)
+                : reinterpret_cast<void*>(&redundancy_gemm_kernel<false, false>);
+}
+}  // namespace
+
+cudaError_t gemm_configure(bool pair, bool rowmax) {
   const int smem = (pair ? gemm_layout<true>().total : gemm_layout<false>().total) + 1024;
-  void* f = pair ? reinterpret_cast<void*>(&redundancy_gemm_kernel<true>)
-                 : reinterpret_cast<void*>(&redundancy_gemm_kernel<false>);
-  return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return cudaFuncSetAttribute(gemm_fn(pair, rowmax), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              smem);
 }
 
-int gemm_max_ctas(bool pair) {
+int gemm_max_ctas(bool pair, bool rowmax) {
   const int smem = (pair ? gemm_layout<true>().total : gemm_layout<false>().total) + 1024;
-  void* f = pair ? reinterpret_cast<void*>(&redundancy_gemm_kernel<true>)
-                 : reinterpret_cast<void*>(&redundancy_gemm_kernel<false>);
+  void* f = gemm_fn(pair, rowmax);
   int dev = 0, nsm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -431,7 +485,7 @@ cudaError_t launch_plan(const int64_t* tok_off, int U, int w, int rows_per_item,
 }
 
 cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const GemmParams& p,
-                        bool pair, int nctas, cudaStream_t st) {
+                        bool pair, bool rowmax, int nctas, cudaStream_t st) {
   const int smem = (pair ? gemm_layout<true>().total : gemm_layout<false>().total) + 1024;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nctas, 1, 1);
@@ -445,8 +499,12 @@ cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const 
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = pair ? 1 : 0;
-  if (pair) return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<true>, amap, bmap, p);
-  return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<false>, amap, bmap, p);
+  if (pair) {
+    if (rowmax) return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<true, true>, amap, bmap, p);
+    return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<true, false>, amap, bmap, p);
+  }
+  if (rowmax) return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<false, true>, amap, bmap, p);
+  return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<false, false>, amap, bmap, p);
 }
 
 }  // namespace rkv

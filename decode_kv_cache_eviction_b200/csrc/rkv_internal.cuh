@@ -13,7 +13,7 @@ constexpr int kTileBytes = kTile * kHeadDim * 2;
 constexpr int kMaxTokensPerUnit = 49152;  // select keeps a unit's keys in shared memory
 constexpr int kMaxRows = 32;         // G * w limit (MMA N of the logits tile)
 constexpr int kScoreThreads = 512;   // 16 warps
-constexpr int kGemmThreads = 384;
+constexpr int kGemmThreads = 640;    // producer, MMA, 2 idle, 16 epilogue warps
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------- score
@@ -138,7 +138,7 @@ __host__ __device__ inline GemmLayout gemm_layout() {
   L.a = o; o += C::kABytes;
   L.b = o; o += C::kStages * C::kBBytes;
   L.rho = o; o += kRhoSlots * 256 * 4;
-  L.rowx = o; o += 128 * 4;
+  L.rowx = o; o += 4 * 128 * 4;
   L.fin = o; o += 32 * 4;
   L.bars = o; o += (2 + 2 * C::kStages + 4 + 2 * kRhoSlots) * 8;
   L.slot = o; o += 16;
@@ -157,9 +157,9 @@ int score_max_clusters(int rp, bool closed, int smem_bytes, int cs);
 cudaError_t launch_plan(const int64_t* tok_off, int U, int w, int rows_per_item, int* item_off,
                         int* unit_cnt, int64_t* rho_off, cudaStream_t st);
 cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const GemmParams& p,
-                        bool pair, int nctas, cudaStream_t st);
-cudaError_t gemm_configure(bool pair);
-int gemm_max_ctas(bool pair);
+                        bool pair, bool rowmax, int nctas, cudaStream_t st);
+cudaError_t gemm_configure(bool pair, bool rowmax);
+int gemm_max_ctas(bool pair, bool rowmax);
 
 cudaError_t launch_select(const int64_t* tok_off, int U, int w, int cmax, const float* a,
                           const float* r, float lam, int budget, int32_t* idx, int32_t* n_kept,

@@ -80,6 +80,11 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       if (tid == 0) n_kept[u] = N;
       continue;
     }
+    if (budget == 0) {  // only the window is kept (the radix step needs want >= 1)
+      for (int t = tid; t < w; t += kSelThreads) out[t] = c + t;
+      if (tid == 0) n_kept[u] = w;
+      continue;
+    }
 
     // ---- 1. keys, min and max
     uint32_t kmin = 0xffffffffu, kmax = 0u;
@@ -198,7 +203,8 @@ __global__ void __launch_bounds__(kSelThreads, 1)
           int slot = 0;
           if (lane == 0 && bal) slot = atomicAdd(&sh[3], __popc(bal));
           slot = __shfl_sync(0xffffffffu, slot, 0);
-          if (m) list[slot + __popc(bal & ((1u << lane) - 1u))] = k;
+          const int pos = slot + __popc(bal & ((1u << lane) - 1u));
+          if (m && pos < kListCap) list[pos] = k;
         }
         __syncthreads();
         nlist = sh[3];
@@ -245,7 +251,8 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       const unsigned be = __ballot_sync(0xffffffffu, e);
       const bool f = g || (e && eseen + __popc(be & lt) < take_eq);
       const unsigned bf = __ballot_sync(0xffffffffu, f);
-      if (f) out[oseen + __popc(bf & lt)] = i;
+      const int pos = oseen + __popc(bf & lt);
+      if (f && pos < budget) out[pos] = i;
       eseen += __popc(be);
       oseen += __popc(bf);
     }

@@ -46,7 +46,7 @@ extern "C" {
 #endif
 
 typedef struct CUstream_st* rkv_stream_t; /* identical to cudaStream_t */
-typedef struct rkv_engine rkv_engine;     /* opaque; owns device workspace only */
+typedef struct rkv_engine rkv_engine;     /* opaque; owns its workspace and staging */
 
 enum {
   RKV_OK = 0,
@@ -59,14 +59,19 @@ enum {
   RKV_ERR_DEVICE = -7       /* a kept index outside its unit (see rkv_check_status) */
 };
 
-/* How rkv_score computes the redundancy row mean m_i. */
+/* How rkv_score computes the redundancy m_i. */
 enum {
   /* Tensor-core K K^T tile products with the norm scaling, diagonal mask,
    * row mean and token softmax fused into the epilogue (N x N never stored). */
   RKV_REDUNDANCY_GEMM = 0,
   /* The same m_i by linearity of the row sum:
    * sum_{j != i} khat_i . khat_j = khat_i . (sum_j khat_j) - khat_i . khat_i. */
-  RKV_REDUNDANCY_CLOSED_FORM = 1
+  RKV_REDUNDANCY_CLOSED_FORM = 1,
+  /* Nearest-duplicate reading of the cosine-similarity redundancy (R-KV,
+   * "冗余打分"): m_i = max_{j != i, j < N} khat_i . khat_j, from the same
+   * tensor-core tiles with a max fold in the epilogue.  A token with an exact
+   * copy anywhere in the unit gets m_i = 1. */
+  RKV_REDUNDANCY_MAX = 2
 };
 
 typedef struct {
@@ -75,7 +80,7 @@ typedef struct {
   int window;         /* w >= 1: window queries and always-kept tail tokens */
   int max_units;      /* capacity: units per batch (>= 1) */
   int64_t max_tokens; /* capacity: total cached rows per batch (>= 1) */
-  int redundancy;     /* RKV_REDUNDANCY_GEMM or RKV_REDUNDANCY_CLOSED_FORM */
+  int redundancy;     /* RKV_REDUNDANCY_GEMM, _CLOSED_FORM or _MAX */
   int flags;          /* 0, or RKV_FLAG_* bits */
 } rkv_config;
 
@@ -106,9 +111,10 @@ int rkv_destroy(rkv_engine* eng);
  *   a [T] fp32: a_i = abar_i / sum_{j in C} abar_j for i in C, where
  *               abar_i = mean over (g, t) of softmax_j(q_{g,t} . k_j / sqrt(d))[i];
  *   r [T] fp32: r_i = exp(m_i) / sum_{j in C} exp(m_j) for i in C, where
- *               m_i = sum_{j != i, j < N} khat_i . khat_j / (N - 1),
+ *               m_i = sum_{j != i, j < N} khat_i . khat_j / (N - 1)
+ *               (RKV_REDUNDANCY_MAX: m_i = max_{j != i, j < N} khat_i . khat_j),
  *               khat = k / ||k|| (0 for a zero key);
- *   m [T] fp32, optional (NULL to skip): the row means m_i.
+ *   m [T] fp32, optional (NULL to skip): the m_i.
  * Row tok_off[u] + i holds token i of unit u; window rows (i >= N_u - w) are 0. */
 int rkv_score(rkv_engine* eng, const rkv_batch* batch, float* a, float* r, float* m,
               rkv_stream_t stream);
@@ -136,6 +142,41 @@ int rkv_compact(rkv_engine* eng, const rkv_batch* batch, const int32_t* idx,
 int rkv_compress(rkv_engine* eng, const rkv_batch* batch, float lambda, int budget,
                  float* a, float* r, int32_t* idx, int32_t* n_kept, void* K_out,
                  void* V_out, rkv_stream_t stream);
+
+/* A batch in HOST memory (rkv_compress_host).  Same layouts as rkv_batch. */
+typedef struct {
+  int num_units;               /* U >= 0 */
+  const int64_t* tok_off;      /* host [U+1]: row offsets, tok_off[0] = 0, nondecreasing */
+  const void* K;               /* host bf16 [T, d] keys */
+  const void* V;               /* host bf16 [T, d] values */
+  const void* Q;               /* host bf16 [U, G, w, d] window queries */
+} rkv_host_batch;
+
+/* rkv_compress from host buffers to host buffers (the path a caller with the
+ * cache in host memory takes; the paper has no counterpart).  Units are cut
+ * into chunks of at most `chunk_tokens` rows (0 selects 1,048,576; raised to the
+ * longest unit and to budget + w if smaller) and at most max_units units, and
+ * the chunks are pipelined through two device staging slots on three internal
+ * streams: copy-in of chunk i+1, scoring / selection / compaction of chunk i and
+ * copy-out of chunk i-1 overlap.  Results equal those of rkv_compress on the
+ * same units, bit for bit.
+ *   idx [U, budget + w] int32, n_kept [U] int32, K_out / V_out bf16
+ *   [U, budget + w, d]: HOST outputs, laid out as for rkv_select / rkv_compact.
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister) for the
+ * copies to overlap; pageable memory works but serialises them.  Everything is
+ * ordered after earlier work on `stream`, and later work on `stream` runs after
+ * the last copy-out; the host buffers must stay untouched until then (e.g.
+ * until rkv_check_status(eng, stream) returns).  The staging (about
+ * 4 * chunk_tokens * 512 bytes of device memory and U + chunks page-locked
+ * int64) is allocated on the first call, grown when a call needs more, and
+ * freed by rkv_destroy.  A call first waits on the host for the engine's
+ * previous rkv_compress_host call to finish.  Not capturable in a CUDA graph.
+ * Errors: those of rkv_compress (all validation happens before anything is
+ * enqueued), RKV_ERR_CAPACITY when one chunk cannot fit the engine's
+ * max_tokens, RKV_ERR_OOM when the staging cannot be allocated. */
+int rkv_compress_host(rkv_engine* eng, const rkv_host_batch* batch, float lambda, int budget,
+                      int32_t* idx, int32_t* n_kept, void* K_out, void* V_out,
+                      int64_t chunk_tokens, rkv_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the engine's device status word:
  * RKV_OK, RKV_ERR_TIMEOUT (a device wait gave up; outputs are invalid) or

@@ -23,6 +23,25 @@ ATOL, RTOL = 1e-6, 1e-3
 SEL_BAND = 1e-5
 
 
+def rand_batch(lengths, G, w, seed=0, dup=0.2, zero_rows=(), device="cuda:0"):
+    """Gaussian keys, values and queries for units of the given lengths; a
+    fraction ``dup`` of each unit's rows are exact copies of earlier rows."""
+    rng = np.random.default_rng(seed)
+    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    T = int(off[-1])
+    K = rng.standard_normal((T, 128)).astype(np.float32)
+    for u in range(len(lengths)):
+        for i in range(1, lengths[u]):
+            if rng.random() < dup:
+                K[off[u] + i] = K[off[u] + rng.integers(0, i)]
+    for z in zero_rows:
+        K[z] = 0
+    V = rng.standard_normal((T, 128)).astype(np.float32)
+    Q = rng.standard_normal((len(lengths), G, w, 128)).astype(np.float32)
+    t = lambda x: torch.from_numpy(x).to(device).to(torch.bfloat16)
+    return Batch(t(K), t(V), t(Q), off)
+
+
 def make_batch(gen_batch: W.Batch) -> Batch:
     return Batch(gen_batch.K, gen_batch.V, gen_batch.Q, gen_batch.tok_off)
 
@@ -65,8 +84,14 @@ def close(x_gpu, x_ora, what):
                            f"oracle={x_ora[bad[:5]].tolist()}")
 
 
+def oracle_mode(mode):
+    """The oracle redundancy that an engine mode computes."""
+    return "max" if mode == "max" else "closed"
+
+
 def check_unit(out, batch: Batch, u, w, lam, budget, redundancy="closed", check_m=True):
-    """Compare unit u of an engine run with the oracle."""
+    """Compare unit u of an engine run with the oracle.  ``redundancy`` names the
+    oracle function: ``closed`` / ``rowblocks`` (row mean) or ``max`` (row max)."""
     k, v, q = unit_inputs(batch, u)
     N = k.shape[0]
     c = N - w
@@ -74,6 +99,8 @@ def check_unit(out, batch: Batch, u, w, lam, budget, redundancy="closed", check_
     _, a_o = ora.importance(q, k)
     if redundancy == "closed":
         m_o, r_o = ora.redundancy_mean_closed_form(k, w)
+    elif redundancy == "max":
+        m_o, r_o = ora.redundancy_max(k, w)
     else:
         m_o, r_o = ora.redundancy_mean(k, w)
     a_g = out["a"][r0:r0 + N]

@@ -57,6 +57,9 @@ def test_struct_layout_matches_header():
       printf("%zu %zu %zu %zu %zu\n", offsetof(rkv_batch, tok_off),
              offsetof(rkv_batch, tok_off_host), offsetof(rkv_batch, K),
              offsetof(rkv_batch, V), offsetof(rkv_batch, Q));
+      printf("%zu %zu %zu %zu %zu\n", sizeof(rkv_host_batch), offsetof(rkv_host_batch, tok_off),
+             offsetof(rkv_host_batch, K), offsetof(rkv_host_batch, V),
+             offsetof(rkv_host_batch, Q));
       return 0;
     }
     """
@@ -74,6 +77,9 @@ def test_struct_layout_matches_header():
                      C.flags.offset, ctypes.sizeof(Bt)]
     assert want2 == [Bt.tok_off.offset, Bt.tok_off_host.offset, Bt.K.offset, Bt.V.offset,
                      Bt.Q.offset]
+    H = B.RkvHostBatch
+    want3 = [int(x) for x in lines[2].split()]
+    assert want3 == [ctypes.sizeof(H), H.tok_off.offset, H.K.offset, H.V.offset, H.Q.offset]
 
 
 def test_status_strings_and_version():
@@ -119,6 +125,8 @@ def test_null_arguments():
     assert L.rkv_select(None, None, None, None, 0.1, 4, None, None, None) == B.RKV_ERR_INVALID_ARG
     assert L.rkv_compact(None, None, None, None, 4, None, None, None) == B.RKV_ERR_INVALID_ARG
     assert L.rkv_check_status(None, None) == B.RKV_ERR_INVALID_ARG
+    assert L.rkv_compress_host(None, None, 0.1, 4, None, None, None, None, 0,
+                               None) == B.RKV_ERR_INVALID_ARG
     assert L.rkv_destroy(None) == B.RKV_OK
     assert L.rkv_launch_count(None) == 0
 

@@ -12,27 +12,10 @@ from decode_kv_cache_eviction_b200 import Batch, Engine, RkvError
 from decode_kv_cache_eviction_b200 import workloads as W
 from oracle import rkv_oracle as ora
 
-from parity import check_unit, make_batch, run_engine
+from parity import check_unit, make_batch, oracle_mode, rand_batch, run_engine
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
-
-
-def rand_batch(lengths, G, w, seed=0, dup=0.2, zero_rows=()):
-    rng = np.random.default_rng(seed)
-    off = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
-    T = int(off[-1])
-    K = rng.standard_normal((T, 128)).astype(np.float32)
-    for u in range(len(lengths)):
-        for i in range(1, lengths[u]):
-            if rng.random() < dup:
-                K[off[u] + i] = K[off[u] + rng.integers(0, i)]
-    for z in zero_rows:
-        K[z] = 0
-    V = rng.standard_normal((T, 128)).astype(np.float32)
-    Q = rng.standard_normal((len(lengths), G, w, 128)).astype(np.float32)
-    t = lambda x: torch.from_numpy(x).to(DEV).to(torch.bfloat16)
-    return Batch(t(K), t(V), t(Q), off)
 
 
 # ----------------------------------------------------------------- select alone
@@ -117,10 +100,14 @@ def test_worked_example_on_gpu():
             np.testing.assert_allclose(out["r"][:4], g["r"], atol=5e-6)
             np.testing.assert_allclose(out["m"][:4], g["m"], atol=5e-6)
             assert out["idx"][0].tolist() == want, (mode, lam)
+    # row max: nearest other unit key of each candidate, 1, 1, 1/sqrt(2), 0
+    out = run_engine(b, 1, 2, 0.1, 2, mode="max")
+    np.testing.assert_allclose(out["m"][:4], [1.0, 1.0, 0.5 ** 0.5, 0.0], atol=5e-6)
+    np.testing.assert_allclose(out["a"][:4], g["a"], atol=5e-6)
 
 
 # ----------------------------------------------------------------- score kernels, small
-@pytest.mark.parametrize("mode", ["closed", "gemm"])
+@pytest.mark.parametrize("mode", ["closed", "gemm", "max"])
 @pytest.mark.parametrize("G,w", [(1, 8), (4, 8), (2, 3), (5, 5), (1, 1), (32, 1)])
 def test_score_small_ragged(mode, G, w):
     lengths = [w, w + 1, 127, 128, 129, 1000, 2500, 5000]
@@ -130,10 +117,27 @@ def test_score_small_ragged(mode, G, w):
     for lam in (0.1,):
         out = run_engine(b, G, w, lam, budget, mode=mode)
         for u in range(len(lengths)):
-            check_unit(out, b, u, w, lam, budget)
+            check_unit(out, b, u, w, lam, budget, redundancy=oracle_mode(mode))
 
 
-@pytest.mark.parametrize("mode", ["closed", "gemm"])
+def test_row_max_flags_every_duplicate():
+    """Row max: a candidate with an exact copy anywhere in its unit (window
+    included) scores m = 1 up to fp32 rounding; the others stay well below."""
+    lengths = [700, 3000, 129]
+    b = rand_batch(lengths, 4, 8, seed=31, dup=0.25)
+    out = run_engine(b, 4, 8, 0.1, 64, mode="max")
+    K = b.K.float().cpu().numpy()
+    for u, n in enumerate(lengths):
+        r0 = int(b.tok_off_host[u])
+        rows = K[r0:r0 + n]
+        _, inv, cnt = np.unique(rows, axis=0, return_inverse=True, return_counts=True)
+        has_copy = cnt[inv.reshape(-1)] > 1
+        m = out["m"][r0:r0 + n - 8]
+        assert np.all(np.abs(m[has_copy[:n - 8]] - 1.0) < 1e-5)
+        assert np.all(m[~has_copy[:n - 8]] < 0.7)
+
+
+@pytest.mark.parametrize("mode", ["closed", "gemm", "max"])
 def test_budget_edges(mode):
     lengths = [300, 300, 300]
     w = 8
@@ -141,7 +145,7 @@ def test_budget_edges(mode):
     for budget in (0, 1, 291, 292, 300):
         out = run_engine(b, 4, w, 0.1, budget, mode=mode)
         for u in range(3):
-            check_unit(out, b, u, w, 0.1, budget)
+            check_unit(out, b, u, w, 0.1, budget, redundancy=oracle_mode(mode))
 
 
 def test_gemm_single_cta_and_pair_agree():
@@ -153,6 +157,12 @@ def test_gemm_single_cta_and_pair_agree():
         check_unit(o1, b, u, 8, 0.1, 256)
     np.testing.assert_allclose(o1["m"], o2["m"], rtol=1e-5, atol=1e-7)
     np.testing.assert_allclose(o2["r"], o3["r"], rtol=1e-4, atol=1e-9)
+    x1 = run_engine(b, 4, 8, 0.1, 256, mode="max", single_cta=True)
+    x2 = run_engine(b, 4, 8, 0.1, 256, mode="max", single_cta=False)
+    for u in range(3):
+        check_unit(x1, b, u, 8, 0.1, 256, redundancy="max")
+    # the same tile products and one max order per row: identical results
+    assert np.array_equal(x1["m"], x2["m"])
 
 
 @pytest.mark.parametrize("G,N", [(4, 32768), (2, 49152)])
@@ -160,9 +170,9 @@ def test_largest_supported_unit(G, N):
     # logits of a unit stay in tensor memory: 32768 tokens at G*w = 32,
     # 49152 (the select limit) at G*w <= 16
     b = rand_batch([N], G, 8, seed=1, dup=0.0)
-    for mode in ("closed", "gemm"):
+    for mode in ("closed", "gemm", "max"):
         out = run_engine(b, G, 8, 0.1, 4096, mode=mode)
-        check_unit(out, b, 0, 8, 0.1, 4096)
+        check_unit(out, b, 0, 8, 0.1, 4096, redundancy=oracle_mode(mode))
 
 
 def test_rejects_too_long_unit_and_capacity():
@@ -194,7 +204,7 @@ def test_rejects_too_long_unit_and_capacity():
 
 def test_repeated_calls_are_deterministic():
     b = rand_batch([4000, 6000], 4, 8, seed=5)
-    for mode in ("closed", "gemm"):
+    for mode in ("closed", "gemm", "max"):
         eng = Engine(4, 8, max_units=2, max_tokens=b.num_tokens, redundancy=mode)
         o1 = run_engine(b, 4, 8, 0.1, 512, engine=eng)
         o2 = run_engine(b, 4, 8, 0.1, 512, engine=eng)
@@ -214,18 +224,18 @@ def _sampled(name, n_sample, modes=("gemm", "closed")):
         for lam in wl.lambdas:
             out = run_engine(b, wl.group, wl.window, lam, wl.budget, mode=mode)
             for u in units:
-                check_unit(out, b, u, wl.window, lam, wl.budget)
+                check_unit(out, b, u, wl.window, lam, wl.budget, redundancy=oracle_mode(mode))
             del out
             torch.cuda.empty_cache()
     return b, units
 
 
 def test_workload_tiny_full():
-    _sampled("tiny", 1)
+    _sampled("tiny", 1, modes=("gemm", "closed", "max"))
 
 
 def test_workload_llama3_layer_full():
-    _sampled("llama3_8b_layer", 8)
+    _sampled("llama3_8b_layer", 8, modes=("gemm", "closed", "max"))
 
 
 def test_workload_tiny_definition_redundancy():
@@ -248,4 +258,4 @@ def test_workload_long_trace_32k_sampled():
 
 @pytest.mark.slow
 def test_workload_ragged_serving_sampled():
-    _sampled("ragged_serving", 8)
+    _sampled("ragged_serving", 8, modes=("gemm", "closed", "max"))
