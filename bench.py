@@ -398,12 +398,26 @@ def measure_e2e(eng, batch: Batch, wl: W.Workload, args, dist: Dist):
     eng.score(batch, a, r)
     eng.select(batch, a, r, args.lam, wl.budget, idx, nk)
     ok = torch.equal(outs[1], nk.cpu()) and torch.equal(outs[0], idx.cpu())
-    h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hQ)) + 8 * len(off)
+    # V crosses the bus whole only when it is not mapped into the device
+    # address space; otherwise the compaction kernel reads the kept rows only
+    v_mapped = _mapped_host(hV)
+    v_bytes = (int(outs[1].sum()) * hV.shape[1] * hV.element_size() if v_mapped
+               else hV.numel() * hV.element_size())
+    h2d = sum(t.numel() * t.element_size() for t in (hK, hQ)) + v_bytes + 8 * len(off)
     d2h = sum(t.numel() * t.element_size() for t in outs)
     return {"value": batch.num_tokens * dist.world / (ms * 1e-3), "unit": UNIT,
             "ms_per_step": ms, "steps": args.e2e_steps, "warmup": 1,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "api": "rkv_compress_host", "outputs_consistent": bool(ok)}
+            "api": "rkv_compress_host", "v_rows_moved": "kept" if v_mapped else "all",
+            "outputs_consistent": bool(ok)}
+
+
+def _mapped_host(t: torch.Tensor) -> bool:
+    """Whether a host tensor is page-locked and visible to the device."""
+    from cuda.bindings import runtime as rt
+    err, attr = rt.cudaPointerGetAttributes(t.data_ptr())
+    return (err == rt.cudaError_t.cudaSuccess and
+            attr.type == rt.cudaMemoryType.cudaMemoryTypeHost and attr.devicePointer != 0)
 
 
 def main():

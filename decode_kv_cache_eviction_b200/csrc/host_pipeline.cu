@@ -6,7 +6,14 @@
 //   compute  : [wait in(i), copy-out(i-2) done] score, select, compact [comp(i)]
 //   copy-out : [wait comp(i)] idx, n_kept, K_out, V_out -> host        [out(i)]
 // Compute is serial on its stream, so the engine's workspace and the shared
-// score scratch are never used by two chunks at once.  A chunk's results are
+// score scratch are never used by two chunks at once.
+//
+// V is needed only for the kept rows (B + w of each unit's N).  When the
+// caller's V is page-locked and mapped into the device address space (every
+// cudaHostAlloc / cudaMallocHost allocation on a 64-bit system with unified
+// addressing), the compaction kernel gathers the kept rows straight from host
+// memory and V is never copied in whole; otherwise each chunk's V is copied
+// like K.  A chunk's results are
 // independent of how the units were split (every kernel works per unit), so
 // the outputs equal those of one rkv_compress over the whole batch.
 #include <algorithm>
@@ -194,6 +201,17 @@ extern "C" int rkv_compress_host(rkv_engine* e, const rkv_host_batch* hb, float 
   }
 
   const int64_t R = static_cast<int64_t>(e->cfg.group) * w;
+  // device view of a page-locked, mapped V (nullptr: copy V chunk by chunk)
+  const char* dV = nullptr;
+  {
+    cudaPointerAttributes pa;
+    if (cudaPointerGetAttributes(&pa, hb->V) == cudaSuccess) {
+      if (pa.type == cudaMemoryTypeHost && pa.devicePointer != nullptr)
+        dV = static_cast<const char*>(pa.devicePointer);
+    } else {
+      cudaGetLastError();   // pageable memory unknown to CUDA: copy it
+    }
+  }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaStream_t s_in = e->hs[0], s_comp = e->hs[1], s_out = e->hs[2];
   auto fail = [&](cudaError_t err) {
@@ -219,7 +237,7 @@ extern "C" int rkv_compress_host(rkv_engine* e, const rkv_host_batch* hb, float 
       return fail(cudaErrorUnknown);
     cudaError_t err = cudaMemcpyAsync(sl.K, hK + c.r0 * kRowBytes, c.rows * kRowBytes,
                                       cudaMemcpyHostToDevice, s_in);
-    if (err == cudaSuccess)
+    if (err == cudaSuccess && !dV)
       err = cudaMemcpyAsync(sl.V, hV + c.r0 * kRowBytes, c.rows * kRowBytes,
                             cudaMemcpyHostToDevice, s_in);
     if (err == cudaSuccess)
@@ -239,7 +257,7 @@ extern "C" int rkv_compress_host(rkv_engine* e, const rkv_host_batch* hb, float 
     b.tok_off = sl.off;
     b.tok_off_host = e->h_off_pinned + c.off_at;
     b.K = sl.K;
-    b.V = sl.V;
+    b.V = dV ? static_cast<const void*>(dV + c.r0 * kRowBytes) : sl.V;
     b.Q = sl.Q;
     rc = rkv_compress(e, &b, lambda, budget, e->h_a, e->h_r, sl.idx, sl.nk, sl.Ko, sl.Vo,
                       reinterpret_cast<rkv_stream_t>(s_comp));

@@ -356,6 +356,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
       : RKV_R8(0), RKV_R8(8), RKV_R8(16), RKV_R8(24)
       : "r"(taddr));
 }
+// 16 lanes x 256-bit, repeated over 8 groups of 8 consecutive columns (64
+// columns).  Thread t receives, for repeat i (columns 8i .. 8i+7 of the
+// access), v[4i], v[4i+1] = lane t/4, columns 8i + 2(t%4) + {0, 1} and
+// v[4i+2], v[4i+3] = lane t/4 + 8, the same columns.
+__device__ __forceinline__ void tmem_ld16x256b_x8(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : RKV_R8(0), RKV_R8(8), RKV_R8(16), RKV_R8(24)
+      : "r"(taddr));
+}
 #undef RKV_R8
 
 // ---------------------------------------------------------------- misc

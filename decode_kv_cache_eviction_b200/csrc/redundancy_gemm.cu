@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int ew = warp - 4;              // epilogue warp 0..15
     const int cg = ew >> 2;               // 64-column group of the tile
     const int q = warp & 3;               // TMEM lane quarter
-    const int rloc = q * 32 + lane;       // row of this CTA's A block
+    const int gq = lane >> 2, tq = lane & 3;   // quad and thread within it
     const float* rho_ring = reinterpret_cast<const float*>(sm + L.rho);
     float* rowx = reinterpret_cast<float*>(sm + L.rowx);
     float* fin = reinterpret_cast<float*>(sm + L.fin);
@@ -245,59 +245,74 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int N = static_cast<int>(__ldg(&p.tok_off[u + 1]) - base);
       const int c = N - p.w;
       const int rbase = blk * C::kRowsPerItem + rank * 128;   // unit-local first row
-      const int i = rbase + rloc;
+      // Each thread accumulates 4 rows of its lane quarter (gq, gq + 8, gq + 16,
+      // gq + 24) over its 16 columns of each 64-column group (8i + 2tq + {0,1}),
+      // two partial values per row.
       constexpr float kInit = kMax ? -INFINITY : 0.f;
-      float s0 = kInit, s1 = kInit, s2 = kInit, s3 = kInit;
+      float a0 = kInit, b0 = kInit, a1 = kInit, b1 = kInit;
+      float a2 = kInit, b2 = kInit, a3 = kInit, b3 = kInit;
       const int ntiles = (N + C::kN - 1) / C::kN;
       for (int t = 0; t < ntiles; ++t, ++rt) {
         const int j0 = t * C::kN;
         const uint32_t rs_slot = rt % kRhoSlots;
-        const float* rs = rho_ring + rs_slot * 256 + cg * 64;
+        const float* rs = rho_ring + rs_slot * 256 + cg * 64 + 2 * tq;
         if (etid == 0) RKV_GSTAMP(1, rt, 0);
         mbar_wait(&acc_full[ab], aph, abort, p.status);
         mbar_wait(&rho_full[rs_slot], (rt / kRhoSlots) & 1, abort, p.status);
         if (etid == 0) RKV_GSTAMP(1, rt, 1);
         __syncwarp();
         tc_fence_after();
+        // this thread's 16 column weights: 8 shared-memory reads per tile, 4x
+        // fewer than one row per thread over all 64 columns would need
+        float2 wt[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) wt[k] = *reinterpret_cast<const float2*>(rs + 8 * k);
         const uint32_t tbase =
             tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + cg * 64;
         const int cw0 = j0 + cg * 64;                // first column of this warp's group
-        const int rw0 = rbase + q * 32;              // first row of this warp
+        const int rw0 = rbase + q * 32;              // first row of this warp's quarter
         const bool masked = ((rw0 < cw0 + 64) && (cw0 < rw0 + 32)) || (kMax && cw0 + 64 > N);
-        const int jd = i - cw0;
-        const int jn = kMax ? N - cw0 : 64;
+        const int dd = rw0 - cw0;                    // diagonal: column - row == dd
+        const int jn = kMax ? N - cw0 : 64;          // first column past the unit
         constexpr uint32_t neutral = kMax ? 0xff800000u : 0u;   // -inf, or 0
-        // 32 columns at a time, so that the values, four partial sums and the
-        // weights fit the 96 registers a thread has at 640 threads per CTA.
-        // Masked groups (rare): the diagonal column i - cw0 and, for the row
-        // max, the columns past the unit are neutralised (-inf * rho is -inf or
-        // NaN, both ignored by fmaxf).  Sums use packed fp32x2 FMAs.
         uint32_t v[32];
-        auto half = [&](int off) {
-          if (masked) {
+        // Masked groups (rare): the diagonal and, for the row max, the columns
+        // past the unit are neutralised (-inf * rho is -inf or NaN, both
+        // ignored by fmaxf).  h selects the 16-lane half of the quarter.
+        auto patch = [&](int h) {
 #pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (k + off == jd || k + off >= jn) v[k] = neutral;
-          }
+          for (int k = 0; k < 8; ++k)
 #pragma unroll
-          for (int cc = 0; cc < 32; cc += 4) {
-            const float4 r4 = *reinterpret_cast<const float4*>(rs + off + cc);
+            for (int e = 0; e < 4; ++e) {
+              const int col = 8 * k + 2 * tq + (e & 1);
+              const int row = 16 * h + gq + ((e >> 1) << 3);
+              if (col - row == dd || col >= jn) v[4 * k + e] = neutral;
+            }
+        };
+        auto fold = [&](float& pa, float& pb, float& qa, float& qb) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
             if constexpr (kMax) {
-              float p0, p1, p2, p3;
-              mul2(p0, p1, __uint_as_float(v[cc + 0]), __uint_as_float(v[cc + 1]), r4.x, r4.y);
-              mul2(p2, p3, __uint_as_float(v[cc + 2]), __uint_as_float(v[cc + 3]), r4.z, r4.w);
-              s0 = fmaxf(s0, p0); s1 = fmaxf(s1, p1); s2 = fmaxf(s2, p2); s3 = fmaxf(s3, p3);
+              float x0, x1, y0, y1;
+              mul2(x0, x1, __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]), wt[k].x,
+                   wt[k].y);
+              mul2(y0, y1, __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]), wt[k].x,
+                   wt[k].y);
+              pa = fmaxf(pa, x0); pb = fmaxf(pb, x1); qa = fmaxf(qa, y0); qb = fmaxf(qb, y1);
             } else {
-              fma2(s0, s1, __uint_as_float(v[cc + 0]), __uint_as_float(v[cc + 1]), r4.x, r4.y);
-              fma2(s2, s3, __uint_as_float(v[cc + 2]), __uint_as_float(v[cc + 3]), r4.z, r4.w);
+              fma2(pa, pb, __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]), wt[k].x,
+                   wt[k].y);
+              fma2(qa, qb, __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]), wt[k].x,
+                   wt[k].y);
             }
           }
         };
-        tmem_ld32(tbase, v);
+        tmem_ld16x256b_x8(tbase, v);                 // lanes 0-15 of the quarter
         tmem_wait_ld();
         if (etid == 0) RKV_GSTAMP(1, rt, 2);
-        half(0);
-        tmem_ld32(tbase + 32, v);
+        if (masked) patch(0);
+        fold(a0, b0, a1, b1);
+        tmem_ld16x256b_x8(tbase + (16u << 16), v);   // lanes 16-31
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -306,22 +321,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           else mbar_arrive(&acc_empty[ab]);
         }
         if (++ab == 2) { ab = 0; aph ^= 1; }
-        half(32);
+        if (masked) patch(1);
+        fold(a2, b2, a3, b3);
         if (etid == 0) RKV_GSTAMP(1, rt, 3);
         __syncwarp();
         if (lane == 0) mbar_arrive(&rho_empty[rs_slot]);
       }
-      // ---- item end: combine the four column groups, write m, count finished blocks
-      float tot = kMax ? fmaxf(fmaxf(s0, s1), fmaxf(s2, s3)) : (s0 + s1) + (s2 + s3);
-      if (cg > 0) rowx[(cg - 1) * 128 + rloc] = tot;
+      // ---- item end: finish the rows over the quad (its four threads hold
+      // disjoint columns), combine the four column groups, write m
+      auto red = [](float x, float y) { return kMax ? fmaxf(x, y) : x + y; };
+      float t0 = red(a0, b0), t1 = red(a1, b1), t2 = red(a2, b2), t3 = red(a3, b3);
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        t0 = red(t0, __shfl_xor_sync(0xffffffffu, t0, o));
+        t1 = red(t1, __shfl_xor_sync(0xffffffffu, t1, o));
+        t2 = red(t2, __shfl_xor_sync(0xffffffffu, t2, o));
+        t3 = red(t3, __shfl_xor_sync(0xffffffffu, t3, o));
+      }
+      // thread tq of the quad owns row gq + 8 tq of the quarter
+      float tot = tq == 0 ? t0 : tq == 1 ? t1 : tq == 2 ? t2 : t3;
+      const int rl = q * 32 + gq + 8 * tq;           // row of this CTA's A block
+      const int i = rbase + rl;
+      if (cg > 0) rowx[(cg - 1) * 128 + rl] = tot;
       named_bar_sync(3, 512);
       if (cg == 0 && i < c) {
         const float rho_i = __ldg(&p.rho[__ldg(&p.rho_off[u]) + i]);
         if constexpr (kMax) {
-          tot = fmaxf(fmaxf(tot, rowx[rloc]), fmaxf(rowx[128 + rloc], rowx[256 + rloc]));
+          tot = fmaxf(fmaxf(tot, rowx[rl]), fmaxf(rowx[128 + rl], rowx[256 + rl]));
           p.m_dst[base + i] = rho_i * tot;
         } else {
-          tot += (rowx[rloc] + rowx[128 + rloc]) + rowx[256 + rloc];
+          tot += (rowx[rl] + rowx[128 + rl]) + rowx[256 + rl];
           p.m_dst[base + i] = rho_i * tot / static_cast<float>(N - 1);
         }
       }

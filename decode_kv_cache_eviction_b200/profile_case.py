@@ -15,7 +15,7 @@ from decode_kv_cache_eviction_b200 import Batch, Engine, workloads as W  # noqa:
 ap = argparse.ArgumentParser()
 ap.add_argument("--units", type=int, default=32)
 ap.add_argument("--n", type=int, default=32768)
-ap.add_argument("--mode", default="gemm", choices=["gemm", "closed"])
+ap.add_argument("--mode", default="gemm", choices=["gemm", "closed", "max"])
 ap.add_argument("--iters", type=int, default=3)
 a = ap.parse_args()
 wl = W.custom(name="long_trace_32k", n_kv_head=a.units, group=4, window=8, budget=4096,

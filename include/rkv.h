@@ -163,7 +163,10 @@ typedef struct {
  *   idx [U, budget + w] int32, n_kept [U] int32, K_out / V_out bf16
  *   [U, budget + w, d]: HOST outputs, laid out as for rkv_select / rkv_compact.
  * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister) for the
- * copies to overlap; pageable memory works but serialises them.  Everything is
+ * copies to overlap; pageable memory works but serialises them.  When V is
+ * page-locked and mapped into the device address space (cudaHostAlloc on a
+ * 64-bit system, or cudaHostRegister with cudaHostRegisterMapped), only the
+ * kept V rows cross the bus: the compaction kernel reads them from host memory.  Everything is
  * ordered after earlier work on `stream`, and later work on `stream` runs after
  * the last copy-out; the host buffers must stay untouched until then (e.g.
  * until rkv_check_status(eng, stream) returns).  The staging (about
