@@ -100,3 +100,11 @@ def run_unit(Q, K, w, budget, lam):
     m, r = redundancy(K, w)
     s = [lam * ai - (1.0 - lam) * ri for ai, ri in zip(a, r)]
     return dict(abar=abar, a=a, m=m, r=r, s=s, idx=select(s, N, w, budget))
+
+
+def evict_in_place(N, idx):
+    """Live-slot mask and ascending free slots, by a plain scan."""
+    kept = set(int(i) for i in idx)
+    keep = [i in kept for i in range(N)]
+    free = [i for i in range(N) if not keep[i]]
+    return keep, free

@@ -162,6 +162,33 @@ def compact(K: np.ndarray, V: np.ndarray, idx: np.ndarray):
     return K[idx], V[idx]
 
 
+def evict_in_place(N: int, idx: np.ndarray):
+    """In-place slot reuse (the ThinKV summary's Continuous Thinking: evicted
+    slots are not compacted away but reused).  Given the kept token indices of
+    a unit, returns (keep [N] bool, free [N - kept] int64): the live-slot mask
+    and the evicted slots in ascending order, which new tokens take next."""
+    keep = np.zeros(N, dtype=bool)
+    keep[np.asarray(idx, dtype=np.int64)] = True
+    free = np.flatnonzero(~keep).astype(np.int64)
+    return keep, free
+
+
+def fill_free_slots(K: np.ndarray, V: np.ndarray, keep: np.ndarray, free: np.ndarray,
+                    K_new: np.ndarray, V_new: np.ndarray):
+    """New tokens overwrite evicted slots (Continuous Thinking): new token t goes
+    to slot free[t], lowest slot first; the slot becomes live.  Returns the
+    updated (K, V, keep); the inputs are not modified.  Needs len(K_new) <=
+    len(free)."""
+    n = len(K_new)
+    assert n <= len(free) and len(V_new) == n
+    K2, V2, keep2 = K.copy(), V.copy(), keep.copy()
+    slots = np.asarray(free[:n], dtype=np.int64)
+    K2[slots] = K_new
+    V2[slots] = V_new
+    keep2[slots] = True
+    return K2, V2, keep2
+
+
 def run_unit(Q, K, V, w: int, budget: int, lam: float, redundancy="rowblocks"):
     """Whole path for one unit.  ``redundancy`` picks the row-mean definition
     (``rowblocks``), its closed form (``closed``) or the row-max reading

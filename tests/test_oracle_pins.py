@@ -355,3 +355,51 @@ def test_row_max_zero_key_and_window_keys_count():
     K = np.array([[1.0, 0.0], [0.0, 0.0], [0.0, 1.0], [1.0, 0.0]])
     m, _ = ora.redundancy_max(K, 1)   # candidates 0..2; key 3 (window) duplicates key 0
     np.testing.assert_allclose(m, [1.0, 0.0, 0.0], atol=1e-15)
+
+
+# ---- in-place slot reuse (eviction mask + free slots) -----------------------
+
+@pytest.mark.parametrize("seed", range(5))
+def test_evict_in_place_matches_scan_and_partitions_slots(seed):
+    rng = np.random.default_rng(300 + seed)
+    N = int(rng.integers(2, 300))
+    w = int(rng.integers(1, min(N, 8) + 1))
+    s = rng.standard_normal(N - w)
+    budget = int(rng.integers(0, N))
+    idx = ora.select(s, N, w, budget)
+    keep, free = ora.evict_in_place(N, idx)
+    keep_l, free_l = loops.evict_in_place(N, idx.tolist())
+    assert keep.tolist() == keep_l and free.tolist() == free_l
+    # kept and free slots partition 0..N-1; free is ascending; the window is live
+    assert sorted(idx.tolist() + free.tolist()) == list(range(N))
+    assert np.all(np.diff(free) > 0)
+    assert keep[N - w:].all()
+    assert keep.sum() == len(idx)
+
+
+def test_in_place_live_rows_equal_gather_compaction():
+    """Reading the live slots in ascending order gives exactly the rows that
+    gather compaction writes."""
+    rng = np.random.default_rng(31)
+    Q, K = _rand_unit(rng, 400, 16, 2, 4, dup=0.2)
+    V = rng.standard_normal(K.shape)
+    out = ora.run_unit(Q, K, V, 4, 50, 0.1, redundancy="closed")
+    keep, free = ora.evict_in_place(400, out["idx"])
+    np.testing.assert_array_equal(K[keep], out["K"])
+    np.testing.assert_array_equal(V[keep], out["V"])
+    assert len(free) == 400 - len(out["idx"])
+
+
+def test_fill_free_slots_takes_lowest_slots_first():
+    K = np.arange(10 * 3, dtype=np.float64).reshape(10, 3)
+    V = -K
+    keep, free = ora.evict_in_place(10, np.array([1, 4, 5, 8, 9]))
+    assert free.tolist() == [0, 2, 3, 6, 7]
+    Kn = np.full((3, 3), 100.0) + np.arange(3)[:, None]
+    K2, V2, keep2 = ora.fill_free_slots(K, V, keep, free, Kn, -Kn)
+    assert np.array_equal(K2[[0, 2, 3]], Kn) and np.array_equal(V2[[0, 2, 3]], -Kn)
+    untouched = [1, 4, 5, 6, 7, 8, 9]
+    assert np.array_equal(K2[untouched], K[untouched])
+    assert keep2.tolist() == [True, True, True, True, True, True, False, False, True, True]
+    with pytest.raises(AssertionError):
+        ora.fill_free_slots(K, V, keep, free, np.zeros((6, 3)), np.zeros((6, 3)))
