@@ -108,3 +108,17 @@ def evict_in_place(N, idx):
     keep = [i in kept for i in range(N)]
     free = [i for i in range(N) if not keep[i]]
     return keep, free
+
+
+def refree_keep_count(p, sinks, T):
+    """Stopping rule by a plain loop over the ranking (sinks, then newest first)."""
+    N = len(p)
+    m = min(sinks, N)
+    order = list(range(m)) + list(range(N - 1, m - 1, -1))
+    total = math.fsum(x * x for x in p)
+    acc = 0.0
+    for k, j in enumerate(order, start=1):
+        acc += p[j] * p[j]
+        if math.sqrt(acc) >= (1.0 - T) * math.sqrt(total):
+            return k
+    return N

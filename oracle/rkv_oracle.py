@@ -156,6 +156,56 @@ def select(s: np.ndarray, N: int, w: int, budget: int):
     return np.concatenate([kept, np.arange(c, N)]).astype(np.int64)
 
 
+def select_with_sinks(s: np.ndarray, N: int, w: int, budget: int, sinks: int):
+    """Kept indices with attention-sink protection and a per-unit budget (the
+    ReFreeKV review keeps the first m tokens as anchors; LU-KV gives each head
+    its own budget).  The first min(sinks, N - w) tokens are always kept, the
+    top-`budget` of the remaining candidates sinks .. N-w-1 are ranked by (s
+    descending, index ascending) as in :func:`select`, and the window follows.
+    Returns sinks, then the selected candidates ascending, then the window;
+    every token when no more than `budget` candidates remain.  With sinks = 0
+    this is :func:`select`."""
+    c = N - w
+    m = min(sinks, c)
+    if c - m <= budget:
+        return np.arange(N, dtype=np.int64)
+    rest = s[m:c]
+    order = np.lexsort((np.arange(c - m), -rest))
+    kept = np.sort(order[:budget]) + m
+    return np.concatenate([np.arange(m), kept, np.arange(c, N)]).astype(np.int64)
+
+
+def last_query_probs(Q: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """The attention row of the newest query (ReFreeKV with k = 1: one row of
+    the attention matrix stands for all of it), averaged over the GQA group:
+    p_j = mean_g softmax_j(q_{g, w-1} . k_j / sqrt(d)), over all N keys."""
+    return attention_probs(Q, K)[:, -1, :].mean(axis=0)
+
+
+def refree_keep_count(p: np.ndarray, sinks: int, T: float) -> int:
+    """ReFreeKV's stopping rule on one attention row p [N].
+
+    Initial ranking: the first m = min(sinks, N) tokens in order, then the
+    others from the newest to the oldest.  Uni-Metric: the Frobenius norm of
+    the attention entries kept.  Keep the shortest prefix of the ranking whose
+    norm reaches (1 - T) of the full row's norm, i.e. the norm lost by cutting
+    there is below T: the smallest k with sum_{first k} p^2 >= (1 - T)^2 sum p^2."""
+    N = len(p)
+    m = min(sinks, N)
+    order = np.concatenate([np.arange(m), np.arange(N - 1, m - 1, -1)])
+    e = p[order] ** 2
+    need = (1.0 - T) ** 2 * e.sum()
+    kept = np.cumsum(e)
+    return int(np.argmax(kept >= need)) + 1
+
+
+def refree_budget(k: int, N: int, w: int, sinks: int) -> int:
+    """The R-KV budget that keeps k tokens in all: k minus the sinks and the
+    window (which are kept anyway), at least 0."""
+    c = N - w
+    return max(0, k - min(sinks, c) - w)
+
+
 def compact(K: np.ndarray, V: np.ndarray, idx: np.ndarray):
     """Gather-based compaction of the surviving rows (the R-KV-style baseline
     named in the ThinKV summary): K'[j] = K[idx[j]], V'[j] = V[idx[j]]."""

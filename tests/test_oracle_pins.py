@@ -403,3 +403,75 @@ def test_fill_free_slots_takes_lowest_slots_first():
     assert keep2.tolist() == [True, True, True, True, True, True, False, False, True, True]
     with pytest.raises(AssertionError):
         ora.fill_free_slots(K, V, keep, free, np.zeros((6, 3)), np.zeros((6, 3)))
+
+
+# ---- sinks + per-unit budgets; ReFreeKV adaptive budget ----------------------
+
+@pytest.mark.parametrize("seed", range(6))
+def test_select_with_sinks_reduces_and_brute_force(seed):
+    rng = np.random.default_rng(400 + seed)
+    N = int(rng.integers(3, 13))
+    w = int(rng.integers(1, 3))
+    s = np.round(rng.standard_normal(N - w), 1)       # ties on purpose
+    for budget in range(0, N - w + 1):
+        assert np.array_equal(ora.select_with_sinks(s, N, w, budget, 0),
+                              ora.select(s, N, w, budget))
+        for sinks in (1, 2, 4):
+            got = ora.select_with_sinks(s, N, w, budget, sinks).tolist()
+            m = min(sinks, N - w)
+            # sinks and window always kept; the middle is the brute-force best subset
+            assert got[:m] == list(range(m)) and got[-w:] == list(range(N - w, N))
+            mid = got[m:len(got) - w]
+            if N - w - m <= budget:
+                assert got == list(range(N))
+            else:
+                sub = loops.select_by_subsets(list(s[m:]), N - m, w, budget)
+                assert mid == [i + m for i in sub[:budget]]
+
+
+def test_last_query_probs_is_last_row_of_attention():
+    rng = np.random.default_rng(9)
+    Q, K = _rand_unit(rng, 50, 8, 3, 4)
+    p = ora.last_query_probs(Q, K)
+    assert p.shape == (50,) and abs(p.sum() - 1.0) < 1e-12
+    # the newest query sees every key: with w = 1, G = 1 it is a plain softmax
+    from scipy.special import softmax as sp_softmax
+    Q1 = Q[:1, -1:, :]
+    np.testing.assert_allclose(ora.last_query_probs(Q1, K),
+                               sp_softmax(K @ Q1[0, 0] / np.sqrt(8)), rtol=1e-12)
+
+
+def test_refree_keep_count_closed_forms():
+    N = 1000
+    # uniform row: norm of the first k entries is sqrt(k/N) of the full norm
+    p = np.full(N, 1.0 / N)
+    for T in (0.01, 0.013, 0.37):     # (1 - T)^2 N away from an integer
+        want = int(np.ceil((1 - T) ** 2 * N))
+        assert ora.refree_keep_count(p, 4, T) == want
+    # all mass on the sinks: the sinks alone suffice
+    p = np.zeros(N); p[:4] = 0.25
+    assert ora.refree_keep_count(p, 4, 0.01) == 4
+    # all mass on the newest token: sinks (ranked first) plus that one
+    p = np.zeros(N); p[-1] = 1.0
+    assert ora.refree_keep_count(p, 4, 0.01) == 5
+    assert ora.refree_keep_count(p, 0, 0.01) == 1
+    # one old token holds all the mass: everything back to it is kept
+    p = np.zeros(N); p[100] = 1.0
+    assert ora.refree_keep_count(p, 4, 0.01) == 4 + (N - 100)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_refree_keep_count_matches_loop(seed):
+    rng = np.random.default_rng(500 + seed)
+    N = int(rng.integers(5, 400))
+    p = rng.random(N) ** 8
+    p /= p.sum()
+    for T in (0.01, 0.05, 0.3):
+        for sinks in (0, 4):
+            assert ora.refree_keep_count(p, sinks, T) == loops.refree_keep_count(list(p), sinks, T)
+
+
+def test_refree_budget_counts_sinks_and_window():
+    assert ora.refree_budget(100, 1000, 8, 4) == 88
+    assert ora.refree_budget(10, 1000, 8, 4) == 0
+    assert ora.refree_budget(5, 6, 8 - 6 + 4, 4) == 0
