@@ -174,6 +174,11 @@ def algorithmic(batch: Batch, wl: W.Workload):
         "select_bytes": float(8 * c.sum() + 4 * U * W_ + 4 * U),
         # kept K and V rows read; the whole [U, B+w] outputs written
         "compact_bytes": float(2 * 2 * d * kept.sum() + 2 * 2 * d * U * W_),
+        # kept indices and counts read; keep mask (1 B) and free list (4 B) per
+        # token and the free counts written
+        "evict_bytes": float(4 * U * W_ + 4 * U + 5 * n.sum() + 4 * U),
+        # K read once, the newest queries, p_last written and read back, budgets
+        "refree_bytes": float((2 * d + 8) * n.sum() + 2 * d * U * wl.group + 8 * U),
     }
 
 
@@ -214,7 +219,7 @@ def kernel_report(per_kernel, alg, pk, src):
             tf = alg["gemm_flops"] / (ms * 1e-3) / 1e12
             ent.update(bound="tensor", achieved=round(tf, 2), unit="TFLOP/s",
                        peak=pk["bf16_tflops_sustained"], frac=round(tf / pk["bf16_tflops_sustained"], 4))
-        elif name in ("score", "select", "compact"):
+        elif name in ("score", "select", "compact", "evict", "refree"):
             gbs = alg[f"{name}_bytes"] / (ms * 1e-3) / 1e9
             ent.update(bound="hbm", achieved=round(gbs, 1), unit="GB/s", peak=hbm,
                        frac=round(gbs / hbm, 4))
@@ -351,6 +356,11 @@ def run_engine(args, dist: Dist):
         secondary = {"redundancy": other, "value": tokens * dist.world / (ms2 * 1e-3),
                      "ms_per_step": ms2, "kernels": rep2}
 
+    in_place = adaptive = None
+    if not args.no_secondary:
+        in_place = measure_in_place(eng, batch, wl, args, dist, alg, pk, src)
+        adaptive = measure_adaptive(eng, batch, wl, args, dist, alg, pk, src)
+
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(eng, batch, wl, args, dist)
@@ -368,8 +378,57 @@ def run_engine(args, dist: Dist):
                 "config": config_of(wl, batch, args.redundancy, args.lam, dist.world),
                 "roofline": roofline, "kernels": rep, "gpu_launches": launches,
                 "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
-                "secondary": secondary}
+                "secondary": secondary, "in_place": in_place, "adaptive": adaptive}
         print(json.dumps(line), flush=True)
+
+
+def measure_adaptive(eng, batch: Batch, wl: W.Workload, args, dist: Dist, alg, pk, src):
+    """The step with the adaptive budget: rkv_refree_budget (T = 1%, 4 sinks,
+    budgets capped at the workload's B) -> score -> rkv_select_ex -> compact."""
+    sinks, T = 4, 0.01
+    a, r = eng.alloc_scores(batch)
+    U, Wd = batch.num_units, wl.budget + sinks + wl.window
+    dev = batch.K.device
+    idx = torch.empty((U, Wd), dtype=torch.int32, device=dev)
+    nk = torch.empty(U, dtype=torch.int32, device=dev)
+    Ko = torch.empty((U, Wd, wl.head_dim), dtype=torch.bfloat16, device=dev)
+    Vo = torch.empty_like(Ko)
+    p_last = torch.empty(batch.num_tokens, device=dev)
+    budgets = torch.empty(U, dtype=torch.int32, device=dev)
+
+    def step():
+        eng.refree_budget(batch, T, sinks, wl.budget, p_last, budgets)
+        eng.score(batch, a, r)
+        eng.select_ex(batch, a, r, args.lam, wl.budget, idx, nk, budgets, sinks)
+        eng.compact(batch, idx, nk, wl.budget + sinks, Ko, Vo)
+
+    ms, per_kernel, _ = timed(step, args.steps, args.warmup, dist, eng)
+    eng.check_status()
+    rep = kernel_report(per_kernel, alg, pk, src)
+    b = budgets.cpu().numpy()
+    return {"value": batch.num_tokens * dist.world / (ms * 1e-3), "ms_per_step": ms,
+            "T": T, "sinks": sinks, "budget_mean": float(b.mean()),
+            "budget_min": int(b.min()), "budget_max": int(b.max()),
+            "kernels": {k: rep[k] for k in ("refree", "select", "compact") if k in rep}}
+
+
+def measure_in_place(eng, batch: Batch, wl: W.Workload, args, dist: Dist, alg, pk, src):
+    """The same step with in-place slot reuse (rkv_evict_in_place: keep mask
+    and free slots) in place of gather compaction."""
+    a, r = eng.alloc_scores(batch)
+    idx, nk = eng.alloc_outputs(batch, wl.budget)[:2]
+    keep, free, nfree = eng.alloc_in_place(batch)
+
+    def step():
+        eng.score(batch, a, r)
+        eng.select(batch, a, r, args.lam, wl.budget, idx, nk)
+        eng.evict_in_place(batch, idx, nk, wl.budget, keep, free, nfree)
+
+    ms, per_kernel, _ = timed(step, args.steps, args.warmup, dist, eng)
+    eng.check_status()
+    rep = kernel_report(per_kernel, alg, pk, src)
+    return {"value": batch.num_tokens * dist.world / (ms * 1e-3), "ms_per_step": ms,
+            "kernels": {k: rep[k] for k in ("select", "evict") if k in rep}}
 
 
 def measure_e2e(eng, batch: Batch, wl: W.Workload, args, dist: Dist):

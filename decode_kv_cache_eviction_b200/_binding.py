@@ -33,9 +33,10 @@ RKV_FLAG_GEMM_SINGLE_CTA = 1
 
 # Every function declared in include/rkv.h.
 EXPORTS = ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact",
-           "rkv_compress", "rkv_compress_host", "rkv_check_status", "rkv_launch_count", "rkv_set_timing",
+           "rkv_compress", "rkv_compress_host", "rkv_evict_in_place", "rkv_fill_slots",
+           "rkv_select_ex", "rkv_refree_budget", "rkv_check_status", "rkv_launch_count", "rkv_set_timing",
            "rkv_read_timing", "rkv_score_noalloc", "rkv_status_string", "rkv_version")
-KERNELS = ("score", "plan", "gemm", "select", "compact")
+KERNELS = ("score", "plan", "gemm", "select", "compact", "evict", "fill", "refree")
 
 
 class RkvConfig(ctypes.Structure):
@@ -85,6 +86,12 @@ def lib():
                                vp, vp]
     L.rkv_compress_host.argtypes = [vp, ctypes.POINTER(RkvHostBatch), f32, i32, vp, vp, vp, vp,
                                     i64, vp]
+    L.rkv_evict_in_place.argtypes = [vp, ctypes.POINTER(RkvBatch), vp, vp, i32, vp, vp, vp, vp]
+    L.rkv_fill_slots.argtypes = [vp, ctypes.POINTER(RkvBatch), vp, vp, vp, vp, vp, vp, vp, vp,
+                                 vp, vp]
+    L.rkv_select_ex.argtypes = [vp, ctypes.POINTER(RkvBatch), vp, vp, f32, i32, vp, i32, vp, vp,
+                                vp]
+    L.rkv_refree_budget.argtypes = [vp, ctypes.POINTER(RkvBatch), f32, i32, i32, vp, vp, vp, vp]
     L.rkv_check_status.argtypes = [vp, vp]
     L.rkv_launch_count.argtypes = [vp]
     L.rkv_launch_count.restype = i64
@@ -96,7 +103,8 @@ def lib():
     L.rkv_status_string.restype = ctypes.c_char_p
     L.rkv_version.argtypes = []
     for name in ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact",
-                 "rkv_compress", "rkv_compress_host", "rkv_check_status", "rkv_set_timing",
+                 "rkv_compress", "rkv_compress_host", "rkv_evict_in_place", "rkv_fill_slots",
+                 "rkv_select_ex", "rkv_refree_budget", "rkv_check_status", "rkv_set_timing",
                  "rkv_read_timing",
                  "rkv_score_noalloc", "rkv_version"):
         getattr(L, name).restype = i32
@@ -220,6 +228,51 @@ class Engine:
                                        _ptr(idx), _ptr(n_kept), _ptr(K_out), _ptr(V_out),
                                        int(chunk_tokens), _stream(stream)),
                "rkv_compress_host")
+
+    def evict_in_place(self, batch: Batch, idx, n_kept, budget: int, keep, free_slots, n_free,
+                       stream=None):
+        """Keep mask and ascending free slots instead of compaction
+        (``rkv_evict_in_place``); keep is uint8 [T], free_slots int32 [T],
+        n_free int32 [U]."""
+        _check(lib().rkv_evict_in_place(self.h, ctypes.byref(batch.c), _ptr(idx), _ptr(n_kept),
+                                        int(budget), _ptr(keep), _ptr(free_slots), _ptr(n_free),
+                                        _stream(stream)), "rkv_evict_in_place")
+
+    def fill_slots(self, batch: Batch, new_off, K_new, V_new, keep, free_slots, n_free,
+                   stream=None):
+        """New tokens overwrite the lowest free slots of their unit
+        (``rkv_fill_slots``), in place in batch.K / batch.V.  ``new_off`` is an
+        int64 sequence of U + 1 row offsets into K_new / V_new."""
+        off = np.ascontiguousarray(np.asarray(new_off, dtype=np.int64))
+        dev = torch.from_numpy(off).to(batch.K.device)
+        _check(lib().rkv_fill_slots(self.h, ctypes.byref(batch.c), _ptr(batch.K), _ptr(batch.V),
+                                    _ptr(dev), off.ctypes.data, _ptr(K_new), _ptr(V_new),
+                                    _ptr(keep), _ptr(free_slots), _ptr(n_free),
+                                    _stream(stream)), "rkv_fill_slots")
+        return dev   # keep the device offsets alive until the caller syncs
+
+    def alloc_in_place(self, batch: Batch):
+        """keep uint8 [T], free_slots int32 [T], n_free int32 [U] on the batch's device."""
+        T, U, dev = batch.num_tokens, batch.num_units, batch.K.device
+        return (torch.empty(T, dtype=torch.uint8, device=dev),
+                torch.empty(T, dtype=torch.int32, device=dev),
+                torch.empty(U, dtype=torch.int32, device=dev))
+
+    def select_ex(self, batch: Batch, a, r, lam: float, budget: int, idx, n_kept, budgets=None,
+                  sinks: int = 0, stream=None):
+        """Selection with attention sinks and optional per-unit budgets
+        (``rkv_select_ex``); idx has row stride budget + sinks + w."""
+        _check(lib().rkv_select_ex(self.h, ctypes.byref(batch.c), _ptr(a), _ptr(r), float(lam),
+                                   int(budget), _ptr(budgets), int(sinks), _ptr(idx),
+                                   _ptr(n_kept), _stream(stream)), "rkv_select_ex")
+
+    def refree_budget(self, batch: Batch, T: float, sinks: int, max_budget: int, p_last, budgets,
+                      keep_count=None, stream=None):
+        """Adaptive per-unit budgets from the newest query's attention row
+        (``rkv_refree_budget``)."""
+        _check(lib().rkv_refree_budget(self.h, ctypes.byref(batch.c), float(T), int(sinks),
+                                       int(max_budget), _ptr(p_last), _ptr(budgets),
+                                       _ptr(keep_count), _stream(stream)), "rkv_refree_budget")
 
     def check_status(self, stream=None):
         _check(lib().rkv_check_status(self.h, _stream(stream)), "device status")

@@ -164,7 +164,7 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   e->max_n = e->max_cs * score_lmax(e->rp);
   if (e->max_n > kMaxTokensPerUnit) e->max_n = kMaxTokensPerUnit;
 
-  if (select_configure() != cudaSuccess) {
+  if (select_configure() != cudaSuccess || inplace_configure() != cudaSuccess) {
     delete e;
     return cuda_fail(cudaErrorUnknown);
   }
@@ -294,7 +294,7 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   p.rho_out = closed ? nullptr : e->rho;
   p.rho_off = closed ? nullptr : e->rho_off;
   p.status = e->status;
-  const int rows_per_item = e->pair ? 256 : 128;
+  const int rows_per_item = e->pair ? GemmCfg<true>::kRowsPerItem : GemmCfg<false>::kRowsPerItem;
   cudaError_t err;
   if (!closed) {   // row blocks for the GEMM and the padded rho layout the score kernel writes
     t_begin(e, RKV_KERNEL_PLAN, st);
@@ -313,8 +313,10 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
 
   // redundancy GEMM
   CUtensorMap amap, bmap;
-  if (make_map(e, &amap, b->K, static_cast<uint64_t>(T), 128) != RKV_OK) return RKV_ERR_CUDA;
-  if (make_map(e, &bmap, b->K, static_cast<uint64_t>(T), e->pair ? 128 : 256) != RKV_OK)
+  if (make_map(e, &amap, b->K, static_cast<uint64_t>(T), GemmCfg<true>::kRowsPerCta) != RKV_OK)
+    return RKV_ERR_CUDA;
+  if (make_map(e, &bmap, b->K, static_cast<uint64_t>(T),
+               e->pair ? GemmCfg<true>::kBRows : GemmCfg<false>::kBRows) != RKV_OK)
     return RKV_ERR_CUDA;
   GemmParams g;
   g.tok_off = b->tok_off;
@@ -362,8 +364,36 @@ int rkv_select(rkv_engine* e, const rkv_batch* b, const float* a, const float* r
     return RKV_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   t_begin(e, RKV_KERNEL_SELECT, st);
-  cudaError_t err = launch_select(b->tok_off, U, e->cfg.window, cmax, a, r, lambda, budget, idx,
-                                  n_kept, st);
+  cudaError_t err = launch_select(b->tok_off, U, e->cfg.window, cmax, a, r, lambda, budget,
+                                  nullptr, 0, budget + e->cfg.window, idx, n_kept, st);
+  t_end(e, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  ++e->launches;
+  return RKV_OK;
+}
+
+int rkv_select_ex(rkv_engine* e, const rkv_batch* b, const float* a, const float* r,
+                  float lambda, int budget, const int32_t* budgets, int sinks, int32_t* idx,
+                  int32_t* n_kept, rkv_stream_t stream) {
+  if (!e) return RKV_ERR_INVALID_ARG;
+  int64_t T = 0;
+  int nmax = 0, cmax = 0;
+  int rc = check_batch(e, b, &T, &nmax, &cmax);
+  if (rc != RKV_OK) return rc;
+  if (!(lambda >= 0.f && lambda <= 1.f) || budget < 0 || sinks < 0) return RKV_ERR_INVALID_ARG;
+  if (!a || !r || !idx || !n_kept) return RKV_ERR_INVALID_ARG;
+  if (!aligned(a, 4) || !aligned(r, 4) || !aligned(idx, 4) || !aligned(n_kept, 4) ||
+      (budgets && !aligned(budgets, 4)))
+    return RKV_ERR_INVALID_ARG;
+  const int U = b->num_units;
+  if (U == 0) return RKV_OK;
+  const int64_t W = static_cast<int64_t>(budget) + sinks + e->cfg.window;
+  if (W >= (static_cast<int64_t>(1) << 30) || U * W >= (static_cast<int64_t>(1) << 31))
+    return RKV_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_begin(e, RKV_KERNEL_SELECT, st);
+  cudaError_t err = launch_select(b->tok_off, U, e->cfg.window, cmax, a, r, lambda, budget,
+                                  budgets, sinks, static_cast<int>(W), idx, n_kept, st);
   t_end(e, st);
   if (err != cudaSuccess) return cuda_fail(err);
   ++e->launches;
@@ -390,6 +420,89 @@ int rkv_compact(rkv_engine* e, const rkv_batch* b, const int32_t* idx, const int
   t_begin(e, RKV_KERNEL_COMPACT, st);
   cudaError_t err = launch_compact(b->tok_off, U, static_cast<int>(W), idx, n_kept, b->K, b->V,
                                    K_out, V_out, e->status, e->nsm, st);
+  t_end(e, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  ++e->launches;
+  return RKV_OK;
+}
+
+int rkv_evict_in_place(rkv_engine* e, const rkv_batch* b, const int32_t* idx,
+                       const int32_t* n_kept, int budget, uint8_t* keep, int32_t* free_slots,
+                       int32_t* n_free, rkv_stream_t stream) {
+  if (!e) return RKV_ERR_INVALID_ARG;
+  int64_t T = 0;
+  int nmax = 0, cmax = 0;
+  int rc = check_batch(e, b, &T, &nmax, &cmax);
+  if (rc != RKV_OK) return rc;
+  if (budget < 0 || !idx || !n_kept || !keep || !free_slots || !n_free) return RKV_ERR_INVALID_ARG;
+  if (!aligned(idx, 4) || !aligned(n_kept, 4) || !aligned(free_slots, 4) || !aligned(n_free, 4))
+    return RKV_ERR_INVALID_ARG;
+  const int U = b->num_units;
+  if (U == 0) return RKV_OK;
+  const int64_t W = static_cast<int64_t>(budget) + e->cfg.window;
+  if (U * W >= (static_cast<int64_t>(1) << 31)) return RKV_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_begin(e, RKV_KERNEL_EVICT, st);
+  cudaError_t err = launch_evict_in_place(b->tok_off, U, nmax, static_cast<int>(W), idx, n_kept,
+                                          keep, free_slots, n_free, e->status, e->nsm, st);
+  t_end(e, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  ++e->launches;
+  return RKV_OK;
+}
+
+int rkv_fill_slots(rkv_engine* e, const rkv_batch* b, void* K, void* V, const int64_t* new_off,
+                   const int64_t* new_off_host, const void* K_new, const void* V_new,
+                   uint8_t* keep, int32_t* free_slots, int32_t* n_free, rkv_stream_t stream) {
+  if (!e) return RKV_ERR_INVALID_ARG;
+  int64_t T = 0;
+  int nmax = 0, cmax = 0;
+  int rc = check_batch(e, b, &T, &nmax, &cmax);
+  if (rc != RKV_OK) return rc;
+  if (!K || !V || !new_off || !new_off_host || !keep || !free_slots || !n_free)
+    return RKV_ERR_INVALID_ARG;
+  const int U = b->num_units;
+  if (new_off_host[0] != 0) return RKV_ERR_INVALID_ARG;
+  for (int u = 0; u < U; ++u)
+    if (new_off_host[u + 1] < new_off_host[u]) return RKV_ERR_INVALID_ARG;
+  const int64_t Tn = new_off_host[U];
+  if (Tn > 0 && (!K_new || !V_new)) return RKV_ERR_INVALID_ARG;
+  if (!aligned(K, 16) || !aligned(V, 16) || (Tn > 0 && (!aligned(K_new, 16) ||
+      !aligned(V_new, 16))) || !aligned(new_off, 8) || !aligned(free_slots, 4) ||
+      !aligned(n_free, 4))
+    return RKV_ERR_INVALID_ARG;
+  if (U == 0 || Tn == 0) return RKV_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_begin(e, RKV_KERNEL_FILL, st);
+  cudaError_t err = launch_fill_slots(b->tok_off, U, new_off, K_new, V_new, K, V, keep,
+                                      free_slots, n_free, e->status, e->nsm, st);
+  t_end(e, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  ++e->launches;
+  return RKV_OK;
+}
+
+int rkv_refree_budget(rkv_engine* e, const rkv_batch* b, float T, int sinks, int max_budget,
+                      float* p_last, int32_t* budgets, int32_t* keep_count,
+                      rkv_stream_t stream) {
+  if (!e) return RKV_ERR_INVALID_ARG;
+  int64_t Tn = 0;
+  int nmax = 0, cmax = 0;
+  int rc = check_batch(e, b, &Tn, &nmax, &cmax);
+  if (rc != RKV_OK) return rc;
+  if (!(T >= 0.f && T < 1.f) || sinks < 0 || max_budget < 0 || !p_last || !budgets || !b->K ||
+      !b->Q)
+    return RKV_ERR_INVALID_ARG;
+  if (!aligned(p_last, 4) || !aligned(budgets, 4) || (keep_count && !aligned(keep_count, 4)) ||
+      !aligned(b->K, 16) || !aligned(b->Q, 16))
+    return RKV_ERR_INVALID_ARG;
+  if (e->cfg.group > 8) return RKV_ERR_UNSUPPORTED;
+  const int U = b->num_units;
+  if (U == 0) return RKV_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  t_begin(e, RKV_KERNEL_REFREE, st);
+  cudaError_t err = launch_refree(b->tok_off, U, e->cfg.group, e->cfg.window, b->Q, b->K, sinks,
+                                  T, max_budget, p_last, budgets, keep_count, e->nsm, st);
   t_end(e, st);
   if (err != cudaSuccess) return cuda_fail(err);
   ++e->launches;

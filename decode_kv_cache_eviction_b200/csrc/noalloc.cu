@@ -173,8 +173,8 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   CUtensorMap kmap, qmap, amap, bmap;
   if (encode(&kmap, b->K, static_cast<uint64_t>(T), kTile) != RKV_OK ||
       encode(&qmap, b->Q, static_cast<uint64_t>(U) * R, rp) != RKV_OK ||
-      encode(&amap, b->K, static_cast<uint64_t>(T), 128) != RKV_OK ||
-      encode(&bmap, b->K, static_cast<uint64_t>(T), 128) != RKV_OK)
+      encode(&amap, b->K, static_cast<uint64_t>(T), GemmCfg<true>::kRowsPerCta) != RKV_OK ||
+      encode(&bmap, b->K, static_cast<uint64_t>(T), GemmCfg<true>::kBRows) != RKV_OK)
     return RKV_ERR_CUDA;
 
   Scratch* s = d->scratch;  // device address, never the host-side symbol
@@ -194,7 +194,8 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   p.rho_out = s->rho;
   p.rho_off = s->rho_off;
   p.status = s->status;
-  if (launch_plan(b->tok_off, U, window, 256, s->item_off, s->unit_cnt, s->rho_off, st) !=
+  constexpr int kRows = GemmCfg<true>::kRowsPerItem;
+  if (launch_plan(b->tok_off, U, window, kRows, s->item_off, s->unit_cnt, s->rho_off, st) !=
       cudaSuccess) {
     cudaGetLastError();
     return RKV_ERR_CUDA;
@@ -206,7 +207,7 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   int64_t items = 0;
   for (int u = 0; u < U; ++u) {
     const int64_t c = off[u + 1] - off[u] - window;
-    if (c > 0) items += (c + 255) / 256;
+    if (c > 0) items += (c + kRows - 1) / kRows;
   }
   if (items == 0) return RKV_OK;
   GemmParams g;

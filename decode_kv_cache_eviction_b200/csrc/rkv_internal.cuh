@@ -162,12 +162,25 @@ cudaError_t gemm_configure(bool pair, bool rowmax);
 int gemm_max_ctas(bool pair, bool rowmax);
 
 cudaError_t launch_select(const int64_t* tok_off, int U, int w, int cmax, const float* a,
-                          const float* r, float lam, int budget, int32_t* idx, int32_t* n_kept,
-                          cudaStream_t st);
+                          const float* r, float lam, int budget, const int32_t* budgets,
+                          int sinks, int W, int32_t* idx, int32_t* n_kept, cudaStream_t st);
 cudaError_t select_configure();
 
 cudaError_t launch_compact(const int64_t* tok_off, int U, int W, const int32_t* idx,
                            const int32_t* n_kept, const void* K, const void* V, void* Ko,
                            void* Vo, int* status, int nsm, cudaStream_t st);
+
+cudaError_t launch_refree(const int64_t* tok_off, int U, int G, int w, const void* Q,
+                          const void* K, int sinks, float T, int max_budget, float* p_last,
+                          int32_t* budgets, int32_t* keep_count, int nsm, cudaStream_t st);
+cudaError_t inplace_configure();
+cudaError_t launch_evict_in_place(const int64_t* tok_off, int U, int nmax, int W,
+                                  const int32_t* idx, const int32_t* n_kept, uint8_t* keep,
+                                  int32_t* free_slots, int32_t* n_free, int* status, int nsm,
+                                  cudaStream_t st);
+cudaError_t launch_fill_slots(const int64_t* tok_off, int U, const int64_t* new_off,
+                              const void* K_new, const void* V_new, void* K, void* V,
+                              uint8_t* keep, int32_t* free_slots, int32_t* n_free, int* status,
+                              int nsm, cudaStream_t st);
 
 }  // namespace rkv

@@ -18,6 +18,10 @@
 //      in ascending index order: each warp owns a contiguous segment of the
 //      candidates, counts its "greater" and "equal" keys, and after one
 //      block-level prefix over the warps writes its positions with ballots.
+// Optional extensions: the first `sinks` tokens are always kept and excluded
+// from the ranking (attention sinks), and each unit may have its own budget
+// (budgets[u], clamped to 0 .. budget).  Row u of idx has stride W and ends in
+// -1 past the n_kept[u] valid entries.
 #include "ptx.cuh"
 #include "rkv_internal.cuh"
 
@@ -48,8 +52,9 @@ __device__ __forceinline__ void prefetch_l2(const void* p, size_t bytes) {
 
 __global__ void __launch_bounds__(kSelThreads, 1)
     select_kernel(const int64_t* __restrict__ tok_off, int U, int w, const float* __restrict__ a,
-                  const float* __restrict__ r, float lam, int budget, int32_t* __restrict__ idx,
-                  int32_t* __restrict__ n_kept) {
+                  const float* __restrict__ r, float lam, int max_budget,
+                  const int32_t* __restrict__ budgets, int sinks, int W,
+                  int32_t* __restrict__ idx, int32_t* __restrict__ n_kept) {
   extern __shared__ uint32_t keys[];
   __shared__ uint32_t hist8[kHistGroups][256];
   __shared__ uint32_t hist[256];
@@ -59,18 +64,22 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   __shared__ int wgt[kSelWarps], weq[kSelWarps], eqb[kSelWarps], outb[kSelWarps];
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
   const float lw = lam, rw = 1.f - lam;
-  const int W = budget + w;
 
   for (int u = blockIdx.x; u < U; u += gridDim.x) {
-    const int64_t base = tok_off[u];
-    const int N = static_cast<int>(tok_off[u + 1] - base);
-    const int c = N - w;
+    const int64_t tbase = tok_off[u];
+    const int N = static_cast<int>(tok_off[u + 1] - tbase);
+    const int c0 = N - w;                       // candidates, sinks included
+    const int m = min(sinks, c0);               // sinks: always kept, not ranked
+    const int c = c0 - m;                       // ranked candidates m .. c0 - 1
+    const int64_t base = tbase + m;             // a, r of ranked candidate i at base + i
+    int budget = max_budget;
+    if (budgets) budget = min(max(budgets[u], 0), max_budget);
     int32_t* out = idx + static_cast<int64_t>(u) * W;
     if (tid == 0 && u + static_cast<int>(gridDim.x) < U) {
       const int u2 = u + gridDim.x;
       const int64_t b2 = tok_off[u2];
       const int64_t c2 = tok_off[u2 + 1] - b2 - w;
-      if (c2 > budget) {
+      if (c2 > 0) {
         prefetch_l2(a + b2, static_cast<size_t>(c2) * 4);
         prefetch_l2(r + b2, static_cast<size_t>(c2) * 4);
       }
@@ -80,11 +89,15 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       if (tid == 0) n_kept[u] = N;
       continue;
     }
-    if (budget == 0) {  // only the window is kept (the radix step needs want >= 1)
-      for (int t = tid; t < w; t += kSelThreads) out[t] = c + t;
-      if (tid == 0) n_kept[u] = w;
-      continue;
+    // sinks, the window after the selected candidates, and the unused tail
+    for (int t = tid; t < W - budget; t += kSelThreads) {
+      if (t < m) out[t] = t;
+      else if (t < m + w) out[budget + t] = c0 + (t - m);
+      else out[budget + t] = -1;
     }
+    if (tid == 0) n_kept[u] = m + budget + w;
+    if (budget == 0) continue;  // the radix step needs want >= 1
+    out += m;                   // selected candidates follow the sinks
 
     // ---- 1. keys, min and max
     uint32_t kmin = 0xffffffffu, kmax = 0u;
@@ -198,13 +211,13 @@ __global__ void __launch_bounds__(kSelThreads, 1)
         for (int i0 = wp * 32; i0 < ((c + 31) & ~31); i0 += kSelThreads) {
           const int i = i0 + lane;
           const uint32_t k = i < c ? keys[i] : 0u;
-          const bool m = i < c && (k & pmask) == prefix;
-          const unsigned bal = __ballot_sync(0xffffffffu, m);
+          const bool hit = i < c && (k & pmask) == prefix;
+          const unsigned bal = __ballot_sync(0xffffffffu, hit);
           int slot = 0;
           if (lane == 0 && bal) slot = atomicAdd(&sh[3], __popc(bal));
           slot = __shfl_sync(0xffffffffu, slot, 0);
           const int pos = slot + __popc(bal & ((1u << lane) - 1u));
-          if (m && pos < kListCap) list[pos] = k;
+          if (hit && pos < kListCap) list[pos] = k;
         }
         __syncthreads();
         nlist = sh[3];
@@ -252,12 +265,10 @@ __global__ void __launch_bounds__(kSelThreads, 1)
       const bool f = g || (e && eseen + __popc(be & lt) < take_eq);
       const unsigned bf = __ballot_sync(0xffffffffu, f);
       const int pos = oseen + __popc(bf & lt);
-      if (f && pos < budget) out[pos] = i;
+      if (f && pos < budget) out[pos] = m + i;
       eseen += __popc(be);
       oseen += __popc(bf);
     }
-    for (int t = tid; t < w; t += kSelThreads) out[budget + t] = c + t;
-    if (tid == 0) n_kept[u] = budget + w;
     __syncthreads();  // shared state is reused by the next unit
   }
 }
@@ -270,8 +281,10 @@ cudaError_t select_configure() {
 }
 
 cudaError_t launch_select(const int64_t* tok_off, int U, int w, int cmax, const float* a,
-                          const float* r, float lam, int budget, int32_t* idx, int32_t* n_kept,
-                          cudaStream_t st) {
+                          const float* r, float lam, int budget, const int32_t* budgets,
+                          int sinks, int W, int32_t* idx, int32_t* n_kept, cudaStream_t st) {
+  // keys of the ranked candidates (budgets[u] <= budget, so a unit with at
+  // most `budget` candidates never needs them)
   const size_t smem = cmax > budget ? static_cast<size_t>(cmax) * 4 : 0;
   int dev = 0, nsm = 0, per = 0;
   cudaGetDevice(&dev);
@@ -284,7 +297,8 @@ cudaError_t launch_select(const int64_t* tok_off, int U, int w, int cmax, const 
   }
   int grid = nsm * per;
   if (grid > U) grid = U;
-  select_kernel<<<grid, kSelThreads, smem, st>>>(tok_off, U, w, a, r, lam, budget, idx, n_kept);
+  select_kernel<<<grid, kSelThreads, smem, st>>>(tok_off, U, w, a, r, lam, budget, budgets, sinks,
+                                                 W, idx, n_kept);
   return cudaGetLastError();
 }
 

@@ -129,6 +129,36 @@ int rkv_score(rkv_engine* eng, const rkv_batch* batch, float* a, float* r, float
 int rkv_select(rkv_engine* eng, const rkv_batch* batch, const float* a, const float* r,
                float lambda, int budget, int32_t* idx, int32_t* n_kept, rkv_stream_t stream);
 
+/* rkv_select with attention sinks and per-unit budgets (sinks: the ReFreeKV
+ * review's anchor tokens; per-head budgets: LU-KV; an adaptive budget from
+ * rkv_refree_budget).  For unit u with c = N_u - w candidates, m = min(sinks, c)
+ * and B_u = budgets ? clamp(budgets[u], 0, budget) : budget:
+ *   - if c - m <= B_u, every token 0 .. N_u - 1 is kept;
+ *   - else tokens 0 .. m-1 (always), then the B_u best of candidates m .. c-1
+ *     by (s descending, index ascending) in ascending order, then the window.
+ *   idx [U, W] int32 with W = budget + sinks + w; entries past n_kept[u] are -1.
+ *   budgets: device [U] int32 or NULL.
+ * For rkv_compact / rkv_evict_in_place on this idx, pass budget + sinks as
+ * their budget (same row stride).  sinks = 0 and budgets = NULL is rkv_select. */
+int rkv_select_ex(rkv_engine* eng, const rkv_batch* batch, const float* a, const float* r,
+                  float lambda, int budget, const int32_t* budgets, int sinks, int32_t* idx,
+                  int32_t* n_kept, rkv_stream_t stream);
+
+/* Adaptive per-unit budget (the ReFreeKV review: initial ranking + Uni-Metric
+ * stop, with k = 1 and threshold T, e.g. 0.01).
+ *   p_last [T] fp32 (output): p_j = mean over the G heads of the newest query's
+ *     attention softmax_j(q_{g, w-1} . k_j / sqrt(d)), over all N_u keys;
+ *   keep_count [U] int32 (output, may be NULL): the smallest k such that the
+ *     first k tokens of the ranking (tokens 0 .. m-1, m = min(sinks, N_u), then
+ *     N_u - 1, N_u - 2, ... down to m) hold sum p^2 >= (1 - T)^2 sum_all p^2,
+ *     i.e. their Frobenius norm is at least (1 - T) of the row's;
+ *   budgets [U] int32 (output): clamp(k - min(sinks, N_u - w) - w, 0,
+ *     max_budget), the rkv_select_ex budget that keeps k tokens in all.
+ * Computed in fp32; requires G <= 8 (RKV_ERR_UNSUPPORTED otherwise). */
+int rkv_refree_budget(rkv_engine* eng, const rkv_batch* batch, float T, int sinks,
+                      int max_budget, float* p_last, int32_t* budgets, int32_t* keep_count,
+                      rkv_stream_t stream);
+
 /* Gather compaction: K_out[u][j] = K[tok_off[u] + idx[u][j]] (and V likewise) for
  * j < n_kept[u]; rows n_kept[u] .. budget + w - 1 are zero.  Bit-exact copies.
  *   K_out, V_out: device bf16 [U, budget + w, d] (must not overlap K, V).
@@ -136,6 +166,36 @@ int rkv_select(rkv_engine* eng, const rkv_batch* batch, const float* a, const fl
 int rkv_compact(rkv_engine* eng, const rkv_batch* batch, const int32_t* idx,
                 const int32_t* n_kept, int budget, void* K_out, void* V_out,
                 rkv_stream_t stream);
+
+/* In-place slot reuse, the alternative to rkv_compact (the ThinKV summary's
+ * Continuous Thinking: evicted slots are reused instead of compacted away).
+ * Rows stay where they are; for unit u, with idx / n_kept as rkv_select wrote
+ * them (row stride budget + w):
+ *   keep [T] uint8: keep[tok_off[u] + i] = 1 if token i is kept, else 0;
+ *   free_slots [T] int32: rows tok_off[u] .. tok_off[u] + n_free[u] - 1 hold the
+ *     evicted token indices of unit u (unit-local) in ascending order; the rest
+ *     of the unit's rows hold -1;
+ *   n_free [U] int32: N_u minus the number of distinct kept indices.
+ * Moves 1 + 4 bytes per cached token instead of rkv_compact's 4 d bytes per
+ * kept token.  A kept index outside 0 .. N_u - 1 (or an n_kept outside
+ * 0 .. budget + w) is ignored and sets RKV_ERR_DEVICE (see rkv_check_status). */
+int rkv_evict_in_place(rkv_engine* eng, const rkv_batch* batch, const int32_t* idx,
+                       const int32_t* n_kept, int budget, uint8_t* keep, int32_t* free_slots,
+                       int32_t* n_free, rkv_stream_t stream);
+
+/* New tokens overwrite evicted slots (Continuous Thinking).  New token t of
+ * unit u, row new_off[u] + t of K_new / V_new (bf16 [new_off[U], d]), is written
+ * to row tok_off[u] + free_slots[tok_off[u] + t] of K and V (the batch's
+ * caches, passed again as writable pointers), lowest free slot first, and
+ * marked live in keep.  The used slots leave the free list (the remaining ones
+ * move to the front) and n_free[u] drops by the count.  new_off is device
+ * [U+1] with a host copy new_off_host (new_off[0] = 0, nondecreasing).  A unit
+ * with more new tokens than free slots takes n_free[u] of them and sets
+ * RKV_ERR_DEVICE; a slot outside the unit is skipped and sets it too. */
+int rkv_fill_slots(rkv_engine* eng, const rkv_batch* batch, void* K, void* V,
+                   const int64_t* new_off, const int64_t* new_off_host, const void* K_new,
+                   const void* V_new, uint8_t* keep, int32_t* free_slots, int32_t* n_free,
+                   rkv_stream_t stream);
 
 /* rkv_score, rkv_select and rkv_compact in one call.  a and r are caller-owned
  * scratch [T] fp32 (they hold the scores afterwards). */
@@ -196,7 +256,10 @@ enum {
   RKV_KERNEL_GEMM = 2,    /* redundancy GEMM + fused epilogue + token softmax */
   RKV_KERNEL_SELECT = 3,  /* joint score + top-B */
   RKV_KERNEL_COMPACT = 4, /* K/V gather */
-  RKV_NUM_KERNELS = 5
+  RKV_KERNEL_EVICT = 5,   /* in-place eviction: keep mask and free slots */
+  RKV_KERNEL_FILL = 6,    /* new tokens into free slots */
+  RKV_KERNEL_REFREE = 7,  /* adaptive budget (newest query's attention row) */
+  RKV_NUM_KERNELS = 8
 };
 
 /* Per-kernel timing.  While enabled, the engine records a pair of CUDA events
