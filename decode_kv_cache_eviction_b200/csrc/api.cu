@@ -242,6 +242,7 @@ int rkv_destroy(rkv_engine* e) {
     for (int i = 0; i < rkv_engine::kMaxEv; ++i)
       for (int k = 0; k < 2; ++k) cudaEventDestroy(e->ev[i][k]);
   rkv_host_pipeline_free(e);
+  cudaFree(e->rf_z);
   cudaFree(e->status);
   cudaFree(e->item_off);
   cudaFree(e->unit_cnt);
@@ -499,10 +500,19 @@ int rkv_refree_budget(rkv_engine* e, const rkv_batch* b, float T, int sinks, int
   if (e->cfg.group > 8) return RKV_ERR_UNSUPPORTED;
   const int U = b->num_units;
   if (U == 0) return RKV_OK;
+  if (!e->rf_z) {
+    const size_t n = static_cast<size_t>(e->cfg.max_tokens) * refree_padded_group(e->cfg.group);
+    if (cudaMalloc(&e->rf_z, n * sizeof(float)) != cudaSuccess) {
+      cudaGetLastError();
+      e->rf_z = nullptr;
+      return RKV_ERR_OOM;
+    }
+  }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   t_begin(e, RKV_KERNEL_REFREE, st);
   cudaError_t err = launch_refree(b->tok_off, U, e->cfg.group, e->cfg.window, b->Q, b->K, sinks,
-                                  T, max_budget, p_last, budgets, keep_count, e->nsm, st);
+                                  T, max_budget, e->rf_z, p_last, budgets, keep_count, e->nsm,
+                                  st);
   t_end(e, st);
   if (err != cudaSuccess) return cuda_fail(err);
   ++e->launches;

@@ -59,6 +59,8 @@ struct rkv_engine {
   cudaEvent_t h_start = nullptr, h_done = nullptr;
   cudaEvent_t h_in[2] = {}, h_comp[2] = {}, h_out[2] = {};
   bool h_made = false;
+  // rkv_refree_budget's logit scratch (max_tokens x padded G floats), on first use
+  float* rf_z = nullptr;
 };
 
 // Frees everything rkv_compress_host allocated (called by rkv_destroy).

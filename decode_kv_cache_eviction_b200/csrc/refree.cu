@@ -5,9 +5,12 @@
 //
 // Per unit (one 256-thread CTA, persistent over units):
 //   pass 1  logits z_g(j) = q_g . k_j / sqrt(d) of the G newest queries for
-//           every key j, online max / sum per head g;
-//   pass 2  the same logits again, p(j) = mean_g exp(z_g(j) - M_g) / S_g,
-//           written to p_last, and e(j) = p(j)^2 summed;
+//           every key j, online max / sum per head g; the logits go to a
+//           scratch array (GP floats per token, one coalesced store per warp
+//           step), so K is read once;
+//   pass 2  the logits back from the scratch (mostly from L2), p(j) =
+//           mean_g exp(z_g(j) - M_g) / S_g, written to p_last, and e(j) =
+//           p(j)^2 summed;
 //   pass 3  the stopping point: the sinks' energy, then the suffix sums from
 //           the newest token down until (1 - T)^2 of the total is reached.
 //
@@ -44,8 +47,9 @@ template <int GP>
 __global__ void __launch_bounds__(kRfThreads)
     refree_kernel(const int64_t* __restrict__ tok_off, int U, int G, int w,
                   const uint16_t* __restrict__ Q, const uint2* __restrict__ K, float scale_log2,
-                  int sinks, float T, int max_budget, float* __restrict__ p_last,
-                  int32_t* __restrict__ budgets, int32_t* __restrict__ keep_count) {
+                  int sinks, float T, int max_budget, float* __restrict__ zbuf,
+                  float* __restrict__ p_last, int32_t* __restrict__ budgets,
+                  int32_t* __restrict__ keep_count) {
   constexpr int TB = 32 / GP;   // tokens per warp step
   __shared__ float red_m[kRfWarps][32], red_s[kRfWarps][32];
   __shared__ float fin_m[GP], fin_s[GP];
@@ -94,8 +98,10 @@ __global__ void __launch_bounds__(kRfThreads)
 
     // ---- pass 1: per-head max and sum of 2^(z - max)
     float rm = -INFINITY, rs = 0.f;
+    float* zu = zbuf + base * GP;   // logit of (token j, head g) at zu[j * GP + g]
     for (int j0 = wp * TB; j0 < N; j0 += kRfWarps * TB) {
       const float z = logit(j0);
+      if (j0 + tl < N) __stcg(&zu[j0 * GP + lane], z);
       if (real && j0 + tl < N) {
         if (z > rm) {
           rs = rs * ex2(rm - z) + 1.f;
@@ -126,7 +132,7 @@ __global__ void __launch_bounds__(kRfThreads)
     const float invG = 1.f / static_cast<float>(G);
     float esum = 0.f;
     for (int j0 = wp * TB; j0 < N; j0 += kRfWarps * TB) {
-      const float z = logit(j0);
+      const float z = j0 + tl < N ? __ldcg(&zu[j0 * GP + lane]) : 0.f;
       float pr = real ? ex2(z - Mg) * invS : 0.f;
 #pragma unroll
       for (int o = 1; o < GP; o <<= 1) pr += __shfl_xor_sync(0xffffffffu, pr, o);
@@ -222,30 +228,35 @@ __global__ void __launch_bounds__(kRfThreads)
 
 template <int GP>
 cudaError_t launch_rf(const int64_t* tok_off, int U, int G, int w, const void* Q, const void* K,
-                      int sinks, float T, int max_budget, float* p_last, int32_t* budgets,
-                      int32_t* keep_count, int nsm, cudaStream_t st) {
+                      int sinks, float T, int max_budget, float* zbuf, float* p_last,
+                      int32_t* budgets, int32_t* keep_count, int nsm, cudaStream_t st) {
   int grid = nsm * 4;
   if (grid > U) grid = U;
   const float scale_log2 = kLog2e / sqrtf(static_cast<float>(kHeadDim));
   refree_kernel<GP><<<grid, kRfThreads, 0, st>>>(
       tok_off, U, G, w, static_cast<const uint16_t*>(Q), static_cast<const uint2*>(K), scale_log2,
-      sinks, T, max_budget, p_last, budgets, keep_count);
+      sinks, T, max_budget, zbuf, p_last, budgets, keep_count);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+int refree_padded_group(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8; }
+
 cudaError_t launch_refree(const int64_t* tok_off, int U, int G, int w, const void* Q,
-                          const void* K, int sinks, float T, int max_budget, float* p_last,
-                          int32_t* budgets, int32_t* keep_count, int nsm, cudaStream_t st) {
-  if (G <= 1) return launch_rf<1>(tok_off, U, G, w, Q, K, sinks, T, max_budget, p_last, budgets,
-                                  keep_count, nsm, st);
-  if (G <= 2) return launch_rf<2>(tok_off, U, G, w, Q, K, sinks, T, max_budget, p_last, budgets,
-                                  keep_count, nsm, st);
-  if (G <= 4) return launch_rf<4>(tok_off, U, G, w, Q, K, sinks, T, max_budget, p_last, budgets,
-                                  keep_count, nsm, st);
-  return launch_rf<8>(tok_off, U, G, w, Q, K, sinks, T, max_budget, p_last, budgets, keep_count,
-                      nsm, st);
+                          const void* K, int sinks, float T, int max_budget, float* zbuf,
+                          float* p_last, int32_t* budgets, int32_t* keep_count, int nsm,
+                          cudaStream_t st) {
+  switch (refree_padded_group(G)) {
+    case 1: return launch_rf<1>(tok_off, U, G, w, Q, K, sinks, T, max_budget, zbuf, p_last,
+                                budgets, keep_count, nsm, st);
+    case 2: return launch_rf<2>(tok_off, U, G, w, Q, K, sinks, T, max_budget, zbuf, p_last,
+                                budgets, keep_count, nsm, st);
+    case 4: return launch_rf<4>(tok_off, U, G, w, Q, K, sinks, T, max_budget, zbuf, p_last,
+                                budgets, keep_count, nsm, st);
+    default: return launch_rf<8>(tok_off, U, G, w, Q, K, sinks, T, max_budget, zbuf, p_last,
+                                 budgets, keep_count, nsm, st);
+  }
 }
 
 }  // namespace rkv

@@ -170,9 +170,11 @@ cudaError_t launch_compact(const int64_t* tok_off, int U, int W, const int32_t* 
                            const int32_t* n_kept, const void* K, const void* V, void* Ko,
                            void* Vo, int* status, int nsm, cudaStream_t st);
 
+int refree_padded_group(int G);   // heads per token in the refree logit scratch
 cudaError_t launch_refree(const int64_t* tok_off, int U, int G, int w, const void* Q,
-                          const void* K, int sinks, float T, int max_budget, float* p_last,
-                          int32_t* budgets, int32_t* keep_count, int nsm, cudaStream_t st);
+                          const void* K, int sinks, float T, int max_budget, float* zbuf,
+                          float* p_last, int32_t* budgets, int32_t* keep_count, int nsm,
+                          cudaStream_t st);
 cudaError_t inplace_configure();
 cudaError_t launch_evict_in_place(const int64_t* tok_off, int U, int nmax, int W,
                                   const int32_t* idx, const int32_t* n_kept, uint8_t* keep,

@@ -17,6 +17,8 @@ ap.add_argument("--units", type=int, default=32)
 ap.add_argument("--n", type=int, default=32768)
 ap.add_argument("--mode", default="gemm", choices=["gemm", "closed", "max"])
 ap.add_argument("--iters", type=int, default=3)
+ap.add_argument("--extras", action="store_true",
+                help="also run the in-place eviction and the adaptive-budget kernels")
 a = ap.parse_args()
 wl = W.custom(name="long_trace_32k", n_kv_head=a.units, group=4, window=8, budget=4096,
               n_min=a.n, dup_frac=0.3, dup_noise=0.05, span_len=(32, 256))
@@ -27,6 +29,13 @@ ra, rr = eng.alloc_scores(b)
 idx, nk, Ko, Vo = eng.alloc_outputs(b, 4096)
 for _ in range(a.iters):
     eng.compress(b, 0.1, 4096, ra, rr, idx, nk, Ko, Vo)
+if a.extras:
+    keep, free, nfree = eng.alloc_in_place(b)
+    p_last = torch.empty(b.num_tokens, device="cuda")
+    budgets = torch.empty(b.num_units, dtype=torch.int32, device="cuda")
+    for _ in range(a.iters):
+        eng.evict_in_place(b, idx, nk, 4096, keep, free, nfree)
+        eng.refree_budget(b, 0.01, 4, 4096, p_last, budgets)
 eng.check_status()
 torch.cuda.synchronize()
 print("ok", b.num_units, b.num_tokens)
