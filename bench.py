@@ -42,7 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # grows in proportion to the units processed).  Set to None whenever the
 # kernel changes after its capture; the figures are in profiles/.
 NCU_TRAFFIC_LONG_TRACE = {"gemm": (136.362496e6 + 5.319936e6) * 64,
-                          "score": (134.491648e6 + 3.696384e6) * 64}
+                          "score": (134.494208e6 + 3.787264e6) * 64}
 
 
 def parse():
