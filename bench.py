@@ -38,11 +38,15 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per launch of a kernel on long_trace_32k, from one
-# ncu capture of the 16-unit profiling case scaled by 1024/16 units (traffic
-# grows in proportion to the units processed).  Set to None whenever the
-# kernel changes after its capture; the figures are in profiles/.
-NCU_TRAFFIC_LONG_TRACE = {"gemm": (136.362496e6 + 5.319936e6) * 64,
-                          "score": (134.494208e6 + 3.787264e6) * 64}
+# ncu capture of a 16- or 64-unit profiling case scaled to 1024 units (traffic
+# grows in proportion to the units processed).  Remove an entry whenever its
+# kernel changes after the capture; the figures are in profiles/.
+NCU_TRAFFIC_LONG_TRACE = {
+    # (redundancy mode, kernel): bytes per launch
+    ("gemm", "gemm"): (136.362496e6 + 5.319936e6) * 64,      # 16-unit capture
+    ("gemm", "score"): (134.494208e6 + 3.787264e6) * 64,     # 16-unit capture
+    ("closed", "score"): (537.811968e6 + 17.450496e6) * 16,  # 64-unit capture
+}
 
 
 def parse():
@@ -340,8 +344,8 @@ def run_engine(args, dist: Dist):
     dom = "score" if args.redundancy == "closed" else "gemm"
     roof = dict(rep[dom])
     traffic = None
-    if wl.name == "long_trace_32k" and args.redundancy == "gemm":
-        traffic = NCU_TRAFFIC_LONG_TRACE.get(dom)
+    if wl.name == "long_trace_32k":
+        traffic = NCU_TRAFFIC_LONG_TRACE.get((args.redundancy, dom))
     roofline = {"kernel": dom, "bound": roof["bound"], "achieved": roof["achieved"],
                 "peak": roof["peak"], "unit": roof["unit"], "frac": roof["frac"],
                 "traffic": traffic, "traffic_unit": "bytes per launch (ncu, scaled)",
