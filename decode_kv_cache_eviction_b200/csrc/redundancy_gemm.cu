@@ -58,6 +58,24 @@ __device__ __forceinline__ int find_unit(const int* item_off, int U, int item) {
   return lo;
 }
 
+// tcgen05.mma without a compiler memory clobber: its operands are ordered by
+// the mbarrier waits before it (which carry one), and the issue loop keeps
+// its descriptors in registers.
+template <int kCtaGroup>
+__device__ __forceinline__ void mma_bf16_nm(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  if constexpr (kCtaGroup == 1)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
 template <bool kPair, bool kMax>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     redundancy_gemm_kernel(const __grid_constant__ CUtensorMap amap,
@@ -187,6 +205,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int N = static_cast<int>(__ldg(&p.tok_off[u + 1]) - base);
         const bool aok = mbar_wait(a_full, ai & 1, abort, p.status);
         const uint32_t aaddr = smem_u32(sm + L.a);
+        uint64_t adesc[8];   // A descriptors of this item's 8 K-steps
+#pragma unroll
+        for (int kq = 0; kq < 8; ++kq)
+          adesc[kq] = desc_kmajor_sw128(aaddr + (kq >> 2) * (C::kABytes / 2) + (kq & 3) * 32);
         const int ntiles = (N + C::kN - 1) / C::kN;
         for (int t = 0; t < ntiles; ++t, ++tcount) {
           RKV_GSTAMP(0, tcount, 0);
@@ -196,14 +218,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           RKV_GSTAMP(0, tcount, 2);
           tc_fence_after();
           if (go) {
-            const uint32_t baddr = smem_u32(sm + L.b + stage * C::kBBytes);
+            // B descriptors: the stage's base plus each K-step's offset in
+            // 16-byte units (the start-address field cannot carry: smem < 256 KB)
+            const uint64_t bdesc0 = desc_kmajor_sw128(smem_u32(sm + L.b + stage * C::kBBytes));
             const uint32_t d = tmem + ab * 256;
 #pragma unroll
             for (int kq = 0; kq < 8; ++kq) {
-              const uint32_t ao = (kq >> 2) * (C::kABytes / 2) + (kq & 3) * 32;
               const uint32_t bo = (kq >> 2) * (C::kBBytes / 2) + (kq & 3) * 32;
-              mma_bf16<C::kCtaGroup>(d, desc_kmajor_sw128(aaddr + ao),
-                                     desc_kmajor_sw128(baddr + bo), idesc, kq > 0);
+              mma_bf16_nm<C::kCtaGroup>(d, adesc[kq], bdesc0 + (bo >> 4), idesc, kq > 0);
             }
             if constexpr (kPair) {
               mma_commit_pair(&b_empty[stage]);
