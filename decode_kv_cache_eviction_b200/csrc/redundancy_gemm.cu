@@ -24,7 +24,8 @@
 // 256-key B tile, which halves the shared-memory traffic per SM.
 //
 // Warp roles (640 threads = 5 warps per SM sub-partition): warp 0 TMA producer,
-// warp 1 MMA issuer (leader CTA only in pair mode) and TMEM owner, warps 4-19
+// warp 1 MMA issuer (leader CTA only in pair mode; the whole warp runs the loop
+// and elects one lane per instruction) and TMEM owner, warps 4-19
 // epilogue (warp % 4 selects the TMEM lane quarter, (warp - 4) / 4 the
 // 64-column quarter of the tile).
 #include "ptx.cuh"
@@ -58,22 +59,38 @@ __device__ __forceinline__ int find_unit(const int* item_off, int U, int item) {
   return lo;
 }
 
-// tcgen05.mma without a compiler memory clobber: its operands are ordered by
-// the mbarrier waits before it (which carry one), and the issue loop keeps
-// its descriptors in registers.
+// MMA and commit issued by the whole (converged) warp, one lane elected inside
+// the instruction sequence: the issue loop's values stay warp-uniform.  The
+// MMA carries no compiler memory clobber; its operands are ordered by the
+// mbarrier waits before it, which do.
 template <int kCtaGroup>
-__device__ __forceinline__ void mma_bf16_nm(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
+__device__ __forceinline__ void mma_bf16_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
   if constexpr (kCtaGroup == 1)
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
   else
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void commit_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void commit_pair_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
 }
 
 template <bool kPair, bool kMax>
@@ -194,7 +211,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && leader) {
+    if (leader) {   // the whole warp, converged; one elected lane issues
       const uint32_t idesc = idesc_bf16_f32(C::kMmaM, C::kN);
       int stage = 0, ab = 0;
       uint32_t ph = 0, aph = 0;
@@ -203,7 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int u = find_unit(p.item_off, p.num_units, item);
         const int64_t base = __ldg(&p.tok_off[u]);
         const int N = static_cast<int>(__ldg(&p.tok_off[u + 1]) - base);
-        const bool aok = mbar_wait(a_full, ai & 1, abort, p.status);
+        const bool aok = __all_sync(0xffffffffu, mbar_wait(a_full, ai & 1, abort, p.status));
         const uint32_t aaddr = smem_u32(sm + L.a);
         uint64_t adesc[8];   // A descriptors of this item's 8 K-steps
 #pragma unroll
@@ -215,6 +232,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           bool go = mbar_wait(&b_full[stage], ph, abort, p.status);
           RKV_GSTAMP(0, tcount, 1);
           go = mbar_wait(&acc_empty[ab], aph ^ 1, abort, p.status) && go && aok;
+          go = __all_sync(0xffffffffu, go);
           RKV_GSTAMP(0, tcount, 2);
           tc_fence_after();
           if (go) {
@@ -225,14 +243,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int kq = 0; kq < 8; ++kq) {
               const uint32_t bo = (kq >> 2) * (C::kBBytes / 2) + (kq & 3) * 32;
-              mma_bf16_nm<C::kCtaGroup>(d, adesc[kq], bdesc0 + (bo >> 4), idesc, kq > 0);
+              mma_bf16_elect<C::kCtaGroup>(d, adesc[kq], bdesc0 + (bo >> 4), idesc, kq > 0);
             }
             if constexpr (kPair) {
-              mma_commit_pair(&b_empty[stage]);
-              mma_commit_pair(&acc_full[ab]);
+              commit_pair_elect(&b_empty[stage]);
+              commit_pair_elect(&acc_full[ab]);
             } else {
-              mma_commit(&b_empty[stage]);
-              mma_commit(&acc_full[ab]);
+              commit_elect(&b_empty[stage]);
+              commit_elect(&acc_full[ab]);
             }
           }
           RKV_GSTAMP(0, tcount, 3);
@@ -240,8 +258,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (++ab == 2) { ab = 0; aph ^= 1; }
         }
         if (aok) {
-          if constexpr (kPair) mma_commit_pair(a_empty);
-          else mma_commit(a_empty);
+          if constexpr (kPair) commit_pair_elect(a_empty);
+          else commit_elect(a_empty);
         }
       }
     }
