@@ -43,7 +43,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel changes after the capture; the figures are in profiles/.
 NCU_TRAFFIC_LONG_TRACE = {
     # (redundancy mode, kernel): bytes per launch
-    ("gemm", "gemm"): (136.362496e6 + 5.319936e6) * 64,      # 16-unit capture
+    ("gemm", "gemm"): (136.425472e6 + 5.207808e6) * 64,      # 16-unit capture
     ("gemm", "score"): (134.494208e6 + 3.787264e6) * 64,     # 16-unit capture
     ("closed", "score"): (537.811968e6 + 17.450496e6) * 16,  # 64-unit capture
 }
