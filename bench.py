@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--workload", default="long_trace_32k", choices=W.WORKLOAD_ORDER)
     ap.add_argument("--redundancy", default="gemm", choices=["gemm", "closed", "max"])
     ap.add_argument("--lam", type=float, default=0.1)
+    ap.add_argument("--dense-gemm", dest="symmetric", action="store_false",
+                    help="run the redundancy GEMM over all tiles instead of the symmetric form")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--e2e-chunk", type=int, default=0,
@@ -174,6 +176,11 @@ def algorithmic(batch: Batch, wl: W.Workload):
         "score_bytes": float((2 * d + 8) * n.sum() + 2 * d * U * wl.group * wl.window),
         # dense-equivalent tile products of the definition (rows in C x all N keys)
         "gemm_flops": float((2 * c * n * d).sum()),
+        # symmetric form: the 256 x 256 tiles actually executed (on and above
+        # the diagonal block of the candidate row blocks)
+        "gemm_sym_flops": float(sum(2 * d * 256 * 256 * (nbr * nbc - nbr * (nbr - 1) // 2)
+                                    for nbr, nbc in zip(((c + 255) // 256).astype(np.int64),
+                                                        ((n + 255) // 256).astype(np.int64)))),
         # a and r read, kept indices and counts written
         "select_bytes": float(8 * c.sum() + 4 * U * W_ + 4 * U),
         # kept K and V rows read; the whole [U, B+w] outputs written
@@ -211,7 +218,7 @@ def timed(fn, steps, warmup, dist: Dist, eng=None):
     return dist.max(ms), per_kernel, launches
 
 
-def kernel_report(per_kernel, alg, pk, src):
+def kernel_report(per_kernel, alg, pk, src, symmetric=False):
     hbm = pk["hbm_gbs"]
     out = {}
     for name, (tot, n) in per_kernel.items():
@@ -220,9 +227,14 @@ def kernel_report(per_kernel, alg, pk, src):
         ms = tot / n
         ent = {"ms": round(ms, 4), "launches": n}
         if name == "gemm":
-            tf = alg["gemm_flops"] / (ms * 1e-3) / 1e12
+            # the tensor-pipe fraction counts the flops the kernel executes
+            # (the symmetric form skips the tiles below the diagonal)
+            flops = alg["gemm_sym_flops"] if symmetric else alg["gemm_flops"]
+            tf = flops / (ms * 1e-3) / 1e12
             ent.update(bound="tensor", achieved=round(tf, 2), unit="TFLOP/s",
                        peak=pk["bf16_tflops_sustained"], frac=round(tf / pk["bf16_tflops_sustained"], 4))
+            if symmetric:
+                ent["dense_equivalent_tflops"] = round(alg["gemm_flops"] / (ms * 1e-3) / 1e12, 2)
         elif name in ("score", "select", "compact", "evict", "refree"):
             gbs = alg[f"{name}_bytes"] / (ms * 1e-3) / 1e9
             ent.update(bound="hbm", achieved=round(gbs, 1), unit="GB/s", peak=hbm,
@@ -258,12 +270,14 @@ def cpu_baseline(batch: Batch, wl: W.Workload, lam: float, seconds: float, redun
                        f"{t_used:.1f} s on {cores} host threads)")}
 
 
-def config_of(wl: W.Workload, batch: Batch, redundancy: str, lam: float, world: int):
+def config_of(wl: W.Workload, batch: Batch, redundancy: str, lam: float, world: int,
+              gemm_form: str = "dense"):
     n = np.diff(batch.tok_off_host)
     return {"workload": wl.name, "units": batch.num_units, "tokens": int(n.sum()),
             "n_min": int(n.min()), "n_max": int(n.max()), "head_dim": wl.head_dim,
             "group": wl.group, "window": wl.window, "budget": wl.budget, "lambda": lam,
-            "redundancy": redundancy, "l2": "inputs larger than L2 (K+V %.1f GiB per GPU)"
+            "redundancy": redundancy, "gemm": gemm_form,
+            "l2": "inputs larger than L2 (K+V %.1f GiB per GPU)"
             % (2 * n.sum() * wl.head_dim * 2 / 2**30),
             "parallelism": f"replicas x{world} (units sharded per GPU, no collective)"}
 
@@ -325,7 +339,9 @@ def run_engine(args, dist: Dist):
     alg = algorithmic(batch, wl)
 
     def measure(mode):
-        eng = Engine(wl.group, wl.window, batch.num_units, tokens, redundancy=mode)
+        sym = mode == "gemm" and args.symmetric
+        eng = Engine(wl.group, wl.window, batch.num_units, tokens, redundancy=mode,
+                     symmetric_gemm=sym)
         a, r = eng.alloc_scores(batch)
         idx, nk, Ko, Vo = eng.alloc_outputs(batch, wl.budget)
         step = lambda: eng.compress(batch, args.lam, wl.budget, a, r, idx, nk, Ko, Vo)
@@ -333,11 +349,12 @@ def run_engine(args, dist: Dist):
         eng.check_status()
         ms, per_kernel, launches = timed(step, args.steps, args.warmup, dist, eng)
         eng.check_status()
-        rep = kernel_report(per_kernel, alg, pk, src)
+        rep = kernel_report(per_kernel, alg, pk, src, symmetric=sym)
         del a, r, idx, nk, Ko, Vo
         return eng, ms, rep, launches
 
     clk = Clocks(dist.local) if dist.rank == 0 else None
+    sym_main = args.redundancy == "gemm" and args.symmetric
     eng, ms, rep, launches = measure(args.redundancy)
     clocks = clk.stop() if clk else None
     value = tokens * dist.world / (ms * 1e-3)
@@ -345,7 +362,7 @@ def run_engine(args, dist: Dist):
     roof = dict(rep[dom])
     traffic = None
     if wl.name == "long_trace_32k":
-        traffic = NCU_TRAFFIC_LONG_TRACE.get((args.redundancy, dom))
+        traffic = NCU_TRAFFIC_LONG_TRACE.get(("gemm_sym" if sym_main else args.redundancy, dom))
     roofline = {"kernel": dom, "bound": roof["bound"], "achieved": roof["achieved"],
                 "peak": roof["peak"], "unit": roof["unit"], "frac": roof["frac"],
                 "traffic": traffic, "traffic_unit": "bytes per launch (ncu, scaled)",
@@ -379,7 +396,8 @@ def run_engine(args, dist: Dist):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": config_of(wl, batch, args.redundancy, args.lam, dist.world),
+                "config": config_of(wl, batch, args.redundancy, args.lam, dist.world,
+                                    "symmetric" if sym_main else "dense"),
                 "roofline": roofline, "kernels": rep, "gpu_launches": launches,
                 "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
                 "secondary": secondary, "in_place": in_place, "adaptive": adaptive}

@@ -30,6 +30,7 @@ RKV_REDUNDANCY_GEMM = 0
 RKV_REDUNDANCY_CLOSED_FORM = 1
 RKV_REDUNDANCY_MAX = 2
 RKV_FLAG_GEMM_SINGLE_CTA = 1
+RKV_FLAG_GEMM_SYMMETRIC = 2
 
 # Every function declared in include/rkv.h.
 EXPORTS = ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact",
@@ -170,11 +171,13 @@ class Engine:
     """One engine = one configuration and its device workspace."""
 
     def __init__(self, group: int, window: int, max_units: int, max_tokens: int,
-                 head_dim: int = 128, redundancy: str = "gemm", single_cta_gemm=False):
+                 head_dim: int = 128, redundancy: str = "gemm", single_cta_gemm=False,
+                 symmetric_gemm=False):
         mode = {"gemm": RKV_REDUNDANCY_GEMM, "closed": RKV_REDUNDANCY_CLOSED_FORM,
                 "max": RKV_REDUNDANCY_MAX}[redundancy]
-        self.cfg = RkvConfig(head_dim, group, window, max_units, max_tokens, mode,
-                             RKV_FLAG_GEMM_SINGLE_CTA if single_cta_gemm else 0)
+        flags = ((RKV_FLAG_GEMM_SINGLE_CTA if single_cta_gemm else 0) |
+                 (RKV_FLAG_GEMM_SYMMETRIC if symmetric_gemm else 0))
+        self.cfg = RkvConfig(head_dim, group, window, max_units, max_tokens, mode, flags)
         self.group, self.window = group, window
         h = ctypes.c_void_p()
         _check(lib().rkv_create(ctypes.byref(self.cfg), ctypes.byref(h)), "rkv_create")

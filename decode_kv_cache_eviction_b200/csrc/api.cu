@@ -106,7 +106,11 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   if (cfg->redundancy != RKV_REDUNDANCY_GEMM && cfg->redundancy != RKV_REDUNDANCY_CLOSED_FORM &&
       cfg->redundancy != RKV_REDUNDANCY_MAX)
     return RKV_ERR_INVALID_ARG;
-  if ((cfg->flags & ~RKV_FLAG_GEMM_SINGLE_CTA) != 0) return RKV_ERR_INVALID_ARG;
+  if ((cfg->flags & ~(RKV_FLAG_GEMM_SINGLE_CTA | RKV_FLAG_GEMM_SYMMETRIC)) != 0)
+    return RKV_ERR_INVALID_ARG;
+  if ((cfg->flags & RKV_FLAG_GEMM_SYMMETRIC) &&
+      ((cfg->flags & RKV_FLAG_GEMM_SINGLE_CTA) || cfg->redundancy != RKV_REDUNDANCY_GEMM))
+    return RKV_ERR_UNSUPPORTED;
   if (cfg->head_dim != kHeadDim) return RKV_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(cfg->group) * cfg->window > kMaxRows) return RKV_ERR_UNSUPPORTED;
   if (cfg->max_tokens >= (static_cast<int64_t>(1) << 31)) return RKV_ERR_UNSUPPORTED;
@@ -131,6 +135,7 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   e->rp = cfg->group * cfg->window <= 16 ? 16 : 32;
   e->pair = (cfg->flags & RKV_FLAG_GEMM_SINGLE_CTA) == 0;
   e->rowmax = cfg->redundancy == RKV_REDUNDANCY_MAX;
+  e->sym = (cfg->flags & RKV_FLAG_GEMM_SYMMETRIC) != 0;
 
   cudaDriverEntryPointQueryResult q;
   void* fn = nullptr;
@@ -169,11 +174,11 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
     return cuda_fail(cudaErrorUnknown);
   }
   if (!closed) {
-    if (gemm_configure(e->pair, e->rowmax) != cudaSuccess) {
+    if (gemm_configure(e->pair, e->rowmax, e->sym) != cudaSuccess) {
       delete e;
       return cuda_fail(cudaErrorUnknown);
     }
-    e->gemm_ctas = gemm_max_ctas(e->pair, e->rowmax);
+    e->gemm_ctas = gemm_max_ctas(e->pair, e->rowmax, e->sym);
     if (e->gemm_ctas <= 0) {
       delete e;
       return RKV_ERR_UNSUPPORTED;
@@ -188,6 +193,8 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
     ok = ok && cudaMalloc(&e->rho, sizeof(float) * nrho) == cudaSuccess;
     ok = ok && cudaMalloc(&e->rho_off, sizeof(int64_t) * (cfg->max_units + 1)) == cudaSuccess;
   }
+  if (e->sym)
+    ok = ok && cudaMalloc(&e->cs_off, sizeof(int64_t) * (cfg->max_units + 1)) == cudaSuccess;
   ok = ok && cudaMemset(e->status, 0, 16) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
@@ -196,6 +203,7 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
     cudaFree(e->unit_cnt);
     cudaFree(e->rho);
     cudaFree(e->rho_off);
+    cudaFree(e->cs_off);
     delete e;
     return RKV_ERR_OOM;
   }
@@ -248,6 +256,8 @@ int rkv_destroy(rkv_engine* e) {
   cudaFree(e->unit_cnt);
   cudaFree(e->rho);
   cudaFree(e->rho_off);
+  cudaFree(e->cs_off);
+  cudaFree(e->cs);
   delete e;
   return RKV_OK;
 }
@@ -270,6 +280,24 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool closed = e->cfg.redundancy == RKV_REDUNDANCY_CLOSED_FORM;
   const int R = e->cfg.group * e->cfg.window;
+  // symmetric form: column-partial scratch for this batch (grown before
+  // anything is enqueued; zeroed on the stream before the GEMM)
+  int64_t cs_need = 0;
+  if (e->sym) {
+    for (int u = 0; u < U; ++u)
+      cs_need += sym_scratch_floats(b->tok_off_host[u + 1] - b->tok_off_host[u], e->cfg.window);
+    if (cs_need > e->cs_cap) {
+      cudaFree(e->cs);
+      e->cs = nullptr;
+      e->cs_cap = 0;
+      if (cudaMalloc(&e->cs, sizeof(float) * cs_need) != cudaSuccess) {
+        cudaGetLastError();
+        e->cs = nullptr;
+        return RKV_ERR_OOM;
+      }
+      e->cs_cap = cs_need;
+    }
+  }
 
   const int cs = score_cluster_size(nmax, e->rp, e->max_cs);
   if (cs == 0) return RKV_ERR_UNSUPPORTED;
@@ -300,7 +328,7 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   if (!closed) {   // row blocks for the GEMM and the padded rho layout the score kernel writes
     t_begin(e, RKV_KERNEL_PLAN, st);
     err = launch_plan(b->tok_off, U, e->cfg.window, rows_per_item, e->item_off, e->unit_cnt,
-                      e->rho_off, st);
+                      e->rho_off, e->sym ? e->cs_off : nullptr, st);
     t_end(e, st);
     if (err != cudaSuccess) return cuda_fail(err);
     ++e->launches;
@@ -330,6 +358,8 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   g.r_dst = r;
   g.unit_cnt = e->unit_cnt;
   g.status = e->status;
+  g.cs = e->sym ? e->cs : nullptr;
+  g.cs_off = e->sym ? e->cs_off : nullptr;
   int64_t items = 0;
   for (int u = 0; u < U; ++u) {
     const int64_t c = b->tok_off_host[u + 1] - b->tok_off_host[u] - e->cfg.window;
@@ -339,8 +369,16 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   int64_t nctas = e->gemm_ctas;
   const int64_t need = items * (e->pair ? 2 : 1);
   if (nctas > need) nctas = need;
+  if (e->sym && cs_need > 0) {
+    err = cudaMemsetAsync(e->cs, 0, sizeof(float) * cs_need, st);
+    if (err != cudaSuccess) return cuda_fail(err);
+  }
   t_begin(e, RKV_KERNEL_GEMM, st);
-  err = launch_gemm(amap, bmap, g, e->pair, e->rowmax, static_cast<int>(nctas), st);
+  err = launch_gemm(amap, bmap, g, e->pair, e->rowmax, e->sym, static_cast<int>(nctas), st);
+  if (err == cudaSuccess && e->sym) {
+    ++e->launches;
+    err = launch_sym_finish(g, e->nsm, st);   // timed together with the GEMM
+  }
   t_end(e, st);
   if (err != cudaSuccess) return cuda_fail(err);
   ++e->launches;

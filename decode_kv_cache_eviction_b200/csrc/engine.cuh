@@ -30,12 +30,16 @@ struct rkv_engine {
   int max_n = 0;               // largest supported N_u
   bool pair = true;
   bool rowmax = false;   // row-max redundancy epilogue
+  bool sym = false;      // symmetric GEMM (tiles on and above the diagonal)
   int gemm_ctas = 0;
   float* rho = nullptr;        // [max_tokens + kRhoAlign * max_units] padded 1/||k||
   int64_t* rho_off = nullptr;  // [max_units + 1]
   int* item_off = nullptr;     // [max_units + 1]
   int* unit_cnt = nullptr;     // [max_units]
   int* status = nullptr;       // [1]
+  int64_t* cs_off = nullptr;   // [max_units + 1] symmetric form: scratch offsets
+  float* cs = nullptr;         // symmetric form: column partials, grown on demand
+  int64_t cs_cap = 0;          // floats allocated in cs
   int64_t launches = 0;
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   // per-kernel timing (rkv_set_timing)

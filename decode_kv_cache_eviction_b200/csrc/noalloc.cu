@@ -101,11 +101,11 @@ int setup(int dev, DeviceState** out) {
     }
     if (d.max_cs[k] == 0) return RKV_ERR_UNSUPPORTED;
   }
-  if (gemm_configure(true, false) != cudaSuccess) {
+  if (gemm_configure(true, false, false) != cudaSuccess) {
     cudaGetLastError();
     return RKV_ERR_CUDA;
   }
-  d.gemm_ctas = gemm_max_ctas(true, false);
+  d.gemm_ctas = gemm_max_ctas(true, false, false);
   if (d.gemm_ctas <= 0) return RKV_ERR_UNSUPPORTED;
   d.ready = true;
   *out = &d;
@@ -195,7 +195,7 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   p.rho_off = s->rho_off;
   p.status = s->status;
   constexpr int kRows = GemmCfg<true>::kRowsPerItem;
-  if (launch_plan(b->tok_off, U, window, kRows, s->item_off, s->unit_cnt, s->rho_off, st) !=
+  if (launch_plan(b->tok_off, U, window, kRows, s->item_off, s->unit_cnt, s->rho_off, nullptr, st) !=
       cudaSuccess) {
     cudaGetLastError();
     return RKV_ERR_CUDA;
@@ -221,9 +221,11 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   g.r_dst = r;
   g.unit_cnt = s->unit_cnt;
   g.status = s->status;
+  g.cs = nullptr;
+  g.cs_off = nullptr;
   int64_t nctas = d->gemm_ctas;
   if (nctas > 2 * items) nctas = 2 * items;
-  if (launch_gemm(amap, bmap, g, true, false, static_cast<int>(nctas), st) != cudaSuccess) {
+  if (launch_gemm(amap, bmap, g, true, false, false, static_cast<int>(nctas), st) != cudaSuccess) {
     cudaGetLastError();
     return RKV_ERR_CUDA;
   }

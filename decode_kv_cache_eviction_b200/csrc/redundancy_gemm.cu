@@ -93,7 +93,7 @@ __device__ __forceinline__ void commit_pair_elect(uint64_t* bar) {
       : "memory");
 }
 
-template <bool kPair, bool kMax>
+template <bool kPair, bool kMax, bool kSym>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     redundancy_gemm_kernel(const __grid_constant__ CUtensorMap amap,
                            const __grid_constant__ CUtensorMap bmap, const GemmParams p) {
@@ -182,7 +182,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
         const int ntiles = (N + C::kN - 1) / C::kN;
-        for (int t = 0; t < ntiles; ++t) {
+        // symmetric form: only the tiles on and above the diagonal block
+        for (int t = kSym ? blk : 0; t < ntiles; ++t) {
           if (mbar_wait(&b_empty[stage], ph ^ 1, abort, p.status)) {
             uint8_t* bd = sm + L.b + stage * C::kBBytes;
             const int yb = static_cast<int>(base + t * C::kN + rank * C::kBRows);
@@ -227,7 +228,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int kq = 0; kq < 8; ++kq)
           adesc[kq] = desc_kmajor_sw128(aaddr + (kq >> 2) * (C::kABytes / 2) + (kq & 3) * 32);
         const int ntiles = (N + C::kN - 1) / C::kN;
-        for (int t = 0; t < ntiles; ++t, ++tcount) {
+        const int t0 = kSym ? item - __ldg(&p.item_off[u]) : 0;
+        for (int t = t0; t < ntiles; ++t, ++tcount) {
           RKV_GSTAMP(0, tcount, 0);
           bool go = mbar_wait(&b_full[stage], ph, abort, p.status);
           RKV_GSTAMP(0, tcount, 1);
@@ -278,6 +280,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int ab = 0;
     uint32_t aph = 0;
     uint32_t rt = 0;   // rho tiles consumed so far
+    int colbuf = 0;    // symmetric form: double buffer of the column exchange
     for (int item = group_id; item < n_items; item += ngroups) {
       const int u = find_unit(p.item_off, p.num_units, item);
       const int blk = item - __ldg(&p.item_off[u]);
@@ -292,8 +295,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       float a0 = kInit, b0 = kInit, a1 = kInit, b1 = kInit;
       float a2 = kInit, b2 = kInit, a3 = kInit, b3 = kInit;
       const int ntiles = (N + C::kN - 1) / C::kN;
-      for (int t = 0; t < ntiles; ++t, ++rt) {
+      // symmetric form: weights rho_i of this thread's 4 rows (for the column
+      // sums) and the scratch segment of this item (256 floats per tile above
+      // the diagonal)
+      float rw[4] = {0.f, 0.f, 0.f, 0.f};
+      int64_t cs_item = 0;
+      if constexpr (kSym) {
+        const float* rho_u = p.rho + __ldg(&p.rho_off[u]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) rw[k] = __ldg(&rho_u[rbase + q * 32 + gq + 8 * k]);
+        cs_item = __ldg(&p.cs_off[u]) +
+                  256 * (static_cast<int64_t>(blk) * (ntiles - 1) -
+                         static_cast<int64_t>(blk) * (blk - 1) / 2);
+      }
+      for (int t = kSym ? blk : 0; t < ntiles; ++t, ++rt) {
         const int j0 = t * C::kN;
+        const bool colsum = kSym && t > blk;   // tile above the diagonal block
         const uint32_t rs_slot = rt % kRhoSlots;
         const float* rs = rho_ring + rs_slot * 256 + cg * 64 + 2 * tq;
         if (etid == 0) RKV_GSTAMP(1, rt, 0);
@@ -347,11 +364,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         };
+        // symmetric form: rho-weighted column partials over this thread's 4
+        // rows, columns 8k + 2tq + {0, 1} (pairs k = 0..7)
+        float cp[16];
+        auto colfold = [&](int h) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            fma2(cp[2 * k], cp[2 * k + 1], __uint_as_float(v[4 * k]),
+                 __uint_as_float(v[4 * k + 1]), rw[2 * h], rw[2 * h]);
+            fma2(cp[2 * k], cp[2 * k + 1], __uint_as_float(v[4 * k + 2]),
+                 __uint_as_float(v[4 * k + 3]), rw[2 * h + 1], rw[2 * h + 1]);
+          }
+        };
+        if constexpr (kSym) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) cp[k] = 0.f;
+        }
         tmem_ld16x256b_x8(tbase, v);                 // lanes 0-15 of the quarter
         tmem_wait_ld();
         if (etid == 0) RKV_GSTAMP(1, rt, 2);
         if (masked) patch(0);
         fold(a0, b0, a1, b1);
+        if (colsum) colfold(0);
         tmem_ld16x256b_x8(tbase + (16u << 16), v);   // lanes 16-31
         tmem_wait_ld();
         tc_fence_before();
@@ -366,6 +400,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (etid == 0) RKV_GSTAMP(1, rt, 3);
         __syncwarp();
         if (lane == 0) mbar_arrive(&rho_empty[rs_slot]);
+        if constexpr (kSym) {
+          if (colsum) {
+            colfold(1);
+            // reduce-scatter over the quad index gq (lane bits 2-4): lane l
+            // keeps the column sums of columns 2l and 2l + 1 of the group
+#pragma unroll
+            for (int sft = 16, n = 8; sft >= 4; sft >>= 1, n >>= 1) {
+              const bool up = (lane & sft) != 0;
+#pragma unroll
+              for (int k = 0; k < n; ++k) {
+                const float send = up ? cp[k] : cp[k + n];
+                const float keep = up ? cp[k + n] : cp[k];
+                cp[k] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+              }
+            }
+            // the four lane quarters of this column group, then one 2-addend
+            // atomic per column pair (the pair's other CTA adds its rows)
+            float2* cx = reinterpret_cast<float2*>(sm + L.colx) + (colbuf * 4 + cg) * 4 * 32;
+            cx[q * 32 + lane] = make_float2(cp[0], cp[1]);
+            named_bar_sync(4 + cg, 128);
+            if (q == 0) {
+              float2 acc = cx[lane];
+#pragma unroll
+              for (int qq = 1; qq < 4; ++qq) {
+                const float2 y = cx[qq * 32 + lane];
+                acc.x += y.x;
+                acc.y += y.y;
+              }
+              // fire-and-forget reduction (no returned value to wait for)
+              float* dst =
+                  p.cs + cs_item + static_cast<int64_t>(t - blk - 1) * 256 + cg * 64 + 2 * lane;
+              asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(dst), "f"(acc.x),
+                           "f"(acc.y)
+                           : "memory");
+            }
+            colbuf ^= 1;
+          }
+        }
       }
       // ---- item end: finish the rows over the quad (its four threads hold
       // disjoint columns), combine the four column groups, write m
@@ -389,10 +461,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if constexpr (kMax) {
           tot = fmaxf(fmaxf(tot, rowx[rl]), fmaxf(rowx[128 + rl], rowx[256 + rl]));
           p.m_dst[base + i] = rho_i * tot;
+        } else if constexpr (kSym) {
+          // this item's columns only (blocks blk ..); the earlier blocks'
+          // share comes from their column partials in the final pass
+          p.m_dst[base + i] = (tot + rowx[rl]) + (rowx[128 + rl] + rowx[256 + rl]);
         } else {
           tot += (rowx[rl] + rowx[128 + rl]) + rowx[256 + rl];
           p.m_dst[base + i] = rho_i * tot / static_cast<float>(N - 1);
         }
+      }
+      if constexpr (kSym) {
+        // the row partials are complete; the finish kernel adds the column
+        // partials and applies the softmax (doing it here would stall a pair)
+        named_bar_sync(3, 512);
+        continue;
       }
       __threadfence();
       named_bar_sync(3, 512);
@@ -403,8 +485,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       named_bar_sync(3, 512);
       if (*last_flag) {
-        // ---- token softmax over the unit's candidates (|m| <= 1: no max shift)
         __threadfence();
+        // ---- token softmax over the unit's candidates (|m| <= 1: no max shift)
         float sum = 0.f;
         for (int ii = etid; ii < c; ii += 512) sum += ex2(__ldcg(&p.m_dst[base + ii]) * kLog2e);
         sum = warp_reduce_sum(sum);
@@ -432,62 +514,139 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // One block: items per unit and their prefix, 256-aligned rho segment
-// offsets, and zeroed unit counters.
+// offsets, zeroed unit counters and (symmetric form, cs_off != null) the
+// offsets of each unit's column-partial scratch.
 __global__ void plan_kernel(const int64_t* tok_off, int U, int w, int rows_per_item,
-                            int* item_off, int* unit_cnt, int64_t* rho_off) {
-  __shared__ long long wsum[2][32];
+                            int* item_off, int* unit_cnt, int64_t* rho_off, int64_t* cs_off) {
+  __shared__ long long wsum[3][32];
   const int tid = threadIdx.x, nt = blockDim.x;
   const int per = (U + nt - 1) / nt;
   const int u0 = min(U, tid * per), u1 = min(U, u0 + per);
-  long long li = 0, lr = 0;   // this thread's items and padded rho length
+  long long li = 0, lr = 0, ls = 0;   // this thread's items, rho and scratch lengths
   for (int u = u0; u < u1; ++u) {
     const int64_t n = tok_off[u + 1] - tok_off[u];
     const int64_t c = n - w;
     li += c > 0 ? (c + rows_per_item - 1) / rows_per_item : 0;
     lr += (n + kRhoAlign - 1) / kRhoAlign * kRhoAlign;
+    ls += sym_scratch_floats(n, w);
     unit_cnt[u] = 0;
   }
-  // block exclusive scans of li and lr
-  long long ii = li, ir = lr;
+  // block exclusive scans of li, lr and ls
+  long long ii = li, ir = lr, is = ls;
   const int lane = tid & 31, wp = tid >> 5;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const long long yi = __shfl_up_sync(0xffffffffu, ii, o);
     const long long yr = __shfl_up_sync(0xffffffffu, ir, o);
-    if (lane >= o) { ii += yi; ir += yr; }
+    const long long ys = __shfl_up_sync(0xffffffffu, is, o);
+    if (lane >= o) { ii += yi; ir += yr; is += ys; }
   }
-  if (lane == 31) { wsum[0][wp] = ii; wsum[1][wp] = ir; }
+  if (lane == 31) { wsum[0][wp] = ii; wsum[1][wp] = ir; wsum[2][wp] = is; }
   __syncthreads();
   if (wp == 0) {
     long long xi = lane < (nt >> 5) ? wsum[0][lane] : 0;
     long long xr = lane < (nt >> 5) ? wsum[1][lane] : 0;
+    long long xs = lane < (nt >> 5) ? wsum[2][lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const long long yi = __shfl_up_sync(0xffffffffu, xi, o);
       const long long yr = __shfl_up_sync(0xffffffffu, xr, o);
-      if (lane >= o) { xi += yi; xr += yr; }
+      const long long ys = __shfl_up_sync(0xffffffffu, xs, o);
+      if (lane >= o) { xi += yi; xr += yr; xs += ys; }
     }
     wsum[0][lane] = xi;
     wsum[1][lane] = xr;
+    wsum[2][lane] = xs;
   }
   __syncthreads();
   long long ri = ii - li + (wp > 0 ? wsum[0][wp - 1] : 0);
   long long rr = ir - lr + (wp > 0 ? wsum[1][wp - 1] : 0);
+  long long rs = is - ls + (wp > 0 ? wsum[2][wp - 1] : 0);
   for (int u = u0; u < u1; ++u) {
     item_off[u] = static_cast<int>(ri);
     rho_off[u] = rr;
+    if (cs_off) cs_off[u] = rs;
     const int64_t n = tok_off[u + 1] - tok_off[u];
     const int64_t c = n - w;
     ri += c > 0 ? (c + rows_per_item - 1) / rows_per_item : 0;
     rr += (n + kRhoAlign - 1) / kRhoAlign * kRhoAlign;
+    rs += sym_scratch_floats(n, w);
   }
   if (u1 == U && u0 < u1) {
     item_off[U] = static_cast<int>(ri);
     rho_off[U] = rr;
+    if (cs_off) cs_off[U] = rs;
   }
   if (U == 0 && tid == 0) {
     item_off[0] = 0;
     rho_off[0] = 0;
+    if (cs_off) cs_off[0] = 0;
+  }
+}
+
+// Symmetric form, after the GEMM: one CTA per unit adds to each candidate row's
+// partial (left in m_dst) the column partials of the earlier row blocks, in
+// block order, scales by rho_i / (N - 1), and applies the token softmax.
+// Block a2's partials for every later row are contiguous (index i - 256
+// (a2 + 1)), so a thread takes 4 consecutive rows and reads one aligned float4
+// per earlier block.
+constexpr int kFinishThreads = 512;
+__global__ void __launch_bounds__(kFinishThreads)
+    sym_finish_kernel(const int64_t* __restrict__ tok_off, int U, int w,
+                      const float* __restrict__ rho, const int64_t* __restrict__ rho_off,
+                      const float* __restrict__ cs, const int64_t* __restrict__ cs_off,
+                      float* m_dst, float* r_dst) {
+  __shared__ float wred[kFinishThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+  for (int u = blockIdx.x; u < U; u += gridDim.x) {
+    const int64_t base = tok_off[u];
+    const int N = static_cast<int>(tok_off[u + 1] - base);
+    const int c = N - w;
+    if (c <= 0) continue;
+    const int nbc = (N + 255) / 256;
+    const float* rho_u = rho + rho_off[u];
+    const int64_t cs0 = cs_off[u];
+    const float inv_nm1 = 1.f / static_cast<float>(N - 1);
+    float esum = 0.f;
+    for (int r0 = 4 * tid; r0 < c; r0 += 4 * kFinishThreads) {
+      const int a = r0 >> 8;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int a2 = 0; a2 < a; ++a2) {
+        const int64_t seg = cs0 + 256 * (static_cast<int64_t>(a2) * (nbc - 1) -
+                                         static_cast<int64_t>(a2) * (a2 - 1) / 2);
+        const float4 y = __ldcs(reinterpret_cast<const float4*>(cs + seg + (r0 - 256 * (a2 + 1))));
+        acc.x += y.x;
+        acc.y += y.y;
+        acc.z += y.z;
+        acc.w += y.w;
+      }
+      const float part[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = r0 + e;
+        if (i < c) {
+          const float m = rho_u[i] * (m_dst[base + i] + part[e]) * inv_nm1;
+          m_dst[base + i] = m;
+          esum += ex2(m * kLog2e);
+        }
+      }
+    }
+    // token softmax (|m| <= 1: no max shift); each thread rereads its own rows
+    esum = warp_reduce_sum(esum);
+    if (lane == 0) wred[wp] = esum;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int k = 0; k < kFinishThreads / 32; ++k) tot += wred[k];
+    const float inv = 1.f / tot;
+    for (int r0 = 4 * tid; r0 < c; r0 += 4 * kFinishThreads)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = r0 + e;
+        if (i < c) r_dst[base + i] = ex2(m_dst[base + i] * kLog2e) * inv;
+      }
+    __syncthreads();   // wred is reused by the next unit
   }
 }
 
@@ -500,23 +659,26 @@ cudaError_t gemm_trace_read(void* dst, size_t bytes) {
 #endif
 
 namespace {
-void* gemm_fn(bool pair, bool rowmax) {
-  if (pair) return rowmax ? reinterpret_cast<void*>(&redundancy_gemm_kernel<true, true>)
-                          : reinterpret_cast<void*>(&redundancy_gemm_kernel<true, false>);
-  return rowmax ? reinterpret_cast<void*>(&redundancy_gemm_kernel<false, true>)
-                : reinterpret_cast<void*>(&redundancy_gemm_kernel<false, false>);
+// The symmetric form exists for CTA pairs and the row mean only (its tiles
+// are 256 x 256 and the column sums are added linearly).
+void* gemm_fn(bool pair, bool rowmax, bool sym) {
+  if (sym) return reinterpret_cast<void*>(&redundancy_gemm_kernel<true, false, true>);
+  if (pair) return rowmax ? reinterpret_cast<void*>(&redundancy_gemm_kernel<true, true, false>)
+                          : reinterpret_cast<void*>(&redundancy_gemm_kernel<true, false, false>);
+  return rowmax ? reinterpret_cast<void*>(&redundancy_gemm_kernel<false, true, false>)
+                : reinterpret_cast<void*>(&redundancy_gemm_kernel<false, false, false>);
 }
 }  // namespace
 
-cudaError_t gemm_configure(bool pair, bool rowmax) {
+cudaError_t gemm_configure(bool pair, bool rowmax, bool sym) {
   const int smem = (pair ? gemm_layout<true>().total : gemm_layout<false>().total) + 1024;
-  return cudaFuncSetAttribute(gemm_fn(pair, rowmax), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              smem);
+  return cudaFuncSetAttribute(gemm_fn(pair, rowmax, sym),
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
-int gemm_max_ctas(bool pair, bool rowmax) {
+int gemm_max_ctas(bool pair, bool rowmax, bool sym) {
   const int smem = (pair ? gemm_layout<true>().total : gemm_layout<false>().total) + 1024;
-  void* f = gemm_fn(pair, rowmax);
+  void* f = gemm_fn(pair, rowmax, sym);
   int dev = 0, nsm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -548,13 +710,23 @@ int gemm_max_ctas(bool pair, bool rowmax) {
 }
 
 cudaError_t launch_plan(const int64_t* tok_off, int U, int w, int rows_per_item, int* item_off,
-                        int* unit_cnt, int64_t* rho_off, cudaStream_t st) {
-  plan_kernel<<<1, 1024, 0, st>>>(tok_off, U, w, rows_per_item, item_off, unit_cnt, rho_off);
+                        int* unit_cnt, int64_t* rho_off, int64_t* cs_off, cudaStream_t st) {
+  plan_kernel<<<1, 1024, 0, st>>>(tok_off, U, w, rows_per_item, item_off, unit_cnt, rho_off,
+                                  cs_off);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sym_finish(const GemmParams& p, int nsm, cudaStream_t st) {
+  int grid = nsm * 4;
+  if (grid > p.num_units) grid = p.num_units;
+  sym_finish_kernel<<<grid, kFinishThreads, 0, st>>>(p.tok_off, p.num_units, p.w, p.rho,
+                                                     p.rho_off, p.cs, p.cs_off, p.m_dst,
+                                                     p.r_dst);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const GemmParams& p,
-                        bool pair, bool rowmax, int nctas, cudaStream_t st) {
+                        bool pair, bool rowmax, bool sym, int nctas, cudaStream_t st) {
   const int smem = (pair ? gemm_layout<true>().total : gemm_layout<false>().total) + 1024;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nctas, 1, 1);
@@ -568,12 +740,16 @@ cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const 
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = pair ? 1 : 0;
+  if (sym)
+    return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<true, false, true>, amap, bmap, p);
   if (pair) {
-    if (rowmax) return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<true, true>, amap, bmap, p);
-    return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<true, false>, amap, bmap, p);
+    if (rowmax)
+      return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<true, true, false>, amap, bmap, p);
+    return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<true, false, false>, amap, bmap, p);
   }
-  if (rowmax) return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<false, true>, amap, bmap, p);
-  return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<false, false>, amap, bmap, p);
+  if (rowmax)
+    return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<false, true, false>, amap, bmap, p);
+  return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<false, false, false>, amap, bmap, p);
 }
 
 }  // namespace rkv

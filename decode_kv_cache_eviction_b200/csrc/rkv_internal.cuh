@@ -109,6 +109,10 @@ struct GemmParams {
   float* r_dst;            // [T] receives r
   int* unit_cnt;           // [U] zeroed by the plan kernel
   int* status;
+  // symmetric form only: zeroed scratch of column partial sums (the two CTAs
+  // of a pair each add their rows' partial) and its per-unit offsets
+  float* cs;               // [cs_off[U]]
+  const int64_t* cs_off;   // [U+1]
 };
 
 template <bool kPair>
@@ -128,7 +132,7 @@ constexpr int kRhoAlign = 256;   // per-unit rho segments start at multiples of 
 constexpr int kRhoSlots = 8;     // ring of 256-column rho tiles in the GEMM kernel
 
 struct GemmLayout {
-  uint32_t a, b, rho, rowx, fin, bars, slot, flags, total;
+  uint32_t a, b, rho, rowx, fin, colx, bars, slot, flags, total;
 };
 template <bool kPair>
 __host__ __device__ inline GemmLayout gemm_layout() {
@@ -140,6 +144,7 @@ __host__ __device__ inline GemmLayout gemm_layout() {
   L.rho = o; o += kRhoSlots * 256 * 4;
   L.rowx = o; o += 4 * 128 * 4;
   L.fin = o; o += 32 * 4;
+  L.colx = o; o += 2 * 4 * 4 * 32 * 8;   // symmetric form: [2][cg][q][lane] float2
   L.bars = o; o += (2 + 2 * C::kStages + 4 + 2 * kRhoSlots) * 8;
   L.slot = o; o += 16;
   L.flags = o; o += 16;
@@ -155,11 +160,20 @@ cudaError_t score_configure(int rp, bool closed, int smem_bytes, int cs);
 int score_max_clusters(int rp, bool closed, int smem_bytes, int cs);
 
 cudaError_t launch_plan(const int64_t* tok_off, int U, int w, int rows_per_item, int* item_off,
-                        int* unit_cnt, int64_t* rho_off, cudaStream_t st);
+                        int* unit_cnt, int64_t* rho_off, int64_t* cs_off, cudaStream_t st);
 cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const GemmParams& p,
-                        bool pair, bool rowmax, int nctas, cudaStream_t st);
-cudaError_t gemm_configure(bool pair, bool rowmax);
-int gemm_max_ctas(bool pair, bool rowmax);
+                        bool pair, bool rowmax, bool sym, int nctas, cudaStream_t st);
+cudaError_t launch_sym_finish(const GemmParams& p, int nsm, cudaStream_t st);
+cudaError_t gemm_configure(bool pair, bool rowmax, bool sym);
+int gemm_max_ctas(bool pair, bool rowmax, bool sym);
+// Column-partial scratch of the symmetric form for one unit: 256 floats per
+// tile above the diagonal of its candidate row blocks.
+__host__ __device__ inline int64_t sym_scratch_floats(int64_t n, int w) {
+  const int64_t c = n - w;
+  if (c <= 0) return 0;
+  const int64_t nbr = (c + 255) / 256, nbc = (n + 255) / 256;
+  return 256 * (nbr * (nbc - 1) - nbr * (nbr - 1) / 2);
+}
 
 cudaError_t launch_select(const int64_t* tok_off, int U, int w, int cmax, const float* a,
                           const float* r, float lam, int budget, const int32_t* budgets,

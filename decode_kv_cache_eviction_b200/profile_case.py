@@ -17,6 +17,7 @@ ap.add_argument("--units", type=int, default=32)
 ap.add_argument("--n", type=int, default=32768)
 ap.add_argument("--mode", default="gemm", choices=["gemm", "closed", "max"])
 ap.add_argument("--iters", type=int, default=3)
+ap.add_argument("--symmetric", action="store_true", help="symmetric redundancy GEMM")
 ap.add_argument("--extras", action="store_true",
                 help="also run the in-place eviction and the adaptive-budget kernels")
 a = ap.parse_args()
@@ -24,7 +25,7 @@ wl = W.custom(name="long_trace_32k", n_kv_head=a.units, group=4, window=8, budge
               n_min=a.n, dup_frac=0.3, dup_noise=0.05, span_len=(32, 256))
 gb = W.generate(wl, seed=0, device="cuda")
 b = Batch(gb.K, gb.V, gb.Q, gb.tok_off)
-eng = Engine(4, 8, b.num_units, b.num_tokens, redundancy=a.mode)
+eng = Engine(4, 8, b.num_units, b.num_tokens, redundancy=a.mode, symmetric_gemm=a.symmetric)
 ra, rr = eng.alloc_scores(b)
 idx, nk, Ko, Vo = eng.alloc_outputs(b, 4096)
 for _ in range(a.iters):

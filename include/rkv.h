@@ -88,7 +88,17 @@ typedef struct {
 enum {
   /* Redundancy GEMM on single CTAs (M = 128 tcgen05 MMAs) instead of CTA
    * pairs (M = 256, cta_group::2).  Same results; slower. */
-  RKV_FLAG_GEMM_SINGLE_CTA = 1
+  RKV_FLAG_GEMM_SINGLE_CTA = 1,
+  /* Row-mean GEMM on the tiles on and above the diagonal only: S is symmetric,
+   * so tile (a, b > a) gives block a its row sums and block b its column sums
+   * (rho-weighted, reduced on CUDA cores and added to a zeroed scratch).  The
+   * unit's last CTA adds the parts in a fixed order.  About half the MMA work;
+   * same results up to fp32 rounding order, and deterministic.  CTA pairs and
+   * RKV_REDUNDANCY_GEMM only (RKV_ERR_UNSUPPORTED otherwise).  The scratch
+   * (256 fp32 per tile above the diagonal, about N_u^2 / 128 bytes per unit) is
+   * allocated by rkv_score when a batch first needs more and freed by
+   * rkv_destroy. */
+  RKV_FLAG_GEMM_SYMMETRIC = 2
 };
 
 typedef struct {

@@ -47,10 +47,14 @@ def make_batch(gen_batch: W.Batch) -> Batch:
 
 
 def run_engine(batch: Batch, group, window, lam, budget, mode="gemm", single_cta=False,
-               engine=None):
+               engine=None, symmetric=False):
+    """Score, select and compact with a fresh engine (mode "gemm_sym" = the
+    symmetric row-mean GEMM)."""
+    if mode == "gemm_sym":
+        mode, symmetric = "gemm", True
     eng = engine or Engine(group, window, max_units=max(1, batch.num_units),
                            max_tokens=max(1, batch.num_tokens), redundancy=mode,
-                           single_cta_gemm=single_cta)
+                           single_cta_gemm=single_cta, symmetric_gemm=symmetric)
     a, r = eng.alloc_scores(batch)
     m = torch.full_like(a, float("nan"))
     a.fill_(float("nan"))
@@ -86,7 +90,7 @@ def close(x_gpu, x_ora, what):
 
 def oracle_mode(mode):
     """The oracle redundancy that an engine mode computes."""
-    return "max" if mode == "max" else "closed"
+    return "max" if mode == "max" else "closed"   # gemm, gemm_sym, closed: the row mean
 
 
 def check_unit(out, batch: Batch, u, w, lam, budget, redundancy="closed", check_m=True):

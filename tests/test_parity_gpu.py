@@ -107,7 +107,7 @@ def test_worked_example_on_gpu():
 
 
 # ----------------------------------------------------------------- score kernels, small
-@pytest.mark.parametrize("mode", ["closed", "gemm", "max"])
+@pytest.mark.parametrize("mode", ["closed", "gemm", "max", "gemm_sym"])
 @pytest.mark.parametrize("G,w", [(1, 8), (4, 8), (2, 3), (5, 5), (1, 1), (32, 1)])
 def test_score_small_ragged(mode, G, w):
     lengths = [w, w + 1, 127, 128, 129, 1000, 2500, 5000]
@@ -137,7 +137,7 @@ def test_row_max_flags_every_duplicate():
         assert np.all(m[~has_copy[:n - 8]] < 0.7)
 
 
-@pytest.mark.parametrize("mode", ["closed", "gemm", "max"])
+@pytest.mark.parametrize("mode", ["closed", "gemm", "max", "gemm_sym"])
 def test_budget_edges(mode):
     lengths = [300, 300, 300]
     w = 8
@@ -165,12 +165,44 @@ def test_gemm_single_cta_and_pair_agree():
     assert np.array_equal(x1["m"], x2["m"])
 
 
+@pytest.mark.parametrize("lengths", [[255, 256, 257, 511, 512, 513, 769], [3000, 4100, 700, 9],
+                                     [20000, 12345]])
+def test_symmetric_gemm_matches_dense(lengths):
+    """Tiles on and above the diagonal only: the same m up to fp32 rounding
+    order, the oracle's kept sets, and bit-identical repeated calls."""
+    b = rand_batch(lengths, 4, 8, seed=len(lengths) * 13)
+    dense = run_engine(b, 4, 8, 0.1, 128, mode="gemm")
+    sym = run_engine(b, 4, 8, 0.1, 128, mode="gemm_sym")
+    for u in range(len(lengths)):
+        check_unit(sym, b, u, 8, 0.1, 128)
+    c_rows = np.zeros(b.num_tokens, bool)
+    for u, n in enumerate(lengths):
+        r0 = int(b.tok_off_host[u])
+        c_rows[r0:r0 + n - 8] = True
+    np.testing.assert_allclose(sym["m"][c_rows], dense["m"][c_rows], rtol=1e-4, atol=1e-7)
+    again = run_engine(b, 4, 8, 0.1, 128, engine=sym["engine"])
+    assert np.array_equal(again["m"], sym["m"]) and np.array_equal(again["r"], sym["r"])
+    assert np.array_equal(again["idx"], sym["idx"])
+
+
+def test_symmetric_flag_rejections():
+    with pytest.raises(RkvError) as ei:
+        Engine(4, 8, 1, 1000, redundancy="closed", symmetric_gemm=True)
+    assert ei.value.code == -2
+    with pytest.raises(RkvError) as ei:
+        Engine(4, 8, 1, 1000, redundancy="max", symmetric_gemm=True)
+    assert ei.value.code == -2
+    with pytest.raises(RkvError) as ei:
+        Engine(4, 8, 1, 1000, single_cta_gemm=True, symmetric_gemm=True)
+    assert ei.value.code == -2
+
+
 @pytest.mark.parametrize("G,N", [(4, 32768), (2, 49152)])
 def test_largest_supported_unit(G, N):
     # logits of a unit stay in tensor memory: 32768 tokens at G*w = 32,
     # 49152 (the select limit) at G*w <= 16
     b = rand_batch([N], G, 8, seed=1, dup=0.0)
-    for mode in ("closed", "gemm", "max"):
+    for mode in ("closed", "gemm", "max", "gemm_sym"):
         out = run_engine(b, G, 8, 0.1, 4096, mode=mode)
         check_unit(out, b, 0, 8, 0.1, 4096, redundancy=oracle_mode(mode))
 
@@ -235,7 +267,7 @@ def test_workload_tiny_full():
 
 
 def test_workload_llama3_layer_full():
-    _sampled("llama3_8b_layer", 8, modes=("gemm", "closed", "max"))
+    _sampled("llama3_8b_layer", 8, modes=("gemm", "closed", "max", "gemm_sym"))
 
 
 def test_workload_tiny_definition_redundancy():
@@ -248,12 +280,12 @@ def test_workload_tiny_definition_redundancy():
 
 @pytest.mark.slow
 def test_workload_r1_llama8b_cache_sampled():
-    _sampled("r1_llama8b_cache", 6)
+    _sampled("r1_llama8b_cache", 6, modes=("gemm", "closed", "gemm_sym"))
 
 
 @pytest.mark.slow
 def test_workload_long_trace_32k_sampled():
-    _sampled("long_trace_32k", 6)
+    _sampled("long_trace_32k", 6, modes=("gemm", "closed", "gemm_sym"))
 
 
 @pytest.mark.slow
