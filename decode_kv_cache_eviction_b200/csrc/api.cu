@@ -280,8 +280,8 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool closed = e->cfg.redundancy == RKV_REDUNDANCY_CLOSED_FORM;
   const int R = e->cfg.group * e->cfg.window;
-  // symmetric form: column-partial scratch for this batch (grown before
-  // anything is enqueued; zeroed on the stream before the GEMM)
+  // symmetric form: partial-sum scratch for this batch (grown before
+  // anything is enqueued; the GEMM writes every element)
   int64_t cs_need = 0;
   if (e->sym) {
     for (int u = 0; u < U; ++u)
@@ -362,17 +362,13 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   g.cs_off = e->sym ? e->cs_off : nullptr;
   int64_t items = 0;
   for (int u = 0; u < U; ++u) {
-    const int64_t c = b->tok_off_host[u + 1] - b->tok_off_host[u] - e->cfg.window;
-    if (c > 0) items += (c + rows_per_item - 1) / rows_per_item;
+    const int64_t n = b->tok_off_host[u + 1] - b->tok_off_host[u];
+    items += gemm_unit_items(n, n - e->cfg.window, rows_per_item, e->sym);
   }
   if (items == 0) return RKV_OK;
   int64_t nctas = e->gemm_ctas;
   const int64_t need = items * (e->pair ? 2 : 1);
   if (nctas > need) nctas = need;
-  if (e->sym && cs_need > 0) {
-    err = cudaMemsetAsync(e->cs, 0, sizeof(float) * cs_need, st);
-    if (err != cudaSuccess) return cuda_fail(err);
-  }
   t_begin(e, RKV_KERNEL_GEMM, st);
   err = launch_gemm(amap, bmap, g, e->pair, e->rowmax, e->sym, static_cast<int>(nctas), st);
   if (err == cudaSuccess && e->sym) {

@@ -23,6 +23,22 @@
 // one M = 256 MMA (cta_group::2): each CTA holds 128 A rows and half of each
 // 256-key B tile, which halves the shared-memory traffic per SM.
 //
+// Symmetric form (kSym, row mean on CTA pairs): S = khat khat^T is symmetric,
+// so only the 256 x 256 tiles (a, b) with a <= b are computed.  A work item is
+// (unit, block b): its 256 keys stay in shared memory as the MMA's B operand
+// while the row blocks a = 0 .. b stream through as the A operand, so TMEM
+// lane = row of block a and column = key of block b.  Per tile the epilogue
+//   - adds rho_i-weighted column sums into registers that persist over the
+//     whole item (block b's share from rows of blocks 0 .. b; the diagonal
+//     tile with its diagonal dropped), reduced across threads once per item;
+//   - for a < b, forms the rho_j-weighted row sums of block a's rows over
+//     block b's columns (a 4-thread reduction, then the four column groups
+//     through shared memory) and stores them to a scratch slot (a, b).
+// Every slot is written by exactly one plain store, so nothing needs zeroing
+// and the result does not depend on timing.  A finish kernel adds, per row,
+// the two CTAs' column sums and the slots (a, b > a) in block order, scales by
+// rho_i / (N - 1) and applies the token softmax.
+//
 // Warp roles (640 threads = 5 warps per SM sub-partition): warp 0 TMA producer,
 // warp 1 MMA issuer (leader CTA only in pair mode; the whole warp runs the loop
 // and elects one lane per instruction) and TMEM owner, warps 4-19
@@ -57,6 +73,15 @@ __device__ __forceinline__ int find_unit(const int* item_off, int U, int item) {
     else hi = mid - 1;
   }
   return lo;
+}
+
+// Block of a work item within its unit.  The symmetric form runs a unit's
+// items from the last block (the most tiles) down, so long items start first.
+template <bool kSym>
+__device__ __forceinline__ int item_block(const int* item_off, int u, int item) {
+  const int i0 = __ldg(&item_off[u]);
+  if constexpr (kSym) return __ldg(&item_off[u + 1]) - 1 - item;
+  return item - i0;
 }
 
 // MMA and commit issued by the whole (converged) warp, one lane elected inside
@@ -164,7 +189,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       float* rho_ring = reinterpret_cast<float*>(sm + L.rho);
       for (int item = group_id; item < n_items; item += ngroups, ++ai) {
         const int u = find_unit(p.item_off, p.num_units, item);
-        const int blk = item - __ldg(&p.item_off[u]);
+        const int blk = item_block<kSym>(p.item_off, u, item);
         const float* rho_u = p.rho + __ldg(&p.rho_off[u]);
         const int64_t base = __ldg(&p.tok_off[u]);
         const int N = static_cast<int>(__ldg(&p.tok_off[u + 1]) - base);
@@ -181,9 +206,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d(ad + C::kABytes / 2, &amap, a_full, 64, ya, pol);
           }
         }
-        const int ntiles = (N + C::kN - 1) / C::kN;
-        // symmetric form: only the tiles on and above the diagonal block
-        for (int t = kSym ? blk : 0; t < ntiles; ++t) {
+        // symmetric form: the row blocks 0 .. blk against the item's block
+        const int ntiles = kSym ? blk + 1 : (N + C::kN - 1) / C::kN;
+        for (int t = 0; t < ntiles; ++t) {
           if (mbar_wait(&b_empty[stage], ph ^ 1, abort, p.status)) {
             uint8_t* bd = sm + L.b + stage * C::kBBytes;
             const int yb = static_cast<int>(base + t * C::kN + rank * C::kBRows);
@@ -199,7 +224,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
           if (++stage == NSB) { stage = 0; ph ^= 1; }
-          // the 256 column weights of this tile (every CTA of a pair loads its own)
+          // the tile's 256 rho values (column weights; row weights in the
+          // symmetric form); every CTA of a pair loads its own
           const uint32_t rs = rt % kRhoSlots;
           if (mbar_wait(&rho_empty[rs], ((rt / kRhoSlots) & 1) ^ 1, abort, p.status)) {
             mbar_arrive_expect_tx(&rho_full[rs], 256 * 4);
@@ -223,13 +249,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int N = static_cast<int>(__ldg(&p.tok_off[u + 1]) - base);
         const bool aok = __all_sync(0xffffffffu, mbar_wait(a_full, ai & 1, abort, p.status));
         const uint32_t aaddr = smem_u32(sm + L.a);
-        uint64_t adesc[8];   // A descriptors of this item's 8 K-steps
+        // descriptors of the item's fixed block for the 8 K-steps: the A
+        // operand, or in the symmetric form the B operand
+        uint64_t fdesc[8];
 #pragma unroll
         for (int kq = 0; kq < 8; ++kq)
-          adesc[kq] = desc_kmajor_sw128(aaddr + (kq >> 2) * (C::kABytes / 2) + (kq & 3) * 32);
-        const int ntiles = (N + C::kN - 1) / C::kN;
-        const int t0 = kSym ? item - __ldg(&p.item_off[u]) : 0;
-        for (int t = t0; t < ntiles; ++t, ++tcount) {
+          fdesc[kq] = desc_kmajor_sw128(aaddr + (kq >> 2) * (C::kABytes / 2) + (kq & 3) * 32);
+        const int ntiles =
+            kSym ? item_block<kSym>(p.item_off, u, item) + 1 : (N + C::kN - 1) / C::kN;
+        for (int t = 0; t < ntiles; ++t, ++tcount) {
           RKV_GSTAMP(0, tcount, 0);
           bool go = mbar_wait(&b_full[stage], ph, abort, p.status);
           RKV_GSTAMP(0, tcount, 1);
@@ -238,14 +266,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           RKV_GSTAMP(0, tcount, 2);
           tc_fence_after();
           if (go) {
-            // B descriptors: the stage's base plus each K-step's offset in
-            // 16-byte units (the start-address field cannot carry: smem < 256 KB)
-            const uint64_t bdesc0 = desc_kmajor_sw128(smem_u32(sm + L.b + stage * C::kBBytes));
+            // streamed-tile descriptors: the stage's base plus each K-step's
+            // offset in 16-byte units (the start-address field cannot carry:
+            // smem < 256 KB)
+            const uint64_t sdesc0 = desc_kmajor_sw128(smem_u32(sm + L.b + stage * C::kBBytes));
             const uint32_t d = tmem + ab * 256;
 #pragma unroll
             for (int kq = 0; kq < 8; ++kq) {
               const uint32_t bo = (kq >> 2) * (C::kBBytes / 2) + (kq & 3) * 32;
-              mma_bf16_elect<C::kCtaGroup>(d, adesc[kq], bdesc0 + (bo >> 4), idesc, kq > 0);
+              if constexpr (kSym)   // A = row block t (streamed), B = the item's block
+                mma_bf16_elect<C::kCtaGroup>(d, sdesc0 + (bo >> 4), fdesc[kq], idesc, kq > 0);
+              else
+                mma_bf16_elect<C::kCtaGroup>(d, fdesc[kq], sdesc0 + (bo >> 4), idesc, kq > 0);
             }
             if constexpr (kPair) {
               commit_pair_elect(&b_empty[stage]);
@@ -266,7 +298,155 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && kSym) {
+    // ------------------------------------------------- epilogue, symmetric form
+    const int ew = warp - 4;              // epilogue warp 0..15
+    const int cg = ew >> 2;               // 64-column group of the tile
+    const int q = warp & 3;               // TMEM lane quarter
+    const int gq = lane >> 2, tq = lane & 3;   // quad and thread within it
+    const float* rho_ring = reinterpret_cast<const float*>(sm + L.rho);
+    float* rowc = reinterpret_cast<float*>(sm + L.rowx);    // [2][3][128] row partials
+    float2* colx = reinterpret_cast<float2*>(sm + L.colx);  // [2][cg][q][32] column sums
+    const uint32_t acc_empty_lead = mapa(smem_u32(acc_empty), 0);
+    const int rq = rank * 128 + q * 32;   // first row of this warp's quarter in a block
+    int ab = 0;
+    uint32_t aph = 0;
+    uint32_t rt = 0;   // rho tiles consumed so far
+    int rb = 0;        // double buffer of the per-tile row exchange
+    int ib = 0;        // double buffer of the per-item column exchange
+    for (int item = group_id; item < n_items; item += ngroups, ib ^= 1) {
+      const int u = find_unit(p.item_off, p.num_units, item);
+      const int blk = item_block<kSym>(p.item_off, u, item);
+      const int nb = __ldg(&p.item_off[u + 1]) - __ldg(&p.item_off[u]);
+      const float* rho_u = p.rho + __ldg(&p.rho_off[u]);
+      float* cs_u = p.cs + __ldg(&p.cs_off[u]);
+      // weights rho_j of this thread's 16 columns of block blk (8k + 2tq + {0, 1})
+      float2 wt[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        wt[k] = __ldg(reinterpret_cast<const float2*>(rho_u + blk * 256 + cg * 64 + 2 * tq + 8 * k));
+      // rho_i-weighted column sums of the item's block over this thread's rows
+      float cp[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) cp[k] = 0.f;
+      for (int t = 0; t <= blk; ++t, ++rt) {
+        const bool diag = t == blk;
+        const uint32_t rs_slot = rt % kRhoSlots;
+        mbar_wait(&acc_full[ab], aph, abort, p.status);
+        mbar_wait(&rho_full[rs_slot], (rt / kRhoSlots) & 1, abort, p.status);
+        __syncwarp();
+        tc_fence_after();
+        // weights of this thread's 4 rows of block t (gq + 8k of the quarter)
+        const float* wr = rho_ring + rs_slot * 256 + rq + gq;
+        const float w0 = wr[0], w1 = wr[8], w2 = wr[16], w3 = wr[24];
+        const uint32_t tbase =
+            tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + cg * 64;
+        // diagonal tile: rows and columns of one block; the diagonal (column -
+        // row == dd in this warp's 32 x 64 sub-block) is dropped
+        const int dd = rq - cg * 64;
+        const bool masked = diag && dd > -32 && dd < 64;
+        uint32_t v[32];
+        auto patch = [&](int h) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int col = 8 * k + 2 * tq + (e & 1);
+              const int row = 16 * h + gq + ((e >> 1) << 3);
+              if (col - row == dd) v[4 * k + e] = 0u;
+            }
+        };
+        // row sums over this thread's 16 columns: rows gq + 16h and gq + 16h + 8,
+        // two partial values each
+        auto rowfold = [&](float& pa, float& pb, float& qa, float& qb) {
+          mul2(pa, pb, __uint_as_float(v[0]), __uint_as_float(v[1]), wt[0].x, wt[0].y);
+          mul2(qa, qb, __uint_as_float(v[2]), __uint_as_float(v[3]), wt[0].x, wt[0].y);
+#pragma unroll
+          for (int k = 1; k < 8; ++k) {
+            fma2(pa, pb, __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]), wt[k].x,
+                 wt[k].y);
+            fma2(qa, qb, __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]), wt[k].x,
+                 wt[k].y);
+          }
+        };
+        auto colfold = [&](float wa, float wb) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            fma2(cp[2 * k], cp[2 * k + 1], __uint_as_float(v[4 * k]),
+                 __uint_as_float(v[4 * k + 1]), wa, wa);
+            fma2(cp[2 * k], cp[2 * k + 1], __uint_as_float(v[4 * k + 2]),
+                 __uint_as_float(v[4 * k + 3]), wb, wb);
+          }
+        };
+        float a0 = 0.f, b0 = 0.f, a1 = 0.f, b1 = 0.f, a2 = 0.f, b2 = 0.f, a3 = 0.f, b3 = 0.f;
+        tmem_ld16x256b_x8(tbase, v);                 // lanes 0-15 of the quarter
+        tmem_wait_ld();
+        if (masked) patch(0);
+        if (!diag) rowfold(a0, b0, a1, b1);
+        colfold(w0, w1);
+        tmem_ld16x256b_x8(tbase + (16u << 16), v);   // lanes 16-31
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_lead + ab * 8);
+        if (++ab == 2) { ab = 0; aph ^= 1; }
+        if (masked) patch(1);
+        if (!diag) rowfold(a2, b2, a3, b3);
+        colfold(w2, w3);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rho_empty[rs_slot]);
+        if (!diag) {
+          // the quad's four threads hold disjoint columns of the same 4 rows:
+          // reduce-scatter so that thread tq keeps row gq + 8 tq
+          const float t0 = a0 + b0, t1 = a1 + b1, t2 = a2 + b2, t3 = a3 + b3;
+          const bool u2 = (lane & 2) != 0, u1 = (lane & 1) != 0;
+          const float k0 = (u2 ? t2 : t0) + __shfl_xor_sync(0xffffffffu, u2 ? t0 : t2, 2);
+          const float k1 = (u2 ? t3 : t1) + __shfl_xor_sync(0xffffffffu, u2 ? t1 : t3, 2);
+          const float rsum = (u1 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, u1 ? k0 : k1, 1);
+          // the four column groups of the quarter, then one store per row
+          const int rl = q * 32 + gq + 8 * tq;
+          float* rc = rowc + rb * 384;
+          if (cg > 0) rc[(cg - 1) * 128 + rl] = rsum;
+          named_bar_sync(8 + q, 128);
+          if (cg == 0) {
+            const float tot = ((rsum + rc[rl]) + rc[128 + rl]) + rc[256 + rl];
+            const int64_t seg = 512 * static_cast<int64_t>(nb) +
+                                256 * (static_cast<int64_t>(t) * (nb - 1) -
+                                       static_cast<int64_t>(t) * (t - 1) / 2);
+            cs_u[seg + static_cast<int64_t>(blk - t - 1) * 256 + rank * 128 + rl] = tot;
+          }
+          rb ^= 1;
+        }
+      }
+      // ---- item end: column sums of block blk over the quad index gq (lane
+      // bits 2-4), reduce-scattered so that lane l keeps columns 2l and 2l + 1
+      // of the group, then the four lane quarters through shared memory
+#pragma unroll
+      for (int sft = 16, n = 8; sft >= 4; sft >>= 1, n >>= 1) {
+        const bool up = (lane & sft) != 0;
+#pragma unroll
+        for (int k = 0; k < n; ++k) {
+          const float send = up ? cp[k] : cp[k + n];
+          const float keep = up ? cp[k + n] : cp[k];
+          cp[k] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+        }
+      }
+      float2* cx = colx + (ib * 4 + cg) * 4 * 32;
+      cx[q * 32 + lane] = make_float2(cp[0], cp[1]);
+      named_bar_sync(4 + cg, 128);
+      if (q == 0) {
+        float2 acc = cx[lane];
+#pragma unroll
+        for (int qq = 1; qq < 4; ++qq) {
+          const float2 y = cx[qq * 32 + lane];
+          acc.x += y.x;
+          acc.y += y.y;
+        }
+        // this CTA's rows' share; the pair's other CTA writes the other slot
+        *reinterpret_cast<float2*>(cs_u + (2 * blk + rank) * 256 + cg * 64 + 2 * lane) = acc;
+      }
+    }
+  } else if (!kSym && warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int etid = threadIdx.x - 128;   // 0..511
     const int ew = warp - 4;              // epilogue warp 0..15
@@ -280,10 +460,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int ab = 0;
     uint32_t aph = 0;
     uint32_t rt = 0;   // rho tiles consumed so far
-    int colbuf = 0;    // symmetric form: double buffer of the column exchange
     for (int item = group_id; item < n_items; item += ngroups) {
       const int u = find_unit(p.item_off, p.num_units, item);
-      const int blk = item - __ldg(&p.item_off[u]);
+      const int blk = item_block<kSym>(p.item_off, u, item);
       const int64_t base = __ldg(&p.tok_off[u]);
       const int N = static_cast<int>(__ldg(&p.tok_off[u + 1]) - base);
       const int c = N - p.w;
@@ -295,22 +474,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       float a0 = kInit, b0 = kInit, a1 = kInit, b1 = kInit;
       float a2 = kInit, b2 = kInit, a3 = kInit, b3 = kInit;
       const int ntiles = (N + C::kN - 1) / C::kN;
-      // symmetric form: weights rho_i of this thread's 4 rows (for the column
-      // sums) and the scratch segment of this item (256 floats per tile above
-      // the diagonal)
-      float rw[4] = {0.f, 0.f, 0.f, 0.f};
-      int64_t cs_item = 0;
-      if constexpr (kSym) {
-        const float* rho_u = p.rho + __ldg(&p.rho_off[u]);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) rw[k] = __ldg(&rho_u[rbase + q * 32 + gq + 8 * k]);
-        cs_item = __ldg(&p.cs_off[u]) +
-                  256 * (static_cast<int64_t>(blk) * (ntiles - 1) -
-                         static_cast<int64_t>(blk) * (blk - 1) / 2);
-      }
-      for (int t = kSym ? blk : 0; t < ntiles; ++t, ++rt) {
+      for (int t = 0; t < ntiles; ++t, ++rt) {
         const int j0 = t * C::kN;
-        const bool colsum = kSym && t > blk;   // tile above the diagonal block
         const uint32_t rs_slot = rt % kRhoSlots;
         const float* rs = rho_ring + rs_slot * 256 + cg * 64 + 2 * tq;
         if (etid == 0) RKV_GSTAMP(1, rt, 0);
@@ -364,28 +529,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         };
-        // symmetric form: rho-weighted column partials over this thread's 4
-        // rows, columns 8k + 2tq + {0, 1} (pairs k = 0..7)
-        float cp[16];
-        auto colfold = [&](int h) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            fma2(cp[2 * k], cp[2 * k + 1], __uint_as_float(v[4 * k]),
-                 __uint_as_float(v[4 * k + 1]), rw[2 * h], rw[2 * h]);
-            fma2(cp[2 * k], cp[2 * k + 1], __uint_as_float(v[4 * k + 2]),
-                 __uint_as_float(v[4 * k + 3]), rw[2 * h + 1], rw[2 * h + 1]);
-          }
-        };
-        if constexpr (kSym) {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) cp[k] = 0.f;
-        }
         tmem_ld16x256b_x8(tbase, v);                 // lanes 0-15 of the quarter
         tmem_wait_ld();
         if (etid == 0) RKV_GSTAMP(1, rt, 2);
         if (masked) patch(0);
         fold(a0, b0, a1, b1);
-        if (colsum) colfold(0);
         tmem_ld16x256b_x8(tbase + (16u << 16), v);   // lanes 16-31
         tmem_wait_ld();
         tc_fence_before();
@@ -400,44 +548,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (etid == 0) RKV_GSTAMP(1, rt, 3);
         __syncwarp();
         if (lane == 0) mbar_arrive(&rho_empty[rs_slot]);
-        if constexpr (kSym) {
-          if (colsum) {
-            colfold(1);
-            // reduce-scatter over the quad index gq (lane bits 2-4): lane l
-            // keeps the column sums of columns 2l and 2l + 1 of the group
-#pragma unroll
-            for (int sft = 16, n = 8; sft >= 4; sft >>= 1, n >>= 1) {
-              const bool up = (lane & sft) != 0;
-#pragma unroll
-              for (int k = 0; k < n; ++k) {
-                const float send = up ? cp[k] : cp[k + n];
-                const float keep = up ? cp[k + n] : cp[k];
-                cp[k] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
-              }
-            }
-            // the four lane quarters of this column group, then one 2-addend
-            // atomic per column pair (the pair's other CTA adds its rows)
-            float2* cx = reinterpret_cast<float2*>(sm + L.colx) + (colbuf * 4 + cg) * 4 * 32;
-            cx[q * 32 + lane] = make_float2(cp[0], cp[1]);
-            named_bar_sync(4 + cg, 128);
-            if (q == 0) {
-              float2 acc = cx[lane];
-#pragma unroll
-              for (int qq = 1; qq < 4; ++qq) {
-                const float2 y = cx[qq * 32 + lane];
-                acc.x += y.x;
-                acc.y += y.y;
-              }
-              // fire-and-forget reduction (no returned value to wait for)
-              float* dst =
-                  p.cs + cs_item + static_cast<int64_t>(t - blk - 1) * 256 + cg * 64 + 2 * lane;
-              asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(dst), "f"(acc.x),
-                           "f"(acc.y)
-                           : "memory");
-            }
-            colbuf ^= 1;
-          }
-        }
       }
       // ---- item end: finish the rows over the quad (its four threads hold
       // disjoint columns), combine the four column groups, write m
@@ -461,20 +571,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if constexpr (kMax) {
           tot = fmaxf(fmaxf(tot, rowx[rl]), fmaxf(rowx[128 + rl], rowx[256 + rl]));
           p.m_dst[base + i] = rho_i * tot;
-        } else if constexpr (kSym) {
-          // this item's columns only (blocks blk ..); the earlier blocks'
-          // share comes from their column partials in the final pass
-          p.m_dst[base + i] = (tot + rowx[rl]) + (rowx[128 + rl] + rowx[256 + rl]);
         } else {
           tot += (rowx[rl] + rowx[128 + rl]) + rowx[256 + rl];
           p.m_dst[base + i] = rho_i * tot / static_cast<float>(N - 1);
         }
-      }
-      if constexpr (kSym) {
-        // the row partials are complete; the finish kernel adds the column
-        // partials and applies the softmax (doing it here would stall a pair)
-        named_bar_sync(3, 512);
-        continue;
       }
       __threadfence();
       named_bar_sync(3, 512);
@@ -515,7 +615,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // One block: items per unit and their prefix, 256-aligned rho segment
 // offsets, zeroed unit counters and (symmetric form, cs_off != null) the
-// offsets of each unit's column-partial scratch.
+// offsets of each unit's scratch.  An item is a block of candidate rows, or in
+// the symmetric form any 256-key block of a unit that has candidates (its
+// columns reach every candidate row).
 __global__ void plan_kernel(const int64_t* tok_off, int U, int w, int rows_per_item,
                             int* item_off, int* unit_cnt, int64_t* rho_off, int64_t* cs_off) {
   __shared__ long long wsum[3][32];
@@ -526,7 +628,7 @@ __global__ void plan_kernel(const int64_t* tok_off, int U, int w, int rows_per_i
   for (int u = u0; u < u1; ++u) {
     const int64_t n = tok_off[u + 1] - tok_off[u];
     const int64_t c = n - w;
-    li += c > 0 ? (c + rows_per_item - 1) / rows_per_item : 0;
+    li += gemm_unit_items(n, c, rows_per_item, cs_off != nullptr);
     lr += (n + kRhoAlign - 1) / kRhoAlign * kRhoAlign;
     ls += sym_scratch_floats(n, w);
     unit_cnt[u] = 0;
@@ -568,7 +670,7 @@ __global__ void plan_kernel(const int64_t* tok_off, int U, int w, int rows_per_i
     if (cs_off) cs_off[u] = rs;
     const int64_t n = tok_off[u + 1] - tok_off[u];
     const int64_t c = n - w;
-    ri += c > 0 ? (c + rows_per_item - 1) / rows_per_item : 0;
+    ri += gemm_unit_items(n, c, rows_per_item, cs_off != nullptr);
     rr += (n + kRhoAlign - 1) / kRhoAlign * kRhoAlign;
     rs += sym_scratch_floats(n, w);
   }
@@ -584,12 +686,11 @@ __global__ void plan_kernel(const int64_t* tok_off, int U, int w, int rows_per_i
   }
 }
 
-// Symmetric form, after the GEMM: one CTA per unit adds to each candidate row's
-// partial (left in m_dst) the column partials of the earlier row blocks, in
-// block order, scales by rho_i / (N - 1), and applies the token softmax.
-// Block a2's partials for every later row are contiguous (index i - 256
-// (a2 + 1)), so a thread takes 4 consecutive rows and reads one aligned float4
-// per earlier block.
+// Symmetric form, after the GEMM: one CTA per unit.  Row i of block a (i < c)
+// gets the two CTAs' column sums of block a, then the row sums of the slots
+// (a, b) for b = a + 1 .. nb - 1 in block order, is scaled by rho_i / (N - 1),
+// and the token softmax follows.  A thread takes 4 consecutive rows (one
+// block) and reads one aligned float4 per slot.
 constexpr int kFinishThreads = 512;
 __global__ void __launch_bounds__(kFinishThreads)
     sym_finish_kernel(const int64_t* __restrict__ tok_off, int U, int w,
@@ -603,19 +704,22 @@ __global__ void __launch_bounds__(kFinishThreads)
     const int N = static_cast<int>(tok_off[u + 1] - base);
     const int c = N - w;
     if (c <= 0) continue;
-    const int nbc = (N + 255) / 256;
+    const int nb = (N + 255) / 256;
     const float* rho_u = rho + rho_off[u];
-    const int64_t cs0 = cs_off[u];
+    const float* cs_u = cs + cs_off[u];
     const float inv_nm1 = 1.f / static_cast<float>(N - 1);
     float esum = 0.f;
     for (int r0 = 4 * tid; r0 < c; r0 += 4 * kFinishThreads) {
-      const int a = r0 >> 8;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      const int a = r0 >> 8, lr = r0 & 255;
+      const float4 d0 = __ldcs(reinterpret_cast<const float4*>(cs_u + (2 * a) * 256 + lr));
+      const float4 d1 = __ldcs(reinterpret_cast<const float4*>(cs_u + (2 * a + 1) * 256 + lr));
+      float4 acc = make_float4(d0.x + d1.x, d0.y + d1.y, d0.z + d1.z, d0.w + d1.w);
+      const float* seg = cs_u + 512 * static_cast<int64_t>(nb) +
+                         256 * (static_cast<int64_t>(a) * (nb - 1) -
+                                static_cast<int64_t>(a) * (a - 1) / 2) + lr;
 #pragma unroll 4
-      for (int a2 = 0; a2 < a; ++a2) {
-        const int64_t seg = cs0 + 256 * (static_cast<int64_t>(a2) * (nbc - 1) -
-                                         static_cast<int64_t>(a2) * (a2 - 1) / 2);
-        const float4 y = __ldcs(reinterpret_cast<const float4*>(cs + seg + (r0 - 256 * (a2 + 1))));
+      for (int b = a + 1; b < nb; ++b) {
+        const float4 y = __ldcs(reinterpret_cast<const float4*>(seg + (b - a - 1) * 256));
         acc.x += y.x;
         acc.y += y.y;
         acc.z += y.z;
@@ -626,7 +730,7 @@ __global__ void __launch_bounds__(kFinishThreads)
       for (int e = 0; e < 4; ++e) {
         const int i = r0 + e;
         if (i < c) {
-          const float m = rho_u[i] * (m_dst[base + i] + part[e]) * inv_nm1;
+          const float m = rho_u[i] * part[e] * inv_nm1;
           m_dst[base + i] = m;
           esum += ex2(m * kLog2e);
         }

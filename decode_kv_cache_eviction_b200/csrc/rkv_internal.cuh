@@ -109,8 +109,8 @@ struct GemmParams {
   float* r_dst;            // [T] receives r
   int* unit_cnt;           // [U] zeroed by the plan kernel
   int* status;
-  // symmetric form only: zeroed scratch of column partial sums (the two CTAs
-  // of a pair each add their rows' partial) and its per-unit offsets
+  // symmetric form only: scratch of column and row partial sums (layout at
+  // sym_scratch_floats) and its per-unit offsets
   float* cs;               // [cs_off[U]]
   const int64_t* cs_off;   // [U+1]
 };
@@ -142,7 +142,7 @@ __host__ __device__ inline GemmLayout gemm_layout() {
   L.a = o; o += C::kABytes;
   L.b = o; o += C::kStages * C::kBBytes;
   L.rho = o; o += kRhoSlots * 256 * 4;
-  L.rowx = o; o += 4 * 128 * 4;
+  L.rowx = o; o += 2 * 3 * 128 * 4;   // [3][128] row partials; symmetric form [2][3][128]
   L.fin = o; o += 32 * 4;
   L.colx = o; o += 2 * 4 * 4 * 32 * 8;   // symmetric form: [2][cg][q][lane] float2
   L.bars = o; o += (2 + 2 * C::kStages + 4 + 2 * kRhoSlots) * 8;
@@ -166,13 +166,22 @@ cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const 
 cudaError_t launch_sym_finish(const GemmParams& p, int nsm, cudaStream_t st);
 cudaError_t gemm_configure(bool pair, bool rowmax, bool sym);
 int gemm_max_ctas(bool pair, bool rowmax, bool sym);
-// Column-partial scratch of the symmetric form for one unit: 256 floats per
-// tile above the diagonal of its candidate row blocks.
+// Scratch of the symmetric form for one unit of nb = ceil(n / 256) blocks:
+// the two CTAs' column sums of every block (2 x 256 floats per block), then
+// for each block a the row sums of the slots (a, b), b = a + 1 .. nb - 1
+// (256 floats each).  128 nb (nb + 3) floats in all; every float is written
+// by exactly one store of the GEMM.
 __host__ __device__ inline int64_t sym_scratch_floats(int64_t n, int w) {
-  const int64_t c = n - w;
+  if (n - w <= 0) return 0;
+  const int64_t nb = (n + 255) / 256;
+  return 128 * nb * (nb + 3);
+}
+// GEMM work items of one unit: its blocks of candidate rows, or in the
+// symmetric form all its 256-key blocks (when it has candidates).
+__host__ __device__ inline int64_t gemm_unit_items(int64_t n, int64_t c, int rows_per_item,
+                                                   bool sym) {
   if (c <= 0) return 0;
-  const int64_t nbr = (c + 255) / 256, nbc = (n + 255) / 256;
-  return 256 * (nbr * (nbc - 1) - nbr * (nbr - 1) / 2);
+  return sym ? (n + 255) / 256 : (c + rows_per_item - 1) / rows_per_item;
 }
 
 cudaError_t launch_select(const int64_t* tok_off, int U, int w, int cmax, const float* a,

@@ -91,13 +91,13 @@ enum {
   RKV_FLAG_GEMM_SINGLE_CTA = 1,
   /* Row-mean GEMM on the tiles on and above the diagonal only: S is symmetric,
    * so tile (a, b > a) gives block a its row sums and block b its column sums
-   * (rho-weighted, reduced on CUDA cores and added to a zeroed scratch).  The
-   * unit's last CTA adds the parts in a fixed order.  About half the MMA work;
-   * same results up to fp32 rounding order, and deterministic.  CTA pairs and
-   * RKV_REDUNDANCY_GEMM only (RKV_ERR_UNSUPPORTED otherwise).  The scratch
-   * (256 fp32 per tile above the diagonal, about N_u^2 / 128 bytes per unit) is
-   * allocated by rkv_score when a batch first needs more and freed by
-   * rkv_destroy. */
+   * (rho-weighted, reduced on CUDA cores).  Every partial sum is written once
+   * to a scratch, and a finish kernel adds the parts in a fixed order.  About
+   * half the MMA work; same results up to fp32 rounding order, and
+   * deterministic.  CTA pairs and RKV_REDUNDANCY_GEMM only
+   * (RKV_ERR_UNSUPPORTED otherwise).  The scratch (128 nb (nb + 3) fp32 for a
+   * unit of nb = ceil(N_u / 256) blocks, about N_u^2 / 128 bytes) is allocated
+   * by rkv_score when a batch first needs more and freed by rkv_destroy. */
   RKV_FLAG_GEMM_SYMMETRIC = 2
 };
 
