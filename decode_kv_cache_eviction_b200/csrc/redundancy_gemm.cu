@@ -32,8 +32,10 @@
 //     whole item (block b's share from rows of blocks 0 .. b; the diagonal
 //     tile with its diagonal dropped), reduced across threads once per item;
 //   - for a < b, forms the rho_j-weighted row sums of block a's rows over
-//     block b's columns (a 4-thread reduction, then the four column groups
-//     through shared memory) and stores them to a scratch slot (a, b).
+//     block b's columns (a 4-thread reduction per 64-column group) and puts
+//     them in a shared-memory ring; warp 2 adds the four column groups and
+//     stores the sums to a scratch slot (a, b), so no epilogue warp waits
+//     for another.
 // Every slot is written by exactly one plain store, so nothing needs zeroing
 // and the result does not depend on timing.  A finish kernel adds, per row,
 // the two CTAs' column sums and the slots (a, b > a) in block order, scales by
@@ -41,9 +43,9 @@
 //
 // Warp roles (640 threads = 5 warps per SM sub-partition): warp 0 TMA producer,
 // warp 1 MMA issuer (leader CTA only in pair mode; the whole warp runs the loop
-// and elects one lane per instruction) and TMEM owner, warps 4-19
-// epilogue (warp % 4 selects the TMEM lane quarter, (warp - 4) / 4 the
-// 64-column quarter of the tile).
+// and elects one lane per instruction) and TMEM owner, warp 2 (symmetric form)
+// row-sum store, warps 4-19 epilogue (warp % 4 selects the TMEM lane quarter,
+// (warp - 4) / 4 the 64-column quarter of the tile).
 #include "ptx.cuh"
 #include "rkv_internal.cuh"
 
@@ -142,6 +144,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* rho_full = acc_empty + 2;      // [kRhoSlots] rho tile landed
   uint64_t* rho_empty = rho_full + kRhoSlots;  // [kRhoSlots] epilogue done with it
+  uint64_t* row_full = rho_empty + kRhoSlots;  // [kRowRing] symmetric form: partials written
+  uint64_t* row_empty = row_full + kRowRing;   // [kRowRing] symmetric form: partials stored
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.slot);
   volatile int* abort = reinterpret_cast<volatile int*>(sm + L.flags);
   volatile int* last_flag = reinterpret_cast<volatile int*>(sm + L.flags + 4);
@@ -160,6 +164,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int b = 0; b < kRhoSlots; ++b) {
       mbar_init(&rho_full[b], 1);
       mbar_init(&rho_empty[b], 16);   // this CTA's 16 epilogue warps
+    }
+    for (int b = 0; b < kRowRing; ++b) {
+      mbar_init(&row_full[b], 16);    // the 16 epilogue warps
+      mbar_init(&row_empty[b], 1);    // the row-store warp
     }
     *abort = 0;
     fence_mbar_init();
@@ -298,6 +306,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     __syncwarp();
+  } else if (warp == 2 && kSym) {
+    // ------------------------------------------------ row-sum store (symmetric)
+    // Per tile below the item's block: the four column groups' partial row
+    // sums of this CTA's 128 rows, added in a fixed order and stored to the
+    // tile's scratch slot.
+    const float* rr = reinterpret_cast<const float*>(sm + L.rowr);
+    uint32_t n = 0;   // row exchanges so far
+    for (int item = group_id; item < n_items; item += ngroups) {
+      const int u = find_unit(p.item_off, p.num_units, item);
+      const int blk = item_block<kSym>(p.item_off, u, item);
+      const int nb = __ldg(&p.item_off[u + 1]) - __ldg(&p.item_off[u]);
+      float* cs_u = p.cs + __ldg(&p.cs_off[u]);
+      for (int t = 0; t < blk; ++t, ++n) {
+        const uint32_t s = n % kRowRing;
+        mbar_wait(&row_full[s], (n / kRowRing) & 1, abort, p.status);
+        const float* x = rr + s * 512;
+        float tot[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int rl = lane + 32 * j;
+          tot[j] = ((x[rl] + x[128 + rl]) + x[256 + rl]) + x[384 + rl];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&row_empty[s]);
+        const int64_t seg = 512 * static_cast<int64_t>(nb) +
+                            256 * (static_cast<int64_t>(t) * (nb - 1) -
+                                   static_cast<int64_t>(t) * (t - 1) / 2);
+        float* dst = cs_u + seg + static_cast<int64_t>(blk - t - 1) * 256 + rank * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[lane + 32 * j] = tot[j];
+      }
+    }
   } else if (warp >= 4 && kSym) {
     // ------------------------------------------------- epilogue, symmetric form
     const int ew = warp - 4;              // epilogue warp 0..15
@@ -305,19 +345,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;               // TMEM lane quarter
     const int gq = lane >> 2, tq = lane & 3;   // quad and thread within it
     const float* rho_ring = reinterpret_cast<const float*>(sm + L.rho);
-    float* rowc = reinterpret_cast<float*>(sm + L.rowx);    // [2][3][128] row partials
+    float* rowr = reinterpret_cast<float*>(sm + L.rowr);    // [kRowRing][cg][128]
     float2* colx = reinterpret_cast<float2*>(sm + L.colx);  // [2][cg][q][32] column sums
     const uint32_t acc_empty_lead = mapa(smem_u32(acc_empty), 0);
     const int rq = rank * 128 + q * 32;   // first row of this warp's quarter in a block
     int ab = 0;
     uint32_t aph = 0;
     uint32_t rt = 0;   // rho tiles consumed so far
-    int rb = 0;        // double buffer of the per-tile row exchange
+    uint32_t nx = 0;   // row exchanges so far
     int ib = 0;        // double buffer of the per-item column exchange
     for (int item = group_id; item < n_items; item += ngroups, ib ^= 1) {
       const int u = find_unit(p.item_off, p.num_units, item);
       const int blk = item_block<kSym>(p.item_off, u, item);
-      const int nb = __ldg(&p.item_off[u + 1]) - __ldg(&p.item_off[u]);
       const float* rho_u = p.rho + __ldg(&p.rho_off[u]);
       float* cs_u = p.cs + __ldg(&p.cs_off[u]);
       // weights rho_j of this thread's 16 columns of block blk (8k + 2tq + {0, 1})
@@ -403,19 +442,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const float k0 = (u2 ? t2 : t0) + __shfl_xor_sync(0xffffffffu, u2 ? t0 : t2, 2);
           const float k1 = (u2 ? t3 : t1) + __shfl_xor_sync(0xffffffffu, u2 ? t1 : t3, 2);
           const float rsum = (u1 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, u1 ? k0 : k1, 1);
-          // the four column groups of the quarter, then one store per row
-          const int rl = q * 32 + gq + 8 * tq;
-          float* rc = rowc + rb * 384;
-          if (cg > 0) rc[(cg - 1) * 128 + rl] = rsum;
-          named_bar_sync(8 + q, 128);
-          if (cg == 0) {
-            const float tot = ((rsum + rc[rl]) + rc[128 + rl]) + rc[256 + rl];
-            const int64_t seg = 512 * static_cast<int64_t>(nb) +
-                                256 * (static_cast<int64_t>(t) * (nb - 1) -
-                                       static_cast<int64_t>(t) * (t - 1) / 2);
-            cs_u[seg + static_cast<int64_t>(blk - t - 1) * 256 + rank * 128 + rl] = tot;
-          }
-          rb ^= 1;
+          // into the ring; the row-store warp adds the four column groups
+          const uint32_t s = nx % kRowRing;
+          mbar_wait(&row_empty[s], ((nx / kRowRing) & 1) ^ 1, abort, p.status);
+          rowr[s * 512 + cg * 128 + q * 32 + gq + 8 * tq] = rsum;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&row_full[s]);
+          ++nx;
         }
       }
       // ---- item end: column sums of block blk over the quad index gq (lane

@@ -130,9 +130,10 @@ struct GemmCfg {
 
 constexpr int kRhoAlign = 256;   // per-unit rho segments start at multiples of this
 constexpr int kRhoSlots = 8;     // ring of 256-column rho tiles in the GEMM kernel
+constexpr int kRowRing = 4;      // symmetric form: ring of per-tile row-partial buffers
 
 struct GemmLayout {
-  uint32_t a, b, rho, rowx, fin, colx, bars, slot, flags, total;
+  uint32_t a, b, rho, rowx, fin, colx, rowr, bars, slot, flags, total;
 };
 template <bool kPair>
 __host__ __device__ inline GemmLayout gemm_layout() {
@@ -142,10 +143,11 @@ __host__ __device__ inline GemmLayout gemm_layout() {
   L.a = o; o += C::kABytes;
   L.b = o; o += C::kStages * C::kBBytes;
   L.rho = o; o += kRhoSlots * 256 * 4;
-  L.rowx = o; o += 2 * 3 * 128 * 4;   // [3][128] row partials; symmetric form [2][3][128]
+  L.rowx = o; o += 4 * 128 * 4;
   L.fin = o; o += 32 * 4;
   L.colx = o; o += 2 * 4 * 4 * 32 * 8;   // symmetric form: [2][cg][q][lane] float2
-  L.bars = o; o += (2 + 2 * C::kStages + 4 + 2 * kRhoSlots) * 8;
+  L.rowr = o; o += kRowRing * 4 * 128 * 4;   // symmetric form: [kRowRing][cg][128 rows]
+  L.bars = o; o += (2 + 2 * C::kStages + 4 + 2 * kRhoSlots + 2 * kRowRing) * 8;
   L.slot = o; o += 16;
   L.flags = o; o += 16;
   L.total = o;
