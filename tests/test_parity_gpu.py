@@ -166,7 +166,9 @@ def test_gemm_single_cta_and_pair_agree():
 
 
 @pytest.mark.parametrize("lengths", [[255, 256, 257, 511, 512, 513, 769], [3000, 4100, 700, 9],
-                                     [20000, 12345]])
+                                     [20000, 12345],
+                                     # last key block holds window tokens only
+                                     [264, 520, 16, 1032, 258, 9]])
 def test_symmetric_gemm_matches_dense(lengths):
     """Tiles on and above the diagonal only: the same m up to fp32 rounding
     order, the oracle's kept sets, and bit-identical repeated calls."""
