@@ -56,7 +56,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="engine", choices=["engine", "reference"])
-    ap.add_argument("--workload", default="long_trace_32k", choices=W.WORKLOAD_ORDER)
+    ap.add_argument("--workload", default="long_trace_32k",
+                    choices=W.WORKLOAD_ORDER + W.EXTRA_WORKLOADS)
     ap.add_argument("--redundancy", default="gemm", choices=["gemm", "closed", "max"])
     ap.add_argument("--lam", type=float, default=0.1)
     ap.add_argument("--dense-gemm", dest="symmetric", action="store_false",
@@ -177,11 +178,11 @@ def algorithmic(batch: Batch, wl: W.Workload):
         "score_bytes": float((2 * d + 8) * n.sum() + 2 * d * U * wl.group * wl.window),
         # dense-equivalent tile products of the definition (rows in C x all N keys)
         "gemm_flops": float((2 * c * n * d).sum()),
-        # symmetric form: the 256 x 256 tiles actually executed (on and above
-        # the diagonal block of the candidate row blocks)
-        "gemm_sym_flops": float(sum(2 * d * 256 * 256 * (nbr * nbc - nbr * (nbr - 1) // 2)
-                                    for nbr, nbc in zip(((c + 255) // 256).astype(np.int64),
-                                                        ((n + 255) // 256).astype(np.int64)))),
+        # symmetric form: the 256 x 256 tiles actually executed, (a, b) with
+        # a <= b over the nb = ceil(N / 256) key blocks of a unit with candidates
+        "gemm_sym_flops": float(sum(2 * d * 256 * 256 * (nb * (nb + 1) // 2)
+                                    for nb, cc in zip(((n + 255) // 256).astype(np.int64), c)
+                                    if cc > 0)),
         # a and r read, kept indices and counts written
         "select_bytes": float(8 * c.sum() + 4 * U * W_ + 4 * U),
         # kept K and V rows read; the whole [U, B+w] outputs written
@@ -378,10 +379,12 @@ def run_engine(args, dist: Dist):
         secondary = {"redundancy": other, "value": tokens * dist.world / (ms2 * 1e-3),
                      "ms_per_step": ms2, "kernels": rep2}
 
-    in_place = adaptive = None
+    in_place = adaptive = sweep = None
     if not args.no_secondary:
         in_place = measure_in_place(eng, batch, wl, args, dist, alg, pk, src)
         adaptive = measure_adaptive(eng, batch, wl, args, dist, alg, pk, src)
+        if len(wl.lambdas) > 1:
+            sweep = measure_lambda_sweep(eng, batch, wl, args, dist, alg, pk, src)
 
     e2e = None
     if not args.no_e2e:
@@ -402,7 +405,38 @@ def run_engine(args, dist: Dist):
                 "roofline": roofline, "kernels": rep, "gpu_launches": launches,
                 "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
                 "secondary": secondary, "in_place": in_place, "adaptive": adaptive}
+        if sweep is not None:
+            line["lambda_sweep"] = sweep
+        if wl.name in W.CADENCE:
+            every, trace = W.CADENCE[wl.name]
+            triggers = (trace - wl.budget) // every
+            line["cadence"] = {"decode_steps_per_trigger": every, "trace_tokens": trace,
+                               "triggers_per_trace": triggers, "ms_per_trigger": ms,
+                               "ms_per_trace": ms * triggers}
         print(json.dumps(line), flush=True)
+
+
+def measure_lambda_sweep(eng, batch: Batch, wl: W.Workload, args, dist: Dist, alg, pk, src):
+    """The workload's lambda sweep: a and r do not depend on lambda, so one
+    score serves every lambda, followed by select + compact per lambda.  The
+    value counts each lambda's eviction of every token."""
+    a, r = eng.alloc_scores(batch)
+    outs = [eng.alloc_outputs(batch, wl.budget) for _ in wl.lambdas]
+
+    def step():
+        eng.score(batch, a, r)
+        for lam, (idx, nk, Ko, Vo) in zip(wl.lambdas, outs):
+            eng.select(batch, a, r, lam, wl.budget, idx, nk)
+            eng.compact(batch, idx, nk, wl.budget, Ko, Vo)
+
+    ms, per_kernel, _ = timed(step, args.steps, args.warmup, dist, eng)
+    eng.check_status()
+    rep = kernel_report(per_kernel, alg, pk, src)
+    kept = [int(o[1].sum().item()) for o in outs]
+    return {"lambdas": list(wl.lambdas),
+            "value": batch.num_tokens * len(wl.lambdas) * dist.world / (ms * 1e-3),
+            "ms_per_step": ms, "kept_tokens": kept,
+            "kernels": {k: rep[k] for k in ("score", "select", "compact") if k in rep}}
 
 
 def measure_adaptive(eng, batch: Batch, wl: W.Workload, args, dist: Dist, alg, pk, src):

@@ -86,6 +86,14 @@ WORKLOADS = {
 WORKLOAD_ORDER = ["tiny", "llama3_8b_layer", "r1_llama8b_cache",
                   "long_trace_32k", "ragged_serving"]
 
+# The R1-Llama-8B cache at its trigger cadence: compression runs every 128
+# decode steps, when the cache holds the B = 2048 kept tokens plus 128 new
+# ones (N = 2176).  CADENCE gives (decode steps per trigger, trace length).
+WORKLOADS["r1_llama8b_cadence"] = Workload("r1_llama8b_cadence", 8, 32, 8, 4, 128, 8, 2048,
+                                           (0.1,), 2176, 2176, 0.25, 0.05, (64, 64), None)
+CADENCE = {"r1_llama8b_cadence": (128, 16384)}
+EXTRA_WORKLOADS = ["r1_llama8b_cadence"]
+
 
 def custom(name="custom", n_seq=1, n_layer=1, n_kv_head=1, group=1, head_dim=128,
            window=8, budget=64, lambdas=(0.1,), n_min=512, n_max=None,

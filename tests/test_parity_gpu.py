@@ -272,6 +272,11 @@ def test_workload_llama3_layer_full():
     _sampled("llama3_8b_layer", 8, modes=("gemm", "closed", "max", "gemm_sym"))
 
 
+def test_workload_r1_cadence_sampled():
+    # the R1-Llama-8B cache at its trigger: B + 128 = 2176 tokens per unit
+    _sampled("r1_llama8b_cadence", 6, modes=("gemm_sym", "closed"))
+
+
 def test_workload_tiny_definition_redundancy():
     """Redundancy checked against the row-block definition (not the closed form)."""
     wl = W.WORKLOADS["tiny"]
