@@ -163,7 +163,7 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   const int R = group * window;
   const int rp = R <= 16 ? 16 : 32;
   const int k = rp == 32 ? 1 : 0;
-  const int cs = score_cluster_size(nmax, rp, d->max_cs[k]);
+  const int cs = score_cluster_size(nmax, rp, d->max_cs[k], U, d->clusters[k]);
   if (cs == 0) return RKV_ERR_UNSUPPORTED;
   int ci = 0;
   while ((1 << ci) < cs) ++ci;

@@ -84,16 +84,20 @@ __host__ __device__ inline int score_stages(int rp, bool closed, int smem_cap) {
   return 0;
 }
 
-// Cluster size for a batch whose longest unit has nmax tokens: about 1024
-// tokens per CTA, enough CTAs for the TMEM-resident logits, at most max_cs.
-// Returns 0 if the unit does not fit.
-inline int score_cluster_size(int nmax, int rp, int max_cs) {
+// Cluster size of the score kernel for a batch of `units` units of at most
+// nmax tokens.  It is the smallest power of two whose CTAs hold a unit's logits
+// in TMEM (at most max_cs).  A unit is spread further, to at most 1024 tokens
+// per CTA, only while the batch has fewer units than clusters of that size can
+// be resident (clusters[log2 cs]): with more units, every extra CTA per unit
+// only adds cluster exchanges.  Returns 0 when no size fits.
+inline int score_cluster_size(int nmax, int rp, int max_cs, int64_t units, const int* clusters) {
   int cs = 1;
-  while (cs < max_cs && (nmax + cs - 1) / cs > 1024) cs <<= 1;
   while ((((nmax + cs - 1) / cs + kTile - 1) / kTile) * kTile > score_lmax(rp)) {
     if (cs >= max_cs) return 0;
     cs <<= 1;
   }
+  auto log2i = [](int x) { int l = 0; while ((1 << l) < x) ++l; return l; };
+  while (cs < max_cs && (nmax + cs - 1) / cs > 1024 && units < clusters[log2i(cs)]) cs <<= 1;
   return cs;
 }
 
