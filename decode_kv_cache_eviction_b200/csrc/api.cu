@@ -299,7 +299,9 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
     }
   }
 
-  const int cs = score_cluster_size(nmax, e->rp, e->max_cs, U, e->score_clusters);
+  const int cs = e->score_cs_fixed > 0
+                     ? e->score_cs_fixed
+                     : score_cluster_size(nmax, e->rp, e->max_cs, U, e->score_clusters);
   if (cs == 0) return RKV_ERR_UNSUPPORTED;
   int ncl = e->score_clusters[cs_index(cs)];
   if (ncl > U) ncl = U;

@@ -26,6 +26,7 @@ struct rkv_engine {
   int nstages = 0;             // score K-tile ring depth
   int score_smem = 0;
   int score_clusters[5] = {};  // active clusters for cluster sizes 1, 2, 4, 8, 16
+  int score_cs_fixed = 0;      // > 0: score cluster size set by rkv_compress_host
   int max_cs = 16;
   int max_n = 0;               // largest supported N_u
   bool pair = true;

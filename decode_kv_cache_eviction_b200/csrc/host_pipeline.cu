@@ -13,14 +13,16 @@
 // cudaHostAlloc / cudaMallocHost allocation on a 64-bit system with unified
 // addressing), the compaction kernel gathers the kept rows straight from host
 // memory and V is never copied in whole; otherwise each chunk's V is copied
-// like K.  A chunk's results are
-// independent of how the units were split (every kernel works per unit), so
-// the outputs equal those of one rkv_compress over the whole batch.
+// like K.  Every kernel works per unit and every chunk scores with the
+// cluster size of the whole batch, so a chunk's results do not depend on how
+// the units were split: the outputs equal those of one rkv_compress over the
+// whole batch.
 #include <algorithm>
 #include <cstring>
 #include <vector>
 
 #include "engine.cuh"
+#include "rkv_internal.cuh"
 
 namespace {
 
@@ -228,6 +230,14 @@ extern "C" int rkv_compress_host(rkv_engine* e, const rkv_host_batch* hb, float 
   const char* hK = static_cast<const char*>(hb->K);
   const char* hV = static_cast<const char*>(hb->V);
   const char* hQ = static_cast<const char*>(hb->Q);
+  // every chunk scores with the cluster size of the whole batch, so each
+  // unit's cross-CTA sums are grouped as rkv_compress on the batch groups them
+  struct FixedClusterSize {
+    rkv_engine* e;
+    FixedClusterSize(rkv_engine* en, int cs) : e(en) { e->score_cs_fixed = cs; }
+    ~FixedClusterSize() { e->score_cs_fixed = 0; }
+  } fixed_cs(e, rkv::score_cluster_size(static_cast<int>(nmax), e->rp, e->max_cs, U,
+                                   e->score_clusters));
   for (size_t i = 0; i < chunks.size(); ++i) {
     const Chunk& c = chunks[i];
     const int s = static_cast<int>(i & 1);
