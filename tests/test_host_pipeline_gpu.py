@@ -106,3 +106,14 @@ def test_host_pipeline_rejections():
     # nothing was enqueued by the rejected calls: the engine still works
     ref = device_reference(b2, 64, "gemm")
     assert_same(ref, run_host(eng, b2, 64, 0))
+
+
+def test_many_units_chunks_keep_the_batch_cluster_size():
+    # 200 units: the whole batch scores with the smallest TMEM-fitting cluster,
+    # while a 2-unit chunk alone would spread its units over more CTAs
+    lengths = [3000 + 13 * (i % 7) for i in range(200)]
+    b = rand_batch(lengths, G, WIN, seed=47)
+    ref = device_reference(b, 256, "closed")
+    eng = Engine(G, WIN, max_units=b.num_units, max_tokens=b.num_tokens, redundancy="closed")
+    for chunk in (0, 7000):
+        assert_same(ref, run_host(eng, b, 256, chunk))
