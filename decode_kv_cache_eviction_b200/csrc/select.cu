@@ -1,8 +1,10 @@
 // Joint eviction (R-KV 联合淘汰): s_i = lambda * a_i - (1 - lambda) * r_i and a
 // deterministic top-B of the candidates.
 //
-// Persistent CTAs (1024 threads) walk the units; while one unit is selected,
-// the next unit's a and r are prefetched into L2.  Per unit:
+// Persistent CTAs walk the units; while one unit is selected, the next unit's
+// a and r are prefetched into L2.  A CTA has 1024 threads for long units and
+// 256 for units of at most 8192 candidates, so that several CTAs share an SM
+// where the per-unit steps are short.  Per unit:
 //   1. s is computed in fp32 and mapped to order-preserving uint32 keys held
 //      in shared memory (one read of a and r); the block also finds the
 //      smallest and largest key.
@@ -28,10 +30,8 @@
 namespace rkv {
 namespace {
 
-constexpr int kSelThreads = 1024;
-constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kHistGroups = 8;    // histograms shared by four warps each
 constexpr int kListCap = 4096;    // keys kept for the digits after the first
+constexpr int kSmallUnitCands = 8192;   // longest unit for the 256-thread CTAs
 
 __device__ __forceinline__ uint32_t order_key(float s) {
   uint32_t b = __float_as_uint(s);
@@ -50,11 +50,14 @@ __device__ __forceinline__ void prefetch_l2(const void* p, size_t bytes) {
   }
 }
 
-__global__ void __launch_bounds__(kSelThreads, 1)
+template <int kSelThreads>
+__global__ void __launch_bounds__(kSelThreads, kSelThreads <= 256 ? 4 : 1)
     select_kernel(const int64_t* __restrict__ tok_off, int U, int w, const float* __restrict__ a,
                   const float* __restrict__ r, float lam, int max_budget,
                   const int32_t* __restrict__ budgets, int sinks, int W,
                   int32_t* __restrict__ idx, int32_t* __restrict__ n_kept) {
+  constexpr int kSelWarps = kSelThreads / 32;
+  constexpr int kHistGroups = kSelWarps / 4;   // histograms shared by four warps each
   extern __shared__ uint32_t keys[];
   __shared__ uint32_t hist8[kHistGroups][256];
   __shared__ uint32_t hist[256];
@@ -119,8 +122,8 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     }
     __syncthreads();
     if (wp == 0) {
-      kmin = wmin[lane];
-      kmax = wmax[lane];
+      kmin = lane < kSelWarps ? wmin[lane] : 0xffffffffu;
+      kmax = lane < kSelWarps ? wmax[lane] : 0u;
 #pragma unroll
       for (int o = 16; o; o >>= 1) {
         kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
@@ -276,8 +279,12 @@ __global__ void __launch_bounds__(kSelThreads, 1)
 }  // namespace
 
 cudaError_t select_configure() {
-  return cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              kMaxTokensPerUnit * 4);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<1024>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kMaxTokensPerUnit * 4);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kSmallUnitCands * 4);
 }
 
 cudaError_t launch_select(const int64_t* tok_off, int U, int w, int cmax, const float* a,
@@ -286,19 +293,26 @@ cudaError_t launch_select(const int64_t* tok_off, int U, int w, int cmax, const 
   // keys of the ranked candidates (budgets[u] <= budget, so a unit with at
   // most `budget` candidates never needs them)
   const size_t smem = cmax > budget ? static_cast<size_t>(cmax) * 4 : 0;
+  const bool small = cmax <= kSmallUnitCands;
+  const void* fn = small ? reinterpret_cast<const void*>(&select_kernel<256>)
+                         : reinterpret_cast<const void*>(&select_kernel<1024>);
+  const int threads = small ? 256 : 1024;
   int dev = 0, nsm = 0, per = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, select_kernel, kSelThreads, smem) !=
-          cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, threads, smem) != cudaSuccess ||
       per < 1) {
     cudaGetLastError();
     per = 1;
   }
   int grid = nsm * per;
   if (grid > U) grid = U;
-  select_kernel<<<grid, kSelThreads, smem, st>>>(tok_off, U, w, a, r, lam, budget, budgets, sinks,
-                                                 W, idx, n_kept);
+  if (small)
+    select_kernel<256><<<grid, 256, smem, st>>>(tok_off, U, w, a, r, lam, budget, budgets, sinks,
+                                               W, idx, n_kept);
+  else
+    select_kernel<1024><<<grid, 1024, smem, st>>>(tok_off, U, w, a, r, lam, budget, budgets,
+                                                 sinks, W, idx, n_kept);
   return cudaGetLastError();
 }
 
