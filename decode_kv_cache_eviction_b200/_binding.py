@@ -168,7 +168,15 @@ class Batch:
 
 
 class Engine:
-    """One engine = one configuration and its device workspace."""
+    """One engine = one configuration and its device workspace.
+
+    redundancy: "gemm" (K Kᵀ tiles on the tensor cores, row mean), "closed"
+    (the same row mean in closed form, fused into the score kernel) or "max"
+    (row max from the GEMM tiles).  single_cta_gemm: M = 128 MMAs on single
+    CTAs instead of CTA pairs.  symmetric_gemm: with "gemm", only the tiles on
+    and above the diagonal (RKV_FLAG_GEMM_SYMMETRIC; about half the MMAs, a
+    partial-sum scratch of about N^2 / 128 bytes per unit).
+    """
 
     def __init__(self, group: int, window: int, max_units: int, max_tokens: int,
                  head_dim: int = 128, redundancy: str = "gemm", single_cta_gemm=False,
