@@ -187,9 +187,10 @@ def refree_keep_count(p: np.ndarray, sinks: int, T: float) -> int:
 
     Initial ranking: the first m = min(sinks, N) tokens in order, then the
     others from the newest to the oldest.  Uni-Metric: the Frobenius norm of
-    the attention entries kept.  Keep the shortest prefix of the ranking whose
-    norm reaches (1 - T) of the full row's norm, i.e. the norm lost by cutting
-    there is below T: the smallest k with sum_{first k} p^2 >= (1 - T)^2 sum p^2."""
+    the attention entries kept, which the review calls their energy.  Cutting
+    stops once the energy lost, the drop of that norm from the full row's, is
+    at most T of it: the smallest k with ||p_first k|| >= (1 - T) ||p||, i.e.
+    sum_{first k} p^2 >= (1 - T)^2 sum p^2."""
     N = len(p)
     m = min(sinks, N)
     order = np.concatenate([np.arange(m), np.arange(N - 1, m - 1, -1)])

@@ -460,6 +460,55 @@ def test_refree_keep_count_closed_forms():
     assert ora.refree_keep_count(p, 4, 0.01) == 4 + (N - 100)
 
 
+def _keep_cut_norm(p, sinks, T):
+    """A rejected reading: stop once the cut-off entries' norm is at most T of
+    the row's norm (planted here only to show that the pins tell it apart)."""
+    N = len(p)
+    m = min(sinks, N)
+    order = np.concatenate([np.arange(m), np.arange(N - 1, m - 1, -1)])
+    e = p[order] ** 2
+    cut = e.sum() - np.cumsum(e)
+    return int(np.argmax(np.sqrt(np.maximum(cut, 0)) <= T * np.sqrt(e.sum()))) + 1
+
+
+def _keep_cut_energy(p, sinks, T):
+    """Another rejected reading: the cut-off entries' squared norm at most T of
+    the row's squared norm."""
+    N = len(p)
+    m = min(sinks, N)
+    order = np.concatenate([np.arange(m), np.arange(N - 1, m - 1, -1)])
+    e = p[order] ** 2
+    cut = e.sum() - np.cumsum(e)
+    return int(np.argmax(cut <= T * e.sum())) + 1
+
+
+def test_refree_reading_is_the_drop_of_the_frobenius_norm():
+    """ReFreeKV review, section 2 ("Uni-Metric"): the metric is the Frobenius
+    norm of the kept attention entries, which the review calls their energy;
+    cutting stops once the energy lost, the drop of that norm, is under T.
+    Hand-worked values, with the two rejected readings giving other counts."""
+    # uniform 1000-token row, T = 1%: the kept norm is sqrt(k / 1000) of the
+    # row's, and sqrt(k / 1000) >= 0.99 first holds at k = 981 (980.1 rounded up)
+    p = np.full(1000, 1e-3)
+    assert ora.refree_keep_count(p, 0, 0.01) == 981
+    assert loops.refree_keep_count(list(p), 0, 0.01) == 981
+    assert _keep_cut_norm(p, 0, 0.01) == 1000     # sqrt((1000 - k) / 1000) <= 0.01
+    assert _keep_cut_energy(p, 0, 0.01) == 990    # (1000 - k) / 1000 <= 0.01
+    # five tokens, one sink, T = 0.1.  Ranking: 0 (sink), 4, 3, 2, 1.
+    # Squares: 0.01, 0.04, 0.09, 0.0225, 0.0625, total 0.225; the kept prefix
+    # needs 0.81 * 0.225 = 0.18225: {0} 0.01, {0,4} 0.0725, {0,4,3} 0.095,
+    # {0,4,3,2} 0.185 -> 4 tokens.  Cutting token 1 alone removes 0.04 of
+    # squared norm, more than 0.01 * 0.225 and 0.1 * 0.225, so both rejected
+    # readings keep all 5.
+    p5 = np.array([0.1, 0.2, 0.3, 0.15, 0.25])
+    assert ora.refree_keep_count(p5, 1, 0.1) == 4
+    assert loops.refree_keep_count(list(p5), 1, 0.1) == 4
+    assert _keep_cut_norm(p5, 1, 0.1) == 5
+    assert _keep_cut_energy(p5, 1, 0.1) == 5
+    # the budget that keeps those 4 tokens of a unit with w = 1: 4 - 1 sink - 1
+    assert ora.refree_budget(4, 5, 1, 1) == 2
+
+
 @pytest.mark.parametrize("seed", range(4))
 def test_refree_keep_count_matches_loop(seed):
     rng = np.random.default_rng(500 + seed)
