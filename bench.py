@@ -45,8 +45,6 @@ NCU_TRAFFIC_LONG_TRACE = {
     # (redundancy mode, kernel): bytes per launch
     ("gemm", "gemm"): (136.425472e6 + 5.207808e6) * 64,      # 16-unit capture
     ("gemm_sym", "gemm"): (137.865728e6 + 109.153536e6) * 64,  # 16-unit capture
-    ("gemm", "score"): (134.494208e6 + 3.787264e6) * 64,     # 16-unit capture
-    ("closed", "score"): (537.811968e6 + 17.450496e6) * 16,  # 64-unit capture
 }
 
 
@@ -343,7 +341,8 @@ def run_engine(args, dist: Dist):
     def measure(mode):
         sym = mode == "gemm" and args.symmetric
         eng = Engine(wl.group, wl.window, batch.num_units, tokens, redundancy=mode,
-                     symmetric_gemm=sym)
+                     symmetric_gemm=sym,
+                     max_unit_tokens=int(np.diff(batch.tok_off_host).max()))
         a, r = eng.alloc_scores(batch)
         idx, nk, Ko, Vo = eng.alloc_outputs(batch, wl.budget)
         step = lambda: eng.compress(batch, args.lam, wl.budget, a, r, idx, nk, Ko, Vo)

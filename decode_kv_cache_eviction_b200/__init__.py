@@ -6,4 +6,4 @@ gather compaction, behind a small C ABI (``include/rkv.h``).
 runs in the library's CUDA kernels.
 """
 from ._binding import (Batch, Engine, EXPORTS, LIB_PATH, RkvError, lib,  # noqa: F401
-                       score_noalloc, status_string)
+                       inject_create_fault, noalloc_check_status, score_noalloc, status_string)

@@ -31,12 +31,16 @@ RKV_REDUNDANCY_CLOSED_FORM = 1
 RKV_REDUNDANCY_MAX = 2
 RKV_FLAG_GEMM_SINGLE_CTA = 1
 RKV_FLAG_GEMM_SYMMETRIC = 2
+RKV_FAULT_NONE = 0
+RKV_FAULT_ALLOC = 1
+RKV_FAULT_DROP_ANNOUNCE = 2
 
 # Every function declared in include/rkv.h.
 EXPORTS = ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact",
            "rkv_compress", "rkv_compress_host", "rkv_evict_in_place", "rkv_fill_slots",
            "rkv_select_ex", "rkv_refree_budget", "rkv_check_status", "rkv_launch_count", "rkv_set_timing",
-           "rkv_read_timing", "rkv_score_noalloc", "rkv_status_string", "rkv_version")
+           "rkv_read_timing", "rkv_score_noalloc", "rkv_noalloc_check_status", "rkv_inject_fault",
+           "rkv_status_string", "rkv_version")
 KERNELS = ("score", "plan", "gemm", "select", "compact", "evict", "fill", "refree")
 
 
@@ -44,7 +48,7 @@ class RkvConfig(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int), ("group", ctypes.c_int),
                 ("window", ctypes.c_int), ("max_units", ctypes.c_int),
                 ("max_tokens", ctypes.c_int64), ("redundancy", ctypes.c_int),
-                ("flags", ctypes.c_int)]
+                ("flags", ctypes.c_int), ("max_unit_tokens", ctypes.c_int64)]
 
 
 class RkvHostBatch(ctypes.Structure):
@@ -100,6 +104,8 @@ def lib():
     L.rkv_read_timing.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_double),
                                   ctypes.POINTER(i64)]
     L.rkv_score_noalloc.argtypes = [i32, i32, ctypes.POINTER(RkvBatch), vp, vp, vp, vp]
+    L.rkv_noalloc_check_status.argtypes = [vp]
+    L.rkv_inject_fault.argtypes = [vp, i32]
     L.rkv_status_string.argtypes = [i32]
     L.rkv_status_string.restype = ctypes.c_char_p
     L.rkv_version.argtypes = []
@@ -107,7 +113,8 @@ def lib():
                  "rkv_compress", "rkv_compress_host", "rkv_evict_in_place", "rkv_fill_slots",
                  "rkv_select_ex", "rkv_refree_budget", "rkv_check_status", "rkv_set_timing",
                  "rkv_read_timing",
-                 "rkv_score_noalloc", "rkv_version"):
+                 "rkv_score_noalloc", "rkv_noalloc_check_status", "rkv_inject_fault",
+                 "rkv_version"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -137,6 +144,18 @@ def score_noalloc(group: int, window: int, batch: "Batch", a, r, m=None, stream=
     scratch (no engine, no allocation by the library)."""
     _check(lib().rkv_score_noalloc(int(group), int(window), ctypes.byref(batch.c), _ptr(a),
                                    _ptr(r), _ptr(m), _stream(stream)), "rkv_score_noalloc")
+
+
+def noalloc_check_status(stream=None):
+    """rkv_noalloc_check_status: raise if a device wait of an rkv_score_noalloc
+    call on the current device timed out since the last check (clears it)."""
+    _check(lib().rkv_noalloc_check_status(_stream(stream)), "noalloc device status")
+
+
+def inject_create_fault(fault: int):
+    """rkv_inject_fault(NULL, fault): the next engine creation's workspace
+    allocation fails (RKV_FAULT_ALLOC), for testing error paths."""
+    _check(lib().rkv_inject_fault(None, int(fault)), "rkv_inject_fault")
 
 
 class Batch:
@@ -175,17 +194,20 @@ class Engine:
     (row max from the GEMM tiles).  single_cta_gemm: M = 128 MMAs on single
     CTAs instead of CTA pairs.  symmetric_gemm: with "gemm", only the tiles on
     and above the diagonal (RKV_FLAG_GEMM_SYMMETRIC; about half the MMAs, a
-    partial-sum scratch of about N^2 / 128 bytes per unit).
+    partial-sum scratch of about N^2 / 128 bytes per unit, allocated here for
+    max_tokens in units of max_unit_tokens).  max_unit_tokens: the longest unit
+    a batch may hold (0: the engine's limit).
     """
 
     def __init__(self, group: int, window: int, max_units: int, max_tokens: int,
                  head_dim: int = 128, redundancy: str = "gemm", single_cta_gemm=False,
-                 symmetric_gemm=False):
+                 symmetric_gemm=False, max_unit_tokens: int = 0):
         mode = {"gemm": RKV_REDUNDANCY_GEMM, "closed": RKV_REDUNDANCY_CLOSED_FORM,
                 "max": RKV_REDUNDANCY_MAX}[redundancy]
         flags = ((RKV_FLAG_GEMM_SINGLE_CTA if single_cta_gemm else 0) |
                  (RKV_FLAG_GEMM_SYMMETRIC if symmetric_gemm else 0))
-        self.cfg = RkvConfig(head_dim, group, window, max_units, max_tokens, mode, flags)
+        self.cfg = RkvConfig(head_dim, group, window, max_units, max_tokens, mode, flags,
+                             max_unit_tokens)
         self.group, self.window = group, window
         h = ctypes.c_void_p()
         _check(lib().rkv_create(ctypes.byref(self.cfg), ctypes.byref(h)), "rkv_create")
@@ -287,6 +309,10 @@ class Engine:
 
     def check_status(self, stream=None):
         _check(lib().rkv_check_status(self.h, _stream(stream)), "device status")
+
+    def inject_fault(self, fault: int):
+        """Arm a one-shot fault (RKV_FAULT_*) for testing error paths."""
+        _check(lib().rkv_inject_fault(self.h, int(fault)), "rkv_inject_fault")
 
     def set_timing(self, enable: bool):
         _check(lib().rkv_set_timing(self.h, 1 if enable else 0), "rkv_set_timing")

@@ -1,6 +1,7 @@
 // C ABI of the engine: argument validation, workspace, tensor maps, launches.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdlib>
 #include <cstring>
 #include <new>
@@ -72,13 +73,38 @@ void t_end(rkv_engine* e, cudaStream_t st) {
   ++e->nev;
 }
 
-int cs_index(int cs) {
-  int i = 0;
-  while ((1 << i) < cs) ++i;
-  return i;
+// Fault injected for the next engine creation (rkv_inject_fault(NULL, ...)).
+int g_create_fault = 0;
+
+// cudaMalloc that fails once when an allocation fault is armed.
+cudaError_t dev_alloc(int* fault, void** p, size_t bytes) {
+  if (*fault == RKV_FAULT_ALLOC) {
+    *fault = 0;
+    *p = nullptr;
+    return cudaErrorMemoryAllocation;
+  }
+  return cudaMalloc(p, bytes);
+}
+
+// Floats of symmetric-form scratch that any batch within the capacities can
+// need.  A unit of n tokens needs 128 nb (nb + 3) with nb = ceil(n / 256) <=
+// x + 1, x = n / 256, so at most 128 (x^2 + 5 x + 4).  Over a batch, sum x^2 <=
+// (L / 256) sum x with L the longest unit, sum x <= max_tokens / 256 and there
+// are at most max_units units; no batch needs more than max_units units of L
+// tokens either.
+int64_t sym_scratch_bound(int64_t max_tokens, int max_units, int64_t max_len) {
+  const double X = static_cast<double>(max_tokens) / 256.0;
+  const double b1 = 128.0 * (static_cast<double>(max_len) / 256.0 * X + 5.0 * X +
+                             4.0 * static_cast<double>(max_units));
+  const double b2 = static_cast<double>(max_units) * sym_scratch_floats(max_len, 0);
+  return static_cast<int64_t>(std::min(b1, b2)) + 1;
 }
 
 }  // namespace
+
+cudaError_t rkv_engine_alloc(rkv_engine* e, void** p, size_t bytes) {
+  return dev_alloc(&e->fault, p, bytes);
+}
 
 extern "C" {
 
@@ -101,7 +127,8 @@ const char* rkv_status_string(int s) {
 int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   if (!cfg || !out) return RKV_ERR_INVALID_ARG;
   *out = nullptr;
-  if (cfg->group < 1 || cfg->window < 1 || cfg->max_units < 1 || cfg->max_tokens < 1)
+  if (cfg->group < 1 || cfg->window < 1 || cfg->max_units < 1 || cfg->max_tokens < 1 ||
+      cfg->max_unit_tokens < 0)
     return RKV_ERR_INVALID_ARG;
   if (cfg->redundancy != RKV_REDUNDANCY_GEMM && cfg->redundancy != RKV_REDUNDANCY_CLOSED_FORM &&
       cfg->redundancy != RKV_REDUNDANCY_MAX)
@@ -132,7 +159,6 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   e->cfg = *cfg;
   e->device = dev;
   e->nsm = nsm;
-  e->rp = cfg->group * cfg->window <= 16 ? 16 : 32;
   e->pair = (cfg->flags & RKV_FLAG_GEMM_SINGLE_CTA) == 0;
   e->rowmax = cfg->redundancy == RKV_REDUNDANCY_MAX;
   e->sym = (cfg->flags & RKV_FLAG_GEMM_SYMMETRIC) != 0;
@@ -147,27 +173,30 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   }
   e->encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
 
-  // Score kernel: deepest K-tile ring that fits; logits of up to 512/rp tiles
-  // per CTA stay in TMEM, so a unit may hold up to max_cs * 512/rp * 128 tokens.
+  // Score kernel: deepest K-tile ring that fits, one persistent CTA per SM.
   const bool closed = cfg->redundancy == RKV_REDUNDANCY_CLOSED_FORM;
+  const int R = cfg->group * cfg->window;
+  e->rp = R <= 16 ? 16 : (R <= 32 ? 32 : 64);
   e->nstages = score_stages(e->rp, closed, kSmemCap);
   e->score_smem = score_layout(e->rp, closed, e->nstages).total + 1024;
-  if (e->nstages == 0 || score_configure(e->rp, closed, e->score_smem, 16) != cudaSuccess) {
+  if (e->nstages == 0 || score_configure(e->rp, closed, e->score_smem) != cudaSuccess) {
     delete e;
     return cuda_fail(cudaErrorUnknown);
   }
-  e->max_cs = 0;
-  for (int i = 0; i < 5; ++i) {
-    e->score_clusters[i] = score_max_clusters(e->rp, closed, e->score_smem, 1 << i);
-    if (e->score_clusters[i] > 0) e->max_cs = 1 << i;
-    else break;
-  }
-  if (e->max_cs == 0) {
+  e->score_ctas = score_max_ctas(e->rp, closed, e->score_smem);
+  if (e->score_ctas <= 0) {
     delete e;
     return RKV_ERR_UNSUPPORTED;
   }
-  e->max_n = e->max_cs * score_lmax(e->rp);
-  if (e->max_n > kMaxTokensPerUnit) e->max_n = kMaxTokensPerUnit;
+  // a unit spans at most 2 * score_ctas chunks; select keeps its keys on chip
+  const int64_t score_n = 2 * static_cast<int64_t>(e->score_ctas) * score_chunk_tokens(e->rp);
+  e->max_n = static_cast<int>(std::min<int64_t>(score_n, kMaxTokensPerUnit));
+  if (cfg->max_unit_tokens < 0 || cfg->max_unit_tokens > e->max_n) {
+    delete e;
+    return cfg->max_unit_tokens < 0 ? RKV_ERR_INVALID_ARG : RKV_ERR_UNSUPPORTED;
+  }
+  if (cfg->max_unit_tokens > 0) e->max_n = static_cast<int>(cfg->max_unit_tokens);
+  e->max_chunks = score_max_chunks(cfg->max_tokens, cfg->max_units, e->score_ctas, e->rp);
 
   if (select_configure() != cudaSuccess || inplace_configure() != cudaSuccess) {
     delete e;
@@ -185,25 +214,46 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
     }
   }
 
-  bool ok = cudaMalloc(&e->status, 16) == cudaSuccess;
-  ok = ok && cudaMalloc(&e->item_off, sizeof(int) * (cfg->max_units + 1)) == cudaSuccess;
-  ok = ok && cudaMalloc(&e->unit_cnt, sizeof(int) * cfg->max_units) == cudaSuccess;
+  int* fault = &g_create_fault;
+  auto alloc = [&](void** p, size_t bytes) { return dev_alloc(fault, p, bytes) == cudaSuccess; };
+  bool ok = alloc(reinterpret_cast<void**>(&e->status), 16);
+  ok = ok && alloc(reinterpret_cast<void**>(&e->chunk_off), sizeof(int) * (cfg->max_units + 1));
+  ok = ok && alloc(reinterpret_cast<void**>(&e->score_cnt),
+                   sizeof(int) * (static_cast<size_t>(cfg->max_units) * kScoreCnt + 1));
+  ok = ok && alloc(reinterpret_cast<void**>(&e->xstat),
+                   sizeof(float) * static_cast<size_t>(e->max_chunks) * score_xs(e->rp, closed));
+  ok = ok && alloc(reinterpret_cast<void**>(&e->xsum),
+                   sizeof(float) * static_cast<size_t>(e->max_chunks) * 2 * kScoreMaxGroups);
   if (!closed) {
     const int64_t nrho = cfg->max_tokens + static_cast<int64_t>(kRhoAlign) * cfg->max_units;
-    ok = ok && cudaMalloc(&e->rho, sizeof(float) * nrho) == cudaSuccess;
-    ok = ok && cudaMalloc(&e->rho_off, sizeof(int64_t) * (cfg->max_units + 1)) == cudaSuccess;
+    ok = ok && alloc(reinterpret_cast<void**>(&e->item_off), sizeof(int) * (cfg->max_units + 1));
+    ok = ok && alloc(reinterpret_cast<void**>(&e->unit_cnt), sizeof(int) * cfg->max_units);
+    ok = ok && alloc(reinterpret_cast<void**>(&e->rho), sizeof(float) * nrho);
+    ok = ok && alloc(reinterpret_cast<void**>(&e->rho_off),
+                     sizeof(int64_t) * (cfg->max_units + 1));
   }
-  if (e->sym)
-    ok = ok && cudaMalloc(&e->cs_off, sizeof(int64_t) * (cfg->max_units + 1)) == cudaSuccess;
+  if (e->sym) {
+    // the partial-sum scratch of the largest batch the capacities allow, so that
+    // rkv_score never allocates
+    e->cs_cap = sym_scratch_bound(cfg->max_tokens, cfg->max_units, e->max_n);
+    ok = ok && alloc(reinterpret_cast<void**>(&e->cs_off), sizeof(int64_t) * (cfg->max_units + 1));
+    ok = ok && alloc(reinterpret_cast<void**>(&e->cs),
+                     sizeof(float) * static_cast<size_t>(std::max<int64_t>(e->cs_cap, 1)));
+  }
   ok = ok && cudaMemset(e->status, 0, 16) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     cudaFree(e->status);
+    cudaFree(e->chunk_off);
+    cudaFree(e->score_cnt);
+    cudaFree(e->xstat);
+    cudaFree(e->xsum);
     cudaFree(e->item_off);
     cudaFree(e->unit_cnt);
     cudaFree(e->rho);
     cudaFree(e->rho_off);
     cudaFree(e->cs_off);
+    cudaFree(e->cs);
     delete e;
     return RKV_ERR_OOM;
   }
@@ -252,6 +302,10 @@ int rkv_destroy(rkv_engine* e) {
   rkv_host_pipeline_free(e);
   cudaFree(e->rf_z);
   cudaFree(e->status);
+  cudaFree(e->chunk_off);
+  cudaFree(e->score_cnt);
+  cudaFree(e->xstat);
+  cudaFree(e->xsum);
   cudaFree(e->item_off);
   cudaFree(e->unit_cnt);
   cudaFree(e->rho);
@@ -263,6 +317,18 @@ int rkv_destroy(rkv_engine* e) {
 }
 
 int64_t rkv_launch_count(const rkv_engine* e) { return e ? e->launches : 0; }
+
+int rkv_inject_fault(rkv_engine* e, int fault) {
+  if (fault != RKV_FAULT_NONE && fault != RKV_FAULT_ALLOC && fault != RKV_FAULT_DROP_ANNOUNCE)
+    return RKV_ERR_INVALID_ARG;
+  if (!e) {
+    if (fault == RKV_FAULT_DROP_ANNOUNCE) return RKV_ERR_INVALID_ARG;
+    g_create_fault = fault;
+    return RKV_OK;
+  }
+  e->fault = fault;
+  return RKV_OK;
+}
 
 int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
               rkv_stream_t stream) {
@@ -280,66 +346,82 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool closed = e->cfg.redundancy == RKV_REDUNDANCY_CLOSED_FORM;
   const int R = e->cfg.group * e->cfg.window;
-  // symmetric form: partial-sum scratch for this batch (grown before
-  // anything is enqueued; the GEMM writes every element)
-  int64_t cs_need = 0;
-  if (e->sym) {
+  ScoreDims d;
+  if (!score_plan(R, b->tok_off_host, U, e->score_ctas, e->score_tpc_fixed, &d))
+    return RKV_ERR_UNSUPPORTED;
+  if (d.chunks > e->max_chunks) return RKV_ERR_CAPACITY;
+  if (e->sym) {   // the scratch sized at creation covers every batch within the capacities
+    int64_t cs_need = 0;
     for (int u = 0; u < U; ++u)
       cs_need += sym_scratch_floats(b->tok_off_host[u + 1] - b->tok_off_host[u], e->cfg.window);
-    if (cs_need > e->cs_cap) {
-      cudaFree(e->cs);
-      e->cs = nullptr;
-      e->cs_cap = 0;
-      if (cudaMalloc(&e->cs, sizeof(float) * cs_need) != cudaSuccess) {
-        cudaGetLastError();
-        e->cs = nullptr;
-        return RKV_ERR_OOM;
-      }
-      e->cs_cap = cs_need;
-    }
+    if (cs_need > e->cs_cap) return RKV_ERR_CAPACITY;
   }
-
-  const int cs = e->score_cs_fixed > 0
-                     ? e->score_cs_fixed
-                     : score_cluster_size(nmax, e->rp, e->max_cs, U, e->score_clusters);
-  if (cs == 0) return RKV_ERR_UNSUPPORTED;
-  int ncl = e->score_clusters[cs_index(cs)];
-  if (ncl > U) ncl = U;
 
   CUtensorMap kmap, qmap;
   if (make_map(e, &kmap, b->K, static_cast<uint64_t>(T), kTile) != RKV_OK) return RKV_ERR_CUDA;
-  if (make_map(e, &qmap, b->Q, static_cast<uint64_t>(U) * R, e->rp) != RKV_OK)
+  if (make_map(e, &qmap, b->Q, static_cast<uint64_t>(U) * R, d.rp) != RKV_OK)
     return RKV_ERR_CUDA;
 
-  ScoreParams p;
+  const int rows_per_item = e->pair ? GemmCfg<true>::kRowsPerItem : GemmCfg<false>::kRowsPerItem;
+  PlanParams pp = {};
+  pp.tok_off = b->tok_off;
+  pp.U = U;
+  pp.w = e->cfg.window;
+  pp.tpc = d.tpc;
+  pp.chunk_off = e->chunk_off;
+  pp.score_cnt = e->score_cnt;
+  pp.score_abort = e->score_cnt + static_cast<int64_t>(e->cfg.max_units) * kScoreCnt;
+  if (!closed) {   // GEMM row blocks and the padded rho layout the score kernel writes
+    pp.rows_per_item = rows_per_item;
+    pp.item_off = e->item_off;
+    pp.unit_cnt = e->unit_cnt;
+    pp.rho_off = e->rho_off;
+    pp.cs_off = e->sym ? e->cs_off : nullptr;
+  }
+  t_begin(e, RKV_KERNEL_PLAN, st);
+  cudaError_t err = launch_plan(pp, st);
+  t_end(e, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  ++e->launches;
+
+  ScoreParams p = {};
   p.tok_off = b->tok_off;
+  p.chunk_off = e->chunk_off;
   p.num_units = U;
+  p.total_chunks = static_cast<int>(d.chunks);
   p.R = R;
   p.w = e->cfg.window;
-  p.cs = cs;
+  p.tpc = d.tpc;
   p.nstages = e->nstages;
   p.scale_log2 = kLog2e / sqrtf(static_cast<float>(kHeadDim));
+  p.wait_ns = e->wait_ns;
+  p.drop_chunk = -1;
+  if (e->fault == RKV_FAULT_DROP_ANNOUNCE) {   // test hook: one announcement goes missing
+    e->fault = 0;
+    p.drop_chunk = 0;
+    p.wait_ns = 50000000ull;
+  }
   p.a_out = a;
   p.r_out = r;
   p.m_out = m;
   p.rho_out = closed ? nullptr : e->rho;
   p.rho_off = closed ? nullptr : e->rho_off;
+  p.cnt = e->score_cnt;
+  p.abort_all = pp.score_abort;
+  p.xstat = e->xstat;
+  p.xsum = e->xsum;
   p.status = e->status;
-  const int rows_per_item = e->pair ? GemmCfg<true>::kRowsPerItem : GemmCfg<false>::kRowsPerItem;
-  cudaError_t err;
-  if (!closed) {   // row blocks for the GEMM and the padded rho layout the score kernel writes
-    t_begin(e, RKV_KERNEL_PLAN, st);
-    err = launch_plan(b->tok_off, U, e->cfg.window, rows_per_item, e->item_off, e->unit_cnt,
-                      e->rho_off, e->sym ? e->cs_off : nullptr, st);
+  for (int gq = 0; gq < d.ngroups; ++gq) {
+    p.group = gq;
+    p.row0 = 64 * gq;
+    p.Rg = std::min(d.rp, R - p.row0);
+    p.final_pass = gq == d.ngroups - 1;
+    t_begin(e, RKV_KERNEL_SCORE, st);
+    err = launch_score(kmap, qmap, p, d.rp, closed, d.grid, st);
     t_end(e, st);
     if (err != cudaSuccess) return cuda_fail(err);
     ++e->launches;
   }
-  t_begin(e, RKV_KERNEL_SCORE, st);
-  err = launch_score(kmap, qmap, p, e->rp, closed, ncl, st);
-  t_end(e, st);
-  if (err != cudaSuccess) return cuda_fail(err);
-  ++e->launches;
   if (closed) return RKV_OK;
 
   // redundancy GEMM
@@ -538,7 +620,8 @@ int rkv_refree_budget(rkv_engine* e, const rkv_batch* b, float T, int sinks, int
   if (U == 0) return RKV_OK;
   if (!e->rf_z) {
     const size_t n = static_cast<size_t>(e->cfg.max_tokens) * refree_padded_group(e->cfg.group);
-    if (cudaMalloc(&e->rf_z, n * sizeof(float)) != cudaSuccess) {
+    if (dev_alloc(&e->fault, reinterpret_cast<void**>(&e->rf_z), n * sizeof(float)) !=
+        cudaSuccess) {
       cudaGetLastError();
       e->rf_z = nullptr;
       return RKV_ERR_OOM;

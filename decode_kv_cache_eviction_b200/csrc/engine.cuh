@@ -22,13 +22,13 @@ struct rkv_engine {
   rkv_config cfg;
   int device = 0;
   int nsm = 0;
-  int rp = 32;                 // padded G*w (MMA N of the logits tile)
+  int rp = 32;                 // padded query rows per score launch (16, 32, 64)
   int nstages = 0;             // score K-tile ring depth
   int score_smem = 0;
-  int score_clusters[5] = {};  // active clusters for cluster sizes 1, 2, 4, 8, 16
-  int score_cs_fixed = 0;      // > 0: score cluster size set by rkv_compress_host
-  int max_cs = 16;
+  int score_ctas = 0;          // persistent score grid (one CTA per SM)
+  int score_tpc_fixed = 0;     // > 0: score chunk size set by rkv_compress_host
   int max_n = 0;               // largest supported N_u
+  int64_t max_chunks = 0;      // score chunks the exchange workspace holds
   bool pair = true;
   bool rowmax = false;   // row-max redundancy epilogue
   bool sym = false;      // symmetric GEMM (tiles on and above the diagonal)
@@ -38,9 +38,15 @@ struct rkv_engine {
   int* item_off = nullptr;     // [max_units + 1]
   int* unit_cnt = nullptr;     // [max_units]
   int* status = nullptr;       // [1]
+  int* chunk_off = nullptr;    // [max_units + 1] score chunks prefix
+  int* score_cnt = nullptr;    // [max_units * kScoreCnt] score exchange counters
+  float* xstat = nullptr;      // [max_chunks * score_xs] score chunk statistics
+  float* xsum = nullptr;       // [max_chunks * 2 * kScoreMaxGroups] score chunk sums
   int64_t* cs_off = nullptr;   // [max_units + 1] symmetric form: scratch offsets
-  float* cs = nullptr;         // symmetric form: column partials, grown on demand
+  float* cs = nullptr;         // symmetric form: partial sums, sized at creation
   int64_t cs_cap = 0;          // floats allocated in cs
+  uint64_t wait_ns = 2000000000ull;   // limit of a score wait on another CTA
+  int fault = 0;               // RKV_FAULT_* armed by rkv_inject_fault
   int64_t launches = 0;
   PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   // per-kernel timing (rkv_set_timing)
@@ -70,3 +76,7 @@ struct rkv_engine {
 
 // Frees everything rkv_compress_host allocated (called by rkv_destroy).
 void rkv_host_pipeline_free(rkv_engine* e);
+
+// cudaMalloc for the engine's lazily grown buffers; fails (once) when an
+// allocation fault has been armed with rkv_inject_fault.
+cudaError_t rkv_engine_alloc(rkv_engine* e, void** p, size_t bytes);

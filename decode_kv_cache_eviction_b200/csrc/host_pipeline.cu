@@ -14,7 +14,7 @@
 // addressing), the compaction kernel gathers the kept rows straight from host
 // memory and V is never copied in whole; otherwise each chunk's V is copied
 // like K.  Every kernel works per unit and every chunk scores with the
-// cluster size of the whole batch, so a chunk's results do not depend on how
+// chunk size of the whole batch, so a chunk's results do not depend on how
 // the units were split: the outputs equal those of one rkv_compress over the
 // whole batch.
 #include <algorithm>
@@ -76,8 +76,10 @@ int reserve_slots(rkv_engine* e, int64_t tokens, int units) {
   free_slots(e);
   const int64_t R = static_cast<int64_t>(e->cfg.group) * e->cfg.window;
   bool ok = true;
+  // an armed allocation fault (rkv_inject_fault) fails the first of these
+  ok = rkv_engine_alloc(e, &e->hslot[0].K, tokens * kRowBytes) == cudaSuccess;
   for (auto& s : e->hslot) {
-    ok = ok && cudaMalloc(&s.K, tokens * kRowBytes) == cudaSuccess;
+    if (!s.K) ok = ok && cudaMalloc(&s.K, tokens * kRowBytes) == cudaSuccess;
     ok = ok && cudaMalloc(&s.V, tokens * kRowBytes) == cudaSuccess;
     ok = ok && cudaMalloc(&s.Q, units * R * kRowBytes) == cudaSuccess;
     ok = ok && cudaMalloc(&s.off, (units + 1) * sizeof(int64_t)) == cudaSuccess;
@@ -182,6 +184,12 @@ extern "C" int rkv_compress_host(rkv_engine* e, const rkv_host_batch* hb, float 
   const int64_t npin = U + static_cast<int64_t>(chunks.size());
   if (npin >= (int64_t{1} << 31)) return RKV_ERR_UNSUPPORTED;
 
+  // every chunk scores with the chunk size of the whole batch, so each unit's
+  // partial sums are grouped as rkv_compress on the batch groups them
+  rkv::ScoreDims whole;
+  if (!rkv::score_plan(e->cfg.group * w, off, U, e->score_ctas, 0, &whole))
+    return RKV_ERR_UNSUPPORTED;
+
   int rc = make_streams(e);
   if (rc != RKV_OK) return rc;
   // the previous call may still be reading the pinned offsets or the slots
@@ -230,14 +238,11 @@ extern "C" int rkv_compress_host(rkv_engine* e, const rkv_host_batch* hb, float 
   const char* hK = static_cast<const char*>(hb->K);
   const char* hV = static_cast<const char*>(hb->V);
   const char* hQ = static_cast<const char*>(hb->Q);
-  // every chunk scores with the cluster size of the whole batch, so each
-  // unit's cross-CTA sums are grouped as rkv_compress on the batch groups them
-  struct FixedClusterSize {
+  struct FixedChunk {
     rkv_engine* e;
-    FixedClusterSize(rkv_engine* en, int cs) : e(en) { e->score_cs_fixed = cs; }
-    ~FixedClusterSize() { e->score_cs_fixed = 0; }
-  } fixed_cs(e, rkv::score_cluster_size(static_cast<int>(nmax), e->rp, e->max_cs, U,
-                                   e->score_clusters));
+    FixedChunk(rkv_engine* en, int tpc) : e(en) { e->score_tpc_fixed = tpc; }
+    ~FixedChunk() { e->score_tpc_fixed = 0; }
+  } fixed_tpc(e, whole.tpc);
   for (size_t i = 0; i < chunks.size(); ++i) {
     const Chunk& c = chunks[i];
     const int s = static_cast<int>(i & 1);

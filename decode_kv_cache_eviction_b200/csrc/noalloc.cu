@@ -1,17 +1,21 @@
 // rkv_score_noalloc: GEMM-mode scoring for callers that cannot allocate device
 // memory.  The scratch that rkv_score keeps in an engine's workspace (1/||k||
-// per row, per-unit row-block offsets and finished-block counters, a status
-// word) lives here in one file-scope __device__ array of fixed size; the call
-// allocates and frees nothing.
+// per row, the score kernel's per-chunk exchange slots and counters, per-unit
+// offsets and finished-block counters, a status word) lives here in one
+// file-scope __device__ array of fixed size; the call allocates and frees
+// nothing.
 //
 // The array's device address is looked up once per device with that device
 // current (cudaGetSymbolAddress); the host-side symbol itself is only a
 // stand-in and is never passed to a kernel.  Every call rewrites the parts it
 // reads: the plan kernel rewrites the offsets and zeroes the counters, the
-// score kernel rewrites 1/||k|| of every row it covers.  Calls that overlap on
-// the GPU share the array and race.
+// score kernel rewrites the exchange slots and 1/||k|| of every row it covers.
+// Calls that overlap on the GPU share the array and race.  The status word is
+// the one part that persists: a device wait that timed out leaves its bit
+// there until rkv_noalloc_check_status reads and clears it.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstddef>
 #include <mutex>
@@ -26,14 +30,22 @@ namespace {
 
 constexpr int kMaxUnits = RKV_NOALLOC_MAX_UNITS;
 constexpr int64_t kMaxTokens = RKV_NOALLOC_MAX_TOKENS;
+constexpr int kMaxRp = 32;                 // G * w <= 32: one score pass
+// chunks of any batch within the limits: score_max_chunks with up to 256 CTAs
+constexpr int kMaxChunks = 8192;
 constexpr int kMaxDevices = 64;
 constexpr int kSmemCap = 227 * 1024;
 
 struct Scratch {
   float rho[kMaxTokens + static_cast<int64_t>(kRhoAlign) * kMaxUnits];
+  float xstat[static_cast<int64_t>(kMaxChunks) * score_xs(kMaxRp, false)];
+  float xsum[static_cast<int64_t>(kMaxChunks) * 2 * kScoreMaxGroups];
   int64_t rho_off[kMaxUnits + 1];
   int item_off[kMaxUnits + 1];
   int unit_cnt[kMaxUnits];
+  int chunk_off[kMaxUnits + 1];
+  int score_cnt[kMaxUnits * kScoreCnt];
+  int score_abort[4];
   int status[4];
 };
 
@@ -42,10 +54,9 @@ __device__ __align__(256) Scratch g_scratch;
 struct DeviceState {
   bool ready = false;
   Scratch* scratch = nullptr;  // device address of g_scratch on this device
-  int clusters[2][5] = {};     // [rp == 32][log2 cluster size]
-  int max_cs[2] = {};
-  int nstages[2] = {};
+  int nstages[2] = {};         // [rp == 32]
   int smem[2] = {};
+  int ctas[2] = {};
   int gemm_ctas = 0;
 };
 
@@ -79,27 +90,26 @@ int setup(int dev, DeviceState** out) {
     }
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
+  // With lazy module loading the module that holds the array, and so the
+  // array itself, may only be loaded here; that is an allocation the caller
+  // could not have accounted for if its memory pool is already reserved.
   void* ptr = nullptr;
-  if (cudaGetSymbolAddress(&ptr, g_scratch) != cudaSuccess || !ptr) {
+  const cudaError_t se = cudaGetSymbolAddress(&ptr, g_scratch);
+  if (se != cudaSuccess || !ptr) {
     cudaGetLastError();
-    return RKV_ERR_CUDA;
+    return se == cudaErrorMemoryAllocation ? RKV_ERR_OOM : RKV_ERR_CUDA;
   }
   d.scratch = static_cast<Scratch*>(ptr);
   for (int k = 0; k < 2; ++k) {
     const int rp = k ? 32 : 16;
     d.nstages[k] = score_stages(rp, false, kSmemCap);
     d.smem[k] = score_layout(rp, false, d.nstages[k]).total + 1024;
-    if (d.nstages[k] == 0 || score_configure(rp, false, d.smem[k], 16) != cudaSuccess) {
+    if (d.nstages[k] == 0 || score_configure(rp, false, d.smem[k]) != cudaSuccess) {
       cudaGetLastError();
       return RKV_ERR_CUDA;
     }
-    d.max_cs[k] = 0;
-    for (int i = 0; i < 5; ++i) {
-      d.clusters[k][i] = score_max_clusters(rp, false, d.smem[k], 1 << i);
-      if (d.clusters[k][i] > 0) d.max_cs[k] = 1 << i;
-      else break;
-    }
-    if (d.max_cs[k] == 0) return RKV_ERR_UNSUPPORTED;
+    d.ctas[k] = score_max_ctas(rp, false, d.smem[k]);
+    if (d.ctas[k] <= 0) return RKV_ERR_UNSUPPORTED;
   }
   if (gemm_configure(true, false, false) != cudaSuccess) {
     cudaGetLastError();
@@ -126,23 +136,26 @@ int encode(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
 
 bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+int fail() {
+  cudaGetLastError();
+  return RKV_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, float* a, float* r,
                                  float* m, rkv_stream_t stream) {
   if (group < 1 || window < 1 || !b || !a || !r) return RKV_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(group) * window > kMaxRows) return RKV_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(group) * window > kMaxRp) return RKV_ERR_UNSUPPORTED;
   const int U = b->num_units;
   if (U < 0 || !b->tok_off || !b->tok_off_host || !b->K || !b->Q) return RKV_ERR_INVALID_ARG;
   if (U > kMaxUnits) return RKV_ERR_CAPACITY;
   const int64_t* off = b->tok_off_host;
   if (off[0] != 0) return RKV_ERR_INVALID_ARG;
-  int nmax = 0;
   for (int u = 0; u < U; ++u) {
     const int64_t n = off[u + 1] - off[u];
     if (n < window) return RKV_ERR_INVALID_ARG;
     if (n > kMaxTokensPerUnit) return RKV_ERR_UNSUPPORTED;
-    if (n > nmax) nmax = static_cast<int>(n);
   }
   const int64_t T = off[U];
   if (T > kMaxTokens) return RKV_ERR_CAPACITY;
@@ -152,58 +165,71 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   if (U == 0) return RKV_OK;
 
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    cudaGetLastError();
-    return RKV_ERR_CUDA;
-  }
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return fail();
   DeviceState* d = nullptr;
   int rc = setup(dev, &d);
   if (rc != RKV_OK) return rc;
 
   const int R = group * window;
-  const int rp = R <= 16 ? 16 : 32;
-  const int k = rp == 32 ? 1 : 0;
-  const int cs = score_cluster_size(nmax, rp, d->max_cs[k], U, d->clusters[k]);
-  if (cs == 0) return RKV_ERR_UNSUPPORTED;
-  int ci = 0;
-  while ((1 << ci) < cs) ++ci;
-  int ncl = d->clusters[k][ci];
-  if (ncl > U) ncl = U;
+  const int k = R > 16 ? 1 : 0;
+  ScoreDims dims;
+  if (!score_plan(R, off, U, d->ctas[k], 0, &dims)) return RKV_ERR_UNSUPPORTED;
+  if (dims.chunks > kMaxChunks) return RKV_ERR_CAPACITY;
 
   CUtensorMap kmap, qmap, amap, bmap;
   if (encode(&kmap, b->K, static_cast<uint64_t>(T), kTile) != RKV_OK ||
-      encode(&qmap, b->Q, static_cast<uint64_t>(U) * R, rp) != RKV_OK ||
+      encode(&qmap, b->Q, static_cast<uint64_t>(U) * R, dims.rp) != RKV_OK ||
       encode(&amap, b->K, static_cast<uint64_t>(T), GemmCfg<true>::kRowsPerCta) != RKV_OK ||
       encode(&bmap, b->K, static_cast<uint64_t>(T), GemmCfg<true>::kBRows) != RKV_OK)
     return RKV_ERR_CUDA;
 
   Scratch* s = d->scratch;  // device address, never the host-side symbol
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  constexpr int kRows = GemmCfg<true>::kRowsPerItem;
 
-  ScoreParams p;
+  PlanParams pp = {};
+  pp.tok_off = b->tok_off;
+  pp.U = U;
+  pp.w = window;
+  pp.tpc = dims.tpc;
+  pp.chunk_off = s->chunk_off;
+  pp.score_cnt = s->score_cnt;
+  pp.score_abort = s->score_abort;
+  pp.rows_per_item = kRows;
+  pp.item_off = s->item_off;
+  pp.unit_cnt = s->unit_cnt;
+  pp.rho_off = s->rho_off;
+  pp.cs_off = nullptr;
+  if (launch_plan(pp, st) != cudaSuccess) return fail();
+
+  ScoreParams p = {};
   p.tok_off = b->tok_off;
+  p.chunk_off = s->chunk_off;
   p.num_units = U;
+  p.total_chunks = static_cast<int>(dims.chunks);
   p.R = R;
+  p.row0 = 0;
+  p.Rg = R;
   p.w = window;
-  p.cs = cs;
+  p.tpc = dims.tpc;
   p.nstages = d->nstages[k];
+  p.group = 0;
+  p.final_pass = 1;
+  p.drop_chunk = -1;
   p.scale_log2 = kLog2e / sqrtf(static_cast<float>(kHeadDim));
+  p.wait_ns = 2000000000ull;
   p.a_out = a;
   p.r_out = r;
   p.m_out = m;
   p.rho_out = s->rho;
   p.rho_off = s->rho_off;
+  p.cnt = s->score_cnt;
+  p.abort_all = s->score_abort;
+  p.xstat = s->xstat;
+  p.xsum = s->xsum;
   p.status = s->status;
-  constexpr int kRows = GemmCfg<true>::kRowsPerItem;
-  if (launch_plan(b->tok_off, U, window, kRows, s->item_off, s->unit_cnt, s->rho_off, nullptr, st) !=
-      cudaSuccess) {
-    cudaGetLastError();
-    return RKV_ERR_CUDA;
-  }
-  if (launch_score(kmap, qmap, p, rp, false, ncl, st) != cudaSuccess) {
-    cudaGetLastError();
-    return RKV_ERR_CUDA;
-  }
+  if (launch_score(kmap, qmap, p, dims.rp, false, dims.grid, st) != cudaSuccess) return fail();
+
   int64_t items = 0;
   for (int u = 0; u < U; ++u) {
     const int64_t c = off[u + 1] - off[u] - window;
@@ -225,9 +251,27 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   g.cs_off = nullptr;
   int64_t nctas = d->gemm_ctas;
   if (nctas > 2 * items) nctas = 2 * items;
-  if (launch_gemm(amap, bmap, g, true, false, false, static_cast<int>(nctas), st) != cudaSuccess) {
-    cudaGetLastError();
-    return RKV_ERR_CUDA;
+  if (launch_gemm(amap, bmap, g, true, false, false, static_cast<int>(nctas), st) != cudaSuccess)
+    return fail();
+  return RKV_OK;
+}
+
+extern "C" int rkv_noalloc_check_status(rkv_stream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return fail();
+  DeviceState* d = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_dev[dev].ready) d = &g_dev[dev];
   }
+  if (!d) return RKV_OK;   // no call has run on this device
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return fail();
+  int h = 0;
+  if (cudaMemcpy(&h, d->scratch->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return fail();
+  if (h != 0 && cudaMemset(d->scratch->status, 0, sizeof(int)) != cudaSuccess) return fail();
+  if (h & kStatusTimeout) return RKV_ERR_TIMEOUT;
+  if (h != 0) return RKV_ERR_CUDA;
   return RKV_OK;
 }

@@ -646,76 +646,96 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// One block: items per unit and their prefix, 256-aligned rho segment
-// offsets, zeroed unit counters and (symmetric form, cs_off != null) the
-// offsets of each unit's scratch.  An item is a block of candidate rows, or in
-// the symmetric form any 256-key block of a unit that has candidates (its
-// columns reach every candidate row).
-__global__ void plan_kernel(const int64_t* tok_off, int U, int w, int rows_per_item,
-                            int* item_off, int* unit_cnt, int64_t* rho_off, int64_t* cs_off) {
-  __shared__ long long wsum[3][32];
+// One block, before the score kernel: the score chunks of every unit and their
+// prefix, zeroed exchange counters and, for the GEMM, items per unit and their
+// prefix, 256-aligned rho segment offsets, zeroed unit counters and (symmetric
+// form, cs_off != null) the offsets of each unit's scratch.  A GEMM item is a
+// block of candidate rows, or in the symmetric form any 256-key block of a unit
+// that has candidates (its columns reach every candidate row).
+__global__ void plan_kernel(const PlanParams pp) {
+  __shared__ long long wsum[4][32];
+  const int U = pp.U;
   const int tid = threadIdx.x, nt = blockDim.x;
   const int per = (U + nt - 1) / nt;
   const int u0 = min(U, tid * per), u1 = min(U, u0 + per);
-  long long li = 0, lr = 0, ls = 0;   // this thread's items, rho and scratch lengths
+  const bool gemm = pp.rows_per_item > 0;
+  const bool sym = pp.cs_off != nullptr;
+  const int64_t chunk_tok = static_cast<int64_t>(pp.tpc) * kTile;
+  if (tid == 0) *pp.score_abort = 0;
+  long long lc = 0, li = 0, lr = 0, ls = 0;   // this thread's chunks, items, rho, scratch
   for (int u = u0; u < u1; ++u) {
-    const int64_t n = tok_off[u + 1] - tok_off[u];
-    const int64_t c = n - w;
-    li += gemm_unit_items(n, c, rows_per_item, cs_off != nullptr);
-    lr += (n + kRhoAlign - 1) / kRhoAlign * kRhoAlign;
-    ls += sym_scratch_floats(n, w);
-    unit_cnt[u] = 0;
+    const int64_t n = pp.tok_off[u + 1] - pp.tok_off[u];
+    lc += (n + chunk_tok - 1) / chunk_tok;
+    for (int e = 0; e < kScoreCnt; ++e) pp.score_cnt[u * kScoreCnt + e] = 0;
+    if (gemm) {
+      li += gemm_unit_items(n, n - pp.w, pp.rows_per_item, sym);
+      lr += (n + kRhoAlign - 1) / kRhoAlign * kRhoAlign;
+      ls += sym_scratch_floats(n, pp.w);
+      pp.unit_cnt[u] = 0;
+    }
   }
-  // block exclusive scans of li, lr and ls
-  long long ii = li, ir = lr, is = ls;
+  // block exclusive scans
+  long long x[4] = {lc, li, lr, ls};
   const int lane = tid & 31, wp = tid >> 5;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const long long yi = __shfl_up_sync(0xffffffffu, ii, o);
-    const long long yr = __shfl_up_sync(0xffffffffu, ir, o);
-    const long long ys = __shfl_up_sync(0xffffffffu, is, o);
-    if (lane >= o) { ii += yi; ir += yr; is += ys; }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const long long y = __shfl_up_sync(0xffffffffu, x[k], o);
+      if (lane >= o) x[k] += y;
+    }
   }
-  if (lane == 31) { wsum[0][wp] = ii; wsum[1][wp] = ir; wsum[2][wp] = is; }
+  if (lane == 31)
+    for (int k = 0; k < 4; ++k) wsum[k][wp] = x[k];
   __syncthreads();
   if (wp == 0) {
-    long long xi = lane < (nt >> 5) ? wsum[0][lane] : 0;
-    long long xr = lane < (nt >> 5) ? wsum[1][lane] : 0;
-    long long xs = lane < (nt >> 5) ? wsum[2][lane] : 0;
+    long long z[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) z[k] = lane < (nt >> 5) ? wsum[k][lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const long long yi = __shfl_up_sync(0xffffffffu, xi, o);
-      const long long yr = __shfl_up_sync(0xffffffffu, xr, o);
-      const long long ys = __shfl_up_sync(0xffffffffu, xs, o);
-      if (lane >= o) { xi += yi; xr += yr; xs += ys; }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const long long y = __shfl_up_sync(0xffffffffu, z[k], o);
+        if (lane >= o) z[k] += y;
+      }
     }
-    wsum[0][lane] = xi;
-    wsum[1][lane] = xr;
-    wsum[2][lane] = xs;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) wsum[k][lane] = z[k];
   }
   __syncthreads();
-  long long ri = ii - li + (wp > 0 ? wsum[0][wp - 1] : 0);
-  long long rr = ir - lr + (wp > 0 ? wsum[1][wp - 1] : 0);
-  long long rs = is - ls + (wp > 0 ? wsum[2][wp - 1] : 0);
+  long long rc = x[0] - lc + (wp > 0 ? wsum[0][wp - 1] : 0);
+  long long ri = x[1] - li + (wp > 0 ? wsum[1][wp - 1] : 0);
+  long long rr = x[2] - lr + (wp > 0 ? wsum[2][wp - 1] : 0);
+  long long rs = x[3] - ls + (wp > 0 ? wsum[3][wp - 1] : 0);
   for (int u = u0; u < u1; ++u) {
-    item_off[u] = static_cast<int>(ri);
-    rho_off[u] = rr;
-    if (cs_off) cs_off[u] = rs;
-    const int64_t n = tok_off[u + 1] - tok_off[u];
-    const int64_t c = n - w;
-    ri += gemm_unit_items(n, c, rows_per_item, cs_off != nullptr);
-    rr += (n + kRhoAlign - 1) / kRhoAlign * kRhoAlign;
-    rs += sym_scratch_floats(n, w);
+    const int64_t n = pp.tok_off[u + 1] - pp.tok_off[u];
+    pp.chunk_off[u] = static_cast<int>(rc);
+    rc += (n + chunk_tok - 1) / chunk_tok;
+    if (gemm) {
+      pp.item_off[u] = static_cast<int>(ri);
+      pp.rho_off[u] = rr;
+      if (sym) pp.cs_off[u] = rs;
+      ri += gemm_unit_items(n, n - pp.w, pp.rows_per_item, sym);
+      rr += (n + kRhoAlign - 1) / kRhoAlign * kRhoAlign;
+      rs += sym_scratch_floats(n, pp.w);
+    }
   }
   if (u1 == U && u0 < u1) {
-    item_off[U] = static_cast<int>(ri);
-    rho_off[U] = rr;
-    if (cs_off) cs_off[U] = rs;
+    pp.chunk_off[U] = static_cast<int>(rc);
+    if (gemm) {
+      pp.item_off[U] = static_cast<int>(ri);
+      pp.rho_off[U] = rr;
+      if (sym) pp.cs_off[U] = rs;
+    }
   }
   if (U == 0 && tid == 0) {
-    item_off[0] = 0;
-    rho_off[0] = 0;
-    if (cs_off) cs_off[0] = 0;
+    pp.chunk_off[0] = 0;
+    if (gemm) {
+      pp.item_off[0] = 0;
+      pp.rho_off[0] = 0;
+      if (sym) pp.cs_off[0] = 0;
+    }
   }
 }
 
@@ -846,10 +866,8 @@ int gemm_max_ctas(bool pair, bool rowmax, bool sym) {
   return 2 * n;
 }
 
-cudaError_t launch_plan(const int64_t* tok_off, int U, int w, int rows_per_item, int* item_off,
-                        int* unit_cnt, int64_t* rho_off, int64_t* cs_off, cudaStream_t st) {
-  plan_kernel<<<1, 1024, 0, st>>>(tok_off, U, w, rows_per_item, item_off, unit_cnt, rho_off,
-                                  cs_off);
+cudaError_t launch_plan(const PlanParams& pp, cudaStream_t st) {
+  plan_kernel<<<1, 1024, 0, st>>>(pp);
   return cudaGetLastError();
 }
 

@@ -11,68 +11,80 @@ constexpr int kHeadDim = 128;        // d (the only supported head size)
 constexpr int kTile = 128;           // tokens per K tile (TMA box rows, MMA M)
 constexpr int kTileBytes = kTile * kHeadDim * 2;
 constexpr int kMaxTokensPerUnit = 49152;  // select keeps a unit's keys in shared memory
-constexpr int kMaxRows = 32;         // G * w limit (MMA N of the logits tile)
+constexpr int kMaxRows = 256;        // G * w limit (row groups of 64 per launch)
 constexpr int kScoreThreads = 512;   // 16 warps
 constexpr int kGemmThreads = 640;    // producer, MMA, 2 idle, 16 epilogue warps
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------- score
+constexpr int kScoreMaxGroups = 4;              // row groups of 64: G * w <= 256
+constexpr int kScoreCnt = 2 * kScoreMaxGroups;  // exchange counters per unit
+
 struct ScoreParams {
   const int64_t* tok_off;  // [U+1]
+  const int* chunk_off;    // [U+1] prefix of chunks per unit
   int num_units;
-  int R;                   // G * w real query rows
+  int total_chunks;
+  int R;                   // G * w query rows of a unit
+  int row0;                // first query row of this launch's group
+  int Rg;                  // rows of this group (<= RP)
   int w;
-  int cs;                  // CTAs per cluster (one unit per cluster)
+  int tpc;                 // tiles of 128 tokens per chunk
   int nstages;             // K tile ring depth
+  int group;               // row group of this launch
+  int final_pass;          // last row group: normalises, computes the redundancy side
+  int drop_chunk;          // fault injection: chunk that skips its first announcement (-1)
   float scale_log2;        // log2(e) / sqrt(d)
+  uint64_t wait_ns;        // limit of a wait on another CTA
   float* a_out;            // [T]
   float* r_out;            // [T]
   float* m_out;            // [T] or null
   float* rho_out;          // 1/||k|| at rho_off[u] + j (pads zeroed), or null
   const int64_t* rho_off;  // [U+1] 256-aligned per-unit offsets into rho_out
+  int* cnt;                // [U][kScoreCnt] announcement counters, zeroed by the plan kernel
+  int* abort_all;          // set when a CTA of this call gives up; zeroed by the plan kernel
+  float* xstat;            // [chunks][score_xs] per-chunk (max, sum) per row [, U]
+  float* xsum;             // [chunks][kScoreMaxGroups][2] per-chunk sums of abar, exp(m)
   int* status;
 };
 
-struct ScoreLayout {
-  uint32_t stages, q, abar, marr, rhoc, rhot, ufin, gath, gath2, mrow, invl, red1, red2, rsum,
-      rowt, xbuf, bars, slot, flags, total;
-};
-
-constexpr int kMaxClusterSize = 16;
 constexpr int kTmemColsTotal = 512;
 
-// Logit tiles of one CTA live in TMEM for the whole unit: 512 columns hold
-// 512 / rp tiles of 128 tokens.
-__host__ __device__ inline int score_res_tiles(int rp) { return kTmemColsTotal / rp; }
-__host__ __device__ inline int score_lmax(int rp) { return score_res_tiles(rp) * kTile; }
-// Floats of one CTA's round-1 partials: (max, sum) per query row [, U].
-__host__ __device__ inline int score_xb(int rp, bool closed) { return 2 * rp + (closed ? 128 : 0); }
-constexpr int kScoreBarsFixed = 32 + 1 + 2 + 2 + 2;  // tile-ready, TMEM-free, Q, Q, exchange
+// Tokens per chunk: two logit buffers of 256 tensor-memory columns, RP per tile.
+__host__ __device__ constexpr int score_chunk_tokens(int rp) { return (256 / rp) * kTile; }
+// Floats of one chunk's exchange slot: (max, sum) per query row [, partial U].
+__host__ __device__ constexpr int score_xs(int rp, bool closed) {
+  return 2 * rp + (closed ? 128 : 0);
+}
+
+struct ScoreLayout {
+  uint32_t stages, q, abuf, marr, red1, red2, rhot, ufin, mpart, upart, mrow, invl, rsum, rowt,
+      bars, slot, flags, issued, total;
+};
 
 __host__ __device__ inline ScoreLayout score_layout(int rp, bool closed, int ns) {
   ScoreLayout L;
   uint32_t o = 0;
-  const int lmax = score_lmax(rp);
+  const int cht = score_chunk_tokens(rp);
   L.stages = o; o += ns * kTileBytes;
   L.q = o; o += 2 * rp * 256;
-  L.abar = o; o += lmax * 4;
-  L.marr = o; if (closed) o += lmax * 4;
-  L.rhoc = o; if (closed) o += lmax * 4;
-  L.rhot = o; if (closed) o += 2 * 128 * 4;
-  L.ufin = o; if (closed) o += 128 * 4;
-  L.gath = o; o += kMaxClusterSize * score_xb(rp, closed) * 4;   // round-1 inbox
-  L.gath2 = o; o += kMaxClusterSize * 4 * 4;                       // round-2 inbox
-  L.mrow = o; o += rp * 4;
-  L.invl = o; o += rp * 4;
+  L.abuf = o; o += 2 * 2 * cht * 4;
+  L.marr = o; if (closed) o += 2 * cht * 4;
   L.red1 = o; o += 4 * rp * 2 * 4;
   L.red2 = o; if (closed) o += 4 * 128 * 4;
+  L.rhot = o; if (closed) o += 2 * 128 * 4;
+  L.ufin = o; if (closed) o += 128 * 4;
+  L.mpart = o; o += 384 * 2 * 4;
+  L.upart = o; if (closed) o += 3 * 128 * 4;
+  L.mrow = o; o += rp * 4;
+  L.invl = o; o += rp * 4;
   L.rsum = o; o += 32 * 4;
-  L.rowt = o; o += 32 * 4;
-  L.xbuf = o; o += (score_xb(rp, closed) + 4) * 4;
+  L.rowt = o; o += 64 * 4;
   o = (o + 15u) & ~15u;
-  L.bars = o; o += (2 * ns + kScoreBarsFixed) * 8;
+  L.bars = o; o += (2 * ns + 32 + 6 + 1) * 8;
   L.slot = o; o += 16;
   L.flags = o; o += 16;
+  L.issued = o; o += 32;
   L.total = o;
   return L;
 }
@@ -84,21 +96,24 @@ __host__ __device__ inline int score_stages(int rp, bool closed, int smem_cap) {
   return 0;
 }
 
-// Cluster size of the score kernel for a batch of `units` units of at most
-// nmax tokens.  It is the smallest power of two whose CTAs hold a unit's logits
-// in TMEM (at most max_cs).  A unit is spread further, to at most 1024 tokens
-// per CTA, only while the batch has fewer units than clusters of that size can
-// be resident (clusters[log2 cs]): with more units, every extra CTA per unit
-// only adds cluster exchanges.  Returns 0 when no size fits.
-inline int score_cluster_size(int nmax, int rp, int max_cs, int64_t units, const int* clusters) {
-  int cs = 1;
-  while ((((nmax + cs - 1) / cs + kTile - 1) / kTile) * kTile > score_lmax(rp)) {
-    if (cs >= max_cs) return 0;
-    cs <<= 1;
-  }
-  auto log2i = [](int x) { int l = 0; while ((1 << l) < x) ++l; return l; };
-  while (cs < max_cs && (nmax + cs - 1) / cs > 1024 && units < clusters[log2i(cs)]) cs <<= 1;
-  return cs;
+// Launch shape of the score kernel for one batch.
+struct ScoreDims {
+  int rp;          // padded query rows per launch (16, 32, 64)
+  int ngroups;     // launches (row groups of 64)
+  int tpc;         // tiles per chunk
+  int64_t chunks;  // chunks of the batch
+  int grid;        // CTAs (<= max_ctas)
+};
+
+// Chooses the chunk size (tpc_fixed > 0 forces it) and grid for a batch of U
+// units with host row offsets `off`; false if G * w > 256 or a unit is too long
+// for the progress rule (every unit within 2 * grid chunks).
+bool score_plan(int R, const int64_t* off, int U, int max_ctas, int tpc_fixed, ScoreDims* d);
+// Upper bound of the chunks of any batch within the capacities.
+inline int64_t score_max_chunks(int64_t max_tokens, int max_units, int max_ctas, int rp) {
+  const int64_t tpc_max = score_chunk_tokens(rp) / kTile;
+  const int64_t a = (max_tokens / kTile + 2 * static_cast<int64_t>(max_units)) / tpc_max + 1;
+  return (a > max_ctas ? a : max_ctas) + max_units;
 }
 
 // ---------------------------------------------------------------- redundancy GEMM
@@ -161,12 +176,26 @@ __host__ __device__ inline GemmLayout gemm_layout() {
 // ---------------------------------------------------------------- launches
 // Each returns a cudaError_t of the launch (cudaSuccess when enqueued).
 cudaError_t launch_score(const CUtensorMap& kmap, const CUtensorMap& qmap, const ScoreParams& p,
-                         int rp, bool closed, int nclusters, cudaStream_t st);
-cudaError_t score_configure(int rp, bool closed, int smem_bytes, int cs);
-int score_max_clusters(int rp, bool closed, int smem_bytes, int cs);
+                         int rp, bool closed, int grid, cudaStream_t st);
+cudaError_t score_configure(int rp, bool closed, int smem_bytes);
+int score_max_ctas(int rp, bool closed, int smem_bytes);
 
-cudaError_t launch_plan(const int64_t* tok_off, int U, int w, int rows_per_item, int* item_off,
-                        int* unit_cnt, int64_t* rho_off, int64_t* cs_off, cudaStream_t st);
+// Per-batch offsets and zeroed counters, one block (before the score kernel).
+struct PlanParams {
+  const int64_t* tok_off;  // [U+1]
+  int U;
+  int w;
+  int tpc;                 // score: tiles per chunk
+  int* chunk_off;          // [U+1] score chunks prefix
+  int* score_cnt;          // [U][kScoreCnt] zeroed
+  int* score_abort;        // [1] zeroed
+  int rows_per_item;       // GEMM: rows per work item (0: no GEMM)
+  int* item_off;           // [U+1] GEMM items prefix (or null)
+  int* unit_cnt;           // [U] zeroed (or null)
+  int64_t* rho_off;        // [U+1] 256-aligned rho offsets (or null)
+  int64_t* cs_off;         // [U+1] symmetric scratch offsets (or null)
+};
+cudaError_t launch_plan(const PlanParams& pp, cudaStream_t st);
 cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const GemmParams& p,
                         bool pair, bool rowmax, bool sym, int nctas, cudaStream_t st);
 cudaError_t launch_sym_finish(const GemmParams& p, int nsm, cudaStream_t st);

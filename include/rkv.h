@@ -13,8 +13,9 @@
  * slot buffer (gather compaction, named as the R-KV-style baseline in the ThinKV
  * summary, "Continuous Thinking" section).
  *
- * Limits: head_dim = 128, G*w <= 32; N_u <= 32768 when G*w > 16, else N_u <= 49152
- * (each cluster of up to 16 CTAs keeps a unit's logits in tensor memory).
+ * Limits: head_dim = 128, G*w <= 256 (up to 64 query rows per pass over K; more
+ * rows take several passes), N_u <= 49152 (the selection keeps a unit's keys in
+ * shared memory).
  *
  * Terms used below.  A *unit* is one (sequence, layer, KV head).  Unit u has
  * N_u cached tokens, stored as rows tok_off[u] .. tok_off[u+1]-1 of K and V.
@@ -51,7 +52,7 @@ typedef struct rkv_engine rkv_engine;     /* opaque; owns its workspace and stag
 enum {
   RKV_OK = 0,
   RKV_ERR_INVALID_ARG = -1, /* null/unaligned pointer, bad size, N_u < w, ... */
-  RKV_ERR_UNSUPPORTED = -2, /* head_dim != 128, G*w > 32, N_u too long, not sm_100 */
+  RKV_ERR_UNSUPPORTED = -2, /* head_dim != 128, G*w > 256, N_u too long, not sm_100 */
   RKV_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
   RKV_ERR_TIMEOUT = -4,     /* a device-side wait ran out of time (see rkv_check_status) */
   RKV_ERR_OOM = -5,         /* workspace allocation failed */
@@ -82,6 +83,8 @@ typedef struct {
   int64_t max_tokens; /* capacity: total cached rows per batch (>= 1) */
   int redundancy;     /* RKV_REDUNDANCY_GEMM, _CLOSED_FORM or _MAX */
   int flags;          /* 0, or RKV_FLAG_* bits */
+  int64_t max_unit_tokens; /* capacity: longest unit N_u (0: the engine's limit);
+                              sizes the symmetric GEMM's scratch */
 } rkv_config;
 
 /* rkv_config.flags */
@@ -97,7 +100,9 @@ enum {
    * deterministic.  CTA pairs and RKV_REDUNDANCY_GEMM only
    * (RKV_ERR_UNSUPPORTED otherwise).  The scratch (128 nb (nb + 3) fp32 for a
    * unit of nb = ceil(N_u / 256) blocks, about N_u^2 / 128 bytes) is allocated
-   * by rkv_score when a batch first needs more and freed by rkv_destroy. */
+   * by rkv_create for the largest batch the capacities allow (max_tokens in
+   * units of max_unit_tokens) and freed by rkv_destroy; rkv_score allocates
+   * nothing. */
   RKV_FLAG_GEMM_SYMMETRIC = 2
 };
 
@@ -111,7 +116,9 @@ typedef struct {
 } rkv_batch;
 
 /* Create an engine and allocate its device workspace on the current device.
- * Fails with RKV_ERR_UNSUPPORTED on a device that is not sm_100. */
+ * Fails with RKV_ERR_UNSUPPORTED on a device that is not sm_100, or when
+ * max_unit_tokens exceeds the engine's limit; RKV_ERR_OOM when the workspace
+ * cannot be allocated (nothing is kept then). */
 int rkv_create(const rkv_config* cfg, rkv_engine** out);
 
 /* Free the workspace (waits for the device to finish using it). NULL is a no-op. */
@@ -125,7 +132,12 @@ int rkv_destroy(rkv_engine* eng);
  *               (RKV_REDUNDANCY_MAX: m_i = max_{j != i, j < N} khat_i . khat_j),
  *               khat = k / ||k|| (0 for a zero key);
  *   m [T] fp32, optional (NULL to skip): the m_i.
- * Row tok_off[u] + i holds token i of unit u; window rows (i >= N_u - w) are 0. */
+ * Row tok_off[u] + i holds token i of unit u; window rows (i >= N_u - w) are 0.
+ * Allocates nothing and never synchronises the host.  The kernels exchange
+ * per-chunk statistics through the engine's workspace and wait on each other
+ * with a bounded wait; a wait that runs out sets RKV_ERR_TIMEOUT in the status
+ * word (rkv_check_status).  RKV_ERR_UNSUPPORTED for a unit longer than the
+ * engine's limit; RKV_ERR_CAPACITY for a batch beyond its capacities. */
 int rkv_score(rkv_engine* eng, const rkv_batch* batch, float* a, float* r, float* m,
               rkv_stream_t stream);
 
@@ -258,6 +270,17 @@ int rkv_compress_host(rkv_engine* eng, const rkv_host_batch* batch, float lambda
  * RKV_ERR_DEVICE (an out-of-range kept index reached rkv_compact). */
 int rkv_check_status(rkv_engine* eng, rkv_stream_t stream);
 
+/* Fault injection, for testing the error paths without faulting a GPU.
+ *   RKV_FAULT_ALLOC: the engine's next device allocation fails (RKV_ERR_OOM);
+ *     with eng = NULL, the next rkv_create's workspace allocation fails;
+ *   RKV_FAULT_DROP_ANNOUNCE: in the next score launch one chunk does not
+ *     announce its statistics, and the waits of that launch give up after
+ *     50 ms, so rkv_check_status then reports RKV_ERR_TIMEOUT;
+ *   RKV_FAULT_NONE: disarm.
+ * A fault fires once.  Returns RKV_ERR_INVALID_ARG for an unknown fault. */
+enum { RKV_FAULT_NONE = 0, RKV_FAULT_ALLOC = 1, RKV_FAULT_DROP_ANNOUNCE = 2 };
+int rkv_inject_fault(rkv_engine* eng, int fault);
+
 /* Number of kernel launches enqueued by this engine since creation. */
 int64_t rkv_launch_count(const rkv_engine* eng);
 
@@ -293,24 +316,36 @@ int rkv_read_timing(rkv_engine* eng, int kernel, double* total_ms, int64_t* laun
  *
  * Computes exactly what rkv_score computes for an engine created with
  * RKV_REDUNDANCY_GEMM (CTA-pair GEMM), with head_dim = 128 and the given group and
- * window.  Its scratch (1/||k|| per row, per-unit row-block and row offsets and
- * counters, a status word) lives in one file-scope __device__ array of about
- * 8.5 MB that every GPU which loads the library holds until the process exits;
- * nothing is allocated or freed per call.  Limits: at most RKV_NOALLOC_MAX_UNITS
+ * window.  Its scratch (1/||k|| per row, the score kernel's per-chunk exchange
+ * slots and counters, per-unit offsets and counters, a status word) lives in one
+ * file-scope __device__ array of about 11 MB that every GPU holding the
+ * library's module keeps until the process exits; nothing is allocated or freed
+ * per call.  Limits: G*w <= 32, N_u <= 49152, at most RKV_NOALLOC_MAX_UNITS
  * units and RKV_NOALLOC_MAX_TOKENS rows per call (larger batches return
- * RKV_ERR_CAPACITY before anything is enqueued), and the rkv_score limits
- * (G*w <= 32; N_u <= 32768 when G*w > 16, else N_u <= 49152).
+ * RKV_ERR_CAPACITY, longer units or larger G*w RKV_ERR_UNSUPPORTED, before
+ * anything is enqueued).
  *
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) and sets kernel attributes with that device current;
- * make that first call before any stream capture.  All calls share the one
- * array and each call rewrites what it reads, so successive calls on one
- * stream are safe, but calls that overlap on the GPU (other streams, other host
- * threads without ordering) race on it.  A device-side wait that times out is
- * recorded only in the array's status word: this call has no status query. */
+ * (cudaGetSymbolAddress) and sets kernel attributes with that device current.
+ * Under CUDA's lazy module loading (the default) that lookup may be the moment
+ * the module, and with it the array, is loaded into the device's memory: make
+ * the first call on each device before reserving a memory pool that leaves no
+ * room for it (it returns RKV_ERR_OOM when the array cannot be loaded), and
+ * before any stream capture.  All calls share the one array and each call
+ * rewrites what it reads, so successive calls on one stream are safe, but calls
+ * that overlap on the GPU (other streams, other host threads without ordering)
+ * race on it.  A device-side wait that times out leaves a bit in the array's
+ * status word; rkv_noalloc_check_status reports and clears it. */
 enum { RKV_NOALLOC_MAX_UNITS = 4096, RKV_NOALLOC_MAX_TOKENS = 1048576 };
 int rkv_score_noalloc(int group, int window, const rkv_batch* batch, float* a, float* r,
                       float* m, rkv_stream_t stream);
+
+/* Status of the rkv_score_noalloc calls on the current device: synchronises
+ * `stream`, then reads and clears the status word of the device's static
+ * scratch.  RKV_OK, RKV_ERR_TIMEOUT (a device wait gave up; the outputs of the
+ * calls since the last check are invalid) or RKV_ERR_CUDA.  Allocates nothing;
+ * RKV_OK when no call has run on the device yet. */
+int rkv_noalloc_check_status(rkv_stream_t stream);
 
 /* Static description of a status code. */
 const char* rkv_status_string(int status);

@@ -51,9 +51,9 @@ def test_struct_layout_matches_header():
     #include <stddef.h>
     #include "rkv.h"
     int main(void) {
-      printf("%zu %zu %zu %zu %zu\n", sizeof(rkv_config), offsetof(rkv_config, max_tokens),
+      printf("%zu %zu %zu %zu %zu %zu\n", sizeof(rkv_config), offsetof(rkv_config, max_tokens),
              offsetof(rkv_config, redundancy), offsetof(rkv_config, flags),
-             sizeof(rkv_batch));
+             offsetof(rkv_config, max_unit_tokens), sizeof(rkv_batch));
       printf("%zu %zu %zu %zu %zu\n", offsetof(rkv_batch, tok_off),
              offsetof(rkv_batch, tok_off_host), offsetof(rkv_batch, K),
              offsetof(rkv_batch, V), offsetof(rkv_batch, Q));
@@ -74,7 +74,7 @@ def test_struct_layout_matches_header():
     want2 = [int(x) for x in lines[1].split()]
     C, Bt = B.RkvConfig, B.RkvBatch
     assert want1 == [ctypes.sizeof(C), C.max_tokens.offset, C.redundancy.offset,
-                     C.flags.offset, ctypes.sizeof(Bt)]
+                     C.flags.offset, C.max_unit_tokens.offset, ctypes.sizeof(Bt)]
     assert want2 == [Bt.tok_off.offset, Bt.tok_off_host.offset, Bt.K.offset, Bt.V.offset,
                      Bt.Q.offset]
     H = B.RkvHostBatch
@@ -108,7 +108,8 @@ def _create(**over):
     (dict(redundancy=7), B.RKV_ERR_INVALID_ARG),
     (dict(flags=8), B.RKV_ERR_INVALID_ARG),
     (dict(head_dim=64), B.RKV_ERR_UNSUPPORTED),
-    (dict(group=8, window=8), B.RKV_ERR_UNSUPPORTED),
+    (dict(group=16, window=17), B.RKV_ERR_UNSUPPORTED),   # G * w = 272 > 256
+    (dict(max_unit_tokens=-1), B.RKV_ERR_INVALID_ARG),
     (dict(max_tokens=1 << 31), B.RKV_ERR_UNSUPPORTED),
 ])
 def test_create_rejects_bad_config(over, code):
@@ -129,6 +130,15 @@ def test_null_arguments():
                                None) == B.RKV_ERR_INVALID_ARG
     assert L.rkv_destroy(None) == B.RKV_OK
     assert L.rkv_launch_count(None) == 0
+
+
+def test_fault_injection_arguments():
+    L = rkv.lib()
+    assert L.rkv_inject_fault(None, 7) == B.RKV_ERR_INVALID_ARG
+    # dropping an announcement needs an engine (it concerns a score launch)
+    assert L.rkv_inject_fault(None, B.RKV_FAULT_DROP_ANNOUNCE) == B.RKV_ERR_INVALID_ARG
+    assert L.rkv_inject_fault(None, B.RKV_FAULT_ALLOC) == B.RKV_OK
+    assert L.rkv_inject_fault(None, B.RKV_FAULT_NONE) == B.RKV_OK
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")

@@ -108,9 +108,9 @@ def test_host_pipeline_rejections():
     assert_same(ref, run_host(eng, b2, 64, 0))
 
 
-def test_many_units_chunks_keep_the_batch_cluster_size():
-    # 200 units: the whole batch scores with the smallest TMEM-fitting cluster,
-    # while a 2-unit chunk alone would spread its units over more CTAs
+def test_many_units_chunks_keep_the_batch_chunk_size():
+    # 200 units: the whole batch scores in chunks of 8 tiles per CTA step,
+    # while a 2-unit host chunk alone would use 1-tile chunks to fill the GPU
     lengths = [3000 + 13 * (i % 7) for i in range(200)]
     b = rand_batch(lengths, G, WIN, seed=47)
     ref = device_reference(b, 256, "closed")

@@ -108,7 +108,10 @@ def test_worked_example_on_gpu():
 
 # ----------------------------------------------------------------- score kernels, small
 @pytest.mark.parametrize("mode", ["closed", "gemm", "max", "gemm_sym"])
-@pytest.mark.parametrize("G,w", [(1, 8), (4, 8), (2, 3), (5, 5), (1, 1), (32, 1)])
+@pytest.mark.parametrize("G,w", [(1, 8), (4, 8), (2, 3), (5, 5), (1, 1), (32, 1),
+                                 # more than 32 query rows: one pass of 64 rows, or
+                                 # several passes over row groups of 64
+                                 (8, 8), (9, 7), (16, 5), (32, 8)])
 def test_score_small_ragged(mode, G, w):
     lengths = [w, w + 1, 127, 128, 129, 1000, 2500, 5000]
     zero_rows = [3 + lengths[0] + lengths[1]]   # a zero key inside unit 2
@@ -199,14 +202,15 @@ def test_symmetric_flag_rejections():
     assert ei.value.code == -2
 
 
-@pytest.mark.parametrize("G,N", [(4, 32768), (2, 49152)])
-def test_largest_supported_unit(G, N):
-    # logits of a unit stay in tensor memory: 32768 tokens at G*w = 32,
-    # 49152 (the select limit) at G*w <= 16
-    b = rand_batch([N], G, 8, seed=1, dup=0.0)
+@pytest.mark.parametrize("G,w,N", [(4, 8, 32768), (2, 8, 49152), (4, 8, 40000), (8, 8, 40000)])
+def test_long_units(G, w, N):
+    """Units longer than 32K tokens and up to 64 query rows; every tile of a
+    unit's chunks streams through one pass (chunk exchanges in global memory)."""
+    b = rand_batch([N], G, w, seed=1, dup=0.0)
     for mode in ("closed", "gemm", "max", "gemm_sym"):
-        out = run_engine(b, G, 8, 0.1, 4096, mode=mode)
-        check_unit(out, b, 0, 8, 0.1, 4096, redundancy=oracle_mode(mode))
+        out = run_engine(b, G, w, 0.1, 4096, mode=mode)
+        check_unit(out, b, 0, w, 0.1, 4096, redundancy=oracle_mode(mode))
+        del out
 
 
 def test_rejects_too_long_unit_and_capacity():
@@ -216,8 +220,10 @@ def test_rejects_too_long_unit_and_capacity():
     with pytest.raises(RkvError) as ei:
         eng.score(b, a, r)
     assert ei.value.code == -2
-    b4 = rand_batch([32769], 4, 8, seed=0, dup=0.0)
-    eng4 = Engine(4, 8, max_units=1, max_tokens=b4.num_tokens, redundancy="gemm")
+    # a unit longer than the engine's declared max_unit_tokens
+    b4 = rand_batch([5000], 4, 8, seed=0, dup=0.0)
+    eng4 = Engine(4, 8, max_units=1, max_tokens=b4.num_tokens, redundancy="gemm",
+                  symmetric_gemm=True, max_unit_tokens=4096)
     with pytest.raises(RkvError) as ei:
         eng4.score(b4, *eng4.alloc_scores(b4))
     assert ei.value.code == -2
