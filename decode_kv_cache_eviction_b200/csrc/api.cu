@@ -176,7 +176,7 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   // Score kernel: deepest K-tile ring that fits, one persistent CTA per SM.
   const bool closed = cfg->redundancy == RKV_REDUNDANCY_CLOSED_FORM;
   const int R = cfg->group * cfg->window;
-  e->rp = R <= 16 ? 16 : (R <= 32 ? 32 : 64);
+  e->rp = R <= 16 ? 16 : 32;
   e->nstages = score_stages(e->rp, closed, kSmemCap);
   e->score_smem = score_layout(e->rp, closed, e->nstages).total + 1024;
   if (e->nstages == 0 || score_configure(e->rp, closed, e->score_smem) != cudaSuccess) {
@@ -218,6 +218,8 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
   auto alloc = [&](void** p, size_t bytes) { return dev_alloc(fault, p, bytes) == cudaSuccess; };
   bool ok = alloc(reinterpret_cast<void**>(&e->status), 16);
   ok = ok && alloc(reinterpret_cast<void**>(&e->chunk_off), sizeof(int) * (cfg->max_units + 1));
+  ok = ok && alloc(reinterpret_cast<void**>(&e->chunk_unit),
+                   sizeof(int) * static_cast<size_t>(e->max_chunks));
   ok = ok && alloc(reinterpret_cast<void**>(&e->score_cnt),
                    sizeof(int) * (static_cast<size_t>(cfg->max_units) * kScoreCnt + 1));
   ok = ok && alloc(reinterpret_cast<void**>(&e->xstat),
@@ -245,6 +247,7 @@ int rkv_create(const rkv_config* cfg, rkv_engine** out) {
     cudaGetLastError();
     cudaFree(e->status);
     cudaFree(e->chunk_off);
+    cudaFree(e->chunk_unit);
     cudaFree(e->score_cnt);
     cudaFree(e->xstat);
     cudaFree(e->xsum);
@@ -303,6 +306,7 @@ int rkv_destroy(rkv_engine* e) {
   cudaFree(e->rf_z);
   cudaFree(e->status);
   cudaFree(e->chunk_off);
+  cudaFree(e->chunk_unit);
   cudaFree(e->score_cnt);
   cudaFree(e->xstat);
   cudaFree(e->xsum);
@@ -369,6 +373,7 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   pp.w = e->cfg.window;
   pp.tpc = d.tpc;
   pp.chunk_off = e->chunk_off;
+  pp.chunk_unit = e->chunk_unit;
   pp.score_cnt = e->score_cnt;
   pp.score_abort = e->score_cnt + static_cast<int64_t>(e->cfg.max_units) * kScoreCnt;
   if (!closed) {   // GEMM row blocks and the padded rho layout the score kernel writes
@@ -387,6 +392,7 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   ScoreParams p = {};
   p.tok_off = b->tok_off;
   p.chunk_off = e->chunk_off;
+  p.chunk_unit = e->chunk_unit;
   p.num_units = U;
   p.total_chunks = static_cast<int>(d.chunks);
   p.R = R;
@@ -413,7 +419,7 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   p.status = e->status;
   for (int gq = 0; gq < d.ngroups; ++gq) {
     p.group = gq;
-    p.row0 = 64 * gq;
+    p.row0 = 32 * gq;
     p.Rg = std::min(d.rp, R - p.row0);
     p.final_pass = gq == d.ngroups - 1;
     t_begin(e, RKV_KERNEL_SCORE, st);

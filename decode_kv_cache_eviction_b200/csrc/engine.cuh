@@ -39,6 +39,7 @@ struct rkv_engine {
   int* unit_cnt = nullptr;     // [max_units]
   int* status = nullptr;       // [1]
   int* chunk_off = nullptr;    // [max_units + 1] score chunks prefix
+  int* chunk_unit = nullptr;   // [max_chunks] unit of each score chunk
   int* score_cnt = nullptr;    // [max_units * kScoreCnt] score exchange counters
   float* xstat = nullptr;      // [max_chunks * score_xs] score chunk statistics
   float* xsum = nullptr;       // [max_chunks * 2 * kScoreMaxGroups] score chunk sums

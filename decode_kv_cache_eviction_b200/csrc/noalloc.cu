@@ -44,6 +44,7 @@ struct Scratch {
   int item_off[kMaxUnits + 1];
   int unit_cnt[kMaxUnits];
   int chunk_off[kMaxUnits + 1];
+  int chunk_unit[kMaxChunks];
   int score_cnt[kMaxUnits * kScoreCnt];
   int score_abort[4];
   int status[4];
@@ -193,6 +194,7 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   pp.w = window;
   pp.tpc = dims.tpc;
   pp.chunk_off = s->chunk_off;
+  pp.chunk_unit = s->chunk_unit;
   pp.score_cnt = s->score_cnt;
   pp.score_abort = s->score_abort;
   pp.rows_per_item = kRows;
@@ -205,6 +207,7 @@ extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, floa
   ScoreParams p = {};
   p.tok_off = b->tok_off;
   p.chunk_off = s->chunk_off;
+  p.chunk_unit = s->chunk_unit;
   p.num_units = U;
   p.total_chunks = static_cast<int>(dims.chunks);
   p.R = R;

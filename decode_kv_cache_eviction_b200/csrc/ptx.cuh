@@ -367,6 +367,21 @@ __device__ __forceinline__ void tmem_ld16x256b_x8(uint32_t taddr, uint32_t (&v)[
       : RKV_R8(0), RKV_R8(8), RKV_R8(16), RKV_R8(24)
       : "r"(taddr));
 }
+// The same access over 4 groups of 8 columns (32 columns): 16 registers,
+// v[4i .. 4i+3] for columns 8i .. 8i+7 as above.
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
+      : RKV_R8(0), RKV_R8(8)
+      : "r"(taddr));
+}
+// Over 2 groups of 8 columns (16 columns): 8 registers.
+__device__ __forceinline__ void tmem_ld16x256b_x2(uint32_t taddr, uint32_t (&v)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : RKV_R8(0)
+               : "r"(taddr));
+}
 #undef RKV_R8
 
 // ---------------------------------------------------------------- misc

@@ -711,7 +711,9 @@ __global__ void plan_kernel(const PlanParams pp) {
   for (int u = u0; u < u1; ++u) {
     const int64_t n = pp.tok_off[u + 1] - pp.tok_off[u];
     pp.chunk_off[u] = static_cast<int>(rc);
-    rc += (n + chunk_tok - 1) / chunk_tok;
+    const long long nc = (n + chunk_tok - 1) / chunk_tok;
+    for (long long q = 0; q < nc; ++q) pp.chunk_unit[rc + q] = u;
+    rc += nc;
     if (gemm) {
       pp.item_off[u] = static_cast<int>(ri);
       pp.rho_off[u] = rr;

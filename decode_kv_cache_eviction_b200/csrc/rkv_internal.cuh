@@ -10,19 +10,22 @@ namespace rkv {
 constexpr int kHeadDim = 128;        // d (the only supported head size)
 constexpr int kTile = 128;           // tokens per K tile (TMA box rows, MMA M)
 constexpr int kTileBytes = kTile * kHeadDim * 2;
-constexpr int kMaxTokensPerUnit = 49152;  // select keeps a unit's keys in shared memory
-constexpr int kMaxRows = 256;        // G * w limit (row groups of 64 per launch)
+// Longest unit: the in-place eviction keeps a byte per token of a unit and the
+// selection a bit per candidate on chip.
+constexpr int kMaxTokensPerUnit = 131072;
+constexpr int kMaxRows = 256;        // G * w limit (row groups of 32 per launch)
 constexpr int kScoreThreads = 512;   // 16 warps
 constexpr int kGemmThreads = 640;    // producer, MMA, 2 idle, 16 epilogue warps
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------- score
-constexpr int kScoreMaxGroups = 4;              // row groups of 64: G * w <= 256
+constexpr int kScoreMaxGroups = 8;              // row groups of 32: G * w <= 256
 constexpr int kScoreCnt = 2 * kScoreMaxGroups;  // exchange counters per unit
 
 struct ScoreParams {
   const int64_t* tok_off;  // [U+1]
   const int* chunk_off;    // [U+1] prefix of chunks per unit
+  const int* chunk_unit;   // [chunks] unit of each chunk
   int num_units;
   int total_chunks;
   int R;                   // G * w query rows of a unit
@@ -58,8 +61,8 @@ __host__ __device__ constexpr int score_xs(int rp, bool closed) {
 }
 
 struct ScoreLayout {
-  uint32_t stages, q, abuf, marr, red1, red2, rhot, ufin, mpart, upart, mrow, invl, rsum, rowt,
-      bars, slot, flags, issued, total;
+  uint32_t stages, q, abuf, marr, rhoc, red1, red2, rhot, ufin, mpart, mrow, invl, rsum, esum,
+      rowt, bars, slot, flags, issued, total;
 };
 
 __host__ __device__ inline ScoreLayout score_layout(int rp, bool closed, int ns) {
@@ -68,18 +71,19 @@ __host__ __device__ inline ScoreLayout score_layout(int rp, bool closed, int ns)
   const int cht = score_chunk_tokens(rp);
   L.stages = o; o += ns * kTileBytes;
   L.q = o; o += 2 * rp * 256;
-  L.abuf = o; o += 2 * 2 * cht * 4;
+  L.abuf = o; o += 2 * cht * 4;
   L.marr = o; if (closed) o += 2 * cht * 4;
+  L.rhoc = o; if (closed) o += 2 * cht * 4;
   L.red1 = o; o += 4 * rp * 2 * 4;
   L.red2 = o; if (closed) o += 4 * 128 * 4;
   L.rhot = o; if (closed) o += 2 * 128 * 4;
   L.ufin = o; if (closed) o += 128 * 4;
-  L.mpart = o; o += 384 * 2 * 4;
-  L.upart = o; if (closed) o += 3 * 128 * 4;
+  L.mpart = o; o += 128 * 2 * 4;
   L.mrow = o; o += rp * 4;
   L.invl = o; o += rp * 4;
-  L.rsum = o; o += 32 * 4;
-  L.rowt = o; o += 64 * 4;
+  L.rsum = o; o += 16 * 4;
+  L.esum = o; o += 16 * 4;
+  L.rowt = o; o += 32 * 4;
   o = (o + 15u) & ~15u;
   L.bars = o; o += (2 * ns + 32 + 6 + 1) * 8;
   L.slot = o; o += 16;
@@ -98,8 +102,8 @@ __host__ __device__ inline int score_stages(int rp, bool closed, int smem_cap) {
 
 // Launch shape of the score kernel for one batch.
 struct ScoreDims {
-  int rp;          // padded query rows per launch (16, 32, 64)
-  int ngroups;     // launches (row groups of 64)
+  int rp;          // padded query rows per launch (16, 32)
+  int ngroups;     // launches (row groups of 32)
   int tpc;         // tiles per chunk
   int64_t chunks;  // chunks of the batch
   int grid;        // CTAs (<= max_ctas)
@@ -187,6 +191,7 @@ struct PlanParams {
   int w;
   int tpc;                 // score: tiles per chunk
   int* chunk_off;          // [U+1] score chunks prefix
+  int* chunk_unit;         // [chunks] unit of each chunk
   int* score_cnt;          // [U][kScoreCnt] zeroed
   int* score_abort;        // [1] zeroed
   int rows_per_item;       // GEMM: rows per work item (0: no GEMM)

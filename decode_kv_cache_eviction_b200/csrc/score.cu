@@ -33,15 +33,22 @@
 // call's abort word, raises its own abort flag and stops working; CTAs waiting
 // on other CTAs see the abort word and give up too.
 //
-// Query rows: RP = 16, 32 or 64 padded rows per launch (G*w real rows).  More
-// than 64 rows run as several launches over row groups of 64; each adds its
-// rows' probabilities to a, and the last one normalises and computes the
-// redundancy part.
+// Query rows: RP = 16 or 32 padded rows per launch (G*w real rows).  More than
+// 32 rows run as several launches over row groups of 32; each adds its rows'
+// probabilities to a, and the last one normalises and computes the redundancy
+// part.
 //
-// Warp roles (512 threads): warp 0 TMA producer, warp 1 MMA issuer and tensor
-// memory owner, warps 4-11 softmax (thread = token row of a tile; tensor-memory
-// lane quarter = warp % 4; warps 4-7 the first half of the query rows, 8-11 the
-// second), warps 12-15 norms and U (thread = token row).
+// Warp roles (512 threads; thread = token row of a tile, tensor-memory lane
+// quarter = warp % 4), each group running on its own so that the K stream
+// never waits for an exchange:
+//   warp 0      TMA producer;
+//   warp 1      MMA issuer and tensor-memory owner;
+//   warps 4-7   pass 1: online statistics of every query row, announced per
+//               chunk (no waits on other CTAs);
+//   warps 8-11  W, merge and pass 2 of x_k-1, then a of x_k-2;
+//   warps 12-15 norms: rho (GEMM form) or rho and U, then m and r (closed form).
+// Only a tensor-memory buffer couples passes 1 and 2: pass 1 of x_k+1 reuses
+// the buffer that pass 2 of x_k-1 releases.
 #include "ptx.cuh"
 #include "rkv_internal.cuh"
 
@@ -57,15 +64,33 @@ constexpr uint64_t kDrainNs = 200000000ull;   // teardown wait for copies in fli
 #ifdef RKV_TRACE
 // Optional phase trace (build with -DRKV_TRACE): globaltimer stamps of the
 // consumer threads' step phases, for the first kTrSteps steps of each CTA.
-constexpr int kTrCtas = 160, kTrSteps = 32, kTrSlots = 10;
+constexpr int kTrCtas = 160, kTrSteps = 32, kTrSlots = 16;
 __device__ unsigned long long g_score_trace[kTrCtas * kTrSteps * kTrSlots];
 #define RKV_STAMP(k, slot)                                                               \
   do {                                                                                   \
     if (ctid == 0 && (k) < kTrSteps && blockIdx.x < kTrCtas)                             \
       g_score_trace[(blockIdx.x * kTrSteps + (k)) * kTrSlots + (slot)] = globaltimer_ns(); \
   } while (0)
+constexpr int kTtCtas = 4, kTtSteps = 16;
+__device__ unsigned long long g_tile_trace[kTtCtas * kTtSteps * 16 * 4];
+#define RKV_TSTAMP(k, t, slot)                                                              \
+  do {                                                                                      \
+    if (ctid == 0 && (k) < kTtSteps && blockIdx.x < kTtCtas && (t) < 16)                    \
+      g_tile_trace[((blockIdx.x * kTtSteps + (k)) * 16 + (t)) * 4 + (slot)] = globaltimer_ns(); \
+  } while (0)
+#define RKV_CLK_BEGIN(var) const long long var = clock64()
+#define RKV_CLK_ADD(acc, var) acc += clock64() - var
+#define RKV_STORE(k, slot, val)                                                          \
+  do {                                                                                   \
+    if (ctid == 0 && (k) < kTrSteps && blockIdx.x < kTrCtas)                             \
+      g_score_trace[(blockIdx.x * kTrSteps + (k)) * kTrSlots + (slot)] = (val);          \
+  } while (0)
 #else
 #define RKV_STAMP(k, slot) do { } while (0)
+#define RKV_TSTAMP(k, t, slot) do { } while (0)
+#define RKV_CLK_BEGIN(var) do { } while (0)
+#define RKV_CLK_ADD(acc, var) do { } while (0)
+#define RKV_STORE(k, slot, val) do { } while (0)
 #endif
 
 struct Chunk {
@@ -82,17 +107,12 @@ struct Chunk {
 __device__ __forceinline__ Chunk chunk_info(const ScoreParams& p, int g) {
   Chunk h;
   h.g = g;
-  int lo = 0, hi = p.num_units - 1;   // largest u with chunk_off[u] <= g
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(&p.chunk_off[mid]) <= g) lo = mid;
-    else hi = mid - 1;
-  }
-  h.u = lo;
-  h.g0 = __ldg(&p.chunk_off[lo]);
-  h.nch = __ldg(&p.chunk_off[lo + 1]) - h.g0;
-  h.base = __ldg(&p.tok_off[lo]);
-  h.n = static_cast<int>(__ldg(&p.tok_off[lo + 1]) - h.base);
+  const int u = __ldg(&p.chunk_unit[g]);
+  h.u = u;
+  h.g0 = __ldg(&p.chunk_off[u]);
+  h.nch = __ldg(&p.chunk_off[u + 1]) - h.g0;
+  h.base = __ldg(&p.tok_off[u]);
+  h.n = static_cast<int>(__ldg(&p.tok_off[u + 1]) - h.base);
   h.c = h.n - p.w;
   h.start = (g - h.g0) * p.tpc * kTile;
   h.len = min(p.tpc * kTile, h.n - h.start);
@@ -187,10 +207,46 @@ __device__ __forceinline__ void lane_merge(float (&m)[RH], float (&s)[RH], int l
   }
 }
 
-template <int RB>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* v) {
-  if constexpr (RB == 8) tmem_ld8(taddr, *reinterpret_cast<uint32_t(*)[8]>(v));
-  else tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(v));
+// Logits of one tile as the 16x256b shape reads them: for lanes 16h .. 16h+15
+// of the warp's quarter, thread t gets v[4i + e] = (token t/4, row 8i + 2(t%4) + e)
+// and v[4i + 2 + e] = (token t/4 + 8, the same row), i < RP / 8, e < 2.
+template <int RP>
+__device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, uint32_t (&v)[RP / 2]) {
+  if constexpr (RP == 16) tmem_ld16x256b_x2(taddr, v);
+  else tmem_ld16x256b_x4(taddr, v);
+}
+
+// Merge per-lane statistics of the NR query rows a lane holds over the 8 lanes
+// that hold the same rows (lane bits 2, 3, 4) with a transposed butterfly.
+// Afterwards slot s (returned) of the lane's rows is merged over all lanes in
+// m[0], s[0]; for NR = 4 two lanes (bit 2) end with the same row.
+template <int NR>
+__device__ __forceinline__ int quad_rows_merge(float (&m)[NR], float (&sx)[NR], int lane) {
+  int slot = 0, half = NR / 2, bit = 16;
+#pragma unroll
+  for (int lv = 0; (NR >> lv) > 1; ++lv, half >>= 1, bit >>= 1) {
+    const bool up = (lane & bit) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float sm_ = up ? m[i] : m[i + half];
+      const float ss_ = up ? sx[i] : sx[i + half];
+      const float km = up ? m[i + half] : m[i];
+      const float ks = up ? sx[i + half] : sx[i];
+      const float om = __shfl_xor_sync(0xffffffffu, sm_, bit);
+      const float os = __shfl_xor_sync(0xffffffffu, ss_, bit);
+      m[i] = km;
+      sx[i] = ks;
+      merge_stat(m[i], sx[i], om, os);
+    }
+    if (up) slot += half;
+  }
+#pragma unroll
+  for (; bit >= 4; bit >>= 1) {   // lane bits not used by the halving above
+    const float om = __shfl_xor_sync(0xffffffffu, m[0], bit);
+    const float os = __shfl_xor_sync(0xffffffffu, sx[0], bit);
+    merge_stat(m[0], sx[0], om, os);
+  }
+  return slot;
 }
 
 // Load the 16 swizzled 16-byte chunks of K-tile row `row` (128 bf16).
@@ -230,10 +286,9 @@ template <int RP, bool CLOSED>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                  const ScoreParams p) {
-  constexpr int RH = RP / 2;                // query rows per softmax warp
-  constexpr int RB = RH < 16 ? RH : 16;     // columns per tensor-memory load
   constexpr int XS = score_xs(RP, CLOSED);  // floats of a chunk's exchange slot
   constexpr int CHT = score_chunk_tokens(RP);
+  constexpr int TPR = 128 / RP;             // pass-2 threads per query row in the merge
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -244,18 +299,20 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const int b0 = static_cast<int>(blockIdx.x);
   // the redundancy side (norms, U, m) runs in the last row-group launch only
   const bool red = p.final_pass != 0;
+  // announcements per chunk on each counter: the statistics (and, closed form,
+  // the norm warps' U), then the sum of abar (and of exp(m))
+  const int nann = (CLOSED && red) ? 2 : 1;
 
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* empty = full + NS;
   uint64_t* tready = empty + NS;   // [2][16] logits of tile t of buffer b are in TMEM
-  uint64_t* tfree = tready + 32;   // [2] softmax warps are done with buffer b
+  uint64_t* tfree = tready + 32;   // [2] pass-2 warps are done with buffer b
   uint64_t* qfull = tfree + 2;     // [2]
   uint64_t* qempty = qfull + 2;    // [2]
   uint64_t* mdone = qempty + 2;    // teardown: every MMA has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.slot);
   volatile int* abort = reinterpret_cast<volatile int*>(sm + L.flags);
   int8_t* lastp = reinterpret_cast<int8_t*>(sm + L.issued);   // [NS + 2] parity of the last copy
-  float* rsum = reinterpret_cast<float*>(sm + L.rsum);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -264,7 +321,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
     for (int k = 0; k < 32; ++k) mbar_init(&tready[k], 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfree[b], 8);
+      mbar_init(&tfree[b], 4);
       mbar_init(&qfull[b], 1);
       mbar_init(&qempty[b], 1);
     }
@@ -273,6 +330,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     *abort = 0;
     fence_mbar_init();
   }
+  if (threadIdx.x < RP)   // window step t of query row r = g * w + t of the group
+    reinterpret_cast<int*>(sm + L.rowt)[threadIdx.x] = (p.row0 + threadIdx.x) % p.w;
   if (warp == 1) {
     tmem_alloc<1>(tmem_slot, kTmemColsTotal);
     tmem_relinquish<1>();
@@ -281,6 +340,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // bit r set for real query rows of this launch's group; window step of a row
+  const uint32_t rmask = p.Rg >= 32 ? 0xffffffffu : ((1u << p.Rg) - 1u);
+  int* row_t = reinterpret_cast<int*>(sm + L.rowt);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -386,41 +448,362 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       drain_wait(mdone, 0);
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ consumers
-    const int ctid = threadIdx.x - 128;      // 0..383
-    const bool is_soft = warp < 12;          // warps 4-11: softmax
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------- statistics warps (pass 1)
+    // thread = 4 tokens x NR query rows of a tile (16x256b loads); no global waits
+    constexpr int NR = RP / 4;               // query rows a thread holds
+    const int ctid = threadIdx.x - 128;      // 0..127
     const int q4 = warp & 3;                 // tensor-memory lane quarter
-    const int row = q4 * 32 + lane;          // token row of the tile
-    const int hh = (warp - 4) >> 2;          // softmax: half of the query rows
-    const int r0 = hh * RH;                  // first query row of a softmax warp
-    float* abuf = reinterpret_cast<float*>(sm + L.abuf);   // [2 slots][2 halves][CHT]
-    float* marr = reinterpret_cast<float*>(sm + L.marr);   // [2 slots][CHT]
+    const int qd = lane >> 2, tq = lane & 3;
     float* red1 = reinterpret_cast<float*>(sm + L.red1);   // [4 quarters][RP][2]
+    uint32_t tph = 0;   // phase bits of tready[32]
+    const bool all_real = p.Rg >= RP;
+    int g = b0;
+    Chunk cur = g < p.total_chunks ? chunk_info(p, g) : no_chunk();
+    for (int k = 0; cur.g >= 0; ++k) {
+      const int buf = k & 1;
+      RKV_STAMP(k, 0);
+      float st_m[NR], st_s[NR];
+#pragma unroll
+      for (int q = 0; q < NR; ++q) { st_m[q] = kNegBig; st_s[q] = 0.f; }
+#ifdef RKV_TRACE
+      long long c_ready = 0, c_tw = 0;
+      const long long c_loop0 = clock64();
+#endif
+      for (int t = 0; t < cur.nt; ++t) {
+        const int bi = buf * 16 + t;
+        RKV_TSTAMP(k, t, 0);
+        RKV_CLK_BEGIN(cr0);
+        mbar_wait(&tready[bi], (tph >> bi) & 1u, abort, p.status);
+        RKV_CLK_ADD(c_ready, cr0);
+        RKV_TSTAMP(k, t, 1);
+        tph ^= 1u << bi;
+        __syncwarp();
+        tc_fence_after();
+        const int t0 = cur.start + kTile * t;
+        const bool inside = t0 + kTile <= cur.c;   // no causal limit or end in this tile
+        uint32_t v[2][RP / 2];
+        RKV_CLK_BEGIN(cw0);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          tmem_ld_tile<RP>(tmem + (static_cast<uint32_t>(q4 * 32 + 16 * h) << 16) +
+                               buf * kBufCols + t * RP, v[h]);
+        tmem_wait_ld();
+        RKV_CLK_ADD(c_tw, cw0);
+        RKV_TSTAMP(k, t, 2);
+        // y = log2-scaled logits (in place of the raw ones), -inf where masked
+        // (padding row, beyond N, causal); the thread's tokens are
+        // qd, qd + 8 (h = 0) and 16 + qd, 24 + qd (h = 1) of the quarter.  A
+        // tile inside the candidates with every query row real needs no mask.
+        if (inside && all_real) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int x = 0; x < RP / 2; ++x)
+              v[h][x] = __float_as_uint(__uint_as_float(v[h][x]) * p.scale_log2);
+        } else {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int ja = t0 + q4 * 32 + 16 * h + qd, jb = ja + 8;
+#pragma unroll
+            for (int i = 0; i < RP / 8; ++i)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int r = 8 * i + 2 * tq + e;
+                const bool real = ((rmask >> r) & 1u) != 0;
+                const bool va = real && (inside || (ja < cur.n && ja <= cur.c + row_t[r]));
+                const bool vb = real && (inside || (jb < cur.n && jb <= cur.c + row_t[r]));
+                v[h][4 * i + e] = __float_as_uint(
+                    va ? __uint_as_float(v[h][4 * i + e]) * p.scale_log2 : -INFINITY);
+                v[h][4 * i + 2 + e] = __float_as_uint(
+                    vb ? __uint_as_float(v[h][4 * i + 2 + e]) * p.scale_log2 : -INFINITY);
+              }
+          }
+        }
+        // online statistics, one update per row and tile (no branches): the
+        // running max takes the tile's max over the thread's four tokens
+#pragma unroll
+        for (int i = 0; i < RP / 8; ++i)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int q = 2 * i + e;
+            const float y0 = __uint_as_float(v[0][4 * i + e]);
+            const float y1 = __uint_as_float(v[0][4 * i + 2 + e]);
+            const float y2 = __uint_as_float(v[1][4 * i + e]);
+            const float y3 = __uint_as_float(v[1][4 * i + 2 + e]);
+            const float mn = fmaxf(st_m[q], fmaxf(fmaxf(y0, y1), fmaxf(y2, y3)));
+            st_s[q] = fmaf(st_s[q], ex2(st_m[q] - mn),
+                           (ex2(y0 - mn) + ex2(y1 - mn)) + (ex2(y2 - mn) + ex2(y3 - mn)));
+            st_m[q] = mn;
+          }
+        RKV_TSTAMP(k, t, 3);
+      }
+#ifdef RKV_TRACE
+      RKV_STORE(k, 7, c_ready);
+      RKV_STORE(k, 8, c_tw);
+      RKV_STORE(k, 15, clock64() - c_loop0);
+#endif
+      // the next chunk's bookkeeping loads overlap the merge below
+      const int gn = g + P;
+      const Chunk nxt = gn < p.total_chunks ? chunk_info(p, gn) : no_chunk();
+      RKV_STAMP(k, 11);
+      const int slot = quad_rows_merge<NR>(st_m, st_s, lane);
+      {
+        const int r = 8 * (slot >> 1) + 2 * tq + (slot & 1);
+        if (NR == 8 || (lane & 4) == 0) {
+          red1[(q4 * RP + r) * 2 + 0] = st_m[0];
+          red1[(q4 * RP + r) * 2 + 1] = st_s[0];
+        }
+      }
+      named_bar_sync(1, 128);
+      float* xs_out = p.xstat + static_cast<int64_t>(cur.g) * XS;
+      if (ctid < RP) {
+        float m = kNegBig, sx = 0.f;
+        for (int q = 0; q < 4; ++q)
+          merge_stat(m, sx, red1[(q * RP + ctid) * 2], red1[(q * RP + ctid) * 2 + 1]);
+        xs_out[2 * ctid] = m;
+        xs_out[2 * ctid + 1] = sx;
+      }
+      named_bar_sync(1, 128);
+      if (ctid == 0 && cur.g != p.drop_chunk) {
+        __threadfence();
+        atomicAdd(&p.cnt[cur.u * kScoreCnt + 2 * p.group], 1);
+      }
+      RKV_STAMP(k, 1);
+      g = gn;
+      cur = nxt;
+    }
+  } else if (warp >= 8 && warp < 12) {
+    // ---------------------------------------------- pass-2 warps
+    // step k: merge the statistics of x_k-1 and turn its logits into abar,
+    // then normalise and write a for x_k-2
+    const int ctid = threadIdx.x - 256;      // 0..127
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    float* abuf = reinterpret_cast<float*>(sm + L.abuf);   // [2 slots][CHT]
+    float* mpart = reinterpret_cast<float*>(sm + L.mpart); // [128][2]
+    float* mrow = reinterpret_cast<float*>(sm + L.mrow);   // [RP]
+    float* invl = reinterpret_cast<float*>(sm + L.invl);   // [RP]
+    float* psum = reinterpret_cast<float*>(sm + L.rsum);   // [4] + inverse sum at [8]
+    Chunk c1 = no_chunk(), c2 = no_chunk();
+    for (int k = 0;; ++k) {
+      const int g = b0 + k * P;
+      const bool have = g < p.total_chunks;
+      if (!have && c1.g < 0 && c2.g < 0) break;
+      // ---- W(x_k-1), pass 2, its sum
+      if (c1.g >= 0) {
+        const int buf = (k - 1) & 1;   // tensor-memory buffer and smem slot of x_k-1
+        if (ctid == 0)
+          wait_count(&p.cnt[c1.u * kScoreCnt + 2 * p.group], nann * c1.nch, abort, p.status,
+                     p.abort_all, p.wait_ns);
+        RKV_STAMP(k, 2);
+        named_bar_sync(2, 128);
+        {
+          // every thread folds a fixed subset of the unit's chunks for one row
+          // (the loads overlap), then the subsets are merged in order: every
+          // CTA of the unit gets identical values
+          const int rr = ctid / TPR, tt = ctid - rr * TPR;
+          const float* xs_in = p.xstat + static_cast<int64_t>(c1.g0) * XS;
+          float M = kNegBig, S = 0.f;
+#pragma unroll 4
+          for (int q = tt; q < c1.nch; q += TPR)
+            merge_stat(M, S, __ldcg(xs_in + q * XS + 2 * rr), __ldcg(xs_in + q * XS + 2 * rr + 1));
+          mpart[2 * ctid] = M;
+          mpart[2 * ctid + 1] = S;
+        }
+        named_bar_sync(2, 128);
+        if (ctid < RP) {
+          float M = kNegBig, S = 0.f;
+#pragma unroll
+          for (int tt = 0; tt < TPR; ++tt)
+            merge_stat(M, S, mpart[2 * (ctid * TPR + tt)], mpart[2 * (ctid * TPR + tt) + 1]);
+          mrow[ctid] = M;
+          invl[ctid] = S > 0.f ? 1.f / S : 0.f;
+        }
+        named_bar_sync(2, 128);
+        RKV_STAMP(k, 3);
+        // p = 2^(y - M) / L = 2^(y - (M + log2 L)) for the NR rows this thread
+        // holds; padding rows (and rows that see no key) get +inf there, so
+        // they add exactly 0
+        constexpr int NR = RP / 4;
+        const int qd = lane >> 2, tq = lane & 3;
+        float ML[NR];
+#pragma unroll
+        for (int i = 0; i < RP / 8; ++i)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int r = 8 * i + 2 * tq + e;
+            const bool real = ((rmask >> r) & 1u) != 0 && invl[r] > 0.f;
+            ML[2 * i + e] = real ? mrow[r] - __log2f(invl[r]) : INFINITY;
+          }
+        float* ab = abuf + buf * CHT;
+        float part = 0.f;
+#ifdef RKV_TRACE
+        long long c_tw2 = 0;
+        const long long c_p2 = clock64();
+#endif
+        for (int t = 0; t < c1.nt; ++t) {
+          const int t0 = c1.start + kTile * t;
+          const bool inside = t0 + kTile <= c1.c;
+          float sum[4];   // tokens qd, qd + 8, 16 + qd, 24 + qd of the quarter
+          uint32_t v[2][RP / 2];
+          RKV_CLK_BEGIN(cw1);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tmem_ld_tile<RP>(tmem + (static_cast<uint32_t>(q4 * 32 + 16 * h) << 16) +
+                                 buf * kBufCols + t * RP, v[h]);
+          tmem_wait_ld();
+          RKV_CLK_ADD(c_tw2, cw1);
+          if (inside) {
+            // padding rows carry an infinite shift, so they add exactly 0
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float pa = 0.f, pb = 0.f;
+#pragma unroll
+              for (int i = 0; i < RP / 8; ++i)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  pa += ex2(fmaf(__uint_as_float(v[h][4 * i + e]), p.scale_log2, -ML[2 * i + e]));
+                  pb += ex2(fmaf(__uint_as_float(v[h][4 * i + 2 + e]), p.scale_log2,
+                                 -ML[2 * i + e]));
+                }
+              sum[2 * h] = pa;
+              sum[2 * h + 1] = pb;
+            }
+          } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int ja = t0 + q4 * 32 + 16 * h + qd, jb = ja + 8;
+              float pa = 0.f, pb = 0.f;
+#pragma unroll
+              for (int i = 0; i < RP / 8; ++i)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const int r = 8 * i + 2 * tq + e;
+                  const bool real = ((rmask >> r) & 1u) != 0;
+                  if (real && ja < c1.n && ja <= c1.c + row_t[r])
+                    pa += ex2(fmaf(__uint_as_float(v[h][4 * i + e]), p.scale_log2, -ML[2 * i + e]));
+                  if (real && jb < c1.n && jb <= c1.c + row_t[r])
+                    pb += ex2(fmaf(__uint_as_float(v[h][4 * i + 2 + e]), p.scale_log2,
+                                   -ML[2 * i + e]));
+                }
+              sum[2 * h] = pa;
+              sum[2 * h + 1] = pb;
+            }
+          }
+          // the four lanes of a quad hold the same tokens' other rows
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            sum[x] += __shfl_xor_sync(0xffffffffu, sum[x], 1);
+            sum[x] += __shfl_xor_sync(0xffffffffu, sum[x], 2);
+          }
+          // lane tq writes token (tq >> 1) * 16 + qd + (tq & 1) * 8 of the quarter
+          const float mine = tq == 0 ? sum[0] : (tq == 1 ? sum[1] : (tq == 2 ? sum[2] : sum[3]));
+          const int trow = q4 * 32 + (tq >> 1) * 16 + qd + (tq & 1) * 8;
+          const int j = t0 + trow;
+          if (j < c1.c) {
+            ab[kTile * t + trow] = mine;
+            part += mine;
+          }
+        }
+#ifdef RKV_TRACE
+        RKV_STORE(k, 9, c_tw2);
+        RKV_STORE(k, 10, clock64() - c_p2);
+#endif
+        // this buffer's logits have been read: the MMA may reuse it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tfree[buf]);
+        RKV_STAMP(k, 4);
+
+        part = warp_reduce_sum(part);
+        if (lane == 0) psum[q4] = part;
+        named_bar_sync(2, 128);
+        if (ctid == 0) {
+          float* xo = p.xsum + static_cast<int64_t>(c1.g) * (2 * kScoreMaxGroups) + 2 * p.group;
+          xo[0] = (psum[0] + psum[1]) + (psum[2] + psum[3]);
+          if (red) {
+            __threadfence();
+            atomicAdd(&p.cnt[c1.u * kScoreCnt + 2 * p.group + 1], 1);
+          }
+        }
+        if (!red) {
+          // an earlier row group: add this group's probabilities to a (not yet
+          // normalised); the last group normalises
+          for (int i = ctid; i < c1.len; i += 128) {
+            const int j = c1.start + i;
+            const int64_t gi = c1.base + j;
+            if (j < c1.c) p.a_out[gi] = p.group > 0 ? p.a_out[gi] + ab[i] : ab[i];
+          }
+        }
+      }
+      // ---- WS(x_k-2) and a of x_k-2
+      if (red && c2.g >= 0) {
+        const int buf = k & 1;   // slot of x_k-2
+        if (warp == 8) {
+          if (lane == 0)
+            wait_count(&p.cnt[c2.u * kScoreCnt + 2 * p.group + 1], nann * c2.nch, abort,
+                       p.status, p.abort_all, p.wait_ns);
+          __syncwarp();
+          // sum over the unit's chunks and row groups, fixed order
+          float sa = 0.f;
+          for (int q = lane; q < c2.nch; q += 32) {
+            const float* xi = p.xsum + static_cast<int64_t>(c2.g0 + q) * (2 * kScoreMaxGroups);
+            float x = 0.f;
+            for (int gq = 0; gq <= p.group; ++gq) x += __ldcg(xi + 2 * gq);
+            sa += x;
+          }
+          sa = warp_reduce_sum(sa);
+          if (lane == 0) psum[8] = sa > 0.f ? 1.f / sa : 0.f;
+        }
+        RKV_STAMP(k, 5);
+        named_bar_sync(2, 128);
+        const float inv_sa = psum[8];
+        const float* ab = abuf + buf * CHT;
+        for (int i = ctid; i < c2.len; i += 128) {
+          const int j = c2.start + i;
+          const int64_t gi = c2.base + j;
+          if (j < c2.c) {
+            float x = ab[i];
+            if (p.group > 0) x = p.a_out[gi] + x;
+            p.a_out[gi] = x * inv_sa;
+          } else {
+            p.a_out[gi] = 0.f;
+            if (!CLOSED) {   // the redundancy GEMM writes the candidates' r and m
+              p.r_out[gi] = 0.f;
+              if (p.m_out) p.m_out[gi] = 0.f;
+            }
+          }
+        }
+        named_bar_sync(2, 128);   // psum and the slot are reused
+        RKV_STAMP(k, 6);
+      }
+      c2 = red ? c1 : no_chunk();
+      c1 = have ? chunk_info(p, g) : no_chunk();
+    }
+  } else if (warp >= 12 && red) {
+    // ---------------------------------------------- norm warps
+    // pass 1: rho = 1/||k|| (GEMM form: stored for the redundancy GEMM; closed
+    // form: U = sum_j rho_j k_j, announced per chunk); closed form pass 2: m_j
+    // of x_k-1 from the K tiles read again and the unit's U, then r of x_k-2
+    const int ctid = threadIdx.x - 384;      // 0..127
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
     float* red2 = reinterpret_cast<float*>(sm + L.red2);   // [4 quarters][128]
     float* rhot = reinterpret_cast<float*>(sm + L.rhot);   // [2][128]
     float* ufin = reinterpret_cast<float*>(sm + L.ufin);   // [128]
-    float* mpart = reinterpret_cast<float*>(sm + L.mpart); // [384][2] merge partials
-    float* upart = reinterpret_cast<float*>(sm + L.upart); // [3][128] U merge partials
-    float* mrow = reinterpret_cast<float*>(sm + L.mrow);   // [RP]
-    float* invl = reinterpret_cast<float*>(sm + L.invl);   // [RP]
-    int* row_t = reinterpret_cast<int*>(sm + L.rowt);      // [RP] window step of a row
-    // bit r set for real query rows of this launch's group
-    const uint64_t rmask = p.Rg >= 64 ? ~0ull : ((1ull << p.Rg) - 1ull);
-    if (ctid < RP) row_t[ctid] = (p.row0 + ctid) % p.w;
-    named_bar_sync(1, kConsumers);
-
-    int stage = 0;      // norm warps: ring position
+    float* rhoc = reinterpret_cast<float*>(sm + L.rhoc);   // [2 slots][CHT] rho of a chunk
+    float* marr = reinterpret_cast<float*>(sm + L.marr);   // [2 slots][CHT]
+    float* esum = reinterpret_cast<float*>(sm + L.esum);   // [4] + inverse sum at [8]
+    int stage = 0;
     uint32_t ph = 0;
-    uint32_t tph = 0;   // softmax warps: phase bits of tready[32]
-    int ntile = 0;      // norm warps: tiles seen (rho broadcast buffer)
+    int ntile = 0;
     Chunk c1 = no_chunk(), c2 = no_chunk();
-
-    // closed form: U += rho_row * k_row over the warp's 32 rows of a tile
+    // U += rho_row * k_row over the warp's 32 rows of a tile
     auto u_accumulate = [&](uint32_t sb, float rho, float (&U4)[4]) {
       float* rt = rhot + (ntile & 1) * 128;
       rt[row] = rho;
-      named_bar_sync(2, 128);
+      named_bar_sync(3, 128);
       const int hd = lane >> 4;
       const uint32_t cidx = (lane & 15) >> 1;
       const uint32_t sub = (lane & 1) * 8;
@@ -441,222 +824,77 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) U4[i] += U8[i] + U8[4 + i];
     };
-
     for (int k = 0;; ++k) {
       const int g = b0 + k * P;
       const bool have = g < p.total_chunks;
       if (!have && c1.g < 0 && c2.g < 0) break;
       const Chunk cur = have ? chunk_info(p, g) : no_chunk();
-
-      RKV_STAMP(k, 0);
-      // ================================================= P1(x_k) and its announcement
+      // ---- pass 1 of x_k
       if (have) {
-        const int buf = k & 1;
-        if (is_soft) {
-          float st_m[RH], st_s[RH];
-#pragma unroll
-          for (int r = 0; r < RH; ++r) { st_m[r] = kNegBig; st_s[r] = 0.f; }
-          for (int t = 0; t < cur.nt; ++t) {
-            const int bi = buf * 16 + t;
-            mbar_wait(&tready[bi], (tph >> bi) & 1u, abort, p.status);
-            tph ^= 1u << bi;
-            __syncwarp();
-            tc_fence_after();
-            uint32_t v[RH];
-            const uint32_t ta =
-                tmem + (static_cast<uint32_t>(q4 * 32) << 16) + buf * kBufCols + t * RP + r0;
-#pragma unroll
-            for (int sb = 0; sb < RH; sb += RB) tmem_ld_cols<RB>(ta + sb, v + sb);
-            tmem_wait_ld();
-            const int t0 = cur.start + kTile * t;
-            const int j = t0 + row;
-            // y = log2-scaled logit, -inf where masked (padding row, beyond N,
-            // causal); only a tile that reaches the window needs the causal limit
-            float y[RH];
-            if (t0 + kTile <= cur.c) {
-#pragma unroll
-              for (int r = 0; r < RH; ++r)
-                y[r] = ((rmask >> (r0 + r)) & 1ull) ? __uint_as_float(v[r]) * p.scale_log2
-                                                    : -INFINITY;
-            } else {
-#pragma unroll
-              for (int r = 0; r < RH; ++r) {
-                const bool vis = ((rmask >> (r0 + r)) & 1ull) && j < cur.n &&
-                                 j <= cur.c + row_t[r0 + r];
-                y[r] = vis ? __uint_as_float(v[r]) * p.scale_log2 : -INFINITY;
-              }
-            }
-            // Lazy running max: the reference only moves when a logit exceeds it
-            // by more than 2^kLazy, so the terms 2^(y - max) stay below 256 and
-            // the common case is branch-free.
-            bool need = false;
-#pragma unroll
-            for (int r = 0; r < RH; ++r) need |= y[r] > st_m[r] + kLazy;
-            if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-              for (int r = 0; r < RH; ++r) {
-                if (y[r] > st_m[r]) {
-                  st_s[r] = st_s[r] * ex2(st_m[r] - y[r]) + 1.f;
-                  st_m[r] = y[r];
-                } else {
-                  st_s[r] += ex2(y[r] - st_m[r]);
-                }
-              }
-            } else {
-#pragma unroll
-              for (int r = 0; r < RH; ++r) st_s[r] += ex2(y[r] - st_m[r]);
-            }
-          }
-          lane_merge<RH>(st_m, st_s, lane);
-          if (lane < RH) {
-            red1[(q4 * RP + r0 + lane) * 2 + 0] = st_m[0];
-            red1[(q4 * RP + r0 + lane) * 2 + 1] = st_s[0];
-          }
-        } else if (red) {
-          // norm warps: ||k|| of row `row`, rho; (GEMM form) rho out;
-          // (closed form) U accumulation
-          float U4[4] = {0.f, 0.f, 0.f, 0.f};
-          for (int t = 0; t < cur.nt; ++t) {
-            const int j = cur.start + kTile * t + row;
-            mbar_wait(&full[stage], ph, abort, p.status);
-            __syncwarp();
-            const uint32_t sb = smem_u32(sm + L.stages + stage * kTileBytes);
-            uint4 xs[16];
-            load_row(sb, row, xs);
-            const float n2 = row_norm2(xs);
-            const float rho = (j < cur.n && n2 > 0.f) ? 1.f / sqrtf(n2) : 0.f;
-            if constexpr (CLOSED) {
-              u_accumulate(sb, rho, U4);
-            } else {
-              if (j < cur.n) p.rho_out[p.rho_off[cur.u] + j] = rho;
-            }
-            ++ntile;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-            if (++stage == NS) { stage = 0; ph ^= 1; }
-          }
-          if constexpr (CLOSED) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) red2[q4 * 128 + lane * 4 + i] = U4[i];
-          } else if (cur.g == cur.g0 + cur.nch - 1) {
-            // the unit's last chunk zeroes the pads of its rho segment
-            const int64_t pe = p.rho_off[cur.u + 1];
-            for (int64_t gi = p.rho_off[cur.u] + cur.n + (ctid - 256); gi < pe; gi += 128)
-              p.rho_out[gi] = 0.f;
-          }
-        }
-        RKV_STAMP(k, 1);
-        named_bar_sync(1, kConsumers);
-        float* xs_out = p.xstat + static_cast<int64_t>(cur.g) * XS;
-        if (ctid < RP) {
-          float m = kNegBig, s = 0.f;
-          for (int q = 0; q < 4; ++q)
-            merge_stat(m, s, red1[(q * RP + ctid) * 2], red1[(q * RP + ctid) * 2 + 1]);
-          xs_out[2 * ctid] = m;
-          xs_out[2 * ctid + 1] = s;
-        }
-        if (CLOSED && red && ctid >= 256) {
-          const int e = ctid - 256;
-          xs_out[2 * RP + e] = ((red2[e] + red2[128 + e]) + red2[256 + e]) + red2[384 + e];
-        }
-        named_bar_sync(1, kConsumers);
-        if (ctid == 0 && cur.g != p.drop_chunk) {
-          __threadfence();
-          atomicAdd(&p.cnt[cur.u * kScoreCnt + 2 * p.group], 1);
-        }
-        RKV_STAMP(k, 2);
-      }
-
-      // ================================================= W(x_k-1), P2(x_k-1), its sums
-      if (c1.g >= 0) {
-        const int buf = (k - 1) & 1;   // tensor-memory buffer and smem slot of x_k-1
-        if (ctid == 0)
-          wait_count(&p.cnt[c1.u * kScoreCnt + 2 * p.group], c1.nch, abort, p.status, p.abort_all,
-                     p.wait_ns);
-        RKV_STAMP(k, 3);
-        named_bar_sync(1, kConsumers);
-        // merge the unit's chunk statistics: every consumer thread folds a fixed
-        // subset of the chunks (the loads overlap), then the subsets are merged
-        // in order, so every CTA of the unit gets identical values
-        {
-          constexpr int TPR = kConsumers / RP;   // threads per query row
-          const int rr = ctid / TPR, tt = ctid - (ctid / TPR) * TPR;
-          const float* xs_in = p.xstat + static_cast<int64_t>(c1.g0) * XS;
-          float M = kNegBig, S = 0.f;
-#pragma unroll 4
-          for (int q = tt; q < c1.nch; q += TPR)
-            merge_stat(M, S, __ldcg(xs_in + q * XS + 2 * rr), __ldcg(xs_in + q * XS + 2 * rr + 1));
-          mpart[2 * ctid] = M;
-          mpart[2 * ctid + 1] = S;
-          if (CLOSED && red) {
-            const int e = ctid & 127, t3 = ctid >> 7;
-            float acc = 0.f;
-#pragma unroll 4
-            for (int q = t3; q < c1.nch; q += 3) acc += __ldcg(xs_in + q * XS + 2 * RP + e);
-            upart[t3 * 128 + e] = acc;
-          }
-        }
-        named_bar_sync(1, kConsumers);
-        if (ctid < RP) {
-          constexpr int TPR = kConsumers / RP;
-          float M = kNegBig, S = 0.f;
-          for (int tt = 0; tt < TPR; ++tt)
-            merge_stat(M, S, mpart[2 * (ctid * TPR + tt)], mpart[2 * (ctid * TPR + tt) + 1]);
-          mrow[ctid] = M;
-          invl[ctid] = S > 0.f ? 1.f / S : 0.f;
-        }
-        if (CLOSED && red && ctid >= 256) {
-          const int e = ctid - 256;
-          ufin[e] = (upart[e] + upart[128 + e]) + upart[256 + e];
-        }
-        named_bar_sync(1, kConsumers);
-        RKV_STAMP(k, 4);
-        float part = 0.f;   // softmax: sum of abar; norm warps: sum of exp(m)
-        if (is_soft) {
-          float M[RH], IL[RH];
-#pragma unroll
-          for (int r = 0; r < RH; ++r) {
-            // padding rows: a huge max and zero weight, so they add exactly 0
-            const bool real = ((rmask >> (r0 + r)) & 1ull) != 0;
-            M[r] = real ? mrow[r0 + r] : 1e30f;
-            IL[r] = real ? invl[r0 + r] : 0.f;
-          }
-          float* ab = abuf + (buf * 2 + hh) * CHT;
-          for (int t = 0; t < c1.nt; ++t) {
-            const int t0 = c1.start + kTile * t;
-            const int j = t0 + row;
-            uint32_t v[RH];
-            const uint32_t ta =
-                tmem + (static_cast<uint32_t>(q4 * 32) << 16) + buf * kBufCols + t * RP + r0;
-#pragma unroll
-            for (int sb = 0; sb < RH; sb += RB) tmem_ld_cols<RB>(ta + sb, v + sb);
-            tmem_wait_ld();
-            float pq[4] = {0.f, 0.f, 0.f, 0.f};
-            if (t0 + kTile <= c1.c) {
-#pragma unroll
-              for (int r = 0; r < RH; ++r)
-                pq[r & 3] = fmaf(ex2(fmaf(__uint_as_float(v[r]), p.scale_log2, -M[r])), IL[r],
-                                 pq[r & 3]);
-            } else {
-#pragma unroll
-              for (int r = 0; r < RH; ++r)
-                if (((rmask >> (r0 + r)) & 1ull) && j < c1.n && j <= c1.c + row_t[r0 + r])
-                  pq[r & 3] = fmaf(ex2(fmaf(__uint_as_float(v[r]), p.scale_log2, -M[r])),
-                                   IL[r], pq[r & 3]);
-            }
-            if (j < c1.c) {
-              const float x = (pq[0] + pq[1]) + (pq[2] + pq[3]);
-              ab[kTile * t + row] = x;
-              part += x;
-            }
-          }
-          // this buffer's logits have been read: the MMA may reuse it
-          tc_fence_before();
+        float U4[4] = {0.f, 0.f, 0.f, 0.f};
+        float* rho_u = CLOSED ? nullptr : p.rho_out + p.rho_off[cur.u];
+        for (int t = 0; t < cur.nt; ++t) {
+          const int j = cur.start + kTile * t + row;
+          mbar_wait(&full[stage], ph, abort, p.status);
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tfree[buf]);
-        } else if (CLOSED && red) {
+          const uint32_t sb = smem_u32(sm + L.stages + stage * kTileBytes);
+          uint4 xs[16];
+          load_row(sb, row, xs);
+          const float n2 = row_norm2(xs);
+          const float rho = (j < cur.n && n2 > 0.f) ? 1.f / sqrtf(n2) : 0.f;
+          if constexpr (CLOSED) {
+            rhoc[(k & 1) * CHT + kTile * t + row] = rho;
+            u_accumulate(sb, rho, U4);
+          } else {
+            if (j < cur.n) rho_u[j] = rho;
+          }
+          ++ntile;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[stage]);
+          if (++stage == NS) { stage = 0; ph ^= 1; }
+        }
+        if constexpr (CLOSED) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) red2[q4 * 128 + lane * 4 + i] = U4[i];
+          named_bar_sync(3, 128);
+          p.xstat[static_cast<int64_t>(cur.g) * XS + 2 * RP + ctid] =
+              ((red2[ctid] + red2[128 + ctid]) + red2[256 + ctid]) + red2[384 + ctid];
+          named_bar_sync(3, 128);
+          if (ctid == 0 && cur.g != p.drop_chunk) {
+            __threadfence();
+            atomicAdd(&p.cnt[cur.u * kScoreCnt + 2 * p.group], 1);
+          }
+        } else if (cur.g == cur.g0 + cur.nch - 1) {
+          // the unit's last chunk zeroes the pads of its rho segment
+          const int64_t pe = p.rho_off[cur.u + 1];
+          for (int64_t gi = p.rho_off[cur.u] + cur.n + ctid; gi < pe; gi += 128)
+            p.rho_out[gi] = 0.f;
+        }
+      }
+      if constexpr (CLOSED) {
+        // ---- W(x_k-1): the unit's U; m of x_k-1 from its tiles read again
+        if (c1.g >= 0) {
+          const int slot = (k - 1) & 1;
+          if (ctid == 0)
+            wait_count(&p.cnt[c1.u * kScoreCnt + 2 * p.group], nann * c1.nch, abort, p.status,
+                       p.abort_all, p.wait_ns);
+          named_bar_sync(3, 128);
+          {
+            const float* xs_in = p.xstat + static_cast<int64_t>(c1.g0) * XS + 2 * RP + ctid;
+            float acc0 = 0.f, acc1 = 0.f;
+            int q = 0;
+            for (; q + 1 < c1.nch; q += 2) {   // two independent loads in flight
+              acc0 += __ldcg(xs_in + q * XS);
+              acc1 += __ldcg(xs_in + (q + 1) * XS);
+            }
+            if (q < c1.nch) acc0 += __ldcg(xs_in + q * XS);
+            ufin[ctid] = acc0 + acc1;
+          }
+          named_bar_sync(3, 128);
           const float inv_nm1 = c1.n > 1 ? 1.f / static_cast<float>(c1.n - 1) : 0.f;
-          float* ma = marr + buf * CHT;
+          float* ma = marr + slot * CHT;
+          const float* rc = rhoc + slot * CHT;
+          float part = 0.f;
           for (int t = 0; t < c1.nt; ++t) {
             const int j = c1.start + kTile * t + row;
             mbar_wait(&full[stage], ph, abort, p.status);
@@ -664,7 +902,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             const uint32_t sb = smem_u32(sm + L.stages + stage * kTileBytes);
             uint4 xs[16];
             load_row(sb, row, xs);
-            const float n2 = row_norm2(xs);
             float dq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int k8 = 0; k8 < 16; ++k8) {
@@ -683,97 +920,61 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             if (lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == NS) { stage = 0; ph ^= 1; }
             if (j < c1.c) {
-              const float rho = (n2 > 0.f) ? 1.f / sqrtf(n2) : 0.f;
+              const float rho = rc[kTile * t + row];
               const float dot = (dq[0] + dq[1]) + (dq[2] + dq[3]);
               const float m = (rho * dot - (rho > 0.f ? 1.f : 0.f)) * inv_nm1;
               ma[kTile * t + row] = m;
               part += ex2(m * kLog2e);
             }
           }
-        }
-        RKV_STAMP(k, 5);
-        part = warp_reduce_sum(part);
-        if (lane == 0) rsum[warp - 4] = part;
-        named_bar_sync(1, kConsumers);
-        if (ctid == 0) {
-          float* xo = p.xsum + static_cast<int64_t>(c1.g) * (2 * kScoreMaxGroups) + 2 * p.group;
-          xo[0] = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) +
-                  ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
-          xo[1] = (rsum[8] + rsum[9]) + (rsum[10] + rsum[11]);
-          if (red) {
+          part = warp_reduce_sum(part);
+          if (lane == 0) esum[q4] = part;
+          named_bar_sync(3, 128);
+          if (ctid == 0) {
+            float* xo =
+                p.xsum + static_cast<int64_t>(c1.g) * (2 * kScoreMaxGroups) + 2 * p.group + 1;
+            *xo = (esum[0] + esum[1]) + (esum[2] + esum[3]);
             __threadfence();
             atomicAdd(&p.cnt[c1.u * kScoreCnt + 2 * p.group + 1], 1);
           }
         }
-        RKV_STAMP(k, 6);
-        if (!red) {
-          // an earlier row group: add this group's probabilities to a (not yet
-          // normalised); the last group normalises
-          const float* a0 = abuf + (buf * 2 + 0) * CHT;
-          const float* a1 = abuf + (buf * 2 + 1) * CHT;
-          for (int i = ctid; i < c1.len; i += kConsumers) {
-            const int j = c1.start + i;
-            const int64_t gi = c1.base + j;
-            if (j < c1.c) {
-              const float x = a0[i] + a1[i];
-              p.a_out[gi] = p.group > 0 ? p.a_out[gi] + x : x;
-            }
+        // ---- WS(x_k-2): r and m of x_k-2
+        if (c2.g >= 0) {
+          const int slot = k & 1;
+          if (warp == 12) {
+            if (lane == 0)
+              wait_count(&p.cnt[c2.u * kScoreCnt + 2 * p.group + 1], nann * c2.nch, abort,
+                         p.status, p.abort_all, p.wait_ns);
+            __syncwarp();
+            float se = 0.f;
+            for (int q = lane; q < c2.nch; q += 32)
+              se += __ldcg(p.xsum + static_cast<int64_t>(c2.g0 + q) * (2 * kScoreMaxGroups) +
+                           2 * p.group + 1);
+            se = warp_reduce_sum(se);
+            if (lane == 0) esum[8] = se > 0.f ? 1.f / se : 0.f;
           }
-        }
-      }
-
-      // ================================================= WS(x_k-2), output of x_k-2
-      if (red && c2.g >= 0) {
-        const int buf = k & 1;   // slot of x_k-2
-        if (warp == 4) {
-          if (lane == 0)
-            wait_count(&p.cnt[c2.u * kScoreCnt + 2 * p.group + 1], c2.nch, abort, p.status,
-                       p.abort_all, p.wait_ns);
-          __syncwarp();
-          // sums over the unit's chunks (and earlier row groups), fixed order
-          float sa = 0.f, se = 0.f;
-          for (int q = lane; q < c2.nch; q += 32) {
-            const float* xi = p.xsum + static_cast<int64_t>(c2.g0 + q) * (2 * kScoreMaxGroups);
-            float x = 0.f;
-            for (int gq = 0; gq <= p.group; ++gq) x += __ldcg(xi + 2 * gq);
-            sa += x;
-            se += __ldcg(xi + 2 * p.group + 1);
-          }
-          sa = warp_reduce_sum(sa);
-          se = warp_reduce_sum(se);
-          if (lane == 0) {
-            rsum[16] = sa > 0.f ? 1.f / sa : 0.f;
-            rsum[17] = se > 0.f ? 1.f / se : 0.f;
-          }
-        }
-        RKV_STAMP(k, 7);
-        named_bar_sync(1, kConsumers);
-        const float inv_sa = rsum[16], inv_se = rsum[17];
-        const float* a0 = abuf + (buf * 2 + 0) * CHT;
-        const float* a1 = abuf + (buf * 2 + 1) * CHT;
-        const float* ma = marr + buf * CHT;
-        for (int i = ctid; i < c2.len; i += kConsumers) {
-          const int j = c2.start + i;
-          const int64_t gi = c2.base + j;
-          if (j < c2.c) {
-            float x = a0[i] + a1[i];
-            if (p.group > 0) x = p.a_out[gi] + x;
-            p.a_out[gi] = x * inv_sa;
-            if constexpr (CLOSED) {
+          named_bar_sync(3, 128);
+          const float inv_se = esum[8];
+          const float* ma = marr + slot * CHT;
+          for (int i = ctid; i < c2.len; i += 128) {
+            const int j = c2.start + i;
+            const int64_t gi = c2.base + j;
+            if (j < c2.c) {
               const float m = ma[i];
               p.r_out[gi] = ex2(m * kLog2e) * inv_se;
               if (p.m_out) p.m_out[gi] = m;
+            } else {
+              p.r_out[gi] = 0.f;
+              if (p.m_out) p.m_out[gi] = 0.f;
             }
-          } else {
-            p.a_out[gi] = 0.f;
-            p.r_out[gi] = 0.f;
-            if (p.m_out) p.m_out[gi] = 0.f;
           }
+          named_bar_sync(3, 128);   // esum and the slot are reused
         }
+        c2 = c1;
+        c1 = cur;
+      } else if (!have) {
+        break;
       }
-      RKV_STAMP(k, 8);
-      c2 = red ? c1 : no_chunk();
-      c1 = cur;
     }
   }
 
@@ -793,8 +994,7 @@ void* score_fn() {
 
 void* pick(int rp, bool closed) {
   if (rp == 16) return closed ? score_fn<16, true>() : score_fn<16, false>();
-  if (rp == 32) return closed ? score_fn<32, true>() : score_fn<32, false>();
-  return closed ? score_fn<64, true>() : score_fn<64, false>();
+  return closed ? score_fn<32, true>() : score_fn<32, false>();
 }
 
 }  // namespace
@@ -818,8 +1018,8 @@ int score_max_ctas(int rp, bool closed, int smem_bytes) {
 }
 
 bool score_plan(int R, const int64_t* off, int U, int max_ctas, int tpc_fixed, ScoreDims* d) {
-  d->rp = R <= 16 ? 16 : (R <= 32 ? 32 : 64);
-  d->ngroups = (R + 63) / 64;
+  d->rp = R <= 16 ? 16 : 32;
+  d->ngroups = (R + 31) / 32;
   if (d->ngroups > kScoreMaxGroups) return false;
   const int tpc_max = score_chunk_tokens(d->rp) / kTile;
   int64_t tiles = 0, tmax = 0;
@@ -873,12 +1073,8 @@ cudaError_t launch_score(const CUtensorMap& kmap, const CUtensorMap& qmap, const
     if (closed) return cudaLaunchKernelEx(&cfg, score_kernel<16, true>, kmap, qmap, p);
     return cudaLaunchKernelEx(&cfg, score_kernel<16, false>, kmap, qmap, p);
   }
-  if (rp == 32) {
-    if (closed) return cudaLaunchKernelEx(&cfg, score_kernel<32, true>, kmap, qmap, p);
-    return cudaLaunchKernelEx(&cfg, score_kernel<32, false>, kmap, qmap, p);
-  }
-  if (closed) return cudaLaunchKernelEx(&cfg, score_kernel<64, true>, kmap, qmap, p);
-  return cudaLaunchKernelEx(&cfg, score_kernel<64, false>, kmap, qmap, p);
+  if (closed) return cudaLaunchKernelEx(&cfg, score_kernel<32, true>, kmap, qmap, p);
+  return cudaLaunchKernelEx(&cfg, score_kernel<32, false>, kmap, qmap, p);
 }
 
 }  // namespace rkv
@@ -886,5 +1082,8 @@ cudaError_t launch_score(const CUtensorMap& kmap, const CUtensorMap& qmap, const
 #ifdef RKV_TRACE
 extern "C" int rkv_debug_score_trace(void* dst, size_t bytes) {
   return static_cast<int>(cudaMemcpyFromSymbol(dst, rkv::g_score_trace, bytes));
+}
+extern "C" int rkv_debug_tile_trace(void* dst, size_t bytes) {
+  return static_cast<int>(cudaMemcpyFromSymbol(dst, rkv::g_tile_trace, bytes));
 }
 #endif

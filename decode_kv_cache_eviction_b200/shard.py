@@ -2,9 +2,12 @@
 
 Units (sequence, layer, KV head) are independent, so a multi-GPU run needs no
 exchange on the data path: each rank compresses a subset of the units.  The
-subsets are balanced by token count (greedy longest-first assignment), which
-balances both the HBM-bound scoring (proportional to N) and, nearly, the
-redundancy GEMM (proportional to N^2) for ragged batches.
+subsets are balanced by a per-unit cost (greedy longest-processing-time-first
+assignment).  With the redundancy GEMM the step is dominated by the N x N tile
+products, so a unit of N tokens costs about N^2 + 320 N (the linear term is the
+HBM-bound scoring and selection: 128 N^2 tensor flops at ~1 PFLOP/s against
+about 264 N bytes at ~6.5 TB/s break even near N = 320); with the closed-form
+redundancy every step is HBM-bound and a unit costs N.
 """
 from __future__ import annotations
 
@@ -14,21 +17,33 @@ from typing import List
 import numpy as np
 
 
-def shard_units(n_tokens, world: int) -> List[np.ndarray]:
-    """Assign unit indices to `world` ranks, balancing the sum of N per rank.
+def unit_cost(n_tokens, redundancy: str = "gemm") -> np.ndarray:
+    """Relative cost of compressing units of the given lengths."""
+    n = np.asarray(n_tokens, dtype=np.float64)
+    if redundancy == "closed":
+        return n
+    if redundancy in ("gemm", "max"):
+        return n * (n + 320.0)
+    raise ValueError(redundancy)
 
-    Longest unit first, each to the currently least-loaded rank (ties to the
+
+def shard_units(n_tokens, world: int, redundancy: str = "gemm") -> List[np.ndarray]:
+    """Assign unit indices to `world` ranks, balancing the summed unit cost
+    (:func:`unit_cost`) per rank.
+
+    Costliest unit first, each to the currently least-loaded rank (ties to the
     lower rank).  Returns, per rank, its unit indices in ascending order."""
     n = np.asarray(n_tokens, dtype=np.int64)
     if world < 1:
         raise ValueError("world must be >= 1")
-    order = np.lexsort((np.arange(len(n)), -n))      # N descending, index ascending
-    heap = [(0, r) for r in range(world)]
+    cost = unit_cost(n, redundancy)
+    order = np.lexsort((np.arange(len(n)), -cost))   # cost descending, index ascending
+    heap = [(0.0, r) for r in range(world)]
     parts = [[] for _ in range(world)]
     for u in order.tolist():
         load, r = heapq.heappop(heap)
         parts[r].append(u)
-        heapq.heappush(heap, (load + int(n[u]), r))
+        heapq.heappush(heap, (load + float(cost[u]), r))
     return [np.array(sorted(p), dtype=np.int64) for p in parts]
 
 

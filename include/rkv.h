@@ -13,9 +13,8 @@
  * slot buffer (gather compaction, named as the R-KV-style baseline in the ThinKV
  * summary, "Continuous Thinking" section).
  *
- * Limits: head_dim = 128, G*w <= 256 (up to 64 query rows per pass over K; more
- * rows take several passes), N_u <= 49152 (the selection keeps a unit's keys in
- * shared memory).
+ * Limits: head_dim = 128, G*w <= 256 (up to 32 query rows per pass over K; more
+ * rows take several passes), N_u <= 131072.
  *
  * Terms used below.  A *unit* is one (sequence, layer, KV head).  Unit u has
  * N_u cached tokens, stored as rows tok_off[u] .. tok_off[u+1]-1 of K and V.
@@ -320,7 +319,7 @@ int rkv_read_timing(rkv_engine* eng, int kernel, double* total_ms, int64_t* laun
  * slots and counters, per-unit offsets and counters, a status word) lives in one
  * file-scope __device__ array of about 11 MB that every GPU holding the
  * library's module keeps until the process exits; nothing is allocated or freed
- * per call.  Limits: G*w <= 32, N_u <= 49152, at most RKV_NOALLOC_MAX_UNITS
+ * per call.  Limits: G*w <= 32, N_u <= 131072, at most RKV_NOALLOC_MAX_UNITS
  * units and RKV_NOALLOC_MAX_TOKENS rows per call (larger batches return
  * RKV_ERR_CAPACITY, longer units or larger G*w RKV_ERR_UNSUPPORTED, before
  * anything is enqueued).

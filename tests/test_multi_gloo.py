@@ -13,16 +13,31 @@ from decode_kv_cache_eviction_b200 import shard
 from decode_kv_cache_eviction_b200 import workloads as W
 
 
-def test_shard_units_partition_and_balance():
+@pytest.mark.parametrize("redundancy", ["gemm", "closed"])
+def test_shard_units_partition_and_balance(redundancy):
     n = W.unit_lengths(W.WORKLOADS["ragged_serving"], 0)
+    cost = shard.unit_cost(n, redundancy)
     for world in (1, 2, 3, 8):
-        parts = shard.shard_units(n, world)
+        parts = shard.shard_units(n, world, redundancy)
         allu = np.sort(np.concatenate(parts))
         np.testing.assert_array_equal(allu, np.arange(len(n)))
-        loads = np.array([n[p].sum() for p in parts])
-        assert loads.max() - loads.min() <= n.max()
+        loads = np.array([cost[p].sum() for p in parts])
+        # greedy LPT: no rank exceeds another by more than the costliest unit
+        assert loads.max() - loads.min() <= cost.max()
         for p in parts:
             assert np.all(np.diff(p) > 0)
+
+
+def test_gemm_sharding_balances_the_quadratic_work():
+    """Units of 2K-8K tokens: balancing N alone can leave the N^2 GEMM work
+    uneven; the GEMM cost model keeps it within a few percent."""
+    rng = np.random.default_rng(0)
+    n = np.concatenate([np.full(40, 8192), np.full(160, 2048)])
+    rng.shuffle(n)
+    for world in (2, 4, 8):
+        parts = shard.shard_units(n, world, "gemm")
+        quad = np.array([(n[p].astype(np.float64) ** 2).sum() for p in parts])
+        assert quad.max() / quad.mean() < 1.05
 
 
 def test_sub_offsets_and_rows():

@@ -21,7 +21,8 @@ DEV = "cuda:0"
 # ----------------------------------------------------------------- select alone
 @pytest.mark.parametrize("lam", [0.0, 0.1, 1.0])
 @pytest.mark.parametrize("lengths,budget", [([1000], 100), ([4096, 300, 9], 256),
-                                            ([20000, 33000], 4096), ([5000], 0)])
+                                            ([20000, 33000], 4096), ([5000], 0),
+                                            ([65536, 131072], 4096)])
 def test_select_bit_exact_given_scores(lam, lengths, budget):
     w = 8
     b = rand_batch(lengths, 1, w, seed=len(lengths) + budget)
@@ -47,6 +48,45 @@ def test_select_bit_exact_given_scores(lam, lengths, budget):
         assert nk[u] == len(want)
         np.testing.assert_array_equal(idx[u, :nk[u]], want)
         assert np.all(idx[u, nk[u]:] == -1)
+
+
+@pytest.mark.parametrize("n,budget", [(40000, 1000), (3000, 2999), (9000, 1)])
+def test_select_all_scores_equal(n, budget):
+    """Every score ties: the bracket around the budget's rank holds every
+    candidate, so the selection runs over all of them; ties go to the lowest
+    indices."""
+    w = 8
+    b = rand_batch([n], 1, w, seed=9)
+    a = torch.full((n,), 2e-4, dtype=torch.float32, device=DEV)
+    r = torch.full((n,), 1e-4, dtype=torch.float32, device=DEV)
+    eng = Engine(1, w, max_units=1, max_tokens=n, redundancy="closed")
+    idx, nk, _, _ = eng.alloc_outputs(b, budget)
+    eng.select(b, a, r, 0.1, budget, idx, nk)
+    eng.check_status()
+    got = idx[0, :nk[0]].cpu().numpy()
+    want = np.arange(n) if n - w <= budget else np.concatenate([np.arange(budget),
+                                                                np.arange(n - w, n)])
+    np.testing.assert_array_equal(got, want)
+
+
+def test_select_two_clusters_and_outliers():
+    """Scores in two tight clusters plus a few extreme outliers (the sample
+    still brackets the budget's rank, or the full selection takes over)."""
+    w, n, budget = 8, 50000, 7000
+    rng = np.random.default_rng(5)
+    a = np.where(rng.random(n) < 0.8, 1e-5 + 1e-9 * rng.random(n), 3e-5 + 1e-9 * rng.random(n))
+    a[rng.choice(n, 20, replace=False)] = 0.5
+    a = a.astype(np.float32)
+    r = np.full(n, 1e-5, np.float32)
+    b = rand_batch([n], 1, w, seed=10)
+    eng = Engine(1, w, max_units=1, max_tokens=n, redundancy="closed")
+    idx, nk, _, _ = eng.alloc_outputs(b, budget)
+    for lam in (1.0, 0.3):
+        eng.select(b, torch.from_numpy(a).to(DEV), torch.from_numpy(r).to(DEV), lam, budget,
+                   idx, nk)
+        eng.check_status()
+        s32 = ora.joint_score(a[:n - w], r[:n - w], np.float32(lam))
+        np.testing.assert_array_equal(idx[0, :nk[0]].cpu().numpy(), ora.select(s32, n, w, budget))
 
 
 # ----------------------------------------------------------------- compaction alone
@@ -202,19 +242,21 @@ def test_symmetric_flag_rejections():
     assert ei.value.code == -2
 
 
-@pytest.mark.parametrize("G,w,N", [(4, 8, 32768), (2, 8, 49152), (4, 8, 40000), (8, 8, 40000)])
+@pytest.mark.parametrize("G,w,N", [(4, 8, 32768), (2, 8, 49152), (4, 8, 40000), (8, 8, 40000),
+                                   (4, 8, 65536), (1, 8, 131072)])
 def test_long_units(G, w, N):
     """Units longer than 32K tokens and up to 64 query rows; every tile of a
     unit's chunks streams through one pass (chunk exchanges in global memory)."""
     b = rand_batch([N], G, w, seed=1, dup=0.0)
-    for mode in ("closed", "gemm", "max", "gemm_sym"):
+    modes = ("closed", "gemm", "max", "gemm_sym") if N <= 65536 else ("closed", "gemm_sym")
+    for mode in modes:
         out = run_engine(b, G, w, 0.1, 4096, mode=mode)
         check_unit(out, b, 0, w, 0.1, 4096, redundancy=oracle_mode(mode))
         del out
 
 
 def test_rejects_too_long_unit_and_capacity():
-    b = rand_batch([49153], 1, 8, seed=0, dup=0.0)
+    b = rand_batch([131073], 1, 8, seed=0, dup=0.0)
     eng = Engine(1, 8, max_units=1, max_tokens=b.num_tokens, redundancy="closed")
     a, r = eng.alloc_scores(b)
     with pytest.raises(RkvError) as ei:
