@@ -489,7 +489,7 @@ int rkv_select(rkv_engine* e, const rkv_batch* b, const float* a, const float* r
     return RKV_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   t_begin(e, RKV_KERNEL_SELECT, st);
-  cudaError_t err = launch_select(b->tok_off, U, e->cfg.window, cmax, a, r, lambda, budget,
+  cudaError_t err = launch_select(b->tok_off, U, T, e->cfg.window, cmax, a, r, lambda, budget,
                                   nullptr, 0, budget + e->cfg.window, idx, n_kept, st);
   t_end(e, st);
   if (err != cudaSuccess) return cuda_fail(err);
@@ -517,7 +517,7 @@ int rkv_select_ex(rkv_engine* e, const rkv_batch* b, const float* a, const float
     return RKV_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   t_begin(e, RKV_KERNEL_SELECT, st);
-  cudaError_t err = launch_select(b->tok_off, U, e->cfg.window, cmax, a, r, lambda, budget,
+  cudaError_t err = launch_select(b->tok_off, U, T, e->cfg.window, cmax, a, r, lambda, budget,
                                   budgets, sinks, static_cast<int>(W), idx, n_kept, st);
   t_end(e, st);
   if (err != cudaSuccess) return cuda_fail(err);

@@ -224,7 +224,8 @@ __host__ __device__ inline int64_t gemm_unit_items(int64_t n, int64_t c, int row
   return sym ? (n + 255) / 256 : (c + rows_per_item - 1) / rows_per_item;
 }
 
-cudaError_t launch_select(const int64_t* tok_off, int U, int w, int cmax, const float* a,
+cudaError_t launch_select(const int64_t* tok_off, int U, int64_t Ttot, int w, int cmax,
+                          const float* a,
                           const float* r, float lam, int budget, const int32_t* budgets,
                           int sinks, int W, int32_t* idx, int32_t* n_kept, cudaStream_t st);
 cudaError_t select_configure();
