@@ -14,7 +14,9 @@ constexpr int kTileBytes = kTile * kHeadDim * 2;
 // selection a bit per candidate on chip.
 constexpr int kMaxTokensPerUnit = 131072;
 constexpr int kMaxRows = 256;        // G * w limit (row groups of 32 per launch)
-constexpr int kScoreThreads = 512;   // 16 warps
+// Score kernel threads: 16 warps, or 20 in the GEMM form (a second set of four
+// pass-2 warps; the closed form's norm warps need the registers instead).
+__host__ __device__ constexpr int score_threads(bool closed) { return closed ? 512 : 640; }
 constexpr int kGemmThreads = 640;    // producer, MMA, 2 idle, 16 epilogue warps
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -61,8 +63,8 @@ __host__ __device__ constexpr int score_xs(int rp, bool closed) {
 }
 
 struct ScoreLayout {
-  uint32_t stages, q, abuf, marr, rhoc, red1, red2, rhot, ufin, mpart, mrow, invl, rsum, esum,
-      rowt, bars, slot, flags, issued, total;
+  uint32_t stages, q, abuf, marr, rhoc, red1, red2, rhot, ufin, mpart, mrow, rsum, esum,
+      osum, rowt, bars, slot, flags, issued, total;
 };
 
 __host__ __device__ inline ScoreLayout score_layout(int rp, bool closed, int ns) {
@@ -72,20 +74,20 @@ __host__ __device__ inline ScoreLayout score_layout(int rp, bool closed, int ns)
   L.stages = o; o += ns * kTileBytes;
   L.q = o; o += 2 * rp * 256;
   L.abuf = o; o += 2 * cht * 4;
-  L.marr = o; if (closed) o += 2 * cht * 4;
+  L.marr = o; if (closed) o += 2 * cht * 4;   // (read by the output warps only when closed)
   L.rhoc = o; if (closed) o += 2 * cht * 4;
   L.red1 = o; o += 4 * rp * 2 * 4;
   L.red2 = o; if (closed) o += 4 * 128 * 4;
   L.rhot = o; if (closed) o += 2 * 128 * 4;
   L.ufin = o; if (closed) o += 128 * 4;
-  L.mpart = o; o += 128 * 2 * 4;
-  L.mrow = o; o += rp * 4;
-  L.invl = o; o += rp * 4;
+  L.mpart = o; o += 256 * 2 * 4;
+  L.mrow = o; o += 2 * rp * 4;   // merged (max, 1 / sum) per query row
   L.rsum = o; o += 16 * 4;
   L.esum = o; o += 16 * 4;
+  L.osum = o; o += 4 * 4;
   L.rowt = o; o += 32 * 4;
   o = (o + 15u) & ~15u;
-  L.bars = o; o += (2 * ns + 32 + 6 + 1) * 8;
+  L.bars = o; o += (2 * ns + 32 + 6 + 1 + 4) * 8;
   L.slot = o; o += 16;
   L.flags = o; o += 16;
   L.issued = o; o += 32;

@@ -283,12 +283,11 @@ __device__ __forceinline__ float row_norm2(const uint4 (&xs)[16]) {
 }
 
 template <int RP, bool CLOSED>
-__global__ void __launch_bounds__(kScoreThreads, 1)
+__global__ void __launch_bounds__(score_threads(CLOSED), 1)
     score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                  const ScoreParams p) {
   constexpr int XS = score_xs(RP, CLOSED);  // floats of a chunk's exchange slot
   constexpr int CHT = score_chunk_tokens(RP);
-  constexpr int TPR = 128 / RP;             // pass-2 threads per query row in the merge
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -310,6 +309,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   uint64_t* qfull = tfree + 2;     // [2]
   uint64_t* qempty = qfull + 2;    // [2]
   uint64_t* mdone = qempty + 2;    // teardown: every MMA has completed
+  uint64_t* sfull = mdone + 1;     // [2] a smem slot holds a chunk's abar (and m)
+  uint64_t* sfree = sfull + 2;     // [2] the output warps are done with a slot
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.slot);
   volatile int* abort = reinterpret_cast<volatile int*>(sm + L.flags);
   int8_t* lastp = reinterpret_cast<int8_t*>(sm + L.issued);   // [NS + 2] parity of the last copy
@@ -321,11 +322,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     }
     for (int k = 0; k < 32; ++k) mbar_init(&tready[k], 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfree[b], 4);
+      mbar_init(&tfree[b], score_threads(CLOSED) == 640 ? 8 : 4);   // pass-2 warps
       mbar_init(&qfull[b], 1);
       mbar_init(&qempty[b], 1);
     }
     mbar_init(mdone, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sfull[b], (CLOSED && red) ? 2 : 1);   // pass-2 warps [+ norm warps]
+      mbar_init(&sfree[b], 1);
+    }
     for (int s = 0; s < NS + 2; ++s) lastp[s] = -1;
     *abort = 0;
     fence_mbar_init();
@@ -448,6 +453,70 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       drain_wait(mdone, 0);
     }
     __syncwarp();
+  } else if (warp == 2 || warp == 3) {
+    // ---------------------------------------------- output warps (final pass)
+    // chunk x_j once its abar (and m) sit in smem slot j % 2: wait for the
+    // sums of every chunk of its unit, write a (and r, m), free the slot
+    if (red) {
+      const int ctid = threadIdx.x - 64;     // 0..63
+      float* abuf = reinterpret_cast<float*>(sm + L.abuf);   // [2 slots][CHT]
+      float* marr = reinterpret_cast<float*>(sm + L.marr);   // [2 slots][CHT]
+      float* osum = reinterpret_cast<float*>(sm + L.osum);   // [2] inverse sums
+      for (int k = 0;; ++k) {
+        const int g = b0 + k * P;
+        if (g >= p.total_chunks) break;
+        const Chunk h = chunk_info(p, g);
+        const int slot = k & 1;
+        mbar_wait(&sfull[slot], (k >> 1) & 1, abort, p.status);
+        if (warp == 2) {
+          if (lane == 0)
+            wait_count(&p.cnt[h.u * kScoreCnt + 2 * p.group + 1], nann * h.nch, abort, p.status,
+                       p.abort_all, p.wait_ns);
+          __syncwarp();
+          // sums over the unit's chunks (and earlier row groups), fixed order
+          float sa = 0.f, se = 0.f;
+          for (int q = lane; q < h.nch; q += 32) {
+            const float* xi = p.xsum + static_cast<int64_t>(h.g0 + q) * (2 * kScoreMaxGroups);
+            float x = 0.f;
+            for (int gq = 0; gq <= p.group; ++gq) x += __ldcg(xi + 2 * gq);
+            sa += x;
+            if (CLOSED) se += __ldcg(xi + 2 * p.group + 1);
+          }
+          sa = warp_reduce_sum(sa);
+          se = warp_reduce_sum(se);
+          if (lane == 0) {
+            osum[0] = sa > 0.f ? 1.f / sa : 0.f;
+            osum[1] = se > 0.f ? 1.f / se : 0.f;
+          }
+        }
+        named_bar_sync(4, 64);
+        RKV_STAMP(k, 5);
+        const float inv_sa = osum[0], inv_se = osum[1];
+        const float* ab = abuf + slot * CHT;
+        const float* ma = marr + slot * CHT;
+        for (int i = ctid; i < h.len; i += 64) {
+          const int j = h.start + i;
+          const int64_t gi = h.base + j;
+          if (j < h.c) {
+            float x = ab[i];
+            if (p.group > 0) x = p.a_out[gi] + x;
+            p.a_out[gi] = x * inv_sa;
+            if constexpr (CLOSED) {
+              const float m = ma[i];
+              p.r_out[gi] = ex2(m * kLog2e) * inv_se;
+              if (p.m_out) p.m_out[gi] = m;
+            }
+          } else {
+            p.a_out[gi] = 0.f;
+            p.r_out[gi] = 0.f;   // the redundancy GEMM writes the candidates' r and m
+            if (p.m_out) p.m_out[gi] = 0.f;
+          }
+        }
+        named_bar_sync(4, 64);
+        RKV_STAMP(k, 6);
+        if (ctid == 0) mbar_arrive(&sfree[slot]);
+      }
+    }
   } else if (warp >= 4 && warp < 8) {
     // ---------------------------------------------- statistics warps (pass 1)
     // thread = 4 tokens x NR query rows of a tile (16x256b loads); no global waits
@@ -573,55 +642,71 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       g = gn;
       cur = nxt;
     }
-  } else if (warp >= 8 && warp < 12) {
+  } else if ((warp >= 8 && warp < 12) || warp >= 16) {
     // ---------------------------------------------- pass-2 warps
-    // step k: merge the statistics of x_k-1 and turn its logits into abar,
-    // then normalise and write a for x_k-2
-    const int ctid = threadIdx.x - 256;      // 0..127
+    // step k: merge the statistics of x_k-1 and turn its logits into abar.
+    // NPAR sets of four warps (warps 8-11 [and 16-19]) take alternate tiles.
+    constexpr int NPAR = (score_threads(CLOSED) - 512) / 128 + 1;
+    constexpr int NP2 = 128 * NPAR;          // pass-2 threads
+    const int tp = warp >= 16 ? 1 : 0;       // this set's tile parity
+    const int ctid = tp * 128 + (threadIdx.x - 256 - (tp ? 256 : 0));   // 0 .. NP2-1
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     float* abuf = reinterpret_cast<float*>(sm + L.abuf);   // [2 slots][CHT]
-    float* mpart = reinterpret_cast<float*>(sm + L.mpart); // [128][2]
-    float* mrow = reinterpret_cast<float*>(sm + L.mrow);   // [RP]
-    float* invl = reinterpret_cast<float*>(sm + L.invl);   // [RP]
+    float* mpart = reinterpret_cast<float*>(sm + L.mpart); // [NP2][2]
+    float* mfin = reinterpret_cast<float*>(sm + L.mrow);   // [RP][2] merged (max, 1 / sum)
     float* psum = reinterpret_cast<float*>(sm + L.rsum);   // [4] + inverse sum at [8]
-    Chunk c1 = no_chunk(), c2 = no_chunk();
+    Chunk c1 = no_chunk();
     for (int k = 0;; ++k) {
       const int g = b0 + k * P;
       const bool have = g < p.total_chunks;
-      if (!have && c1.g < 0 && c2.g < 0) break;
+      if (!have && c1.g < 0) break;
       // ---- W(x_k-1), pass 2, its sum
       if (c1.g >= 0) {
         const int buf = (k - 1) & 1;   // tensor-memory buffer and smem slot of x_k-1
         if (ctid == 0)
           wait_count(&p.cnt[c1.u * kScoreCnt + 2 * p.group], nann * c1.nch, abort, p.status,
                      p.abort_all, p.wait_ns);
+        // the slot's previous chunk (x_k-3) has been written out
+        if (red) mbar_wait(&sfree[buf], (((k - 1) >> 1) & 1) ^ 1, abort, p.status);
         RKV_STAMP(k, 2);
-        named_bar_sync(2, 128);
+        named_bar_sync(2, NP2);
         {
           // every thread folds a fixed subset of the unit's chunks for one row
-          // (the loads overlap), then the subsets are merged in order: every
-          // CTA of the unit gets identical values
-          const int rr = ctid / TPR, tt = ctid - rr * TPR;
-          const float* xs_in = p.xstat + static_cast<int64_t>(c1.g0) * XS;
+          // (eight loads in flight at a time), then the subsets are merged in
+          // order: every CTA of the unit gets identical values
+          constexpr int TPRX = NP2 / RP;   // threads per query row
+          const int rr = ctid / TPRX, tt = ctid - rr * TPRX;
+          const float* xs_in = p.xstat + static_cast<int64_t>(c1.g0) * XS + 2 * rr;
           float M = kNegBig, S = 0.f;
-#pragma unroll 4
-          for (int q = tt; q < c1.nch; q += TPR)
-            merge_stat(M, S, __ldcg(xs_in + q * XS + 2 * rr), __ldcg(xs_in + q * XS + 2 * rr + 1));
+          for (int q0 = tt; q0 < c1.nch; q0 += 8 * TPRX) {
+            float lm[8], ls[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+              const int q = q0 + x * TPRX;
+              lm[x] = q < c1.nch ? __ldcg(xs_in + q * XS) : kNegBig;
+              ls[x] = q < c1.nch ? __ldcg(xs_in + q * XS + 1) : 0.f;
+            }
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              if (q0 + x * TPRX < c1.nch) merge_stat(M, S, lm[x], ls[x]);
+          }
           mpart[2 * ctid] = M;
           mpart[2 * ctid + 1] = S;
         }
-        named_bar_sync(2, 128);
+        named_bar_sync(2, NP2);
         if (ctid < RP) {
+          constexpr int TPRX = NP2 / RP;
           float M = kNegBig, S = 0.f;
 #pragma unroll
-          for (int tt = 0; tt < TPR; ++tt)
-            merge_stat(M, S, mpart[2 * (ctid * TPR + tt)], mpart[2 * (ctid * TPR + tt) + 1]);
-          mrow[ctid] = M;
-          invl[ctid] = S > 0.f ? 1.f / S : 0.f;
+          for (int tt = 0; tt < TPRX; ++tt)
+            merge_stat(M, S, mpart[2 * (ctid * TPRX + tt)], mpart[2 * (ctid * TPRX + tt) + 1]);
+          mfin[2 * ctid] = M;
+          mfin[2 * ctid + 1] = S > 0.f ? 1.f / S : 0.f;
         }
-        named_bar_sync(2, 128);
+        named_bar_sync(2, NP2);
         RKV_STAMP(k, 3);
+        const float* mrow2 = mfin;   // (max, 1 / sum) per query row
         // p = 2^(y - M) / L = 2^(y - (M + log2 L)) for the NR rows this thread
         // holds; padding rows (and rows that see no key) get +inf there, so
         // they add exactly 0
@@ -633,8 +718,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int r = 8 * i + 2 * tq + e;
-            const bool real = ((rmask >> r) & 1u) != 0 && invl[r] > 0.f;
-            ML[2 * i + e] = real ? mrow[r] - __log2f(invl[r]) : INFINITY;
+            const float il = mrow2[2 * r + 1];
+            const bool real = ((rmask >> r) & 1u) != 0 && il > 0.f;
+            ML[2 * i + e] = real ? mrow2[2 * r] - __log2f(il) : INFINITY;
           }
         float* ab = abuf + buf * CHT;
         float part = 0.f;
@@ -642,7 +728,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         long long c_tw2 = 0;
         const long long c_p2 = clock64();
 #endif
-        for (int t = 0; t < c1.nt; ++t) {
+        for (int t = tp; t < c1.nt; t += NPAR) {
           const int t0 = c1.start + kTile * t;
           const bool inside = t0 + kTile <= c1.c;
           float sum[4];   // tokens qd, qd + 8, 16 + qd, 24 + qd of the quarter
@@ -717,68 +803,30 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         RKV_STAMP(k, 4);
 
         part = warp_reduce_sum(part);
-        if (lane == 0) psum[q4] = part;
-        named_bar_sync(2, 128);
+        if (lane == 0) psum[tp * 4 + q4] = part;
+        named_bar_sync(2, NP2);
         if (ctid == 0) {
           float* xo = p.xsum + static_cast<int64_t>(c1.g) * (2 * kScoreMaxGroups) + 2 * p.group;
-          xo[0] = (psum[0] + psum[1]) + (psum[2] + psum[3]);
+          float sa = (psum[0] + psum[1]) + (psum[2] + psum[3]);
+          if (NPAR > 1) sa += (psum[4] + psum[5]) + (psum[6] + psum[7]);
+          xo[0] = sa;
           if (red) {
             __threadfence();
             atomicAdd(&p.cnt[c1.u * kScoreCnt + 2 * p.group + 1], 1);
+            mbar_arrive(&sfull[buf]);   // the output warps may write this chunk out
           }
         }
         if (!red) {
           // an earlier row group: add this group's probabilities to a (not yet
           // normalised); the last group normalises
-          for (int i = ctid; i < c1.len; i += 128) {
+          for (int i = ctid; i < c1.len; i += NP2) {
             const int j = c1.start + i;
             const int64_t gi = c1.base + j;
             if (j < c1.c) p.a_out[gi] = p.group > 0 ? p.a_out[gi] + ab[i] : ab[i];
           }
         }
       }
-      // ---- WS(x_k-2) and a of x_k-2
-      if (red && c2.g >= 0) {
-        const int buf = k & 1;   // slot of x_k-2
-        if (warp == 8) {
-          if (lane == 0)
-            wait_count(&p.cnt[c2.u * kScoreCnt + 2 * p.group + 1], nann * c2.nch, abort,
-                       p.status, p.abort_all, p.wait_ns);
-          __syncwarp();
-          // sum over the unit's chunks and row groups, fixed order
-          float sa = 0.f;
-          for (int q = lane; q < c2.nch; q += 32) {
-            const float* xi = p.xsum + static_cast<int64_t>(c2.g0 + q) * (2 * kScoreMaxGroups);
-            float x = 0.f;
-            for (int gq = 0; gq <= p.group; ++gq) x += __ldcg(xi + 2 * gq);
-            sa += x;
-          }
-          sa = warp_reduce_sum(sa);
-          if (lane == 0) psum[8] = sa > 0.f ? 1.f / sa : 0.f;
-        }
-        RKV_STAMP(k, 5);
-        named_bar_sync(2, 128);
-        const float inv_sa = psum[8];
-        const float* ab = abuf + buf * CHT;
-        for (int i = ctid; i < c2.len; i += 128) {
-          const int j = c2.start + i;
-          const int64_t gi = c2.base + j;
-          if (j < c2.c) {
-            float x = ab[i];
-            if (p.group > 0) x = p.a_out[gi] + x;
-            p.a_out[gi] = x * inv_sa;
-          } else {
-            p.a_out[gi] = 0.f;
-            if (!CLOSED) {   // the redundancy GEMM writes the candidates' r and m
-              p.r_out[gi] = 0.f;
-              if (p.m_out) p.m_out[gi] = 0.f;
-            }
-          }
-        }
-        named_bar_sync(2, 128);   // psum and the slot are reused
-        RKV_STAMP(k, 6);
-      }
-      c2 = red ? c1 : no_chunk();
+      named_bar_sync(2, NP2);   // psum is reused
       c1 = have ? chunk_info(p, g) : no_chunk();
     }
   } else if (warp >= 12 && red) {
@@ -798,7 +846,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     int stage = 0;
     uint32_t ph = 0;
     int ntile = 0;
-    Chunk c1 = no_chunk(), c2 = no_chunk();
+    Chunk c1 = no_chunk();
     // U += rho_row * k_row over the warp's 32 rows of a tile
     auto u_accumulate = [&](uint32_t sb, float rho, float (&U4)[4]) {
       float* rt = rhot + (ntile & 1) * 128;
@@ -827,7 +875,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     for (int k = 0;; ++k) {
       const int g = b0 + k * P;
       const bool have = g < p.total_chunks;
-      if (!have && c1.g < 0 && c2.g < 0) break;
+      if (!have && c1.g < 0) break;
       const Chunk cur = have ? chunk_info(p, g) : no_chunk();
       // ---- pass 1 of x_k
       if (have) {
@@ -878,17 +926,19 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           if (ctid == 0)
             wait_count(&p.cnt[c1.u * kScoreCnt + 2 * p.group], nann * c1.nch, abort, p.status,
                        p.abort_all, p.wait_ns);
+          mbar_wait(&sfree[slot], (((k - 1) >> 1) & 1) ^ 1, abort, p.status);
           named_bar_sync(3, 128);
           {
-            const float* xs_in = p.xstat + static_cast<int64_t>(c1.g0) * XS + 2 * RP + ctid;
-            float acc0 = 0.f, acc1 = 0.f;
-            int q = 0;
-            for (; q + 1 < c1.nch; q += 2) {   // two independent loads in flight
-              acc0 += __ldcg(xs_in + q * XS);
-              acc1 += __ldcg(xs_in + (q + 1) * XS);
+            // thread = one dimension of U, the unit's chunks in order
+            const float* ui = p.xstat + static_cast<int64_t>(c1.g0) * XS + 2 * RP + ctid;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int q0 = 0; q0 < c1.nch; q0 += 8) {
+#pragma unroll
+              for (int x = 0; x < 8; ++x)
+                if (q0 + x < c1.nch) acc[x] += __ldcg(ui + (q0 + x) * XS);
             }
-            if (q < c1.nch) acc0 += __ldcg(xs_in + q * XS);
-            ufin[ctid] = acc0 + acc1;
+            ufin[ctid] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
+                         ((acc[4] + acc[5]) + (acc[6] + acc[7]));
           }
           named_bar_sync(3, 128);
           const float inv_nm1 = c1.n > 1 ? 1.f / static_cast<float>(c1.n - 1) : 0.f;
@@ -936,41 +986,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             *xo = (esum[0] + esum[1]) + (esum[2] + esum[3]);
             __threadfence();
             atomicAdd(&p.cnt[c1.u * kScoreCnt + 2 * p.group + 1], 1);
+            mbar_arrive(&sfull[slot]);
           }
+          named_bar_sync(3, 128);   // esum is reused
         }
-        // ---- WS(x_k-2): r and m of x_k-2
-        if (c2.g >= 0) {
-          const int slot = k & 1;
-          if (warp == 12) {
-            if (lane == 0)
-              wait_count(&p.cnt[c2.u * kScoreCnt + 2 * p.group + 1], nann * c2.nch, abort,
-                         p.status, p.abort_all, p.wait_ns);
-            __syncwarp();
-            float se = 0.f;
-            for (int q = lane; q < c2.nch; q += 32)
-              se += __ldcg(p.xsum + static_cast<int64_t>(c2.g0 + q) * (2 * kScoreMaxGroups) +
-                           2 * p.group + 1);
-            se = warp_reduce_sum(se);
-            if (lane == 0) esum[8] = se > 0.f ? 1.f / se : 0.f;
-          }
-          named_bar_sync(3, 128);
-          const float inv_se = esum[8];
-          const float* ma = marr + slot * CHT;
-          for (int i = ctid; i < c2.len; i += 128) {
-            const int j = c2.start + i;
-            const int64_t gi = c2.base + j;
-            if (j < c2.c) {
-              const float m = ma[i];
-              p.r_out[gi] = ex2(m * kLog2e) * inv_se;
-              if (p.m_out) p.m_out[gi] = m;
-            } else {
-              p.r_out[gi] = 0.f;
-              if (p.m_out) p.m_out[gi] = 0.f;
-            }
-          }
-          named_bar_sync(3, 128);   // esum and the slot are reused
-        }
-        c2 = c1;
         c1 = cur;
       } else if (!have) {
         break;
@@ -1006,7 +1025,7 @@ cudaError_t score_configure(int rp, bool closed, int smem_bytes) {
 
 int score_max_ctas(int rp, bool closed, int smem_bytes) {
   int per = 0, dev = 0, nsm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, pick(rp, closed), kScoreThreads,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, pick(rp, closed), score_threads(closed),
                                                     smem_bytes) != cudaSuccess ||
       cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
@@ -1061,7 +1080,7 @@ cudaError_t launch_score(const CUtensorMap& kmap, const CUtensorMap& qmap, const
   const ScoreLayout L = score_layout(rp, closed, p.nstages);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kScoreThreads, 1, 1);
+  cfg.blockDim = dim3(score_threads(closed), 1, 1);
   cfg.dynamicSmemBytes = L.total + 1024;
   cfg.stream = st;
   cudaLaunchAttribute at[1];
