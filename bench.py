@@ -440,8 +440,12 @@ def measure_lambda_sweep(eng, batch: Batch, wl: W.Workload, args, dist: Dist, al
 
 def measure_adaptive(eng, batch: Batch, wl: W.Workload, args, dist: Dist, alg, pk, src):
     """The step with the adaptive budget: rkv_refree_budget (T = 1%, 4 sinks,
-    budgets capped at the workload's B) -> score -> rkv_select_ex -> compact."""
-    sinks, T = 4, 0.01
+    budgets capped at the workload's B) -> score -> rkv_select_ex -> compact.
+    The queries are scaled by 3 so that attention is peaked, as in a trained
+    model; with the workload's unit-variance queries nearly every unit would
+    need the whole cap and the budgets would not vary."""
+    sinks, T, q_scale = 4, 0.01, 3.0
+    batch = Batch(batch.K, batch.V, batch.Q * q_scale, batch.tok_off_host)
     a, r = eng.alloc_scores(batch)
     U, Wd = batch.num_units, wl.budget + sinks + wl.window
     dev = batch.K.device
@@ -463,7 +467,7 @@ def measure_adaptive(eng, batch: Batch, wl: W.Workload, args, dist: Dist, alg, p
     rep = kernel_report(per_kernel, alg, pk, src)
     b = budgets.cpu().numpy()
     return {"value": batch.num_tokens * dist.world / (ms * 1e-3), "ms_per_step": ms,
-            "T": T, "sinks": sinks, "budget_mean": float(b.mean()),
+            "T": T, "sinks": sinks, "query_scale": q_scale, "budget_mean": float(b.mean()),
             "budget_min": int(b.min()), "budget_max": int(b.max()),
             "kernels": {k: rep[k] for k in ("refree", "select", "compact") if k in rep}}
 

@@ -53,7 +53,8 @@ def attention_probs(Q: np.ndarray, K: np.ndarray) -> np.ndarray:
     cached token).  Masked entries are exactly 0."""
     G, w, d = Q.shape
     N = K.shape[0]
-    z = np.einsum("gtd,nd->gtn", Q, K) / np.sqrt(d)
+    # every logit q_{g,t} . k_j at once: one [G*w, d] x [d, N] matrix product
+    z = (Q.reshape(G * w, d) @ K.T).reshape(G, w, N) / np.sqrt(d)
     pos = N - w + np.arange(w)                       # position of query t
     visible = np.arange(N)[None, :] <= pos[:, None]  # [w, N]
     z = np.where(visible[None], z, -np.inf)

@@ -142,3 +142,114 @@ def check_unit(out, batch: Batch, u, w, lam, budget, redundancy="closed", check_
     assert torch.count_nonzero(Kc[nk:].view(torch.int16)) == 0
     assert torch.count_nonzero(Vc[nk:].view(torch.int16)) == 0
     return dict(a=a_o, r=r_o, m=m_o, s=s_o)
+
+
+def _kept_set_valid(s, got, c, budget):
+    """True when ``got`` (the engine's ascending candidate ids, ``budget`` of
+    them) is a top-``budget`` set of ``s`` up to the near-tie band: every kept
+    score is >= the budget-th largest minus the band and every dropped one <=
+    it plus the band.  The same test as the set comparison in
+    :func:`check_unit`, without sorting all c scores."""
+    sb = -np.partition(-s, budget - 1)[budget - 1]
+    band = SEL_BAND * np.max(np.abs(s))
+    kept = np.zeros(c, bool)
+    kept[got] = True
+    ok = s[kept].min() >= sb - band
+    if c > budget:
+        ok = ok and s[~kept].max() <= sb + band
+    return ok
+
+
+def check_all_units(batch: Batch, group, w, budget, lambdas, mode, threads=8,
+                    block_tokens=1 << 22):
+    """Every unit of ``batch`` against the oracle: one engine score call in
+    ``mode``, then select + compact for each lambda.  a, r, m of every
+    candidate within the tolerance (window rows exactly 0); the kept set of
+    every unit and lambda valid up to the tie band, ascending, the window
+    after it, -1 past nk; K'/V' bit-exact gathers of the engine's own indices
+    (checked on the device).  The oracle (importance and the O(N d) closed
+    form of the row mean) runs unit by unit on ``threads`` host threads."""
+    from concurrent.futures import ThreadPoolExecutor
+    if mode == "gemm_sym":
+        eng = Engine(group, w, max_units=batch.num_units, max_tokens=batch.num_tokens,
+                     redundancy="gemm", symmetric_gemm=True)
+    else:
+        eng = Engine(group, w, max_units=batch.num_units, max_tokens=batch.num_tokens,
+                     redundancy=mode)
+    U = batch.num_units
+    off = batch.tok_off_host
+    a, r = eng.alloc_scores(batch)
+    m = torch.full_like(a, float("nan"))
+    eng.score(batch, a, r, m)
+    eng.check_status()
+    ah, rh, mh = (t.cpu().numpy() for t in (a, r, m))
+    del m
+    idx_h, nk_h = [], []
+    off_dev = torch.from_numpy(off[:-1].astype(np.int64)).to(batch.K.device)
+    for lam in lambdas:
+        idx, nk, Ko, Vo = eng.alloc_outputs(batch, budget)
+        eng.select(batch, a, r, lam, budget, idx, nk)
+        eng.compact(batch, idx, nk, budget, Ko, Vo)
+        eng.check_status()
+        # compaction, on the device, in blocks of units
+        ub = max(1, (1 << 28) // (Ko.shape[1] * 256))
+        for u0 in range(0, U, ub):
+            u1 = min(U, u0 + ub)
+            ib = idx[u0:u1].long()
+            valid = ib >= 0
+            assert torch.equal(valid.sum(1).int(), nk[u0:u1]), "nk disagrees with the -1 fill"
+            src = (ib + off_dev[u0:u1, None]).clamp(min=0)
+            for X, Xo in ((batch.K, Ko), (batch.V, Vo)):
+                want = X[src].view(torch.int16)
+                want[~valid] = 0
+                assert torch.equal(Xo[u0:u1].view(torch.int16), want), \
+                    f"lambda {lam}: compaction differs in units {u0}..{u1 - 1}"
+        idx_h.append(idx.cpu().numpy())
+        nk_h.append(nk.cpu().numpy())
+        del idx, nk, Ko, Vo
+    del a, r
+    eng.close()
+    torch.cuda.empty_cache()
+    Qh = batch.Q.double().cpu().numpy()
+
+    def one(u, k):
+        N = k.shape[0]
+        c = N - w
+        lo = int(off[u])
+        _, a_o = ora.importance(Qh[u], k)
+        m_o, r_o = ora.redundancy_mean_closed_form(k, w)
+        close(ah[lo:lo + c], a_o, f"unit {u} a")
+        close(rh[lo:lo + c], r_o, f"unit {u} r")
+        close(mh[lo:lo + c], m_o, f"unit {u} m")
+        assert np.all(ah[lo + c:lo + N] == 0) and np.all(rh[lo + c:lo + N] == 0), \
+            f"unit {u}: window rows must be 0"
+        for li, lam in enumerate(lambdas):
+            nk = int(nk_h[li][u])
+            got = idx_h[li][u]
+            assert np.all(got[nk:] == -1), f"unit {u}: -1 fill"
+            got = got[:nk]
+            if c <= budget:
+                assert np.array_equal(got, np.arange(N)), f"unit {u} lambda {lam}: keep all"
+                continue
+            assert nk == budget + w
+            assert np.all(np.diff(got) > 0), f"unit {u} lambda {lam}: not ascending"
+            assert np.array_equal(got[budget:], np.arange(c, N)), f"unit {u}: window"
+            s = ora.joint_score(a_o, r_o, lam)
+            assert _kept_set_valid(s, got[:budget], c, budget), \
+                f"unit {u} lambda {lam}: kept set differs outside the tie band"
+        return u
+
+    with ThreadPoolExecutor(threads) as ex:
+        u0 = 0
+        while u0 < U:
+            u1 = u0 + 1
+            while u1 < U and off[u1 + 1] - off[u0] <= block_tokens:
+                u1 += 1
+            Kh = batch.K[int(off[u0]):int(off[u1])].cpu()   # one copy per block
+            futs = [ex.submit(lambda u=u: one(u, Kh[int(off[u] - off[u0]):
+                                                     int(off[u + 1] - off[u0])].double().numpy()))
+                    for u in range(u0, u1)]
+            for f in futs:
+                f.result()
+            u0 = u1
+    return U

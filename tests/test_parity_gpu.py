@@ -1,6 +1,6 @@
 """GPU engine vs the fp64 oracle, through the C ABI (see tests/parity.py for the
 tolerances).  Ordered from the integer kernels (select, compaction) to the
-score kernels, then edge cases, then the full-size workloads on sampled units."""
+score kernels, then edge cases, then the full-size workloads on sampled units and on every unit."""
 import json
 import os
 
@@ -12,7 +12,7 @@ from decode_kv_cache_eviction_b200 import Batch, Engine, RkvError
 from decode_kv_cache_eviction_b200 import workloads as W
 from oracle import rkv_oracle as ora
 
-from parity import check_unit, make_batch, oracle_mode, rand_batch, run_engine
+from parity import check_all_units, check_unit, make_batch, oracle_mode, rand_batch, run_engine
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -133,7 +133,7 @@ def test_worked_example_on_gpu():
     Q *= 8.0
     t = lambda x: torch.from_numpy(x).to(DEV).to(torch.bfloat16)
     b = Batch(t(K), t(K), t(Q), np.array([0, 6]))
-    for mode in ("closed", "gemm"):
+    for mode in ("closed", "gemm", "gemm_sym"):
         for lam, want in g["idx"].items():
             out = run_engine(b, 1, 2, float(lam), 2, mode=mode)
             np.testing.assert_allclose(out["a"][:4], g["a"], atol=5e-6)
@@ -345,4 +345,19 @@ def test_workload_long_trace_32k_sampled():
 
 @pytest.mark.slow
 def test_workload_ragged_serving_sampled():
-    _sampled("ragged_serving", 8, modes=("gemm", "closed", "max"))
+    _sampled("ragged_serving", 8, modes=("gemm", "closed", "max", "gemm_sym"))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,mode", [("r1_llama8b_cache", "gemm_sym"),
+                                       ("long_trace_32k", "gemm_sym"),
+                                       ("long_trace_32k", "closed"),
+                                       ("ragged_serving", "gemm_sym"),
+                                       ("ragged_serving", "closed")])
+def test_workload_all_units(name, mode):
+    """Every unit of the full-size workload (the bench's inputs, seed 0) against
+    the oracle, at each of the workload's lambdas (0, 0.1 and 1 for the ragged
+    serving batch)."""
+    wl = W.WORKLOADS[name]
+    b = make_batch(W.generate(wl, seed=0, device=DEV))
+    assert check_all_units(b, wl.group, wl.window, wl.budget, wl.lambdas, mode) == wl.num_units
