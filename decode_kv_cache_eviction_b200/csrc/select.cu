@@ -1,28 +1,31 @@
 // Joint eviction (R-KV 联合淘汰): s_i = lambda * a_i - (1 - lambda) * r_i and a
 // deterministic top-B of the candidates: the B largest by (s descending, index
-// ascending), written in ascending index order.
+// ascending), written in ascending index order.  A NaN score ranks below every
+// number (ties among NaNs by index, like the other ties).
 //
 // One CTA per unit (several CTAs share an SM).  s is mapped to an
-// order-preserving uint32 key; keys are recomputed from a and r wherever they
-// are needed, so a unit of any length needs no shared-memory copy of them.
-//   1. Sample: the keys of S candidates in evenly spaced blocks of 8 (whole
-//      32-byte sectors).  Two order statistics of the sample, about four
-//      standard deviations of the sampling error above and below the budget's
-//      rank, give splitters hi >= lo.
+// order-preserving uint32 key where a key is needed; a unit of any length needs
+// no shared-memory copy of its scores.
+//   1. Sample: the keys of S candidates in evenly spaced blocks of 16 (whole
+//      64-byte segments of a and of r).  Two order statistics of the sample,
+//      about four standard deviations of the sampling error above and below the
+//      budget's rank, give splitters hi >= lo (as keys and as floats).
 //   2. Classify (the one pass that reads a and r from HBM): every candidate is
-//      above the bracket (key > hi, kept for sure), inside it (lo <= key <= hi,
-//      appended with its index to a short list) or below.  A warp handles runs
-//      of 32 consecutive candidates, sixteen runs' loads in flight at once, so
-//      the "above" ballot of a run is directly one 32-bit word of the kept
-//      bitmap.
+//      above the bracket (s > hi, kept for sure), inside it (lo <= s <= hi,
+//      appended with its index to a short list) or below.  A warp takes runs of
+//      128 positions, lane l the aligned float4 of positions 4l .. 4l+3 of a
+//      and of r, four runs' loads in flight.  Plain float compares against the
+//      splitters decide (the key order is the float order); only list entries
+//      get a key.  List slots come from four ballots per run and one shared
+//      atomic per warp and run.
 //   3. If the budget's rank falls inside the bracket and the list fits, the
 //      exact threshold key T and the tie cut (keys equal to T are taken lowest
 //      index first) are found by radix selection on the list alone, and the
 //      kept list entries are added to the bitmap.  Otherwise (rare: many equal
 //      keys, or a sample far from the data) the same selection runs over all
 //      candidates, reading a and r again.
-//   4. The bitmap is turned into ascending indices: one block-wide prefix of
-//      the words' popcounts, then each thread writes the set bits of its words.
+//   4. The bitmap is turned into ascending indices: each warp takes a
+//      contiguous share of the words, one word per lane at a time.
 // Optional extensions: the first `sinks` tokens are always kept and excluded
 // from the ranking (attention sinks), and each unit may have its own budget
 // (budgets[u], clamped to 0 .. budget).  Row u of idx has stride W and ends in
@@ -35,8 +38,8 @@ namespace {
 
 #ifdef RKV_TRACE
 // Optional phase trace (build with -DRKV_TRACE): globaltimer stamps of the
-// first kStCtas units' phases.
-constexpr int kStCtas = 64, kStSlots = 8;
+// first kStCtas units' phases (slot 6: the SM, slot 7: kernel entry).
+constexpr int kStCtas = 1024, kStSlots = 8;
 __device__ unsigned long long g_sel_trace[kStCtas * kStSlots];
 #define RKV_SSTAMP(slot)                                                                  \
   do {                                                                                    \
@@ -53,19 +56,24 @@ constexpr int kSample = 2048;     // sample size (at most the candidate count)
 constexpr int kListCap = 3072;    // bracket entries kept on chip
 constexpr float kSpread = 4.f;    // bracket half-width in sampling standard deviations
 
+// Order-preserving key of a score: -0 and +0 get the key of +0, a NaN key 0
+// (below every number's key, which is at least that of -inf, 0x007fffff).
 __device__ __forceinline__ uint32_t order_key(float s) {
-  uint32_t b = __float_as_uint(s);
-  if ((b << 1) == 0) b = 0;  // -0 and +0 compare equal
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  const uint32_t b = __float_as_uint(__fadd_rn(s, 0.f));   // -0 + 0 = +0
+  const uint32_t k = b ^ (static_cast<uint32_t>(static_cast<int32_t>(b) >> 31) | 0x80000000u);
+  return s == s ? k : 0u;
+}
+// The float whose key is k (k = 0 gives a NaN, which no compare accepts).
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
 struct SelShared {
   uint32_t hist[512];
   union {                        // the sample is done with before the list fills
     uint32_t sample[kSample];
-    uint32_t lkey[kListCap];
+    uint2 list[kListCap];        // bracket entries: (score bits, candidate index)
   };
-  int32_t lidx[kListCap];
   int nlist;
   int cnt_above;
   int sh[8];
@@ -262,6 +270,14 @@ __global__ void __launch_bounds__(kSelThreads, 7)
   const float lw = lam, rw = 1.f - lam;
   const int u = blockIdx.x;
   if (u >= U) return;
+#ifdef RKV_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < kStCtas) {
+    g_sel_trace[blockIdx.x * kStSlots + 7] = globaltimer_ns();
+    unsigned smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    g_sel_trace[blockIdx.x * kStSlots + 6] = smid;
+  }
+#endif
 
   const int64_t tbase = tok_off[u];
   const int N = static_cast<int>(tok_off[u + 1] - tbase);
@@ -303,21 +319,45 @@ __global__ void __launch_bounds__(kSelThreads, 7)
   const int nruns = (npos + 127) >> 7;
   const int nwords = (npos + 31) >> 5;
 
-  // ---- 1. sample and splitters: S / 8 evenly spaced blocks of 8 consecutive
-  // candidates (whole 32-byte sectors of a and r), S about c / 8 within
-  // [256, kSample]
-  const int S = min(c, min(kSample, max(256, ((c / 8) + 7) & ~7)));
+  // runs [run_lo, run_hi) take 128-bit loads: every element they touch lies in
+  // [0, T) (p0 >= -3, so only run 0 can start before the array)
+  int run_lo = 0, run_hi = 0;
+  if (vec_ok) {
+    run_lo = p0 >= 0 ? 0 : 1;
+    run_hi = static_cast<int>(min(static_cast<int64_t>(nruns), (Ttot - p0) / 128));
+  }
+  // lane's float4 of run run_lo (in bounds whenever run_lo < run_hi)
+  const int64_t g_lo = p0 + static_cast<int64_t>(run_lo) * 128 + 4 * lane;
+  const float4* a4 = reinterpret_cast<const float4*>(a + (run_lo < run_hi ? g_lo : 0));
+  const float4* r4 = reinterpret_cast<const float4*>(r + (run_lo < run_hi ? g_lo : 0));
+  constexpr int kRuns = 4;   // runs per warp and iteration of the classification
+  // the warp's first classification iteration into L2 while the sample and
+  // the splitters are worked out
+  if ((lane & 7) == 0) {
+#pragma unroll
+    for (int x = 0; x < kRuns; ++x) {
+      const int run = wp * kRuns + x;
+      if (run >= run_lo && run < run_hi) {
+        prefetch_l2(a4 + 32 * (run - run_lo));
+        prefetch_l2(r4 + 32 * (run - run_lo));
+      }
+    }
+  }
+
+  // ---- 1. sample and splitters: S / 16 evenly spaced blocks of 16 consecutive
+  // candidates (64-byte segments of a and r), S about c / 8 within
+  // [256, kSample]; every candidate when S = c
+  const int S = min(c, min(kSample, max(256, ((c / 8) + 15) & ~15)));
   {
-    const int nblk = S / 8;
+    const int nblk = S >> 4;
+    const float step = nblk > 1 ? static_cast<float>(c - 16) / static_cast<float>(nblk - 1) : 0.f;
     constexpr int kPer = kSample / kSelThreads;   // sample keys per thread (at most)
     float sa[kPer], sr[kPer];
 #pragma unroll
     for (int x = 0; x < kPer; ++x) {   // every load first, then the keys
       const int j = tid + x * kSelThreads;
-      int i = j;   // fewer than 8 candidates in a block's place: take them all
-      if (j < nblk * 8)
-        i = static_cast<int>((static_cast<int64_t>(j >> 3) * (c - 8)) / max(nblk - 1, 1)) +
-            (j & 7);
+      int i = j;   // all candidates, or fewer than 16 in a block's place: take them
+      if (S < c && j < nblk * 16) i = static_cast<int>(static_cast<float>(j >> 4) * step) + (j & 15);
       i = min(i, c - 1);
       sa[x] = j < S ? __ldg(au + i) : 0.f;
       sr[x] = j < S ? __ldg(ru + i) : 0.f;
@@ -353,22 +393,24 @@ __global__ void __launch_bounds__(kSelThreads, 7)
   // offset of candidate 0 within its 16-byte group of scores, so that a run of
   // 128 positions is 32 aligned float4 of a and of r: lane l takes positions
   // 4l .. 4l+3, and the kept bitmap is kept per position (bit p).  Runs that
-  // would read outside [0, T) take bounds-checked scalar loads.
-  constexpr int kRuns = 4;   // runs per warp and iteration, all loads in flight
+  // would read outside [0, T) take bounds-checked scalar loads.  s > f_hi and
+  // lo <= key(s) <= hi are float compares (false for a NaN, whose key is the
+  // lowest); only the list entries' keys are formed.
+  const float f_hi = key_float(hi), f_lo = key_float(lo);
   int above = 0;
   for (int r0 = wp * kRuns; r0 < nruns; r0 += kSelWarps * kRuns) {
     float4 A[kRuns], R[kRuns];
 #pragma unroll
     for (int x = 0; x < kRuns; ++x) {
-      const int64_t ge = p0 + static_cast<int64_t>(r0 + x) * 128 + 4 * lane;   // element of a, r
-      if (r0 + x < nruns && ge >= 0 && ge + 3 < Ttot && vec_ok) {
-        A[x] = __ldg(reinterpret_cast<const float4*>(a + ge));
-        R[x] = __ldg(reinterpret_cast<const float4*>(r + ge));
-      } else {
+      const int run = r0 + x;
+      if (run >= run_lo && run < run_hi) {
+        A[x] = __ldg(a4 + 32 * (run - run_lo));
+        R[x] = __ldg(r4 + 32 * (run - run_lo));
+      } else if (run < nruns) {
         float ta[4], tr[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int i = (r0 + x) * 128 + 4 * lane + e - delta;
+          const int i = run * 128 + 4 * lane + e - delta;
           ta[e] = (i >= 0 && i < c) ? __ldg(au + i) : 0.f;
           tr[e] = (i >= 0 && i < c) ? __ldg(ru + i) : 0.f;
         }
@@ -376,49 +418,63 @@ __global__ void __launch_bounds__(kSelThreads, 7)
         R[x] = make_float4(tr[0], tr[1], tr[2], tr[3]);
       }
     }
+    // the warp's next iteration into L2 while this one is processed (one
+    // prefetch per 128-byte line)
+    if ((lane & 7) == 0) {
+#pragma unroll
+      for (int x = 0; x < kRuns; ++x) {
+        const int run = r0 + kSelWarps * kRuns + x;
+        if (run >= run_lo && run < run_hi) {
+          prefetch_l2(a4 + 32 * (run - run_lo));
+          prefetch_l2(r4 + 32 * (run - run_lo));
+        }
+      }
+    }
 #pragma unroll
     for (int x = 0; x < kRuns; ++x) {
-      if (r0 + x >= nruns) break;
+      const int run = r0 + x;
+      if (run >= nruns) break;
       const float av[4] = {A[x].x, A[x].y, A[x].z, A[x].w};
       const float rv[4] = {R[x].x, R[x].y, R[x].z, R[x].w};
-      uint32_t nab = 0, nin = 0, keys[4];
-      const int i0 = (r0 + x) * 128 + 4 * lane - delta;
+      const int i0 = run * 128 + 4 * lane - delta;
+      float sv[4];
+      uint32_t nab = 0, nin = 0;
+      if (run * 128 >= delta && run * 128 + 128 - delta <= c) {
+        // every position of the run holds a candidate
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool v = i0 + e >= 0 && i0 + e < c;
-        const uint32_t k = order_key(__fsub_rn(__fmul_rn(lw, av[e]), __fmul_rn(rw, rv[e])));
-        keys[e] = k;
-        nab |= (v && k > hi) ? (1u << e) : 0u;
-        nin |= (v && k >= lo && k <= hi) ? (1u << e) : 0u;
+        for (int e = 0; e < 4; ++e) {
+          sv[e] = __fsub_rn(__fmul_rn(lw, av[e]), __fmul_rn(rw, rv[e]));
+          const bool g = sv[e] > f_hi;
+          nab |= g ? (1u << e) : 0u;
+          nin |= (!g && sv[e] >= f_lo) ? (1u << e) : 0u;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          sv[e] = __fsub_rn(__fmul_rn(lw, av[e]), __fmul_rn(rw, rv[e]));
+          const bool v = i0 + e >= 0 && i0 + e < c;
+          const bool g = sv[e] > f_hi;
+          nab |= (v && g) ? (1u << e) : 0u;
+          nin |= (v && !g && sv[e] >= f_lo) ? (1u << e) : 0u;
+        }
       }
-      // bitmap word 4 (r0 + x) + l / 8 holds the nibbles of lanes 8 (l / 8) ..
+      // bitmap word 4 run + l / 8 holds the nibbles of lanes 8 (l / 8) ..
       uint32_t wv = nab << (4 * (lane & 7));
       wv |= __shfl_xor_sync(0xffffffffu, wv, 1);
       wv |= __shfl_xor_sync(0xffffffffu, wv, 2);
       wv |= __shfl_xor_sync(0xffffffffu, wv, 4);
-      if ((lane & 7) == 0) bits[(r0 + x) * 4 + (lane >> 3)] = wv;
+      if ((lane & 7) == 0) bits[run * 4 + (lane >> 3)] = wv;
       above += __popc(nab);
-      // bracket entries go to the list (warp prefix of the counts)
-      const int cnt = __popc(nin);
-      if (__any_sync(0xffffffffu, cnt > 0)) {
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        int pos0 = 0;
-        if (lane == 31) pos0 = atomicAdd(&s.nlist, incl);
-        pos0 = __shfl_sync(0xffffffffu, pos0, 31);
-        int my = pos0 + incl - cnt;
+      // bracket entries (score bits, index): the lanes that have some take
+      // their slots with one shared atomic each
+      if (nin) {
+        int q = atomicAdd(&s.nlist, __popc(nin));
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           if ((nin >> e) & 1u) {
-            if (my < kListCap) {
-              s.lkey[my] = keys[e];
-              s.lidx[my] = i0 + e;
-            }
-            ++my;
+            if (q < kListCap)
+              s.list[q] = make_uint2(__float_as_uint(sv[e]), static_cast<uint32_t>(i0 + e));
+            ++q;
           }
       }
     }
@@ -434,7 +490,7 @@ __global__ void __launch_bounds__(kSelThreads, 7)
   if (want >= 1 && want <= nl && nl <= kListCap) {
     // ---- 3. exact threshold inside the bracket
     auto get_list = [&](int i, uint32_t& v) {
-      v = s.lkey[i];
+      v = order_key(__uint_as_float(s.list[i].x));
       return true;
     };
     int gt, eq;
@@ -446,15 +502,17 @@ __global__ void __launch_bounds__(kSelThreads, 7)
       // ... unless only some are: the take_eq-th smallest index among the list
       // keys equal to T (values ~index: the largest is the smallest index)
       auto get_tied = [&](int i, uint32_t& v) {
-        v = ~static_cast<uint32_t>(s.lidx[i]);
-        return s.lkey[i] == T;
+        const uint2 en = s.list[i];
+        v = ~en.y;
+        return order_key(__uint_as_float(en.x)) == T;
       };
       int dummy2;
       imax = static_cast<int>(~kth_largest(s, get_tied, nl, take_eq, 0u, 32, &dummy2));
     }
     for (int i = tid; i < nl; i += kSelThreads) {
-      const uint32_t k = s.lkey[i];
-      const int ii = s.lidx[i];
+      const uint2 en = s.list[i];
+      const uint32_t k = order_key(__uint_as_float(en.x));
+      const int ii = static_cast<int>(en.y);
       if (k > T || (k == T && ii <= imax))
         atomicOr(&bits[(ii + delta) >> 5], 1u << ((ii + delta) & 31));
     }
@@ -488,30 +546,38 @@ __global__ void __launch_bounds__(kSelThreads, 7)
   __syncthreads();
 
   RKV_SSTAMP(4);
-  // ---- 4. bitmap -> ascending indices
-  const int per = (nwords + kSelThreads - 1) / kSelThreads;
-  const int w0 = min(nwords, tid * per), w1 = min(nwords, w0 + per);
+  // ---- 4. bitmap -> ascending indices: warp wp takes a contiguous share of
+  // the words, one word per lane at a time
+  const int perw = (nwords + kSelWarps - 1) / kSelWarps;
+  const int w0 = min(nwords, wp * perw), w1 = min(nwords, w0 + perw);
   int cnt = 0;
-  for (int q = w0; q < w1; ++q) cnt += __popc(bits[q]);
-  // block exclusive scan of cnt
-  int incl = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) s.wred[wp] = static_cast<uint32_t>(incl);
+  for (int q = w0 + lane; q < w1; q += 32) cnt += __popc(bits[q]);
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if (lane == 0) s.wred[wp] = static_cast<uint32_t>(cnt);
   __syncthreads();
-  int wbase = 0;
-  for (int q = 0; q < wp; ++q) wbase += static_cast<int>(s.wred[q]);
-  int pos = wbase + incl - cnt;
-  for (int q = w0; q < w1; ++q) {
-    uint32_t x = bits[q];
-    while (x) {
-      const int b = __ffs(x) - 1;
+  int pos = 0;
+  for (int q = 0; q < wp; ++q) pos += static_cast<int>(s.wred[q]);
+  for (int q0 = w0; q0 < w1; q0 += 32) {
+    const int q = q0 + lane;
+    uint32_t x = q < w1 ? bits[q] : 0u;
+    const int n = __popc(x);
+    int incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int my = pos + incl - n;
+    pos += __shfl_sync(0xffffffffu, incl, 31);
+    const int ob = m + q * 32 - delta;   // index of bit 0 of the word
+    while (x) {   // two set bits per step
+      const int b0 = __ffs(x) - 1;
       x &= x - 1;
-      if (pos < budget) out[pos] = m + q * 32 + b - delta;
-      ++pos;
+      const int b1 = __ffs(x) - 1;   // -1: no second bit
+      x &= x - 1;
+      if (my < budget) out[my] = ob + b0;
+      if (b1 >= 0 && my + 1 < budget) out[my + 1] = ob + b1;
+      my += 2;
     }
   }
   RKV_SSTAMP(5);

@@ -143,7 +143,8 @@ int rkv_score(rkv_engine* eng, const rkv_batch* batch, float* a, float* r, float
 /* Joint eviction (R-KV 联合淘汰): s_i = lambda * a_i - (1 - lambda) * r_i for i in C
  * (fp32); keep the min(budget, N_u - w) candidates ranked first by (s descending,
  * index ascending), in ascending index order, followed by the window
- * N_u - w .. N_u - 1.  When N_u - w <= budget every token 0 .. N_u - 1 is kept.
+ * N_u - w .. N_u - 1.  -0 and +0 tie; a NaN score ranks below every number.
+ * When N_u - w <= budget every token 0 .. N_u - 1 is kept.
  *   idx [U, budget + w] int32: kept token indices (unit-local); unused slots -1;
  *   n_kept [U] int32: number of valid slots of each unit.
  * lambda must lie in [0, 1]; budget >= 0. */

@@ -50,6 +50,37 @@ def test_select_bit_exact_given_scores(lam, lengths, budget):
         assert np.all(idx[u, nk[u]:] == -1)
 
 
+@pytest.mark.parametrize("nan_frac", [0.1, 0.95])
+def test_select_nan_and_signed_zero_scores(nan_frac):
+    """A NaN score ranks below every number and -0 ties with +0 (index order),
+    as in the oracle's ranking; with most scores NaN the bracket cannot hold the
+    budget's rank and the selection runs over all candidates."""
+    w, budget = 8, 700
+    lengths = [5000, 3001, 700 + w + 5]
+    b = rand_batch(lengths, 1, w, seed=11)
+    rng = np.random.default_rng(12)
+    T = b.num_tokens
+    a = (rng.random(T).astype(np.float32) - 0.5) * 1e-3
+    r = rng.random(T).astype(np.float32) * 1e-3
+    a[rng.random(T) < nan_frac] = np.nan
+    z = rng.random(T) < 0.05           # exact zeros of either sign: s = +-0
+    a[z] = np.where(rng.random(z.sum()) < 0.5, np.float32(-0.0), np.float32(0.0))
+    r[z] = 0.0
+    eng = Engine(1, w, max_units=len(lengths), max_tokens=T, redundancy="closed")
+    ta, tr = torch.from_numpy(a).to(DEV), torch.from_numpy(r).to(DEV)
+    idx, nk, _, _ = eng.alloc_outputs(b, budget)
+    eng.select(b, ta, tr, 0.3, budget, idx, nk)
+    eng.check_status()
+    idx, nk = idx.cpu().numpy(), nk.cpu().numpy()
+    for u, N in enumerate(lengths):
+        r0 = int(b.tok_off_host[u])
+        c = N - w
+        s32 = ora.joint_score(a[r0:r0 + c], r[r0:r0 + c], np.float32(0.3))
+        want = ora.select(s32, N, w, budget)
+        assert nk[u] == len(want)
+        np.testing.assert_array_equal(idx[u, :nk[u]], want)
+
+
 @pytest.mark.parametrize("n,budget", [(40000, 1000), (3000, 2999), (9000, 1)])
 def test_select_all_scores_equal(n, budget):
     """Every score ties: the bracket around the budget's rank holds every
