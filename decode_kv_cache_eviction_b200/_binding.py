@@ -40,7 +40,7 @@ EXPORTS = ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact"
            "rkv_compress", "rkv_compress_host", "rkv_evict_in_place", "rkv_fill_slots",
            "rkv_select_ex", "rkv_refree_budget", "rkv_check_status", "rkv_launch_count", "rkv_set_timing",
            "rkv_read_timing", "rkv_score_noalloc", "rkv_noalloc_check_status", "rkv_inject_fault",
-           "rkv_status_string", "rkv_version")
+           "rkv_debug_intermediates", "rkv_status_string", "rkv_version")
 KERNELS = ("score", "plan", "gemm", "select", "compact", "evict", "fill", "refree")
 
 
@@ -106,6 +106,7 @@ def lib():
     L.rkv_score_noalloc.argtypes = [i32, i32, ctypes.POINTER(RkvBatch), vp, vp, vp, vp]
     L.rkv_noalloc_check_status.argtypes = [vp]
     L.rkv_inject_fault.argtypes = [vp, i32]
+    L.rkv_debug_intermediates.argtypes = [vp, ctypes.POINTER(RkvBatch), vp, vp, vp]
     L.rkv_status_string.argtypes = [i32]
     L.rkv_status_string.restype = ctypes.c_char_p
     L.rkv_version.argtypes = []
@@ -114,7 +115,7 @@ def lib():
                  "rkv_select_ex", "rkv_refree_budget", "rkv_check_status", "rkv_set_timing",
                  "rkv_read_timing",
                  "rkv_score_noalloc", "rkv_noalloc_check_status", "rkv_inject_fault",
-                 "rkv_version"):
+                 "rkv_debug_intermediates", "rkv_version"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -313,6 +314,12 @@ class Engine:
     def inject_fault(self, fault: int):
         """Arm a one-shot fault (RKV_FAULT_*) for testing error paths."""
         _check(lib().rkv_inject_fault(self.h, int(fault)), "rkv_inject_fault")
+
+    def debug_intermediates(self, batch: Batch, rho=None, U=None, stream=None):
+        """rho [T] and/or U [U, 128] of the last score call on this batch
+        (``rkv_debug_intermediates``)."""
+        _check(lib().rkv_debug_intermediates(self.h, ctypes.byref(batch.c), _ptr(rho), _ptr(U),
+                                             _stream(stream)), "rkv_debug_intermediates")
 
     def set_timing(self, enable: bool):
         _check(lib().rkv_set_timing(self.h, 1 if enable else 0), "rkv_set_timing")

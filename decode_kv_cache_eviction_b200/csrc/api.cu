@@ -125,6 +125,7 @@ const char* rkv_status_string(int s) {
 }
 
 int rkv_create(const rkv_config* cfg, rkv_engine** out) {
+  NvtxRange nvtx_("rkv_create");
   if (!cfg || !out) return RKV_ERR_INVALID_ARG;
   *out = nullptr;
   if (cfg->group < 1 || cfg->window < 1 || cfg->max_units < 1 || cfg->max_tokens < 1 ||
@@ -297,6 +298,7 @@ int rkv_read_timing(rkv_engine* e, int kernel, double* total_ms, int64_t* launch
 }
 
 int rkv_destroy(rkv_engine* e) {
+  NvtxRange nvtx_("rkv_destroy");
   if (!e) return RKV_OK;
   cudaDeviceSynchronize();
   if (e->ev_made)
@@ -336,6 +338,7 @@ int rkv_inject_fault(rkv_engine* e, int fault) {
 
 int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
               rkv_stream_t stream) {
+  NvtxRange nvtx_("rkv_score");
   if (!e) return RKV_ERR_INVALID_ARG;
   int64_t T = 0;
   int nmax = 0, cmax = 0;
@@ -473,6 +476,7 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
 
 int rkv_select(rkv_engine* e, const rkv_batch* b, const float* a, const float* r, float lambda,
                int budget, int32_t* idx, int32_t* n_kept, rkv_stream_t stream) {
+  NvtxRange nvtx_("rkv_select");
   if (!e) return RKV_ERR_INVALID_ARG;
   int64_t T = 0;
   int nmax = 0, cmax = 0;
@@ -500,6 +504,7 @@ int rkv_select(rkv_engine* e, const rkv_batch* b, const float* a, const float* r
 int rkv_select_ex(rkv_engine* e, const rkv_batch* b, const float* a, const float* r,
                   float lambda, int budget, const int32_t* budgets, int sinks, int32_t* idx,
                   int32_t* n_kept, rkv_stream_t stream) {
+  NvtxRange nvtx_("rkv_select_ex");
   if (!e) return RKV_ERR_INVALID_ARG;
   int64_t T = 0;
   int nmax = 0, cmax = 0;
@@ -527,6 +532,7 @@ int rkv_select_ex(rkv_engine* e, const rkv_batch* b, const float* a, const float
 
 int rkv_compact(rkv_engine* e, const rkv_batch* b, const int32_t* idx, const int32_t* n_kept,
                 int budget, void* K_out, void* V_out, rkv_stream_t stream) {
+  NvtxRange nvtx_("rkv_compact");
   if (!e) return RKV_ERR_INVALID_ARG;
   int64_t T = 0;
   int nmax = 0, cmax = 0;
@@ -554,6 +560,7 @@ int rkv_compact(rkv_engine* e, const rkv_batch* b, const int32_t* idx, const int
 int rkv_evict_in_place(rkv_engine* e, const rkv_batch* b, const int32_t* idx,
                        const int32_t* n_kept, int budget, uint8_t* keep, int32_t* free_slots,
                        int32_t* n_free, rkv_stream_t stream) {
+  NvtxRange nvtx_("rkv_evict_in_place");
   if (!e) return RKV_ERR_INVALID_ARG;
   int64_t T = 0;
   int nmax = 0, cmax = 0;
@@ -579,6 +586,7 @@ int rkv_evict_in_place(rkv_engine* e, const rkv_batch* b, const int32_t* idx,
 int rkv_fill_slots(rkv_engine* e, const rkv_batch* b, void* K, void* V, const int64_t* new_off,
                    const int64_t* new_off_host, const void* K_new, const void* V_new,
                    uint8_t* keep, int32_t* free_slots, int32_t* n_free, rkv_stream_t stream) {
+  NvtxRange nvtx_("rkv_fill_slots");
   if (!e) return RKV_ERR_INVALID_ARG;
   int64_t T = 0;
   int nmax = 0, cmax = 0;
@@ -610,6 +618,7 @@ int rkv_fill_slots(rkv_engine* e, const rkv_batch* b, void* K, void* V, const in
 int rkv_refree_budget(rkv_engine* e, const rkv_batch* b, float T, int sinks, int max_budget,
                       float* p_last, int32_t* budgets, int32_t* keep_count,
                       rkv_stream_t stream) {
+  NvtxRange nvtx_("rkv_refree_budget");
   if (!e) return RKV_ERR_INVALID_ARG;
   int64_t Tn = 0;
   int nmax = 0, cmax = 0;
@@ -646,6 +655,7 @@ int rkv_refree_budget(rkv_engine* e, const rkv_batch* b, float T, int sinks, int
 
 int rkv_compress(rkv_engine* e, const rkv_batch* b, float lambda, int budget, float* a, float* r,
                  int32_t* idx, int32_t* n_kept, void* K_out, void* V_out, rkv_stream_t stream) {
+  NvtxRange nvtx_("rkv_compress");
   if (!e) return RKV_ERR_INVALID_ARG;
   // validate everything before enqueuing anything
   int64_t T = 0;
@@ -664,7 +674,32 @@ int rkv_compress(rkv_engine* e, const rkv_batch* b, float lambda, int budget, fl
   return rkv_compact(e, b, idx, n_kept, budget, K_out, V_out, stream);
 }
 
+int rkv_debug_intermediates(rkv_engine* e, const rkv_batch* b, float* rho, float* U_out,
+                            rkv_stream_t stream) {
+  NvtxRange nvtx_("rkv_debug_intermediates");
+  if (!e) return RKV_ERR_INVALID_ARG;
+  int64_t T = 0;
+  int nmax = 0, cmax = 0;
+  int rc = check_batch(e, b, &T, &nmax, &cmax);
+  if (rc != RKV_OK) return rc;
+  if ((rho && !aligned(rho, 4)) || (U_out && !aligned(U_out, 4))) return RKV_ERR_INVALID_ARG;
+  const bool closed = e->cfg.redundancy == RKV_REDUNDANCY_CLOSED_FORM;
+  if ((rho && closed) || (U_out && !closed)) return RKV_ERR_UNSUPPORTED;
+  const int U = b->num_units;
+  if (U == 0) return RKV_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaSuccess;
+  if (rho) err = launch_gather_rho(b->tok_off, e->rho_off, U, e->rho, rho, st);
+  if (err == cudaSuccess && U_out)
+    err = launch_sum_unit_U(e->chunk_off, U, e->xstat, score_xs(e->rp, true), 2 * e->rp, U_out,
+                            st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  e->launches += (rho ? 1 : 0) + (U_out ? 1 : 0);
+  return RKV_OK;
+}
+
 int rkv_check_status(rkv_engine* e, rkv_stream_t stream) {
+  NvtxRange nvtx_("rkv_check_status");
   if (!e) return RKV_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return cuda_fail(cudaErrorUnknown);

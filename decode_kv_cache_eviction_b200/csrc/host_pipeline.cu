@@ -140,6 +140,7 @@ void rkv_host_pipeline_free(rkv_engine* e) {
 extern "C" int rkv_compress_host(rkv_engine* e, const rkv_host_batch* hb, float lambda,
                                  int budget, int32_t* idx, int32_t* n_kept, void* K_out,
                                  void* V_out, int64_t chunk_tokens, rkv_stream_t stream) {
+  rkv::NvtxRange nvtx_("rkv_compress_host");
   if (!e || !hb) return RKV_ERR_INVALID_ARG;
   const int U = hb->num_units;
   const int w = e->cfg.window;

@@ -146,6 +146,7 @@ int fail() {
 
 extern "C" int rkv_score_noalloc(int group, int window, const rkv_batch* b, float* a, float* r,
                                  float* m, rkv_stream_t stream) {
+  NvtxRange nvtx_("rkv_score_noalloc");
   if (group < 1 || window < 1 || !b || !a || !r) return RKV_ERR_INVALID_ARG;
   if (static_cast<int64_t>(group) * window > kMaxRp) return RKV_ERR_UNSUPPORTED;
   const int U = b->num_units;

@@ -3,9 +3,19 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 namespace rkv {
+
+// Host-side NVTX range around one public call (a named span in Nsight
+// Systems; a no-op without a tool attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kHeadDim = 128;        // d (the only supported head size)
 constexpr int kTile = 128;           // tokens per K tile (TMA box rows, MMA M)
@@ -231,6 +241,11 @@ cudaError_t launch_select(const int64_t* tok_off, int U, int64_t Ttot, int w, in
                           const float* r, float lam, int budget, const int32_t* budgets,
                           int sinks, int W, int32_t* idx, int32_t* n_kept, cudaStream_t st);
 cudaError_t select_configure();
+// Intermediate arrays of the last score call (rkv_debug_intermediates).
+cudaError_t launch_gather_rho(const int64_t* tok_off, const int64_t* rho_off, int U,
+                              const float* rho, float* out, cudaStream_t st);
+cudaError_t launch_sum_unit_U(const int* chunk_off, int U, const float* xstat, int xs, int u0,
+                              float* out, cudaStream_t st);
 
 cudaError_t launch_compact(const int64_t* tok_off, int U, int W, const int32_t* idx,
                            const int32_t* n_kept, const void* K, const void* V, void* Ko,

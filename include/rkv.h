@@ -281,6 +281,18 @@ int rkv_check_status(rkv_engine* eng, rkv_stream_t stream);
 enum { RKV_FAULT_NONE = 0, RKV_FAULT_ALLOC = 1, RKV_FAULT_DROP_ANNOUNCE = 2 };
 int rkv_inject_fault(rkv_engine* eng, int fault);
 
+/* Intermediate arrays of the last rkv_score call on this engine, for checks
+ * against their definitions.  batch must be the batch that call scored,
+ * unchanged, and no other rkv_score call may run in between.
+ *   rho: device [T] fp32 or NULL: rho_j = 1/||k_j|| (0 for a zero key) of every
+ *        token, as the redundancy GEMM consumes it (GEMM modes only);
+ *   U:   device [U, 128] fp32 or NULL: U = sum_j k_j/||k_j|| over each unit's
+ *        N_u keys (closed-form redundancy only).
+ * Asking for rho in the closed form or U in a GEMM mode returns
+ * RKV_ERR_UNSUPPORTED.  Enqueued on stream; no allocation. */
+int rkv_debug_intermediates(rkv_engine* eng, const rkv_batch* batch, float* rho, float* U,
+                            rkv_stream_t stream);
+
 /* Number of kernel launches enqueued by this engine since creation. */
 int64_t rkv_launch_count(const rkv_engine* eng);
 

@@ -12,7 +12,8 @@ from decode_kv_cache_eviction_b200 import Batch, Engine, RkvError
 from decode_kv_cache_eviction_b200 import workloads as W
 from oracle import rkv_oracle as ora
 
-from parity import check_all_units, check_unit, make_batch, oracle_mode, rand_batch, run_engine
+from parity import (check_all_units, check_unit, make_batch, oracle_mode, rand_batch, run_engine,
+                    unit_inputs)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -192,6 +193,52 @@ def test_score_small_ragged(mode, G, w):
         out = run_engine(b, G, w, lam, budget, mode=mode)
         for u in range(len(lengths)):
             check_unit(out, b, u, w, lam, budget, redundancy=oracle_mode(mode))
+
+
+@pytest.mark.parametrize("G,w", [(4, 8), (8, 8)])   # one row group, then two
+def test_intermediates_rho_and_U(G, w):
+    """The score kernel's intermediates against their definitions: rho_j =
+    1/||k_j|| (0 for a zero key), which the redundancy GEMM consumes, and the
+    closed form's U = sum_j k_j/||k_j|| per unit."""
+    lengths = [w, w + 1, 127, 1000, 5000, 33000]
+    zero_rows = [3 + lengths[0] + lengths[1]]
+    b = rand_batch(lengths, G, w, seed=G + 31, zero_rows=zero_rows)
+    T, U = b.num_tokens, b.num_units
+    for mode in ("gemm", "gemm_sym", "max"):
+        eng = Engine(G, w, max_units=U, max_tokens=T,
+                     redundancy="gemm" if mode == "gemm_sym" else mode,
+                     symmetric_gemm=mode == "gemm_sym")
+        a, r = eng.alloc_scores(b)
+        eng.score(b, a, r)
+        rho = torch.full((T,), float("nan"), device=DEV)
+        eng.debug_intermediates(b, rho=rho)
+        eng.check_status()
+        with pytest.raises(RkvError):
+            eng.debug_intermediates(b, U=torch.empty((U, 128), device=DEV))
+        rho = rho.double().cpu().numpy()
+        for u in range(U):
+            k = unit_inputs(b, u)[0]
+            nrm = ora.key_norms(k)
+            want = np.where(nrm > 0, 1.0 / np.where(nrm > 0, nrm, 1.0), 0.0)
+            lo, hi = int(b.tok_off_host[u]), int(b.tok_off_host[u + 1])
+            np.testing.assert_allclose(rho[lo:hi], want, rtol=1e-5, atol=0, err_msg=f"{mode} unit {u}")
+        eng.close()
+    eng = Engine(G, w, max_units=U, max_tokens=T, redundancy="closed")
+    a, r = eng.alloc_scores(b)
+    eng.score(b, a, r)
+    Ug = torch.full((U, 128), float("nan"), device=DEV)
+    eng.debug_intermediates(b, U=Ug)
+    eng.check_status()
+    with pytest.raises(RkvError):
+        eng.debug_intermediates(b, rho=torch.empty(T, device=DEV))
+    Ug = Ug.double().cpu().numpy()
+    for u in range(U):
+        kh = ora.unit_keys(unit_inputs(b, u)[0])
+        want = kh.sum(axis=0)
+        # fp32 sums of N terms of magnitude <= 1: bound by the sum of magnitudes
+        lim = 4e-5 * np.abs(kh).sum(axis=0) + 1e-6
+        assert np.all(np.abs(Ug[u] - want) <= lim), (u, np.max(np.abs(Ug[u] - want) / lim))
+    eng.close()
 
 
 def test_row_max_flags_every_duplicate():
