@@ -15,6 +15,9 @@ using namespace rkv;
 
 namespace {
 
+// Bytes rounded up to a 256-byte boundary (sub-buffers of one allocation).
+size_t round_up(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
 constexpr int kSmemCap = 227 * 1024;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -633,23 +636,51 @@ int rkv_refree_budget(rkv_engine* e, const rkv_batch* b, float T, int sinks, int
   if (e->cfg.group > 8) return RKV_ERR_UNSUPPORTED;
   const int U = b->num_units;
   if (U == 0) return RKV_OK;
+  // scratch, on first use: logits [max_tokens x GP], per-unit chunk offsets,
+  // per-chunk head statistics and energies
+  const int GP = refree_padded_group(e->cfg.group);
+  const int64_t max_ch = refree_max_chunks(e->cfg.max_tokens, e->cfg.max_units);
+  const size_t z_bytes = round_up(sizeof(float) * static_cast<size_t>(e->cfg.max_tokens) * GP);
+  const size_t off_bytes = round_up(sizeof(int) * (static_cast<size_t>(e->cfg.max_units) + 1));
+  const size_t cs_bytes = round_up(sizeof(float2) * static_cast<size_t>(max_ch) * GP);
+  const size_t ce_bytes = round_up(sizeof(float) * static_cast<size_t>(max_ch));
   if (!e->rf_z) {
-    const size_t n = static_cast<size_t>(e->cfg.max_tokens) * refree_padded_group(e->cfg.group);
-    if (dev_alloc(&e->fault, reinterpret_cast<void**>(&e->rf_z), n * sizeof(float)) !=
-        cudaSuccess) {
+    if (dev_alloc(&e->fault, reinterpret_cast<void**>(&e->rf_z),
+                  z_bytes + off_bytes + cs_bytes + ce_bytes) != cudaSuccess) {
       cudaGetLastError();
       e->rf_z = nullptr;
       return RKV_ERR_OOM;
     }
   }
+  int64_t nchunks = 0;
+  for (int u = 0; u < U; ++u)
+    nchunks += (b->tok_off_host[u + 1] - b->tok_off_host[u] + kRfChunk - 1) / kRfChunk;
+  uint8_t* scr = reinterpret_cast<uint8_t*>(e->rf_z);
+  RefreeArgs ra;
+  ra.tok_off = b->tok_off;
+  ra.U = U;
+  ra.nchunks = nchunks;
+  ra.G = e->cfg.group;
+  ra.w = e->cfg.window;
+  ra.Q = b->Q;
+  ra.K = b->K;
+  ra.sinks = sinks;
+  ra.T = T;
+  ra.max_budget = max_budget;
+  ra.zbuf = reinterpret_cast<float*>(scr);
+  ra.chunk_off = reinterpret_cast<int*>(scr + z_bytes);
+  ra.cstat = reinterpret_cast<float2*>(scr + z_bytes + off_bytes);
+  ra.cenergy = reinterpret_cast<float*>(scr + z_bytes + off_bytes + cs_bytes);
+  ra.p_last = p_last;
+  ra.budgets = budgets;
+  ra.keep_count = keep_count;
+  ra.nsm = e->nsm;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   t_begin(e, RKV_KERNEL_REFREE, st);
-  cudaError_t err = launch_refree(b->tok_off, U, e->cfg.group, e->cfg.window, b->Q, b->K, sinks,
-                                  T, max_budget, e->rf_z, p_last, budgets, keep_count, e->nsm,
-                                  st);
+  cudaError_t err = launch_refree(ra, st);
   t_end(e, st);
   if (err != cudaSuccess) return cuda_fail(err);
-  ++e->launches;
+  e->launches += nchunks > 0 ? 4 : 1;
   return RKV_OK;
 }
 

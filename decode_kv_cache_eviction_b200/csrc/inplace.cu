@@ -4,10 +4,11 @@
 // that new tokens overwrite, lowest slot first.
 //
 // evict_in_place_kernel: one CTA per unit (persistent over units).  The kept
-//   indices are scattered into a shared-memory byte mask, the mask is written
-//   out, and the free list is the mask's complement compacted with a block
-//   scan (ballots within warps, one prefix over the 32 warps per 1024-slot
-//   tile), written in ascending order.
+//   indices set bits of a shared-memory bitmap; one block scan over the
+//   words' free counts (each thread a contiguous run of words) gives every
+//   word the number of free slots before it; then warps walk the words, lane
+//   = slot, and write the keep bytes and the free slots (ascending) with one
+//   coalesced store each per word.
 // fill_slots_kernel: one CTA per unit.  New token t is copied (16 threads per
 //   256-byte row, 128-bit accesses) to slot free[t]; the slot is marked live;
 //   then the remaining free slots move to the front of the list, tile by tile
@@ -19,23 +20,26 @@
 namespace rkv {
 namespace {
 
-constexpr int kIpThreads = 1024;
+constexpr int kIpThreads = 256;
 constexpr int kIpWarps = kIpThreads / 32;
+constexpr int kIpWords = kMaxTokensPerUnit / 32;   // kept bitmap words of the longest unit
 
-__global__ void __launch_bounds__(kIpThreads, 1)
-    evict_in_place_kernel(const int64_t* __restrict__ tok_off, int U, int W,
+__global__ void __launch_bounds__(kIpThreads)
+    evict_in_place_kernel(const int64_t* __restrict__ tok_off, int U, int W, int wcap,
                           const int32_t* __restrict__ idx, const int32_t* __restrict__ n_kept,
                           uint8_t* __restrict__ keep, int32_t* __restrict__ free_slots,
                           int32_t* __restrict__ n_free, int* status) {
-  extern __shared__ uint8_t smask[];
+  // kept bitmap (bit i of word i / 32) and, per word, the free slots before it
+  extern __shared__ uint32_t sm_ip[];
+  uint32_t* bits = sm_ip;                            // [wcap]
+  int* wbase = reinterpret_cast<int*>(sm_ip + wcap);  // [wcap]
   __shared__ int wsum[kIpWarps];
-  __shared__ int running;
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
   for (int u = blockIdx.x; u < U; u += gridDim.x) {
     const int64_t base = tok_off[u];
     const int N = static_cast<int>(tok_off[u + 1] - base);
-    for (int i = tid; i < N; i += kIpThreads) smask[i] = 0;
-    if (tid == 0) running = 0;
+    const int nw = (N + 31) >> 5;
+    for (int q = tid; q < nw; q += kIpThreads) bits[q] = 0u;
     __syncthreads();
     int nk = n_kept[u];
     if (nk < 0 || nk > W) {
@@ -45,38 +49,66 @@ __global__ void __launch_bounds__(kIpThreads, 1)
     const int32_t* iu = idx + static_cast<int64_t>(u) * W;
     for (int j = tid; j < nk; j += kIpThreads) {
       const int k = iu[j];
-      if (k >= 0 && k < N) smask[k] = 1;
+      if (k >= 0 && k < N) atomicOr(&bits[k >> 5], 1u << (k & 31));
       else atomicOr(status, kStatusBadIndex);
     }
     __syncthreads();
-    for (int i = tid; i < N; i += kIpThreads) keep[base + i] = smask[i];
-    // free list: ascending complement of the mask
-    for (int t0 = 0; t0 < N; t0 += kIpThreads) {
-      const int i = t0 + tid;
-      const bool f = i < N && smask[i] == 0;
-      const unsigned bal = __ballot_sync(0xffffffffu, f);
-      if (lane == 0) wsum[wp] = __popc(bal);
-      __syncthreads();
-      if (wp == 0) {
-        const int v = wsum[lane];
-        int incl = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        wsum[lane] = incl - v;   // exclusive prefix of the warps
-      }
-      __syncthreads();
-      const int at = running + wsum[wp] + __popc(bal & ((1u << lane) - 1u));
-      if (f) free_slots[base + at] = i;
-      __syncthreads();   // everyone has read running and wsum
-      if (tid == kIpThreads - 1) running = at + (f ? 1 : 0);
-      __syncthreads();
+    // free slots per word; thread tid takes the contiguous words
+    // [tid * per, (tid + 1) * per) and the block scans the per-thread totals
+    const int per = (nw + kIpThreads - 1) / kIpThreads;
+    const int q0 = min(nw, tid * per), q1 = min(nw, q0 + per);
+    int cnt = 0;
+    for (int q = q0; q < q1; ++q) {
+      const int valid = min(32, N - 32 * q);
+      const uint32_t vm = valid == 32 ? 0xffffffffu : ((1u << valid) - 1u);
+      cnt += __popc(~bits[q] & vm);
     }
-    const int nf = running;
-    for (int i = nf + tid; i < N; i += kIpThreads) free_slots[base + i] = -1;
-    if (tid == 0) n_free[u] = nf;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[wp] = incl;
+    __syncthreads();
+    if (wp == 0) {
+      const int v = lane < kIpWarps ? wsum[lane] : 0;
+      int x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane < kIpWarps) wsum[lane] = x - v;   // exclusive prefix of the warps
+    }
+    __syncthreads();
+    int run = wsum[wp] + incl - cnt;
+    for (int q = q0; q < q1; ++q) {
+      wbase[q] = run;
+      const int valid = min(32, N - 32 * q);
+      const uint32_t vm = valid == 32 ? 0xffffffffu : ((1u << valid) - 1u);
+      run += __popc(~bits[q] & vm);
+    }
+    __syncthreads();
+    // warps walk the words: lane = slot within the word, so the keep bytes and
+    // the free slots of a word go out as one coalesced store each
+    for (int q = wp; q < nw; q += kIpWarps) {
+      const uint32_t x = bits[q];
+      const int i = 32 * q + lane;
+      const bool in = i < N;
+      const bool kept = (x >> lane) & 1u;
+      if (in) keep[base + i] = kept ? 1 : 0;
+      const unsigned fb = __ballot_sync(0xffffffffu, in && !kept);
+      if (in && !kept) free_slots[base + wbase[q] + __popc(fb & ((1u << lane) - 1u))] = i;
+    }
+    int nfree = 0;   // free slots before the last word, plus its own
+    if (nw > 0) {
+      const int valid = N - 32 * (nw - 1);
+      const uint32_t vm = valid == 32 ? 0xffffffffu : ((1u << valid) - 1u);
+      nfree = wbase[nw - 1] + __popc(~bits[nw - 1] & vm);
+    }
+    for (int i = nfree + tid; i < N; i += kIpThreads) free_slots[base + i] = -1;
+    if (tid == 0) n_free[u] = nfree;
     __syncthreads();   // shared state is reused by the next unit
   }
 }
@@ -132,17 +164,18 @@ __global__ void __launch_bounds__(kFillThreads)
 
 cudaError_t inplace_configure() {
   return cudaFuncSetAttribute(evict_in_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              kMaxTokensPerUnit);
+                              2 * kIpWords * 4);
 }
 
 cudaError_t launch_evict_in_place(const int64_t* tok_off, int U, int nmax, int W,
                                   const int32_t* idx, const int32_t* n_kept, uint8_t* keep,
                                   int32_t* free_slots, int32_t* n_free, int* status, int nsm,
                                   cudaStream_t st) {
-  int grid = nsm * 2;
+  int grid = nsm * 8;
   if (grid > U) grid = U;
-  evict_in_place_kernel<<<grid, kIpThreads, static_cast<size_t>(nmax), st>>>(
-      tok_off, U, W, idx, n_kept, keep, free_slots, n_free, status);
+  const int wcap = (nmax + 31) / 32;   // bitmap words of the longest unit
+  evict_in_place_kernel<<<grid, kIpThreads, static_cast<size_t>(2 * wcap) * 4, st>>>(
+      tok_off, U, W, wcap, idx, n_kept, keep, free_slots, n_free, status);
   return cudaGetLastError();
 }
 

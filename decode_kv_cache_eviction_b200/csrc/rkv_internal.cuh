@@ -252,10 +252,28 @@ cudaError_t launch_compact(const int64_t* tok_off, int U, int W, const int32_t* 
                            void* Vo, int* status, int nsm, cudaStream_t st);
 
 int refree_padded_group(int G);   // heads per token in the refree logit scratch
-cudaError_t launch_refree(const int64_t* tok_off, int U, int G, int w, const void* Q,
-                          const void* K, int sinks, float T, int max_budget, float* zbuf,
-                          float* p_last, int32_t* budgets, int32_t* keep_count, int nsm,
-                          cudaStream_t st);
+constexpr int kRfChunk = 2048;    // tokens per refree work chunk
+int64_t refree_max_chunks(int64_t max_tokens, int max_units);
+struct RefreeArgs {
+  const int64_t* tok_off;
+  int U;
+  int64_t nchunks;      // sum over units of ceil(N_u / kRfChunk)
+  int G, w;
+  const void* Q;
+  const void* K;
+  int sinks;
+  float T;
+  int max_budget;
+  int* chunk_off;       // scratch [U + 1]
+  float* zbuf;          // scratch [T_tokens * padded G]
+  float2* cstat;        // scratch [nchunks * padded G]
+  float* cenergy;       // scratch [nchunks]
+  float* p_last;
+  int32_t* budgets;
+  int32_t* keep_count;
+  int nsm;
+};
+cudaError_t launch_refree(const RefreeArgs& a, cudaStream_t st);
 cudaError_t inplace_configure();
 cudaError_t launch_evict_in_place(const int64_t* tok_off, int U, int nmax, int W,
                                   const int32_t* idx, const int32_t* n_kept, uint8_t* keep,
