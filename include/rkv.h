@@ -177,8 +177,10 @@ int rkv_select_ex(rkv_engine* eng, const rkv_batch* batch, const float* a, const
  *   budgets [U] int32 (output): clamp(k - min(sinks, N_u - w) - w, 0,
  *     max_budget), the rkv_select_ex budget that keeps k tokens in all.
  * Computed in fp32; requires G <= 8 (RKV_ERR_UNSUPPORTED otherwise).  The
- * first call allocates a logit scratch of max_tokens x (G rounded up to a power
- * of two) floats, kept until rkv_destroy (RKV_ERR_OOM if that fails). */
+ * first call allocates a scratch, kept until rkv_destroy (RKV_ERR_OOM if that
+ * fails): max_tokens x GP logit floats (GP = G rounded up to a power of two),
+ * max_units + 1 chunk offsets, and per 2048-token chunk GP (max, sum) pairs and
+ * one energy, for max_tokens / 2048 + max_units chunks. */
 int rkv_refree_budget(rkv_engine* eng, const rkv_batch* batch, float T, int sinks,
                       int max_budget, float* p_last, int32_t* budgets, int32_t* keep_count,
                       rkv_stream_t stream);
