@@ -33,6 +33,9 @@ constexpr int64_t kMaxTokens = RKV_NOALLOC_MAX_TOKENS;
 constexpr int kMaxRp = 32;                 // G * w <= 32: one score pass
 // chunks of any batch within the limits: score_max_chunks with up to 256 CTAs
 constexpr int kMaxChunks = 8192;
+static_assert(score_max_chunks(kMaxTokens, kMaxUnits, 256, 16) <= kMaxChunks &&
+                  score_max_chunks(kMaxTokens, kMaxUnits, 256, 32) <= kMaxChunks,
+              "static chunk scratch covers every batch within the limits");
 constexpr int kMaxDevices = 64;
 constexpr int kSmemCap = 227 * 1024;
 

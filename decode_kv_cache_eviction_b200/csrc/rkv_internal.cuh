@@ -126,7 +126,7 @@ struct ScoreDims {
 // for the progress rule (every unit within 2 * grid chunks).
 bool score_plan(int R, const int64_t* off, int U, int max_ctas, int tpc_fixed, ScoreDims* d);
 // Upper bound of the chunks of any batch within the capacities.
-inline int64_t score_max_chunks(int64_t max_tokens, int max_units, int max_ctas, int rp) {
+constexpr int64_t score_max_chunks(int64_t max_tokens, int max_units, int max_ctas, int rp) {
   const int64_t tpc_max = score_chunk_tokens(rp) / kTile;
   const int64_t a = (max_tokens / kTile + 2 * static_cast<int64_t>(max_units)) / tpc_max + 1;
   return (a > max_ctas ? a : max_ctas) + max_units;
