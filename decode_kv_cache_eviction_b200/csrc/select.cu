@@ -50,10 +50,18 @@ __device__ unsigned long long g_sel_trace[kStCtas * kStSlots];
 #define RKV_SSTAMP(slot) do { } while (0)
 #endif
 
-constexpr int kSelThreads = 128;
-constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kSample = 2048;     // sample size (at most the candidate count)
-constexpr int kListCap = 3072;    // bracket entries kept on chip
+// Launch shape and on-chip capacities: threads, sample size (at most the
+// candidate count), bracket entries kept on chip.  Units of at most
+// kShortMaxCand candidates take the short shape, so that twice as many units
+// (and their latency-bound phases) share an SM.
+template <int NT, int SMP, int LC, int MINB>
+struct SelCfg {
+  static constexpr int kThreads = NT, kWarps = NT / 32, kSample = SMP, kListCap = LC,
+                       kMinBlocks = MINB;
+};
+using LongSel = SelCfg<128, 2048, 3072, 7>;
+using ShortSel = SelCfg<64, 1024, 1536, 14>;
+constexpr int kShortMaxCand = 8192;
 constexpr float kSpread = 4.f;    // bracket half-width in sampling standard deviations
 
 // Order-preserving key of a score: -0 and +0 get the key of +0, a NaN key 0
@@ -68,17 +76,18 @@ __device__ __forceinline__ float key_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
+template <class C>
 struct SelShared {
   uint32_t hist[512];
   union {                        // the sample is done with before the list fills
-    uint32_t sample[kSample];
-    uint2 list[kListCap];        // bracket entries: (score bits, candidate index)
+    uint32_t sample[C::kSample];
+    uint2 list[C::kListCap];        // bracket entries: (score bits, candidate index)
   };
   int nlist;
   int cnt_above;
   int sh[8];
-  uint32_t wred[kSelWarps];
-  uint32_t wred2[kSelWarps];
+  uint32_t wred[C::kWarps];
+  uint32_t wred2[C::kWarps];
 };
 
 // Block-wide: the k-th largest (1 <= k <= number of matches) of the values
@@ -86,8 +95,8 @@ struct SelShared {
 // significant digit first.  `lo_bits` is the number of low bits in which the
 // values may differ (bits above are common to all: `prefix`).  Returns the
 // value; *above receives the number of matching values strictly greater.
-template <class Get>
-__device__ uint32_t kth_largest(SelShared& s, Get get, int n, int k, uint32_t prefix,
+template <class C, class Get>
+__device__ uint32_t kth_largest(SelShared<C>& s, Get get, int n, int k, uint32_t prefix,
                                 int lo_bits, int* above, int* equal = nullptr) {
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
   uint32_t pmask = lo_bits >= 32 ? 0u : ~((1u << lo_bits) - 1u);
@@ -98,9 +107,9 @@ __device__ uint32_t kth_largest(SelShared& s, Get get, int n, int k, uint32_t pr
     const int d = min(8, lo);
     const int shift = lo - d;
     const uint32_t dmask = (1u << d) - 1u;
-    for (int b = tid; b < 256; b += kSelThreads) s.hist[b] = 0u;
+    for (int b = tid; b < 256; b += C::kThreads) s.hist[b] = 0u;
     __syncthreads();
-    for (int i = tid; i < n; i += kSelThreads) {
+    for (int i = tid; i < n; i += C::kThreads) {
       uint32_t v;
       if (get(i, v) && (v & pmask) == prefix) atomicAdd(&s.hist[(v >> shift) & dmask], 1u);
     }
@@ -153,7 +162,8 @@ __device__ uint32_t kth_largest(SelShared& s, Get get, int n, int k, uint32_t pr
 // shared memory, by radix selection on both ranks at once: while the two
 // prefixes agree one histogram serves both, afterwards each value counts in
 // the histogram of the prefix it matches.
-__device__ void two_kth_largest(SelShared& s, const uint32_t* vals, int n, int k1, int k2,
+template <class C>
+__device__ void two_kth_largest(SelShared<C>& s, const uint32_t* vals, int n, int k1, int k2,
                                 uint32_t prefix, int lo_bits, uint32_t* out1, uint32_t* out2) {
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
   uint32_t pmask = lo_bits >= 32 ? 0u : ~((1u << lo_bits) - 1u);
@@ -165,9 +175,9 @@ __device__ void two_kth_largest(SelShared& s, const uint32_t* vals, int n, int k
     const int shift = lo - d;
     const uint32_t dmask = (1u << d) - 1u;
     const bool same = p1 == p2;
-    for (int b = tid; b < 512; b += kSelThreads) s.hist[b] = 0u;
+    for (int b = tid; b < 512; b += C::kThreads) s.hist[b] = 0u;
     __syncthreads();
-    for (int i = tid; i < n; i += kSelThreads) {
+    for (int i = tid; i < n; i += C::kThreads) {
       const uint32_t v = vals[i];
       const uint32_t bin = (v >> shift) & dmask;
       if ((v & pmask) == p1) atomicAdd(&s.hist[bin], 1u);
@@ -220,11 +230,11 @@ __device__ void two_kth_largest(SelShared& s, const uint32_t* vals, int n, int k
 }
 
 // Block-wide min and max of get(i) over the valid i in [0, n).
-template <class Get>
-__device__ void min_max(SelShared& s, Get get, int n, uint32_t* mn, uint32_t* mx) {
+template <class C, class Get>
+__device__ void min_max(SelShared<C>& s, Get get, int n, uint32_t* mn, uint32_t* mx) {
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
   uint32_t a = 0xffffffffu, b = 0u;
-  for (int i = tid; i < n; i += kSelThreads) {
+  for (int i = tid; i < n; i += C::kThreads) {
     uint32_t v;
     if (get(i, v)) {
       a = min(a, v);
@@ -244,7 +254,7 @@ __device__ void min_max(SelShared& s, Get get, int n, uint32_t* mn, uint32_t* mx
   a = 0xffffffffu;
   b = 0u;
 #pragma unroll
-  for (int q = 0; q < kSelWarps; ++q) {
+  for (int q = 0; q < C::kWarps; ++q) {
     a = min(a, s.wred[q]);
     b = max(b, s.wred2[q]);
   }
@@ -258,13 +268,14 @@ __device__ __forceinline__ int diff_bits(uint32_t a, uint32_t b) {
   return d ? 32 - __clz(d) : 0;
 }
 
-__global__ void __launch_bounds__(kSelThreads, 7)
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, C::kMinBlocks)
     select_kernel(const int64_t* __restrict__ tok_off, int U, int64_t Ttot, int w,
                   const float* __restrict__ a,
                   const float* __restrict__ r, float lam, int max_budget,
                   const int32_t* __restrict__ budgets, int sinks, int W,
                   int32_t* __restrict__ idx, int32_t* __restrict__ n_kept) {
-  __shared__ SelShared s;
+  __shared__ SelShared<C> s;
   extern __shared__ uint32_t bits[];   // kept bitmap, ceil(c / 32) words
   const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
   const float lw = lam, rw = 1.f - lam;
@@ -289,12 +300,12 @@ __global__ void __launch_bounds__(kSelThreads, 7)
   if (budgets) budget = min(max(budgets[u], 0), max_budget);
   int32_t* out = idx + static_cast<int64_t>(u) * W;
   if (c <= budget) {  // every token is kept
-    for (int i = tid; i < W; i += kSelThreads) out[i] = i < N ? i : -1;
+    for (int i = tid; i < W; i += C::kThreads) out[i] = i < N ? i : -1;
     if (tid == 0) n_kept[u] = N;
     return;
   }
   // sinks, the window after the selected candidates, and the unused tail
-  for (int t = tid; t < W - budget; t += kSelThreads) {
+  for (int t = tid; t < W - budget; t += C::kThreads) {
     if (t < m) out[t] = t;
     else if (t < m + w) out[budget + t] = c0 + (t - m);
     else out[budget + t] = -1;
@@ -346,16 +357,16 @@ __global__ void __launch_bounds__(kSelThreads, 7)
 
   // ---- 1. sample and splitters: S / 16 evenly spaced blocks of 16 consecutive
   // candidates (64-byte segments of a and r), S about c / 8 within
-  // [256, kSample]; every candidate when S = c
-  const int S = min(c, min(kSample, max(256, ((c / 8) + 15) & ~15)));
+  // [256, C::kSample]; every candidate when S = c
+  const int S = min(c, min(C::kSample, max(256, ((c / 8) + 15) & ~15)));
   {
     const int nblk = S >> 4;
     const float step = nblk > 1 ? static_cast<float>(c - 16) / static_cast<float>(nblk - 1) : 0.f;
-    constexpr int kPer = kSample / kSelThreads;   // sample keys per thread (at most)
+    constexpr int kPer = C::kSample / C::kThreads;   // sample keys per thread (at most)
     float sa[kPer], sr[kPer];
 #pragma unroll
     for (int x = 0; x < kPer; ++x) {   // every load first, then the keys
-      const int j = tid + x * kSelThreads;
+      const int j = tid + x * C::kThreads;
       int i = j;   // all candidates, or fewer than 16 in a block's place: take them
       if (S < c && j < nblk * 16) i = static_cast<int>(static_cast<float>(j >> 4) * step) + (j & 15);
       i = min(i, c - 1);
@@ -364,7 +375,7 @@ __global__ void __launch_bounds__(kSelThreads, 7)
     }
 #pragma unroll
     for (int x = 0; x < kPer; ++x) {
-      const int j = tid + x * kSelThreads;
+      const int j = tid + x * C::kThreads;
       if (j < S) s.sample[j] = order_key(__fsub_rn(__fmul_rn(lw, sa[x]), __fmul_rn(rw, sr[x])));
     }
   }
@@ -398,7 +409,7 @@ __global__ void __launch_bounds__(kSelThreads, 7)
   // lowest); only the list entries' keys are formed.
   const float f_hi = key_float(hi), f_lo = key_float(lo);
   int above = 0;
-  for (int r0 = wp * kRuns; r0 < nruns; r0 += kSelWarps * kRuns) {
+  for (int r0 = wp * kRuns; r0 < nruns; r0 += C::kWarps * kRuns) {
     float4 A[kRuns], R[kRuns];
 #pragma unroll
     for (int x = 0; x < kRuns; ++x) {
@@ -423,7 +434,7 @@ __global__ void __launch_bounds__(kSelThreads, 7)
     if ((lane & 7) == 0) {
 #pragma unroll
       for (int x = 0; x < kRuns; ++x) {
-        const int run = r0 + kSelWarps * kRuns + x;
+        const int run = r0 + C::kWarps * kRuns + x;
         if (run >= run_lo && run < run_hi) {
           prefetch_l2(a4 + 32 * (run - run_lo));
           prefetch_l2(r4 + 32 * (run - run_lo));
@@ -472,7 +483,7 @@ __global__ void __launch_bounds__(kSelThreads, 7)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           if ((nin >> e) & 1u) {
-            if (q < kListCap)
+            if (q < C::kListCap)
               s.list[q] = make_uint2(__float_as_uint(sv[e]), static_cast<uint32_t>(i0 + e));
             ++q;
           }
@@ -487,7 +498,7 @@ __global__ void __launch_bounds__(kSelThreads, 7)
   const int nl = s.nlist;
   const int want = budget - A;   // keys still to take from the bracket
 
-  if (want >= 1 && want <= nl && nl <= kListCap) {
+  if (want >= 1 && want <= nl && nl <= C::kListCap) {
     // ---- 3. exact threshold inside the bracket
     auto get_list = [&](int i, uint32_t& v) {
       v = order_key(__uint_as_float(s.list[i].x));
@@ -509,7 +520,7 @@ __global__ void __launch_bounds__(kSelThreads, 7)
       int dummy2;
       imax = static_cast<int>(~kth_largest(s, get_tied, nl, take_eq, 0u, 32, &dummy2));
     }
-    for (int i = tid; i < nl; i += kSelThreads) {
+    for (int i = tid; i < nl; i += C::kThreads) {
       const uint2 en = s.list[i];
       const uint32_t k = order_key(__uint_as_float(en.x));
       const int ii = static_cast<int>(en.y);
@@ -535,7 +546,7 @@ __global__ void __launch_bounds__(kSelThreads, 7)
     int dummy2;
     const uint32_t cut = kth_largest(s, get_tied, c, take_eq, 0u, 32, &dummy2);
     const int imax = static_cast<int>(~cut);
-    for (int wd = wp; wd < nwords; wd += kSelWarps) {
+    for (int wd = wp; wd < nwords; wd += C::kWarps) {
       const int i = wd * 32 + lane - delta;
       const bool v = i >= 0 && i < c;
       const uint32_t k = v ? key_at(i) : 0u;
@@ -548,7 +559,7 @@ __global__ void __launch_bounds__(kSelThreads, 7)
   RKV_SSTAMP(4);
   // ---- 4. bitmap -> ascending indices: warp wp takes a contiguous share of
   // the words, one word per lane at a time
-  const int perw = (nwords + kSelWarps - 1) / kSelWarps;
+  const int perw = (nwords + C::kWarps - 1) / C::kWarps;
   const int w0 = min(nwords, wp * perw), w1 = min(nwords, w0 + perw);
   int cnt = 0;
   for (int q = w0 + lane; q < w1; q += 32) cnt += __popc(bits[q]);
@@ -590,8 +601,12 @@ size_t bitmap_bytes(int c) { return static_cast<size_t>((c + 3 + 127) / 128) * 1
 }  // namespace
 
 cudaError_t select_configure() {
-  return cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(bitmap_bytes(kMaxTokensPerUnit)));
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<LongSel>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(bitmap_bytes(kMaxTokensPerUnit)));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(select_kernel<ShortSel>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(bitmap_bytes(kShortMaxCand)));
 }
 
 cudaError_t launch_select(const int64_t* tok_off, int U, int64_t Ttot, int w, int cmax,
@@ -599,9 +614,14 @@ cudaError_t launch_select(const int64_t* tok_off, int U, int64_t Ttot, int w, in
                           const float* r, float lam, int budget, const int32_t* budgets,
                           int sinks, int W, int32_t* idx, int32_t* n_kept, cudaStream_t st) {
   // the kept bitmap: every position of the longest unit, in whole runs of 128
-  const size_t smem = bitmap_bytes(cmax > 0 ? cmax : 0);
-  select_kernel<<<U, kSelThreads, smem, st>>>(tok_off, U, Ttot, w, a, r, lam, budget, budgets,
-                                              sinks, W, idx, n_kept);
+  const int c = cmax > 0 ? cmax : 0;
+  const size_t smem = bitmap_bytes(c);
+  if (c <= kShortMaxCand)
+    select_kernel<ShortSel><<<U, ShortSel::kThreads, smem, st>>>(
+        tok_off, U, Ttot, w, a, r, lam, budget, budgets, sinks, W, idx, n_kept);
+  else
+    select_kernel<LongSel><<<U, LongSel::kThreads, smem, st>>>(
+        tok_off, U, Ttot, w, a, r, lam, budget, budgets, sinks, W, idx, n_kept);
   return cudaGetLastError();
 }
 
