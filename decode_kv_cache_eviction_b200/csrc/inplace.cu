@@ -47,10 +47,21 @@ __global__ void __launch_bounds__(kIpThreads)
       nk = nk < 0 ? 0 : W;
     }
     const int32_t* iu = idx + static_cast<int64_t>(u) * W;
-    for (int j = tid; j < nk; j += kIpThreads) {
-      const int k = iu[j];
-      if (k >= 0 && k < N) atomicOr(&bits[k >> 5], 1u << (k & 31));
-      else atomicOr(status, kStatusBadIndex);
+    // kept indices, eight loads in flight per thread before their atomics
+    for (int j0 = tid; j0 < nk; j0 += 8 * kIpThreads) {
+      int kk[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const int j = j0 + x * kIpThreads;
+        kk[x] = j < nk ? __ldg(&iu[j]) : 0;
+      }
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        if (j0 + x * kIpThreads >= nk) break;
+        const int k = kk[x];
+        if (k >= 0 && k < N) atomicOr(&bits[k >> 5], 1u << (k & 31));
+        else atomicOr(status, kStatusBadIndex);
+      }
     }
     __syncthreads();
     // free slots per word; thread tid takes the contiguous words
