@@ -3,9 +3,11 @@
 // ascending), written in ascending index order.  A NaN score ranks below every
 // number (ties among NaNs by index, like the other ties).
 //
-// One CTA per unit (several CTAs share an SM).  s is mapped to an
-// order-preserving uint32 key where a key is needed; a unit of any length needs
-// no shared-memory copy of its scores.
+// One CTA per unit: 128 threads (seven per SM) when the longest unit has more
+// than kShortMaxCand candidates, else 64 threads with half the sample and list
+// capacity (fourteen per SM).  s is mapped to an order-preserving uint32 key
+// where a key is needed; a unit of any length needs no shared-memory copy of
+// its scores.
 //   1. Sample: the keys of S candidates in evenly spaced blocks of 16 (whole
 //      64-byte segments of a and of r).  Two order statistics of the sample,
 //      about four standard deviations of the sampling error above and below the
