@@ -103,14 +103,27 @@ __global__ void __launch_bounds__(kIpThreads)
     __syncthreads();
     // warps walk the words: lane = slot within the word, so the keep bytes and
     // the free slots of a word go out as one coalesced store each
-    for (int q = wp; q < nw; q += kIpWarps) {
-      const uint32_t x = bits[q];
-      const int i = 32 * q + lane;
-      const bool in = i < N;
-      const bool kept = (x >> lane) & 1u;
-      if (in) keep[base + i] = kept ? 1 : 0;
-      const unsigned fb = __ballot_sync(0xffffffffu, in && !kept);
-      if (in && !kept) free_slots[base + wbase[q] + __popc(fb & ((1u << lane) - 1u))] = i;
+    // four words per step, their shared-memory loads issued together
+    for (int q0 = wp; q0 < nw; q0 += 4 * kIpWarps) {
+      uint32_t x[4];
+      int wb[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int q = q0 + e * kIpWarps;
+        x[e] = q < nw ? bits[q] : 0u;
+        wb[e] = q < nw ? wbase[q] : 0;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int q = q0 + e * kIpWarps;
+        if (q >= nw) break;
+        const int i = 32 * q + lane;
+        const bool in = i < N;
+        const bool kept = (x[e] >> lane) & 1u;
+        if (in) keep[base + i] = kept ? 1 : 0;
+        const unsigned fb = __ballot_sync(0xffffffffu, in && !kept);
+        if (in && !kept) free_slots[base + wb[e] + __popc(fb & ((1u << lane) - 1u))] = i;
+      }
     }
     int nfree = 0;   // free slots before the last word, plus its own
     if (nw > 0) {
