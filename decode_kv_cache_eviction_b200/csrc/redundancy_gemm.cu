@@ -41,11 +41,14 @@
 // the two CTAs' column sums and the slots (a, b > a) in block order, scales by
 // rho_i / (N - 1) and applies the token softmax.
 //
-// Warp roles (640 threads = 5 warps per SM sub-partition): warp 0 TMA producer,
-// warp 1 MMA issuer (leader CTA only in pair mode; the whole warp runs the loop
-// and elects one lane per instruction) and TMEM owner, warp 2 (symmetric form)
-// row-sum store, warps 4-19 epilogue (warp % 4 selects the TMEM lane quarter,
-// (warp - 4) / 4 the 64-column quarter of the tile).
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (leader CTA only in pair
+// mode; the whole warp runs the loop and elects one lane per instruction) and
+// TMEM owner, then the epilogue warps, warp % 4 selecting the TMEM lane
+// quarter.  Row-block form (640 threads = 5 warps per SM sub-partition):
+// warps 4-19, (warp - 4) / 4 the 64-column quarter of the tile.  Symmetric
+// form (384 threads): warp 2 row-sum store, warps 4-11, (warp - 4) / 4 the
+// 128-column half of the tile; with 168 registers a thread, a warp keeps two
+// TMEM loads' worth of the tile and the column sums of its 32 columns.
 #include "ptx.cuh"
 #include "rkv_internal.cuh"
 
@@ -66,6 +69,11 @@ __device__ unsigned long long g_gemm_trace[kGTCtas * 2 * kGT * 4];
 #else
 #define RKV_GSTAMP(role, tile, slot) do { } while (0)
 #endif
+
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
+};
 
 __device__ __forceinline__ int find_unit(const int* item_off, int U, int item) {
   int lo = 0, hi = U - 1;  // largest u with item_off[u] <= item
@@ -121,11 +129,12 @@ __device__ __forceinline__ void commit_pair_elect(uint64_t* bar) {
 }
 
 template <bool kPair, bool kMax, bool kSym>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads(kSym), 1)
     redundancy_gemm_kernel(const __grid_constant__ CUtensorMap amap,
                            const __grid_constant__ CUtensorMap bmap, const GemmParams p) {
   using C = GemmCfg<kPair>;
   constexpr int NSB = C::kStages;
+  constexpr int kEpiWarps = (gemm_threads(kSym) - 128) / 32;   // per CTA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -159,14 +168,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kPair ? 32 : 16);
+      mbar_init(&acc_empty[b], kPair ? 2 * kEpiWarps : kEpiWarps);
     }
     for (int b = 0; b < kRhoSlots; ++b) {
       mbar_init(&rho_full[b], 1);
-      mbar_init(&rho_empty[b], 16);   // this CTA's 16 epilogue warps
+      mbar_init(&rho_empty[b], kEpiWarps);   // this CTA's epilogue warps
     }
     for (int b = 0; b < kRowRing; ++b) {
-      mbar_init(&row_full[b], 16);    // the 16 epilogue warps
+      mbar_init(&row_full[b], kEpiWarps);   // the epilogue warps
       mbar_init(&row_empty[b], 1);    // the row-store warp
     }
     *abort = 0;
@@ -308,9 +317,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else if (warp == 2 && kSym) {
     // ------------------------------------------------ row-sum store (symmetric)
-    // Per tile below the item's block: the four column groups' partial row
-    // sums of this CTA's 128 rows, added in a fixed order and stored to the
-    // tile's scratch slot.
+    // Per tile below the item's block: the two column halves' partial row
+    // sums of this CTA's 128 rows, added and stored to the tile's scratch slot.
     const float* rr = reinterpret_cast<const float*>(sm + L.rowr);
     uint32_t n = 0;   // row exchanges so far
     for (int item = group_id; item < n_items; item += ngroups) {
@@ -326,7 +334,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int rl = lane + 32 * j;
-          tot[j] = ((x[rl] + x[128 + rl]) + x[256 + rl]) + x[384 + rl];
+          tot[j] = x[rl] + x[128 + rl];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&row_empty[s]);
@@ -340,12 +348,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp >= 4 && kSym) {
     // ------------------------------------------------- epilogue, symmetric form
-    const int ew = warp - 4;              // epilogue warp 0..15
-    const int cg = ew >> 2;               // 64-column group of the tile
+    // 8 warps: warp % 4 selects the TMEM lane quarter, (warp - 4) / 4 the
+    // 128-column half of the tile.  Per tile a warp reads four 32-register
+    // chunks (16 lanes x 64 columns each), two in flight: the load of the next
+    // chunk overlaps the folds of the current one.
+    const int ew = warp - 4;              // epilogue warp 0..7
+    const int ch = ew >> 2;               // 128-column half of the tile
     const int q = warp & 3;               // TMEM lane quarter
     const int gq = lane >> 2, tq = lane & 3;   // quad and thread within it
     const float* rho_ring = reinterpret_cast<const float*>(sm + L.rho);
-    float* rowr = reinterpret_cast<float*>(sm + L.rowr);    // [kRowRing][cg][128]
+    float* rowr = reinterpret_cast<float*>(sm + L.rowr);    // [kRowRing][ch][128]
     float2* colx = reinterpret_cast<float2*>(sm + L.colx);  // [2][cg][q][32] column sums
     const uint32_t acc_empty_lead = mapa(smem_u32(acc_empty), 0);
     const int rq = rank * 128 + q * 32;   // first row of this warp's quarter in a block
@@ -359,82 +371,93 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int blk = item_block<kSym>(p.item_off, u, item);
       const float* rho_u = p.rho + __ldg(&p.rho_off[u]);
       float* cs_u = p.cs + __ldg(&p.cs_off[u]);
-      // weights rho_j of this thread's 16 columns of block blk (8k + 2tq + {0, 1})
-      float2 wt[8];
+      // weights rho_j of this thread's 32 columns of block blk: column group
+      // cg = 2 ch + c, columns 8k + 2tq + {0, 1} of the group
+      float2 wt[2][8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        wt[k] = __ldg(reinterpret_cast<const float2*>(rho_u + blk * 256 + cg * 64 + 2 * tq + 8 * k));
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          wt[c][k] = __ldg(reinterpret_cast<const float2*>(rho_u + blk * 256 + ch * 128 + c * 64 +
+                                                           2 * tq + 8 * k));
       // rho_i-weighted column sums of the item's block over this thread's rows
-      float cp[16];
+      float cp[2][16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) cp[k] = 0.f;
-      for (int t = 0; t <= blk; ++t, ++rt) {
-        const bool diag = t == blk;
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int k = 0; k < 16; ++k) cp[c][k] = 0.f;
+      // One tile: the row blocks t < blk, then the diagonal tile t = blk.
+      auto tile = [&](auto diag_tag) {
+        constexpr bool kDiag = decltype(diag_tag)::value;
         const uint32_t rs_slot = rt % kRhoSlots;
+        if (ew == 0 && lane == 0) RKV_GSTAMP(1, rt, 0);
         mbar_wait(&acc_full[ab], aph, abort, p.status);
         mbar_wait(&rho_full[rs_slot], (rt / kRhoSlots) & 1, abort, p.status);
+        if (ew == 0 && lane == 0) RKV_GSTAMP(1, rt, 1);
         __syncwarp();
         tc_fence_after();
         // weights of this thread's 4 rows of block t (gq + 8k of the quarter)
         const float* wr = rho_ring + rs_slot * 256 + rq + gq;
         const float w0 = wr[0], w1 = wr[8], w2 = wr[16], w3 = wr[24];
         const uint32_t tbase =
-            tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + cg * 64;
-        // diagonal tile: rows and columns of one block; the diagonal (column -
-        // row == dd in this warp's 32 x 64 sub-block) is dropped
-        const int dd = rq - cg * 64;
-        const bool masked = diag && dd > -32 && dd < 64;
-        uint32_t v[32];
-        auto patch = [&](int h) {
+            tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + ch * 128;
+        uint32_t va[32], vb[32];
+        // One chunk (16 lanes h of the quarter x 64 columns of group c): the
+        // column sums take rows gq + 16h (weight wa) and gq + 16h + 8 (wb);
+        // off the diagonal the row sums of those two rows take the chunk's 16
+        // columns, two partial values each.  On the diagonal tile (rows and
+        // columns of one block) the element column - row == dd, local to the
+        // warp's 32 x 64 sub-block, is dropped and the row sums are skipped:
+        // block blk's rows get their share from the column sums.
+        auto fold = [&](uint32_t (&v)[32], int h, int c, const float2 (&w)[8], float (&cc)[16],
+                        float& pa, float& pb, float& qa, float& qb, float wa, float wb) {
+          if constexpr (kDiag) {
+            const int dd = rq - ch * 128 - 64 * c;
+            if (dd > -32 && dd < 64) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
+              for (int k = 0; k < 8; ++k)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int col = 8 * k + 2 * tq + (e & 1);
-              const int row = 16 * h + gq + ((e >> 1) << 3);
-              if (col - row == dd) v[4 * k + e] = 0u;
+                for (int e = 0; e < 4; ++e) {
+                  const int col = 8 * k + 2 * tq + (e & 1);
+                  const int row = 16 * h + gq + ((e >> 1) << 3);
+                  if (col - row == dd) v[4 * k + e] = 0u;
+                }
             }
-        };
-        // row sums over this thread's 16 columns: rows gq + 16h and gq + 16h + 8,
-        // two partial values each
-        auto rowfold = [&](float& pa, float& pb, float& qa, float& qb) {
-          mul2(pa, pb, __uint_as_float(v[0]), __uint_as_float(v[1]), wt[0].x, wt[0].y);
-          mul2(qa, qb, __uint_as_float(v[2]), __uint_as_float(v[3]), wt[0].x, wt[0].y);
-#pragma unroll
-          for (int k = 1; k < 8; ++k) {
-            fma2(pa, pb, __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]), wt[k].x,
-                 wt[k].y);
-            fma2(qa, qb, __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]), wt[k].x,
-                 wt[k].y);
           }
-        };
-        auto colfold = [&](float wa, float wb) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            fma2(cp[2 * k], cp[2 * k + 1], __uint_as_float(v[4 * k]),
-                 __uint_as_float(v[4 * k + 1]), wa, wa);
-            fma2(cp[2 * k], cp[2 * k + 1], __uint_as_float(v[4 * k + 2]),
-                 __uint_as_float(v[4 * k + 3]), wb, wb);
+            const float x0 = __uint_as_float(v[4 * k]), x1 = __uint_as_float(v[4 * k + 1]);
+            const float y0 = __uint_as_float(v[4 * k + 2]), y1 = __uint_as_float(v[4 * k + 3]);
+            if constexpr (!kDiag) fma2(pa, pb, x0, x1, w[k].x, w[k].y);
+            fma2(cc[2 * k], cc[2 * k + 1], x0, x1, wa, wa);
+            if constexpr (!kDiag) fma2(qa, qb, y0, y1, w[k].x, w[k].y);
+            fma2(cc[2 * k], cc[2 * k + 1], y0, y1, wb, wb);
           }
         };
         float a0 = 0.f, b0 = 0.f, a1 = 0.f, b1 = 0.f, a2 = 0.f, b2 = 0.f, a3 = 0.f, b3 = 0.f;
-        tmem_ld16x256b_x8(tbase, v);                 // lanes 0-15 of the quarter
-        tmem_wait_ld();
-        if (masked) patch(0);
-        if (!diag) rowfold(a0, b0, a1, b1);
-        colfold(w0, w1);
-        tmem_ld16x256b_x8(tbase + (16u << 16), v);   // lanes 16-31
-        tmem_wait_ld();
+        // chunk order: (lanes 0-15, group 0), (0-15, 1), (16-31, 0), (16-31, 1)
+        tmem_ld16x256b_x8(tbase, va);
+        tmem_wait_ld_dep(va);
+        tmem_ld16x256b_x8(tbase + 64, vb);
+        fold(va, 0, 0, wt[0], cp[0], a0, b0, a1, b1, w0, w1);
+        tmem_wait_ld_dep(vb);
+        tmem_ld16x256b_x8(tbase + (16u << 16), va);
+        fold(vb, 0, 1, wt[1], cp[1], a0, b0, a1, b1, w0, w1);
+        tmem_wait_ld_dep(va);
+        tmem_ld16x256b_x8(tbase + (16u << 16) + 64, vb);
+        fold(va, 1, 0, wt[0], cp[0], a2, b2, a3, b3, w2, w3);
+        tmem_wait_ld_dep(vb);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_lead + ab * 8);
+        if (ew == 0 && lane == 0) RKV_GSTAMP(1, rt, 2);
         if (++ab == 2) { ab = 0; aph ^= 1; }
-        if (masked) patch(1);
-        if (!diag) rowfold(a2, b2, a3, b3);
-        colfold(w2, w3);
+        fold(vb, 1, 1, wt[1], cp[1], a2, b2, a3, b3, w2, w3);
         __syncwarp();
         if (lane == 0) mbar_arrive(&rho_empty[rs_slot]);
-        if (!diag) {
+        if (ew == 0 && lane == 0) RKV_GSTAMP(1, rt, 3);
+        ++rt;
+        if constexpr (!kDiag) {
           // the quad's four threads hold disjoint columns of the same 4 rows:
           // reduce-scatter so that thread tq keeps row gq + 8 tq
           const float t0 = a0 + b0, t1 = a1 + b1, t2 = a2 + b2, t3 = a3 + b3;
@@ -442,41 +465,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const float k0 = (u2 ? t2 : t0) + __shfl_xor_sync(0xffffffffu, u2 ? t0 : t2, 2);
           const float k1 = (u2 ? t3 : t1) + __shfl_xor_sync(0xffffffffu, u2 ? t1 : t3, 2);
           const float rsum = (u1 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, u1 ? k0 : k1, 1);
-          // into the ring; the row-store warp adds the four column groups
+          // into the ring; the row-store warp adds the two column halves
           const uint32_t s = nx % kRowRing;
           mbar_wait(&row_empty[s], ((nx / kRowRing) & 1) ^ 1, abort, p.status);
-          rowr[s * 512 + cg * 128 + q * 32 + gq + 8 * tq] = rsum;
+          rowr[s * 512 + ch * 128 + q * 32 + gq + 8 * tq] = rsum;
           __syncwarp();
           if (lane == 0) mbar_arrive(&row_full[s]);
           ++nx;
         }
-      }
+      };
+      for (int t = 0; t < blk; ++t) tile(BoolTag<false>{});
+      tile(BoolTag<true>{});
       // ---- item end: column sums of block blk over the quad index gq (lane
       // bits 2-4), reduce-scattered so that lane l keeps columns 2l and 2l + 1
-      // of the group, then the four lane quarters through shared memory
+      // of each group, then the four lane quarters through shared memory
 #pragma unroll
-      for (int sft = 16, n = 8; sft >= 4; sft >>= 1, n >>= 1) {
-        const bool up = (lane & sft) != 0;
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
-        for (int k = 0; k < n; ++k) {
-          const float send = up ? cp[k] : cp[k + n];
-          const float keep = up ? cp[k + n] : cp[k];
-          cp[k] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+        for (int sft = 16, n = 8; sft >= 4; sft >>= 1, n >>= 1) {
+          const bool up = (lane & sft) != 0;
+#pragma unroll
+          for (int k = 0; k < n; ++k) {
+            const float send = up ? cp[c][k] : cp[c][k + n];
+            const float keep = up ? cp[c][k + n] : cp[c][k];
+            cp[c][k] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
+          }
         }
+        float2* cx = colx + (ib * 4 + 2 * ch + c) * 4 * 32;
+        cx[q * 32 + lane] = make_float2(cp[c][0], cp[c][1]);
       }
-      float2* cx = colx + (ib * 4 + cg) * 4 * 32;
-      cx[q * 32 + lane] = make_float2(cp[0], cp[1]);
-      named_bar_sync(4 + cg, 128);
+      named_bar_sync(4 + ch, 128);
       if (q == 0) {
-        float2 acc = cx[lane];
 #pragma unroll
-        for (int qq = 1; qq < 4; ++qq) {
-          const float2 y = cx[qq * 32 + lane];
-          acc.x += y.x;
-          acc.y += y.y;
+        for (int c = 0; c < 2; ++c) {
+          const float2* cx = colx + (ib * 4 + 2 * ch + c) * 4 * 32;
+          float2 acc = cx[lane];
+#pragma unroll
+          for (int qq = 1; qq < 4; ++qq) {
+            const float2 y = cx[qq * 32 + lane];
+            acc.x += y.x;
+            acc.y += y.y;
+          }
+          // this CTA's rows' share; the pair's other CTA writes the other slot
+          *reinterpret_cast<float2*>(cs_u + (2 * blk + rank) * 256 + ch * 128 + c * 64 +
+                                     2 * lane) = acc;
         }
-        // this CTA's rows' share; the pair's other CTA writes the other slot
-        *reinterpret_cast<float2*>(cs_u + (2 * blk + rank) * 256 + cg * 64 + 2 * lane) = acc;
       }
     }
   } else if (!kSym && warp >= 4) {
@@ -812,8 +845,8 @@ __global__ void __launch_bounds__(kFinishThreads)
 }  // namespace
 
 #ifdef RKV_TRACE
-cudaError_t gemm_trace_read(void* dst, size_t bytes) {
-  return cudaMemcpyFromSymbol(dst, g_gemm_trace, bytes);
+extern "C" int rkv_debug_gemm_trace(void* dst, size_t bytes) {
+  return static_cast<int>(cudaMemcpyFromSymbol(dst, g_gemm_trace, bytes));
 }
 #endif
 
@@ -843,7 +876,8 @@ int gemm_max_ctas(bool pair, bool rowmax, bool sym) {
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (!pair) {
     int per = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, f, kGemmThreads, smem) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, f, gemm_threads(sym), smem) !=
+        cudaSuccess) {
       cudaGetLastError();
       return 0;
     }
@@ -851,7 +885,7 @@ int gemm_max_ctas(bool pair, bool rowmax, bool sym) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * nsm, 1, 1);
-  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.blockDim = dim3(gemm_threads(sym), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
@@ -887,7 +921,7 @@ cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const 
   const int smem = (pair ? gemm_layout<true>().total : gemm_layout<false>().total) + 1024;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nctas, 1, 1);
-  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.blockDim = dim3(gemm_threads(sym), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute at[1];

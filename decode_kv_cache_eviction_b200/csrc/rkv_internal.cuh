@@ -28,6 +28,8 @@ constexpr int kMaxRows = 256;        // G * w limit (row groups of 32 per launch
 // pass-2 warps; the closed form's norm warps need the registers instead).
 __host__ __device__ constexpr int score_threads(bool closed) { return closed ? 512 : 640; }
 constexpr int kGemmThreads = 640;    // producer, MMA, 2 idle, 16 epilogue warps
+// The symmetric form: producer, MMA, row-sum store, 1 idle, 8 epilogue warps.
+__host__ __device__ constexpr int gemm_threads(bool sym) { return sym ? 384 : kGemmThreads; }
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------- score
