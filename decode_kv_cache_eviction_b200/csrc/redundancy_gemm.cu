@@ -241,14 +241,16 @@ __global__ void __launch_bounds__(gemm_threads(kSym), 1)
             }
           }
           if (++stage == NSB) { stage = 0; ph ^= 1; }
-          // the tile's 256 rho values (column weights; row weights in the
-          // symmetric form); every CTA of a pair loads its own
-          const uint32_t rs = rt % kRhoSlots;
-          if (mbar_wait(&rho_empty[rs], ((rt / kRhoSlots) & 1) ^ 1, abort, p.status)) {
-            mbar_arrive_expect_tx(&rho_full[rs], 256 * 4);
-            bulk_load(rho_ring + rs * 256, rho_u + t * C::kN, 256 * 4, &rho_full[rs]);
+          // the tile's 256 rho values (column weights of the row-block form);
+          // every CTA of a pair loads its own
+          if constexpr (!kSym) {
+            const uint32_t rs = rt % kRhoSlots;
+            if (mbar_wait(&rho_empty[rs], ((rt / kRhoSlots) & 1) ^ 1, abort, p.status)) {
+              mbar_arrive_expect_tx(&rho_full[rs], 256 * 4);
+              bulk_load(rho_ring + rs * 256, rho_u + t * C::kN, 256 * 4, &rho_full[rs]);
+            }
+            ++rt;
           }
-          ++rt;
         }
       }
     }
@@ -356,7 +358,6 @@ __global__ void __launch_bounds__(gemm_threads(kSym), 1)
     const int ch = ew >> 2;               // 128-column half of the tile
     const int q = warp & 3;               // TMEM lane quarter
     const int gq = lane >> 2, tq = lane & 3;   // quad and thread within it
-    const float* rho_ring = reinterpret_cast<const float*>(sm + L.rho);
     float* rowr = reinterpret_cast<float*>(sm + L.rowr);    // [kRowRing][ch][128]
     float2* colx = reinterpret_cast<float2*>(sm + L.colx);  // [2][cg][q][32] column sums
     const uint32_t acc_empty_lead = mapa(smem_u32(acc_empty), 0);
@@ -387,18 +388,25 @@ __global__ void __launch_bounds__(gemm_threads(kSym), 1)
 #pragma unroll
         for (int k = 0; k < 16; ++k) cp[c][k] = 0.f;
       // One tile: the row blocks t < blk, then the diagonal tile t = blk.
-      auto tile = [&](auto diag_tag) {
+      // weights of this thread's 4 rows of block t (gq + 8k of the quarter),
+      // loaded one tile ahead
+      const float* wrow = rho_u + rq + gq;
+      float nw0 = __ldg(wrow), nw1 = __ldg(wrow + 8), nw2 = __ldg(wrow + 16), nw3 = __ldg(wrow + 24);
+      auto tile = [&](auto diag_tag, int t) {
         constexpr bool kDiag = decltype(diag_tag)::value;
-        const uint32_t rs_slot = rt % kRhoSlots;
+        const float w0 = nw0, w1 = nw1, w2 = nw2, w3 = nw3;
+        if constexpr (!kDiag) {   // the next tile of the item exists
+          const float* wn = wrow + (t + 1) * 256;
+          nw0 = __ldg(wn);
+          nw1 = __ldg(wn + 8);
+          nw2 = __ldg(wn + 16);
+          nw3 = __ldg(wn + 24);
+        }
         if (ew == 0 && lane == 0) RKV_GSTAMP(1, rt, 0);
         mbar_wait(&acc_full[ab], aph, abort, p.status);
-        mbar_wait(&rho_full[rs_slot], (rt / kRhoSlots) & 1, abort, p.status);
         if (ew == 0 && lane == 0) RKV_GSTAMP(1, rt, 1);
         __syncwarp();
         tc_fence_after();
-        // weights of this thread's 4 rows of block t (gq + 8k of the quarter)
-        const float* wr = rho_ring + rs_slot * 256 + rq + gq;
-        const float w0 = wr[0], w1 = wr[8], w2 = wr[16], w3 = wr[24];
         const uint32_t tbase =
             tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + ch * 128;
         uint32_t va[32], vb[32];
@@ -453,8 +461,6 @@ __global__ void __launch_bounds__(gemm_threads(kSym), 1)
         if (ew == 0 && lane == 0) RKV_GSTAMP(1, rt, 2);
         if (++ab == 2) { ab = 0; aph ^= 1; }
         fold(vb, 1, 1, wt[1], cp[1], a2, b2, a3, b3, w2, w3);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&rho_empty[rs_slot]);
         if (ew == 0 && lane == 0) RKV_GSTAMP(1, rt, 3);
         ++rt;
         if constexpr (!kDiag) {
@@ -474,8 +480,8 @@ __global__ void __launch_bounds__(gemm_threads(kSym), 1)
           ++nx;
         }
       };
-      for (int t = 0; t < blk; ++t) tile(BoolTag<false>{});
-      tile(BoolTag<true>{});
+      for (int t = 0; t < blk; ++t) tile(BoolTag<false>{}, t);
+      tile(BoolTag<true>{}, blk);
       // ---- item end: column sums of block blk over the quad index gq (lane
       // bits 2-4), reduce-scattered so that lane l keeps columns 2l and 2l + 1
       // of each group, then the four lane quarters through shared memory
