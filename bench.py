@@ -44,7 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC_LONG_TRACE = {
     # (redundancy mode, kernel): bytes per launch
     ("gemm", "gemm"): (136.425472e6 + 5.207808e6) * 64,      # 16-unit capture
-    ("gemm_sym", "gemm"): (137.865728e6 + 109.153536e6) * 64,  # 16-unit capture
+    ("gemm_sym", "gemm"): (137.337344e6 + 109.282048e6) * 64,  # 16-unit capture
 }
 
 
