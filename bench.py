@@ -190,6 +190,11 @@ def algorithmic(batch: Batch, wl: W.Workload):
         "evict_bytes": float(4 * U * W_ + 4 * U + 5 * n.sum() + 4 * U),
         # K read once, the newest queries, p_last written and read back, budgets
         "refree_bytes": float((2 * d + 8) * n.sum() + 2 * d * U * wl.group + 8 * U),
+        # symmetric form's finish: the partial-sum scratch (128 nb (nb + 3)
+        # floats per unit with candidates) and rho read, m and r written
+        "finish_bytes": float(sum(4 * 128 * nb * (nb + 3) + 12 * cc
+                                  for nb, cc in zip(((n + 255) // 256).astype(np.int64), c)
+                                  if cc > 0)),
     }
 
 
@@ -235,7 +240,7 @@ def kernel_report(per_kernel, alg, pk, src, symmetric=False):
                        peak=pk["bf16_tflops_sustained"], frac=round(tf / pk["bf16_tflops_sustained"], 4))
             if symmetric:
                 ent["dense_equivalent_tflops"] = round(alg["gemm_flops"] / (ms * 1e-3) / 1e12, 2)
-        elif name in ("score", "select", "compact", "evict", "refree"):
+        elif name in ("score", "select", "compact", "evict", "refree", "finish"):
             gbs = alg[f"{name}_bytes"] / (ms * 1e-3) / 1e9
             ent.update(bound="hbm", achieved=round(gbs, 1), unit="GB/s", peak=hbm,
                        frac=round(gbs / hbm, 4))

@@ -41,7 +41,7 @@ EXPORTS = ("rkv_create", "rkv_destroy", "rkv_score", "rkv_select", "rkv_compact"
            "rkv_select_ex", "rkv_refree_budget", "rkv_check_status", "rkv_launch_count", "rkv_set_timing",
            "rkv_read_timing", "rkv_score_noalloc", "rkv_noalloc_check_status", "rkv_inject_fault",
            "rkv_debug_intermediates", "rkv_status_string", "rkv_version")
-KERNELS = ("score", "plan", "gemm", "select", "compact", "evict", "fill", "refree")
+KERNELS = ("score", "plan", "gemm", "select", "compact", "evict", "fill", "refree", "finish")
 
 
 class RkvConfig(ctypes.Structure):

@@ -467,11 +467,13 @@ int rkv_score(rkv_engine* e, const rkv_batch* b, float* a, float* r, float* m,
   if (nctas > need) nctas = need;
   t_begin(e, RKV_KERNEL_GEMM, st);
   err = launch_gemm(amap, bmap, g, e->pair, e->rowmax, e->sym, static_cast<int>(nctas), st);
+  t_end(e, st);
   if (err == cudaSuccess && e->sym) {
     ++e->launches;
-    err = launch_sym_finish(g, e->nsm, st);   // timed together with the GEMM
+    t_begin(e, RKV_KERNEL_FINISH, st);
+    err = launch_sym_finish(g, e->nsm, st);
+    t_end(e, st);
   }
-  t_end(e, st);
   if (err != cudaSuccess) return cuda_fail(err);
   ++e->launches;
   return RKV_OK;

@@ -308,15 +308,17 @@ enum {
   RKV_KERNEL_EVICT = 5,   /* in-place eviction: keep mask and free slots */
   RKV_KERNEL_FILL = 6,    /* new tokens into free slots */
   RKV_KERNEL_REFREE = 7,  /* adaptive budget (newest query's attention row) */
-  RKV_NUM_KERNELS = 8
+  RKV_KERNEL_FINISH = 8,  /* symmetric GEMM form: partial sums -> m, token softmax -> r */
+  RKV_NUM_KERNELS = 9
 };
 
 /* Per-kernel timing.  While enabled, the engine records a pair of CUDA events
  * on the launch stream around each of its kernel launches (up to 4096 pairs
  * between reads).  rkv_read_timing synchronises on those events and returns,
  * for `kernel`, the summed device time in milliseconds and the number of
- * launches since the previous read (of any kernel), then forgets them.
- * rkv_set_timing(eng, 0) disables recording and drops unread events. */
+ * launches recorded since timing was last set; reading drops nothing.
+ * rkv_set_timing (either value) drops the recorded events, and
+ * rkv_set_timing(eng, 0) also stops recording. */
 int rkv_set_timing(rkv_engine* eng, int enable);
 int rkv_read_timing(rkv_engine* eng, int kernel, double* total_ms, int64_t* launches);
 
