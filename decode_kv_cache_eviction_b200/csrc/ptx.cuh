@@ -334,15 +334,6 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-// The same wait, tied to the registers of one 16-register load.
-__device__ __forceinline__ void tmem_wait_ld_dep16(uint32_t (&v)[16]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
-                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
-                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15])
-               :
-               : "memory");
-}
 // The same wait, tied to the registers of one load: their uses cannot be
 // scheduled above it (needed when a later load is in flight meanwhile).
 #define RKV_RW8(i) "+r"(v[i + 0]), "+r"(v[i + 1]), "+r"(v[i + 2]), "+r"(v[i + 3]), \

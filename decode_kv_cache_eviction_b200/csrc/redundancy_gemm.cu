@@ -685,422 +685,6 @@ __global__ void __launch_bounds__(gemm_threads(kSym), 1)
   }
 }
 
-// ---------------------------------------------------------------- symmetric form
-// Items of two key blocks.  An item (unit, pair j) holds key blocks b0 = 2j and
-// b1 = 2j + 1 (b1 absent when the unit's block count is odd and j is the last
-// pair) in shared memory as the MMA's B operand, 128 keys of each per CTA.  The
-// row blocks a = 0 .. b1 stream through the ring as the A operand, and each
-// streamed tile meets both fixed blocks: 8 MMAs into accumulator 0 (block b0,
-// for a <= b0) and 8 into accumulator 1 (block b1), so a streamed tile is read
-// from L2 once for two tiles of products.  Epilogue group g (4 warps, one per
-// TMEM lane quarter, each 32 rows x 256 columns) drains accumulator g, so each
-// group has two tiles' worth of MMA time per tile it folds.
-//   - Column sums of block b_g over the rows of blocks 0 .. b_g stay in
-//     registers over the item (64 per thread); the diagonal tile a = b_g has
-//     its diagonal dropped and gives no row sums.
-//   - Row sums of block a over the columns of b_g (a < b_g): a quad
-//     reduce-scatter, then the 4-deep ring to warp 2, which adds the two
-//     groups' values and stores one scratch slot (a, j) per row block and
-//     item.  A group with no tile for an exchange (group 0 at its diagonal,
-//     group 1 of a single-block item) puts zeros in the ring.
-// Scratch per unit of nb blocks, np = ceil(nb / 2) pairs: the two CTAs' column
-// sums of every block (1024 np floats), then for row block A its slots (A, j),
-// j = ceil(A / 2) .. np - 1, 256 floats each, starting at
-// 1024 np + 256 (A np - floor(A^2 / 4)).
-constexpr int kSymStages = 4;   // streamed-tile ring depth (32 KiB per stage and CTA)
-struct SymLayout {
-  uint32_t fix, b, wsm, rowr, colx, bars, slot, flags, total;
-};
-__host__ __device__ inline SymLayout sym_layout() {
-  SymLayout L;
-  uint32_t o = 0;
-  L.fix = o; o += 4 * 16384;               // [block][K half][128 rows x 128 B]
-  L.b = o; o += kSymStages * 32768;        // streamed row blocks
-  L.wsm = o; o += 2 * 256 * 4;             // [group][256] column weights, permuted
-  L.rowr = o; o += kRowRing * 512 * 4;     // [kRowRing][group][128 rows]
-  L.colx = o; o += 2 * 4 * 4 * 32 * 8;     // [group][64-column group][q][lane] float2
-  L.bars = o; o += (2 + 2 * kSymStages + 4 + 2 * kRowRing) * 8;
-  L.slot = o; o += 16;
-  L.flags = o; o += 16;
-  L.total = o;
-  return L;
-}
-__device__ __forceinline__ int64_t sym_row_seg(int A, int np) {
-  return 1024 * static_cast<int64_t>(np) +
-         256 * (static_cast<int64_t>(A) * np - (static_cast<int64_t>(A) * A) / 4);
-}
-
-__global__ void __launch_bounds__(384, 1)
-    redundancy_gemm_sym_kernel(const __grid_constant__ CUtensorMap amap,
-                               const __grid_constant__ CUtensorMap bmap, const GemmParams p) {
-  constexpr int NSB = kSymStages;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
-  const SymLayout L = sym_layout();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rank = static_cast<int>(cluster_ctarank());
-  const int group_id = static_cast<int>(cluster_id_x());
-  const int ngroups = static_cast<int>(cluster_count_x());
-  const bool leader = rank == 0;
-
-  uint64_t* a_full = reinterpret_cast<uint64_t*>(sm + L.bars);
-  uint64_t* a_empty = a_full + 1;
-  uint64_t* b_full = a_empty + 1;
-  uint64_t* b_empty = b_full + NSB;
-  uint64_t* acc_full = b_empty + NSB;      // [2] accumulator g holds a tile
-  uint64_t* acc_empty = acc_full + 2;      // [2] group g has read it (both CTAs)
-  uint64_t* row_full = acc_empty + 2;      // [kRowRing] both groups' row partials written
-  uint64_t* row_empty = row_full + kRowRing;   // [kRowRing] partials stored
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.slot);
-  volatile int* abort = reinterpret_cast<volatile int*>(sm + L.flags);
-
-  if (threadIdx.x == 0) {
-    mbar_init(a_full, 1);
-    mbar_init(a_empty, 1);
-    for (int s = 0; s < NSB; ++s) {
-      mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], 1);
-    }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(&acc_full[g], 1);
-      mbar_init(&acc_empty[g], 8);   // the group's 4 warps in each CTA of the pair
-    }
-    for (int b = 0; b < kRowRing; ++b) {
-      mbar_init(&row_full[b], 8);    // the 8 epilogue warps
-      mbar_init(&row_empty[b], 1);   // the row-store warp
-    }
-    *abort = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc<2>(tmem_slot, 512);
-    tmem_relinquish<2>();
-  }
-  tc_fence_before();
-  cluster_sync_all();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const int n_items = __ldg(&p.item_off[p.num_units]);
-
-  // item -> unit, pair j (a unit's pairs from the last down), its blocks
-  struct Item {
-    int u, j, np, nb, b0;
-    bool two;
-    int64_t base;
-  };
-  auto decode = [&](int item) {
-    Item it;
-    it.u = find_unit(p.item_off, p.num_units, item);
-    const int i0 = __ldg(&p.item_off[it.u]);
-    it.np = __ldg(&p.item_off[it.u + 1]) - i0;
-    it.j = it.np - 1 - (item - i0);
-    it.base = __ldg(&p.tok_off[it.u]);
-    const int N = static_cast<int>(__ldg(&p.tok_off[it.u + 1]) - it.base);
-    it.nb = (N + 255) / 256;
-    it.b0 = 2 * it.j;
-    it.two = it.b0 + 1 < it.nb;
-    return it;
-  };
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&amap);
-      prefetch_tmap(&bmap);
-      const uint64_t pol = policy_evict_normal();
-      const uint32_t a_full_lead = mapa(smem_u32(a_full), 0);
-      int stage = 0;
-      uint32_t ph = 0;
-      int ai = 0;
-      for (int item = group_id; item < n_items; item += ngroups, ++ai) {
-        const Item it = decode(item);
-        if (mbar_wait(a_empty, (ai & 1) ^ 1, abort, p.status)) {
-          const int nblk = it.two ? 2 : 1;
-          if (leader) mbar_arrive_expect_tx(a_full, 2 * nblk * 32768);
-          for (int k = 0; k < nblk; ++k) {
-            uint8_t* fd = sm + L.fix + k * 32768;
-            const int ya = static_cast<int>(it.base + (it.b0 + k) * 256 + rank * 128);
-            tma_load_2d_pair(fd, &amap, a_full_lead, 0, ya, pol);
-            tma_load_2d_pair(fd + 16384, &amap, a_full_lead, 64, ya, pol);
-          }
-        }
-        const int nA = it.two ? it.b0 + 2 : it.b0 + 1;   // row blocks 0 .. nA - 1
-        for (int a = 0; a < nA; ++a) {
-          if (mbar_wait(&b_empty[stage], ph ^ 1, abort, p.status)) {
-            uint8_t* bd = sm + L.b + stage * 32768;
-            const int yb = static_cast<int>(it.base + a * 256 + rank * 128);
-            const uint32_t bf_lead = mapa(smem_u32(&b_full[stage]), 0);
-            if (leader) mbar_arrive_expect_tx(&b_full[stage], 2 * 32768);
-            tma_load_2d_pair(bd, &bmap, bf_lead, 0, yb, pol);
-            tma_load_2d_pair(bd + 16384, &bmap, bf_lead, 64, yb, pol);
-          }
-          if (++stage == NSB) { stage = 0; ph ^= 1; }
-        }
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (leader) {   // the whole warp, converged; one elected lane issues
-      const uint32_t idesc = idesc_bf16_f32(256, 256);
-      int stage = 0;
-      uint32_t ph = 0;
-      uint32_t use[2] = {0, 0};   // tiles put in accumulator g so far
-      int ai = 0;
-      for (int item = group_id; item < n_items; item += ngroups, ++ai) {
-        const Item it = decode(item);
-        const bool aok = __all_sync(0xffffffffu, mbar_wait(a_full, ai & 1, abort, p.status));
-        const uint32_t faddr = smem_u32(sm + L.fix);
-        uint64_t fdesc[8];   // block b0; block b1 is 32 KiB further (2048 in 16-byte units)
-#pragma unroll
-        for (int kq = 0; kq < 8; ++kq)
-          fdesc[kq] = desc_kmajor_sw128(faddr + (kq >> 2) * 16384 + (kq & 3) * 32);
-        const int nA = it.two ? it.b0 + 2 : it.b0 + 1;
-        for (int a = 0; a < nA; ++a) {
-          const bool bok = mbar_wait(&b_full[stage], ph, abort, p.status);
-          const uint64_t sdesc0 = desc_kmajor_sw128(smem_u32(sm + L.b + stage * 32768));
-          bool all_ok = bok && aok;
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            if (g == 0 ? a > it.b0 : !it.two) continue;
-            bool go = mbar_wait(&acc_empty[g], (use[g] & 1) ^ 1, abort, p.status) && bok && aok;
-            go = __all_sync(0xffffffffu, go);
-            tc_fence_after();
-            if (go) {
-              const uint32_t d = tmem + g * 256;
-#pragma unroll
-              for (int kq = 0; kq < 8; ++kq) {
-                const uint32_t bo = (kq >> 2) * 16384 + (kq & 3) * 32;
-                mma_bf16_elect<2>(d, sdesc0 + (bo >> 4), fdesc[kq] + g * 2048, idesc, kq > 0);
-              }
-              commit_pair_elect(&acc_full[g]);
-            }
-            all_ok = all_ok && go;
-            ++use[g];
-          }
-          if (all_ok) commit_pair_elect(&b_empty[stage]);
-          if (++stage == NSB) { stage = 0; ph ^= 1; }
-        }
-        if (aok) commit_pair_elect(a_empty);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ row-sum store
-    // Per exchange (row block a of the item): both groups' partial row sums of
-    // this CTA's 128 rows, added and stored to the scratch slot (a, j).
-    const float* rr = reinterpret_cast<const float*>(sm + L.rowr);
-    uint32_t n = 0;   // row exchanges so far
-    for (int item = group_id; item < n_items; item += ngroups) {
-      const Item it = decode(item);
-      float* cs_u = p.cs + __ldg(&p.cs_off[it.u]);
-      const int nex = it.two ? it.b0 + 1 : it.b0;
-      for (int a = 0; a < nex; ++a, ++n) {
-        const uint32_t s = n % kRowRing;
-        mbar_wait(&row_full[s], (n / kRowRing) & 1, abort, p.status);
-        const float* x = rr + s * 512;
-        float tot[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int rl = lane + 32 * m;
-          tot[m] = x[rl] + x[128 + rl];
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&row_empty[s]);
-        float* dst = cs_u + sym_row_seg(a, it.np) +
-                     static_cast<int64_t>(it.j - (a + 1) / 2) * 256 + rank * 128;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) dst[lane + 32 * m] = tot[m];
-      }
-    }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ epilogue
-    const int g = (warp - 4) >> 2;        // group: accumulator and key block b0 + g
-    const int q = warp & 3;               // TMEM lane quarter
-    const int gq = lane >> 2, tq = lane & 3;
-    const int t128 = q * 32 + lane;       // thread within the group
-    float* wsm = reinterpret_cast<float*>(sm + L.wsm) + g * 256;
-    float* rowr = reinterpret_cast<float*>(sm + L.rowr);
-    float2* colx = reinterpret_cast<float2*>(sm + L.colx) + g * (4 * 4 * 32);
-    const uint32_t acc_empty_lead = mapa(smem_u32(&acc_empty[g]), 0);
-    const int rq = rank * 128 + q * 32;   // first row of this warp's quarter in a block
-    const uint32_t tgrp = tmem + (static_cast<uint32_t>(q * 32) << 16) + g * 256;
-    uint32_t use = 0;   // tiles drained from accumulator g so far
-    uint32_t nx = 0;    // row exchanges so far
-    auto exchange = [&](float rsum) {
-      const uint32_t s = nx % kRowRing;
-      mbar_wait(&row_empty[s], ((nx / kRowRing) & 1) ^ 1, abort, p.status);
-      rowr[s * 512 + g * 128 + q * 32 + gq + 8 * tq] = rsum;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&row_full[s]);
-      ++nx;
-    };
-    for (int item = group_id; item < n_items; item += ngroups) {
-      const Item it = decode(item);
-      if (g == 1 && !it.two) {
-        // no block b1: zeros for the row exchanges of the rows below b0
-        for (int a = 0; a < it.b0; ++a) exchange(0.f);
-        continue;
-      }
-      const int bg = it.b0 + g;
-      const float* rho_u = p.rho + __ldg(&p.rho_off[it.u]);
-      float* cs_u = p.cs + __ldg(&p.cs_off[it.u]);
-      // column weights rho_j of block bg, permuted so that for 32-column group
-      // c the quad thread tq finds the weights of its columns 32c + 8k + 2tq +
-      // {0, 1}, k = 0..3, as 8 consecutive floats
-      {
-        const int jj = 2 * t128;
-        const float2 wv = __ldg(reinterpret_cast<const float2*>(rho_u + bg * 256 + jj));
-        const int c = jj >> 5, k = (jj & 31) >> 3, tw = (jj & 7) >> 1;
-        *reinterpret_cast<float2*>(wsm + ((c * 4 + tw) * 4 + k) * 2) = wv;
-      }
-      named_bar_sync(4 + g, 128);
-      // rho_i-weighted column sums of block bg over this thread's rows:
-      // cp[c2][2k' + e] for column 64 c2 + 8k' + 2tq + e
-      float cp[4][16];
-#pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2)
-#pragma unroll
-        for (int k = 0; k < 16; ++k) cp[c2][k] = 0.f;
-      // weights of this thread's 4 rows of block a (gq + 8k of the quarter),
-      // loaded one tile ahead
-      const float* wrow = rho_u + rq + gq;
-      float nw0 = __ldg(wrow), nw1 = __ldg(wrow + 8), nw2 = __ldg(wrow + 16), nw3 = __ldg(wrow + 24);
-      auto tile = [&](auto diag_tag, int a) {
-        constexpr bool kDiag = decltype(diag_tag)::value;
-        const float w0 = nw0, w1 = nw1, w2 = nw2, w3 = nw3;
-        if constexpr (!kDiag) {   // the next tile of the group exists
-          const float* wn = wrow + (a + 1) * 256;
-          nw0 = __ldg(wn);
-          nw1 = __ldg(wn + 8);
-          nw2 = __ldg(wn + 16);
-          nw3 = __ldg(wn + 24);
-        }
-        mbar_wait(&acc_full[g], use & 1, abort, p.status);
-        __syncwarp();
-        tc_fence_after();
-        float a0 = 0.f, b0 = 0.f, a1 = 0.f, b1 = 0.f, a2 = 0.f, b2 = 0.f, a3 = 0.f, b3 = 0.f;
-        // chunk i = 8h + c: TMEM lanes 16h .. 16h + 15 of the quarter, columns
-        // 32c .. 32c + 31; a thread holds rows gq + 16h (v[4k], v[4k+1]) and
-        // gq + 16h + 8 (v[4k+2], v[4k+3]) at columns 32c + 8k + 2tq + {0, 1}
-        auto fold = [&](uint32_t (&v)[16], int h, int c) {
-          const float4 W0 = *reinterpret_cast<const float4*>(wsm + (c * 4 + tq) * 8);
-          const float4 W1 = *reinterpret_cast<const float4*>(wsm + (c * 4 + tq) * 8 + 4);
-          const float2 wc[4] = {make_float2(W0.x, W0.y), make_float2(W0.z, W0.w),
-                                make_float2(W1.x, W1.y), make_float2(W1.z, W1.w)};
-          if constexpr (kDiag) {
-            // rows and columns of one block: drop column - row == dd, local
-            // to the warp's 32 x 32 sub-block
-            const int dd = rq - 32 * c;
-            if (dd > -32 && dd < 32) {
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int col = 8 * k + 2 * tq + (e & 1);
-                  const int row = 16 * h + gq + ((e >> 1) << 3);
-                  if (col - row == dd) v[4 * k + e] = 0u;
-                }
-            }
-          }
-          float& pa = h ? a2 : a0;
-          float& pb = h ? b2 : b0;
-          float& qa = h ? a3 : a1;
-          float& qb = h ? b3 : b1;
-          const float wa = h ? w2 : w0, wb = h ? w3 : w1;
-          float* cc = &cp[c >> 1][8 * (c & 1)];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float x0 = __uint_as_float(v[4 * k]), x1 = __uint_as_float(v[4 * k + 1]);
-            const float y0 = __uint_as_float(v[4 * k + 2]), y1 = __uint_as_float(v[4 * k + 3]);
-            if constexpr (!kDiag) fma2(pa, pb, x0, x1, wc[k].x, wc[k].y);
-            fma2(cc[2 * k], cc[2 * k + 1], x0, x1, wa, wa);
-            if constexpr (!kDiag) fma2(qa, qb, y0, y1, wc[k].x, wc[k].y);
-            fma2(cc[2 * k], cc[2 * k + 1], y0, y1, wb, wb);
-          }
-        };
-        uint32_t va[16], vb[16];
-        tmem_ld16x256b_x4(tgrp, va);
-        tmem_wait_ld_dep16(va);
-#pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-          // chunk i in va, chunk i + 1 into vb meanwhile
-          tmem_ld16x256b_x4(tgrp + (static_cast<uint32_t>(((i + 1) >> 3) * 16) << 16) +
-                                32 * ((i + 1) & 7), vb);
-          fold(va, i >> 3, i & 7);
-          tmem_wait_ld_dep16(vb);
-          if (i + 2 < 16) {
-            tmem_ld16x256b_x4(tgrp + (static_cast<uint32_t>(((i + 2) >> 3) * 16) << 16) +
-                                  32 * ((i + 2) & 7), va);
-          } else {
-            // every chunk is in registers: hand the accumulator back
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_lead);
-          }
-          fold(vb, (i + 1) >> 3, (i + 1) & 7);
-          if (i + 2 < 16) tmem_wait_ld_dep16(va);
-        }
-        ++use;
-        if constexpr (!kDiag) {
-          // the quad's four threads hold disjoint columns of the same 4 rows:
-          // reduce-scatter so that thread tq keeps row gq + 8 tq
-          const float t0 = a0 + b0, t1 = a1 + b1, t2 = a2 + b2, t3 = a3 + b3;
-          const bool u2 = (lane & 2) != 0, u1 = (lane & 1) != 0;
-          const float k0 = (u2 ? t2 : t0) + __shfl_xor_sync(0xffffffffu, u2 ? t0 : t2, 2);
-          const float k1 = (u2 ? t3 : t1) + __shfl_xor_sync(0xffffffffu, u2 ? t1 : t3, 2);
-          exchange((u1 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, u1 ? k0 : k1, 1));
-        }
-      };
-      for (int a = 0; a < bg; ++a) tile(BoolTag<false>{}, a);
-      tile(BoolTag<true>{}, bg);
-      // group 0's diagonal row block b0 has a slot only for block b1's columns
-      if (g == 0 && it.two) exchange(0.f);
-      // ---- item end: column sums over the quad index gq (lane bits 2-4),
-      // reduce-scattered so that lane l keeps columns 2l and 2l + 1 of each
-      // 64-column group, then the four lane quarters through shared memory
-#pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2) {
-#pragma unroll
-        for (int sft = 16, n = 8; sft >= 4; sft >>= 1, n >>= 1) {
-          const bool up = (lane & sft) != 0;
-#pragma unroll
-          for (int k = 0; k < n; ++k) {
-            const float send = up ? cp[c2][k] : cp[c2][k + n];
-            const float keep = up ? cp[c2][k + n] : cp[c2][k];
-            cp[c2][k] = keep + __shfl_xor_sync(0xffffffffu, send, sft);
-          }
-        }
-        colx[(c2 * 4 + q) * 32 + lane] = make_float2(cp[c2][0], cp[c2][1]);
-      }
-      named_bar_sync(4 + g, 128);
-      if (q == 0) {
-#pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2) {
-          float2 acc = colx[(c2 * 4) * 32 + lane];
-#pragma unroll
-          for (int qq = 1; qq < 4; ++qq) {
-            const float2 y = colx[(c2 * 4 + qq) * 32 + lane];
-            acc.x += y.x;
-            acc.y += y.y;
-          }
-          // this CTA's rows' share; the pair's other CTA writes the other slot
-          *reinterpret_cast<float2*>(cs_u + (2 * bg + rank) * 256 + 64 * c2 + 2 * lane) = acc;
-        }
-      }
-    }
-  }
-
-  // ---------------------------------------------------------------- teardown
-  tc_fence_before();
-  cluster_sync_all();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc<2>(tmem, 512);
-  }
-}
-
 // One block, before the score kernel: the score chunks of every unit and their
 // prefix, zeroed exchange counters and, for the GEMM, items per unit and their
 // prefix, 256-aligned rho segment offsets, zeroed unit counters and (symmetric
@@ -1197,10 +781,10 @@ __global__ void plan_kernel(const PlanParams pp) {
 }
 
 // Symmetric form, after the GEMM: one CTA per unit.  Row i of block a (i < c)
-// gets the two CTAs' column sums of block a, then the row sums of its slots
-// (a, j) in pair order, is scaled by rho_i / (N - 1), and the token softmax
-// follows.  A thread takes 4 consecutive rows (one block) and reads one
-// aligned float4 per slot.
+// gets the two CTAs' column sums of block a, then the row sums of the slots
+// (a, b) for b = a + 1 .. nb - 1 in block order, is scaled by rho_i / (N - 1),
+// and the token softmax follows.  A thread takes 4 consecutive rows (one
+// block) and reads one aligned float4 per slot.
 constexpr int kFinishThreads = 512;
 __global__ void __launch_bounds__(kFinishThreads)
     sym_finish_kernel(const int64_t* __restrict__ tok_off, int U, int w,
@@ -1224,14 +808,12 @@ __global__ void __launch_bounds__(kFinishThreads)
       const float4 d0 = __ldcs(reinterpret_cast<const float4*>(cs_u + (2 * a) * 256 + lr));
       const float4 d1 = __ldcs(reinterpret_cast<const float4*>(cs_u + (2 * a + 1) * 256 + lr));
       float4 acc = make_float4(d0.x + d1.x, d0.y + d1.y, d0.z + d1.z, d0.w + d1.w);
-      // row block a's slots: pairs j = ceil(a / 2) .. np - 1, except the
-      // unwritten (nb - 1, np - 1) of an odd nb
-      const int np = (nb + 1) / 2;
-      const float* seg = cs_u + sym_row_seg(a, np) + lr;
-      const int nslots = np - (a + 1) / 2 - ((nb & 1) && a == nb - 1 ? 1 : 0);
+      const float* seg = cs_u + 512 * static_cast<int64_t>(nb) +
+                         256 * (static_cast<int64_t>(a) * (nb - 1) -
+                                static_cast<int64_t>(a) * (a - 1) / 2) + lr;
 #pragma unroll 4
-      for (int k = 0; k < nslots; ++k) {
-        const float4 y = __ldcs(reinterpret_cast<const float4*>(seg + k * 256));
+      for (int b = a + 1; b < nb; ++b) {
+        const float4 y = __ldcs(reinterpret_cast<const float4*>(seg + (b - a - 1) * 256));
         acc.x += y.x;
         acc.y += y.y;
         acc.z += y.z;
@@ -1278,26 +860,22 @@ namespace {
 // The symmetric form exists for CTA pairs and the row mean only (its tiles
 // are 256 x 256 and the column sums are added linearly).
 void* gemm_fn(bool pair, bool rowmax, bool sym) {
-  if (sym) return reinterpret_cast<void*>(&redundancy_gemm_sym_kernel);
+  if (sym) return reinterpret_cast<void*>(&redundancy_gemm_kernel<true, false, true>);
   if (pair) return rowmax ? reinterpret_cast<void*>(&redundancy_gemm_kernel<true, true, false>)
                           : reinterpret_cast<void*>(&redundancy_gemm_kernel<true, false, false>);
   return rowmax ? reinterpret_cast<void*>(&redundancy_gemm_kernel<false, true, false>)
                 : reinterpret_cast<void*>(&redundancy_gemm_kernel<false, false, false>);
 }
-int gemm_smem(bool pair, bool sym) {
-  if (sym) return static_cast<int>(sym_layout().total) + 1024;
-  return static_cast<int>(pair ? gemm_layout<true>().total : gemm_layout<false>().total) + 1024;
-}
 }  // namespace
 
 cudaError_t gemm_configure(bool pair, bool rowmax, bool sym) {
-  const int smem = gemm_smem(pair, sym);
+  const int smem = (pair ? gemm_layout<true>().total : gemm_layout<false>().total) + 1024;
   return cudaFuncSetAttribute(gemm_fn(pair, rowmax, sym),
                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
 int gemm_max_ctas(bool pair, bool rowmax, bool sym) {
-  const int smem = gemm_smem(pair, sym);
+  const int smem = (pair ? gemm_layout<true>().total : gemm_layout<false>().total) + 1024;
   void* f = gemm_fn(pair, rowmax, sym);
   int dev = 0, nsm = 0;
   cudaGetDevice(&dev);
@@ -1346,7 +924,7 @@ cudaError_t launch_sym_finish(const GemmParams& p, int nsm, cudaStream_t st) {
 
 cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const GemmParams& p,
                         bool pair, bool rowmax, bool sym, int nctas, cudaStream_t st) {
-  const int smem = gemm_smem(pair, sym);
+  const int smem = (pair ? gemm_layout<true>().total : gemm_layout<false>().total) + 1024;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nctas, 1, 1);
   cfg.blockDim = dim3(gemm_threads(sym), 1, 1);
@@ -1359,7 +937,8 @@ cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const 
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = pair ? 1 : 0;
-  if (sym) return cudaLaunchKernelEx(&cfg, redundancy_gemm_sym_kernel, amap, bmap, p);
+  if (sym)
+    return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<true, false, true>, amap, bmap, p);
   if (pair) {
     if (rowmax)
       return cudaLaunchKernelEx(&cfg, redundancy_gemm_kernel<true, true, false>, amap, bmap, p);

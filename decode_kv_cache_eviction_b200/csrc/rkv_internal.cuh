@@ -220,27 +220,22 @@ cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const 
 cudaError_t launch_sym_finish(const GemmParams& p, int nsm, cudaStream_t st);
 cudaError_t gemm_configure(bool pair, bool rowmax, bool sym);
 int gemm_max_ctas(bool pair, bool rowmax, bool sym);
-// Scratch of the symmetric form for one unit of nb = ceil(n / 256) blocks in
-// np = ceil(nb / 2) pairs (a work item holds key blocks 2j and 2j + 1): the
-// two CTAs' column sums of every block (2 x 256 floats per block, 1024 np in
-// all), then for each row block A its row sums over the columns of the pairs
-// j = ceil(A / 2) .. np - 1 (one 256-float slot each, starting at
-// 1024 np + 256 (A np - floor(A^2 / 4))).  The slot (nb - 1, np - 1) of an odd
-// nb is never written: that pair has block nb - 1 alone, its diagonal.  Every
-// other float is written by exactly one store of the GEMM.
+// Scratch of the symmetric form for one unit of nb = ceil(n / 256) blocks:
+// the two CTAs' column sums of every block (2 x 256 floats per block), then
+// for each block a the row sums of the slots (a, b), b = a + 1 .. nb - 1
+// (256 floats each).  128 nb (nb + 3) floats in all; every float is written
+// by exactly one store of the GEMM.
 __host__ __device__ inline int64_t sym_scratch_floats(int64_t n, int w) {
   if (n - w <= 0) return 0;
-  const int64_t nb = (n + 255) / 256, np = (nb + 1) / 2;
-  // column sums of every block (both CTAs of a pair), then the row slots
-  // (A, j) for j = ceil(A / 2) .. np - 1
-  return 1024 * np + 256 * (nb * np - nb * nb / 4);
+  const int64_t nb = (n + 255) / 256;
+  return 128 * nb * (nb + 3);
 }
 // GEMM work items of one unit: its blocks of candidate rows, or in the
-// symmetric form the pairs of its 256-key blocks (when it has candidates).
+// symmetric form all its 256-key blocks (when it has candidates).
 __host__ __device__ inline int64_t gemm_unit_items(int64_t n, int64_t c, int rows_per_item,
                                                    bool sym) {
   if (c <= 0) return 0;
-  return sym ? ((n + 255) / 256 + 1) / 2 : (c + rows_per_item - 1) / rows_per_item;
+  return sym ? (n + 255) / 256 : (c + rows_per_item - 1) / rows_per_item;
 }
 
 cudaError_t launch_select(const int64_t* tok_off, int U, int64_t Ttot, int w, int cmax,
