@@ -32,10 +32,12 @@
 //     whole item (block b's share from rows of blocks 0 .. b; the diagonal
 //     tile with its diagonal dropped), reduced across threads once per item;
 //   - for a < b, forms the rho_j-weighted row sums of block a's rows over
-//     block b's columns (a 4-thread reduction per 64-column group) and puts
-//     them in a shared-memory ring; warp 2 adds the four column groups and
-//     stores the sums to a scratch slot (a, b), so no epilogue warp waits
-//     for another.
+//     block b's columns (a 4-thread reduction per 128-column half) and puts
+//     them in a shared-memory ring; warp 2 adds the two halves and stores
+//     the sums to a scratch slot (a, b), so no epilogue warp waits for
+//     another.
+// The row weights rho_i of block a come from L2, loaded a tile ahead; the
+// column weights of block b are held in registers for the item.
 // Every slot is written by exactly one plain store, so nothing needs zeroing
 // and the result does not depend on timing.  A finish kernel adds, per row,
 // the two CTAs' column sums and the slots (a, b > a) in block order, scales by
