@@ -34,6 +34,17 @@ def test_header_and_binding_agree():
     assert header_functions() == sorted(B.EXPORTS)
 
 
+def test_kernel_timing_ids_match_header():
+    """The binding's per-kernel timing names are the header's RKV_KERNEL_*
+    enum, in value order, and RKV_NUM_KERNELS counts them."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    ids = {m.group(1).lower(): int(m.group(2))
+           for m in re.finditer(r"\bRKV_KERNEL_([A-Z]+)\s*=\s*(\d+)", text)}
+    num = int(re.search(r"\bRKV_NUM_KERNELS\s*=\s*(\d+)", text).group(1))
+    assert sorted(ids.values()) == list(range(num))
+    assert tuple(sorted(ids, key=ids.get)) == B.KERNELS
+
+
 def test_library_exports_every_header_symbol():
     out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
