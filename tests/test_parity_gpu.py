@@ -269,6 +269,29 @@ def test_budget_edges(mode):
             check_unit(out, b, u, w, 0.1, budget, redundancy=oracle_mode(mode))
 
 
+@pytest.mark.parametrize("mode", ["closed", "gemm", "max", "gemm_sym"])
+def test_units_without_candidates(mode):
+    """Units of exactly w tokens have no candidates: every token is kept, a and
+    r are zero there, and the units around them are unaffected (the GEMM forms
+    give such units no work items)."""
+    w = 8
+    lengths = [8, 300, 8, 9, 264, 8]
+    b = rand_batch(lengths, 4, w, seed=23)
+    out = run_engine(b, 4, w, 0.1, 16, mode=mode)
+    for u in range(len(lengths)):
+        check_unit(out, b, u, w, 0.1, 16, redundancy=oracle_mode(mode))
+
+
+def test_unit_shorter_than_window_is_rejected():
+    b = rand_batch([300, 5, 300], 4, 8, seed=29)
+    eng = Engine(4, 8, max_units=3, max_tokens=b.num_tokens, redundancy="closed")
+    a, r = eng.alloc_scores(b)
+    with pytest.raises(RkvError) as e:
+        eng.score(b, a, r)
+    assert e.value.code == -1   # RKV_ERR_INVALID_ARG
+    eng.close()
+
+
 def test_gemm_single_cta_and_pair_agree():
     b = rand_batch([3000, 4100, 700], 4, 8, seed=11)
     o1 = run_engine(b, 4, 8, 0.1, 256, mode="gemm", single_cta=True)
