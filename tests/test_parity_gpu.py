@@ -282,6 +282,22 @@ def test_units_without_candidates(mode):
         check_unit(out, b, u, w, 0.1, 16, redundancy=oracle_mode(mode))
 
 
+@pytest.mark.parametrize("mode", ["closed", "gemm_sym"])
+def test_many_small_units(mode):
+    """About 2000 short units in one batch (many score chunks, GEMM items and
+    select CTAs of the short shape), checked on every 7th unit and on every
+    unit's kept count."""
+    w = 8
+    rng = np.random.default_rng(37)
+    lengths = rng.choice([8, 9, 16, 33, 100, 257, 300], size=2000).tolist()
+    b = rand_batch(lengths, 4, w, seed=41, dup=0.1)
+    out = run_engine(b, 4, w, 0.1, 12, mode=mode)
+    for u in range(0, len(lengths), 7):
+        check_unit(out, b, u, w, 0.1, 12, redundancy=oracle_mode(mode))
+    want = [n if n - w <= 12 else 12 + w for n in lengths]
+    assert out["nk"].tolist() == want
+
+
 def test_unit_shorter_than_window_is_rejected():
     b = rand_batch([300, 5, 300], 4, 8, seed=29)
     eng = Engine(4, 8, max_units=3, max_tokens=b.num_tokens, redundancy="closed")
