@@ -56,8 +56,6 @@ namespace rkv {
 namespace {
 
 constexpr float kNegBig = -1e30f;  // initial running max (finite: no inf - inf)
-constexpr float kLazy = 8.f;       // log2 headroom before the running max moves
-constexpr int kConsumers = 384;    // softmax + norm threads
 constexpr int kBufCols = 256;      // tensor-memory columns per logit buffer
 constexpr uint64_t kDrainNs = 200000000ull;   // teardown wait for copies in flight
 
@@ -651,7 +649,6 @@ __global__ void __launch_bounds__(score_threads(CLOSED), 1)
     const int tp = warp >= 16 ? 1 : 0;       // this set's tile parity
     const int ctid = tp * 128 + (threadIdx.x - 256 - (tp ? 256 : 0));   // 0 .. NP2-1
     const int q4 = warp & 3;
-    const int row = q4 * 32 + lane;
     float* abuf = reinterpret_cast<float*>(sm + L.abuf);   // [2 slots][CHT]
     float* mpart = reinterpret_cast<float*>(sm + L.mpart); // [NP2][2]
     float* mfin = reinterpret_cast<float*>(sm + L.mrow);   // [RP][2] merged (max, 1 / sum)
